@@ -1,0 +1,364 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself
+(closed forms, invariants the pages fix, brute force on tiny inputs, independent
+library routines, finite differences).  No GPU."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, amp=1.0):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape) * amp
+
+
+# ----------------------------------------------------------------------------- plan
+
+def test_plan_golden_small():
+    """Hand-derived plans for S=8, cp=2 and S=12, cp=3 (golden file, derivation in it)."""
+    with open(os.path.join(GOLDEN, "plan_small.json")) as f:
+        gold = json.load(f)
+    for case in gold["cases"]:
+        p = oracle.plan(case["S"], case["cp"], case["rotate"], case.get("cu_seqlens"))
+        for key in ("perm", "inv_perm", "src", "doc_start", "rank_cu_off", "rank_cu", "pairs"):
+            assert p[key].tolist() == case[key], (case["name"], key)
+
+
+@pytest.mark.parametrize("S,cp", [(512, 2), (8192, 4), (32768, 8), (65536, 8), (131072, 8),
+                                  (96, 3), (40, 5), (4, 1)])
+def test_plan_equal_causal_work(S, cp):
+    """Head/tail pairing gives every rank the same causal pair count:
+    C^2 (2cp-1) + C (C+1), and the ranks together hold S(S+1)/2 pairs."""
+    p = oracle.plan(S, cp)
+    C = S // (2 * cp)
+    assert (p["pairs"] == C * C * (2 * cp - 1) + C * (C + 1)).all()
+    assert int(p["pairs"].sum()) == S * (S + 1) // 2
+    perm, inv = p["perm"], p["inv_perm"]
+    assert sorted(perm.tolist()) == list(range(S))            # a bijection
+    assert (perm[inv] == np.arange(S)).all() and (inv[perm] == np.arange(S)).all()
+
+
+def test_plan_surveyed_pair_counts():
+    expected = {512: 65664, 8192: 8389632, 32768: 67110912, 65536: 268439552,
+                131072: 1073750016}
+    for S, cp in [(512, 2), (8192, 4), (32768, 8), (65536, 8), (131072, 8)]:
+        assert int(oracle.plan(S, cp)["pairs"][0]) == expected[S]
+
+
+def test_plan_cp1_identity():
+    p = oracle.plan(64, 1)
+    assert p["perm"].tolist() == list(range(64))
+    assert p["src"].tolist() == [0]
+
+
+@pytest.mark.parametrize("cp", [2, 3, 4, 8])
+def test_plan_ring_and_allgather_orders(cp):
+    """Ring: step 0 is local and each step takes the left neighbour's shard, so every
+    shard is visited once; all-gather visits shards in rank order."""
+    S = 2 * cp * 4
+    ring = oracle.plan(S, cp, "ring")["src"].reshape(cp, cp)
+    ag = oracle.plan(S, cp, "allgather")["src"].reshape(cp, cp)
+    for r in range(cp):
+        assert ag[r].tolist() == list(range(cp))
+        assert ring[r, 0] == r
+        assert sorted(ring[r].tolist()) == list(range(cp))
+        for s in range(1, cp):
+            # what rank r sees at step s is what its left neighbour saw at step s-1
+            assert ring[r, s] == ring[(r - 1) % cp, s - 1]
+
+
+def test_plan_rejects_bad_configs():
+    with pytest.raises(ValueError):
+        oracle.plan(100, 3)          # 100 % 6 != 0
+    with pytest.raises(ValueError):
+        oracle.plan(64, 0)
+    with pytest.raises(ValueError):
+        oracle.plan(64, 2, "allgather", np.array([0, 10, 60], np.int32))   # last != S
+    with pytest.raises(ValueError):
+        oracle.plan(64, 2, "allgather", np.array([0, 30, 30, 64], np.int32))  # empty doc
+
+
+def test_plan_docs_pairs_and_segments():
+    lens = synth.doc_lengths(65536, 3)
+    cu = synth.cu_seqlens(lens)
+    p = oracle.plan(65536, 8, "ring", cu)
+    L = np.asarray(lens, dtype=np.int64)
+    assert int(p["pairs"].sum()) == int((L * (L + 1) // 2).sum())
+    # every local segment lies inside one chunk and one document
+    C = 65536 // 16
+    for r in range(8):
+        seg = p["rank_cu"][p["rank_cu_off"][r]:p["rank_cu_off"][r + 1]]
+        assert seg[0] == 0 and seg[-1] == 2 * C and C in seg
+        for a, b in zip(seg[:-1], seg[1:]):
+            assert b > a
+            orig = p["perm"][r * 2 * C + a:r * 2 * C + b]
+            assert (np.diff(orig) == 1).all()
+            assert len(set(p["doc_start"][r * 2 * C + a:r * 2 * C + b].tolist())) == 1
+
+
+def test_doc_lengths_recipe():
+    lens = synth.doc_lengths(65536, 3)
+    assert sum(lens) == 65536
+    assert all(128 <= n <= 32768 for n in lens[:-1]) and lens[-1] >= 1
+    # the median of a long draw sits near 2048
+    many = synth.doc_lengths(10_000_000, 11)
+    assert 1800 < float(np.median(many[:-1])) < 2300
+
+
+# -------------------------------------------------------------------- forward pins
+
+def brute_force(q, k, v, ds, scale):
+    """Materialised masked score matrix and an explicit softmax (tiny inputs only)."""
+    B, Hq, S, D = q.shape
+    g = Hq // k.shape[1]
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, S))
+    qi = np.arange(S)[:, None]
+    ki = np.arange(S)[None, :]
+    mask = (ki <= qi) & (ki >= ds[:, None])
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * q[b, h] @ k[b, h // g].T
+            s = np.where(mask, s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            p = e / e.sum(axis=1, keepdims=True)
+            o[b, h] = p @ v[b, h // g]
+            lse[b, h] = (m[:, 0] + np.log(e.sum(axis=1)))
+    return o, lse
+
+
+@pytest.mark.parametrize("Hq,Hkv,S,D,docs", [(2, 2, 16, 8, None), (4, 2, 24, 4, [0, 5, 6, 24]),
+                                             (3, 1, 33, 5, [0, 20, 33])])
+def test_fwd_brute_force(Hq, Hkv, S, D, docs):
+    q, k, v = rnd((2, Hq, S, D), 1), rnd((2, Hkv, S, D), 2), rnd((2, Hkv, S, D), 3)
+    cu = None if docs is None else np.array(docs, np.int32)
+    ds = oracle.doc_start(S, cu)
+    o, lse = oracle.fwd(q, k, v, ds)
+    bo, bl = brute_force(q, k, v, ds, 1 / math.sqrt(D))
+    np.testing.assert_allclose(o, bo, atol=1e-12)
+    np.testing.assert_allclose(lse, bl, atol=1e-12)
+
+
+def test_fwd_closed_forms():
+    """Row 0 sees only key 0: O = V[0], LSE = scale q0.k0.  With K = 0 every admitted
+    score is 0: O is the running mean of V and LSE = ln(#admitted keys)."""
+    S, D = 40, 16
+    q, k, v = rnd((1, 2, S, D), 4), rnd((1, 2, S, D), 5), rnd((1, 2, S, D), 6)
+    o, lse = oracle.fwd(q, k, v)
+    sc = 1 / math.sqrt(D)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], atol=1e-14)
+    np.testing.assert_allclose(lse[:, :, 0], sc * (q[:, :, 0] * k[:, :, 0]).sum(-1), atol=1e-14)
+    cu = np.array([0, 7, 19, 40], np.int32)
+    ds = oracle.doc_start(S, cu)
+    o, lse = oracle.fwd(q, np.zeros_like(k), v, ds)
+    for t in range(S):
+        np.testing.assert_allclose(o[:, :, t], v[:, :, ds[t]:t + 1].mean(axis=2), atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, t], math.log(t - ds[t] + 1), atol=1e-13)
+
+
+def test_fwd_rows_sum_to_one():
+    """Softmax rows sum to 1: with V = 1 every output element is exactly 1."""
+    S, D = 64, 8
+    q, k = rnd((1, 2, S, D), 7, 3.0), rnd((1, 2, S, D), 8, 3.0)
+    o, _ = oracle.fwd(q, k, np.ones((1, 2, S, D)), oracle.doc_start(S, [0, 10, 64]))
+    np.testing.assert_allclose(o, 1.0, atol=1e-13)
+
+
+def test_fwd_matches_torch_sdpa_gqa():
+    """Independent library routine: torch SDPA (fp64, causal, GQA by head groups)."""
+    B, Hq, Hkv, S, D = 1, 8, 2, 96, 32
+    q, k, v = rnd((B, Hq, S, D), 9), rnd((B, Hkv, S, D), 10), rnd((B, Hkv, S, D), 11)
+    o, _ = oracle.fwd(q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=True,
+        enable_gqa=True).numpy()
+    np.testing.assert_allclose(o, ref, atol=1e-12)
+
+
+def test_fwd_doc_mask_matches_per_document_sdpa():
+    """Packed documents: each document is causal attention on its own slice."""
+    S, D = 80, 16
+    q, k, v = rnd((1, 4, S, D), 12), rnd((1, 2, S, D), 13), rnd((1, 2, S, D), 14)
+    cu = np.array([0, 9, 10, 41, 80], np.int32)
+    o, _ = oracle.fwd(q, k, v, oracle.doc_start(S, cu))
+    for a, b in zip(cu[:-1], cu[1:]):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[:, :, a:b]), torch.from_numpy(k[:, :, a:b]),
+            torch.from_numpy(v[:, :, a:b]), is_causal=True, enable_gqa=True).numpy()
+        np.testing.assert_allclose(o[:, :, a:b], ref, atol=1e-12)
+
+
+def test_fwd_rows_equals_full():
+    S, D = 50, 8
+    q, k, v = rnd((2, 4, S, D), 15), rnd((2, 2, S, D), 16), rnd((2, 2, S, D), 17)
+    ds = oracle.doc_start(S, [0, 20, 50])
+    o, lse = oracle.fwd(q, k, v, ds)
+    rows = np.array([0, 3, 49, 2 * S + 21, 7 * S + 49])
+    ro, rl = oracle.fwd_rows(q, k, v, rows, ds)
+    np.testing.assert_allclose(ro, o.reshape(-1, D)[rows], atol=1e-14)
+    np.testing.assert_allclose(rl, lse.reshape(-1)[rows], atol=1e-14)
+
+
+# ------------------------------------------------------------- sharding + merge pins
+
+@pytest.mark.parametrize("cp,rotate,docs", [(2, "allgather", None), (2, "ring", None),
+                                            (4, "ring", None), (4, "allgather", [0, 3, 40, 41, 64]),
+                                            (8, "ring", [0, 17, 64]), (1, "allgather", None)])
+def test_sharded_merged_equals_unsharded(cp, rotate, docs):
+    """The principle the method rests on: attending Q_i to every K_j,V_j and combining
+    the partials gives exactly unsharded attention (to rounding)."""
+    S, D = 64, 8
+    q, k, v = rnd((1, 4, S, D), 18), rnd((1, 2, S, D), 19), rnd((1, 2, S, D), 20)
+    cu = None if docs is None else np.array(docs, np.int32)
+    o, lse = oracle.fwd(q, k, v, oracle.doc_start(S, cu))
+    so, sl = oracle.cp_fwd(q, k, v, cp, rotate, cu)
+    perm = oracle.plan(S, cp, rotate, cu)["perm"]
+    np.testing.assert_allclose(so, o[:, :, perm], atol=1e-12)
+    np.testing.assert_allclose(sl, lse[:, :, perm], atol=1e-12)
+
+
+def test_local_only_attention_breaks_parity():
+    """If only the local shard is attended (CP communication silently off), the result
+    is wrong: dropping steps s > 0 must fail parity."""
+    S, D, cp = 64, 8, 4
+    q, k, v = rnd((1, 2, S, D), 21), rnd((1, 2, S, D), 22), rnd((1, 2, S, D), 23)
+    o, _ = oracle.fwd(q, k, v)
+    lo, _ = oracle.cp_fwd(q, k, v, cp, "ring", steps=1)
+    perm = oracle.plan(S, cp)["perm"]
+    assert np.abs(lo - o[:, :, perm]).max() > 0.1
+
+
+def test_merge_identity_and_halves():
+    R, D = 30, 8
+    S = 40
+    q, k, v = rnd((1, 1, S, D), 24), rnd((1, 1, S, D), 25), rnd((1, 1, S, D), 26)
+    o, lse = oracle.fwd(q, k, v)
+    # identity: merging with an all-(-inf) partial
+    po = rnd((1, R, D), 27)
+    pl = rnd((1, R), 28)
+    mo, ml = oracle.lse_merge(np.concatenate([po, np.zeros((1, R, D))]),
+                              np.concatenate([pl, np.full((1, R), -np.inf)]))
+    np.testing.assert_allclose(mo, po[0], atol=1e-15)
+    np.testing.assert_allclose(ml, pl[0], atol=1e-15)
+    # halves of each row's key set: with the identity permutation and cp=2, "rank" 1
+    # holds rows 20..39 and the two "shards" are keys [0,20) and [20,40)
+    perm = np.arange(S, dtype=np.int32)
+    ds = np.zeros(S, np.int32)
+    first = oracle.partial(q, k, v, perm, 2, 1, 0, ds)
+    second = oracle.partial(q, k, v, perm, 2, 1, 1, ds)
+    mo, ml = oracle.lse_merge(np.stack([first[0][0], second[0][0]]),
+                              np.stack([first[1][0], second[1][0]]))
+    np.testing.assert_allclose(mo, o[0, 0, 20:], atol=1e-13)
+    np.testing.assert_allclose(ml, lse[0, 0, 20:], atol=1e-13)
+    # rows 0..19 against keys 20..39: every row empty -> (0, -inf)
+    empty = oracle.partial(q, k, v, perm, 2, 0, 1, ds)
+    assert np.isneginf(empty[1]).all() and (empty[0] == 0).all()
+
+
+def test_merge_associative():
+    P, R, D = 3, 20, 4
+    po, pl = rnd((P, R, D), 29), rnd((P, R), 30)
+    pl[1, :5] = -np.inf
+    full = oracle.lse_merge(po, pl)
+    ab = oracle.lse_merge(po[:2], pl[:2])
+    nested = oracle.lse_merge(np.stack([ab[0], po[2]]), np.stack([ab[1], pl[2]]))
+    np.testing.assert_allclose(full[0], nested[0], atol=1e-13)
+    np.testing.assert_allclose(full[1], nested[1], atol=1e-13)
+
+
+# ------------------------------------------------------------------- backward pins
+
+def _loss(q, k, v, dout, ds):
+    o, _ = oracle.fwd(q, k, v, ds)
+    return float((o * dout).sum())
+
+
+def test_bwd_finite_differences():
+    """Central differences in fp64 of L = sum(O * dO) on a tiny GQA + doc-mask case."""
+    B, Hq, Hkv, S, D = 1, 4, 2, 16, 8
+    q, k, v = rnd((B, Hq, S, D), 31), rnd((B, Hkv, S, D), 32), rnd((B, Hkv, S, D), 33)
+    dout = rnd((B, Hq, S, D), 34)
+    ds = oracle.doc_start(S, [0, 6, 16])
+    o, lse = oracle.fwd(q, k, v, ds)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds)
+    eps = 1e-6
+    g = np.random.default_rng(35)
+    for name, x, gx in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(12):
+            idx = tuple(int(g.integers(0, n)) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], dout, ds)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], dout, ds)
+            assert abs((lp - lm) / (2 * eps) - gx[idx]) < 1e-6, (name, idx)
+
+
+def test_bwd_matches_torch_autograd():
+    B, Hq, Hkv, S, D = 1, 4, 2, 48, 16
+    q, k, v = rnd((B, Hq, S, D), 36), rnd((B, Hkv, S, D), 37), rnd((B, Hkv, S, D), 38)
+    dout = rnd((B, Hq, S, D), 39)
+    o, lse = oracle.fwd(q, k, v)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True,
+                                                          enable_gqa=True)
+    to.backward(torch.from_numpy(dout))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+
+
+def test_bwd_sum_properties():
+    """Rows of P sum to 1, so sum_k dV_k = sum of dO over the group's rows, and
+    sum_k dK_k = 0 (since sum_k P dP = Dq)."""
+    B, Hq, Hkv, S, D = 1, 6, 2, 40, 8
+    q, k, v = rnd((B, Hq, S, D), 40), rnd((B, Hkv, S, D), 41), rnd((B, Hkv, S, D), 42)
+    dout = rnd((B, Hq, S, D), 43)
+    ds = oracle.doc_start(S, [0, 13, 40])
+    o, lse = oracle.fwd(q, k, v, ds)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds)
+    g = Hq // Hkv
+    for hk in range(Hkv):
+        np.testing.assert_allclose(dv[0, hk].sum(0), dout[0, hk * g:(hk + 1) * g].sum((0, 1)),
+                                   atol=1e-12)
+        np.testing.assert_allclose(dk[0, hk].sum(0), 0.0, atol=1e-12)
+
+
+def test_bwd_sampled_equals_full():
+    B, Hq, Hkv, S, D = 1, 4, 2, 36, 8
+    q, k, v = rnd((B, Hq, S, D), 44), rnd((B, Hkv, S, D), 45), rnd((B, Hkv, S, D), 46)
+    dout = rnd((B, Hq, S, D), 47)
+    ds = oracle.doc_start(S, [0, 11, 36])
+    o, lse = oracle.fwd(q, k, v, ds)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds)
+    rows = np.array([0, 5, 35, S + 12, 3 * S + 35])
+    np.testing.assert_allclose(oracle.bwd_dq_rows(q, k, v, dout, rows, ds),
+                               dq.reshape(-1, D)[rows], atol=1e-13)
+    keys = np.array([0, 10, 11, 35, S + 20])
+    sk, sv = oracle.bwd_dkv_keys(q, k, v, dout, keys, ds)
+    np.testing.assert_allclose(sk, dk.reshape(-1, D)[keys], atol=1e-13)
+    np.testing.assert_allclose(sv, dv.reshape(-1, D)[keys], atol=1e-13)
+
+
+# --------------------------------------------------------------- arithmetic pins
+
+def test_flop_convention_and_memory_estimate():
+    # 4*D*Hq per unmasked pair; the table's fwd FLOPs
+    assert abs(oracle.flops(2, 64, oracle.causal_pairs(512)) - 6.72e7) / 6.72e7 < 1e-3
+    assert abs(oracle.flops(32, 128, oracle.causal_pairs(131072)) - 1.407e14) / 1.407e14 < 1e-3
+    assert oracle.flops(8, 128, 100, backward=True) == 3 * oracle.flops(8, 128, 100)
+    # the concept guide's vanilla attention-matrix estimate: 128k*128k*2 B = 32 GiB per head
+    assert 131072 * 131072 * 2 == 32 * 2 ** 30
