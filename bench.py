@@ -1,0 +1,417 @@
+"""Benchmark: zigzag context-parallel causal attention on B200.
+
+One step = the whole hot path on one batch of seeded synthetic input already in
+HBM: cp_plan_shards (plan + gather of Q, K, V, dO into shard order),
+cp_attn_fwd (per-rank attention over the K/V shards in visit order, partials
+combined by the LSE-merge kernel), cp_attn_bwd (dQ, dK, dV).
+
+Metric: causal CP-attention TFLOPS, fwd+bwd, on the workload named in
+config.workload (default: 128k tokens, 32/8 GQA heads, head_dim 128, cp 8,
+all-gather order).  FLOPs follow the convention 4*D*Hq per unmasked pair for the
+forward and 3x that for forward + backward; the unmasked pair count comes from
+the library's own planner.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--rotate allgather|ring] [--impl native|reference]
+With N > 1 (launched by torchrun) every rank runs its own replica of the
+workload on its own GPU: the path has no cross-GPU exchange on one GPU's worth
+of virtual ranks, so there is no data-path collective; the barrier and the
+max-over-ranks timing use torch.distributed.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_init(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return dist
+
+
+def dist_barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def dist_max(dist, x: float, device=None) -> float:
+    """Max of a float over ranks (identity on one rank)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(value_per_rank_units: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return value_per_rank_units * world / (ms_max * 1e-3)
+
+
+# --------------------------------------------------------------------- peaks and clocks
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return dict(bf16=float(p["bf16_tflops"]), bf16_sustained=float(p["bf16_tflops_sustained"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=1400.0, hbm=FALLBACK_HBM_GBS,
+                    source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- CPU baseline (oracle)
+
+def cpu_baseline(w: synth.Workload, budget_tokens: int = 3072):
+    """The oracle, as it stands, on a bounded sample of the workload: forward and
+    backward of the first `budget_tokens` tokens of one KV group (all its query
+    heads), FLOPs by the same convention."""
+    import oracle  # test infrastructure: the only place the benchmark runs it
+    import torch
+    oracle.build()
+    g = w.num_heads // w.num_kv_heads
+    S = budget_tokens
+    t = synth.attn_inputs(1, g, 1, S, w.head_dim, w.seed, amp=w.amp, with_dout=True)
+    q, k, v, do = (t[n].to(torch.float64).numpy() for n in ("q", "k", "v", "do"))
+    cu = None
+    if w.docs:
+        lens = synth.doc_lengths(S, w.seed, w.doc_median, w.doc_sigma, w.doc_clip)
+        cu = synth.cu_seqlens(lens)
+    ds = oracle.doc_start(S, cu)
+    t0 = time.perf_counter()
+    o, lse = oracle.fwd(q, k, v, ds)
+    oracle.bwd(q, k, v, o, lse, do, ds)
+    dt = time.perf_counter() - t0
+    pairs = oracle.causal_pairs(S, cu)
+    flops = oracle.flops(g, w.head_dim, pairs, backward=True)
+    return dict(value=flops / dt / 1e12, unit="TFLOPS", cores=oracle.num_threads(), kind="oracle",
+                sample=f"fwd+bwd of the first {S} tokens of KV group 0 ({g} query heads, "
+                       f"head_dim {w.head_dim}), fp64 C oracle, {dt:.1f} s"), dt
+
+
+# --------------------------------------------------------------------- native arm
+
+KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_dkdv": 6.0, "bwd_dq": 2.0}   # x D*Hq*pairs
+
+
+def run_native(args, w, rank, world, local_rank):
+    import torch
+    import context_zigzag_cp_b200 as cz
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = dist_init(world, "nccl")
+    peaks = load_peaks()
+    rotate = args.rotate or w.rotate
+
+    t = synth.workload_inputs(w, device=device, with_dout=True)
+    cu = None if t["cu_seqlens"] is None else torch.from_numpy(t["cu_seqlens"]).to(device)
+    prob = cz.Problem(w.batch, w.seq_len, w.cp, w.num_heads, w.num_kv_heads, w.head_dim, rotate,
+                      cu, merge="separate")
+    prob_fused = prob.with_merge("fused")
+    plan = cz.Plan(prob)
+    q, k, v, do = t["q"], t["k"], t["v"], t["do"]
+    qs, ks, vs, dos = (torch.empty_like(x) for x in (q, k, v, do))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_f = torch.empty(max(cz.fwd_workspace_bytes(prob), 256), dtype=torch.uint8, device=device)
+    ws_b = torch.empty(max(cz.bwd_workspace_bytes(prob), 256), dtype=torch.uint8, device=device)
+
+    def step():
+        plan.build([q, k, v, do], [qs, ks, vs, dos])
+        cz.attn_fwd(prob, plan, qs, ks, vs, o, lse, ws=ws_f)
+        cz.attn_bwd(prob, plan, qs, ks, vs, o, lse, dos, dq, dk, dv, ws=ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = cz.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    pairs = int(plan.pairs.sum().item()) * w.batch
+    fwd_flops = 4.0 * w.head_dim * w.num_heads * pairs
+    step_flops = 3.0 * fwd_flops
+
+    # ---- timed region: K steps, barrier + synchronize on both sides
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch0 = cz.launch_count()
+    with ClockSampler(local_rank) as clocks:
+        dist_barrier(dist, device)
+        torch.cuda.synchronize()
+        ev0.record()
+        for _ in range(args.steps):
+            step()
+        ev1.record()
+        torch.cuda.synchronize()
+        dist_barrier(dist, device)
+    launches = (cz.launch_count() - n_launch0)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = dist_max(dist, ms, device)
+    value = aggregate(step_flops / 1e12, world, ms_max)
+
+    # ---- per-kernel times inside one traced step (same stream)
+    with cz.LaunchTrace(256) as tr:
+        step()
+    per = {}
+    for name, kms in tr.launches():
+        a = per.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += kms
+    kernels = {n: {"launches": c, "ms": round(t_, 4)} for n, (c, t_) in per.items()}
+    for n, share in KERNEL_FLOP_SHARE.items():
+        if n in kernels:
+            kernels[n]["tflops"] = round(share * w.head_dim * w.num_heads * pairs /
+                                         (kernels[n]["ms"] / kernels[n]["launches"]) / 1e9, 1)
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    dom_flops = KERNEL_FLOP_SHARE.get(dom, 0.0) * w.head_dim * w.num_heads * pairs
+    dom_ms = kernels[dom]["ms"] / kernels[dom]["launches"]
+    achieved = dom_flops / dom_ms / 1e9 if dom_flops else 0.0
+    peak = peaks["bf16_sustained"]
+
+    # ---- forward alone, both merge modes (device time of the cp_attn_fwd call)
+    def time_fwd(pr, n=3):
+        cz.attn_fwd(pr, plan, qs, ks, vs, o, lse, ws=ws_f)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            cz.attn_fwd(pr, plan, qs, ks, vs, o, lse, ws=ws_f)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    fwd_ms = dist_max(dist, time_fwd(prob), device)
+    fused_ms = dist_max(dist, time_fwd(prob_fused), device)
+
+    # ---- end to end through the public API with pinned host buffers
+    hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
+    ho, hl = torch.empty_like(o, device="cpu").pin_memory(), torch.empty_like(lse, device="cpu").pin_memory()
+    hdq, hdk, hdv = (torch.empty_like(x, device="cpu").pin_memory() for x in (dq, dk, dv))
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+    d2h = sum(x.numel() * x.element_size() for x in (ho, hl, hdq, hdk, hdv))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        do.copy_(hdo, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    dist_barrier(dist, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(max(1, args.steps // 2)):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(dist, e0.elapsed_time(e1) / max(1, args.steps // 2), device)
+    st = cz.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed region")
+
+    out = None
+    if rank == 0:
+        clk = clocks.summary()
+        base, _ = cpu_baseline(w) if not args.no_cpu_baseline else (None, 0)
+        out = {
+            "metric": "causal CP-attention TFLOPS fwd+bwd on 1 B200",
+            "value": round(value, 2),
+            "unit": "TFLOPS",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_max, 3),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO)",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "cp": w.cp,
+                       "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+                       "head_dim": w.head_dim, "rotate": rotate,
+                       "mask": "doc" if w.docs else "causal", "merge": "separate",
+                       "l2": "inputs larger than L2 (Q alone is %.0f MiB)" % (
+                           q.numel() * 2 / 2 ** 20),
+                       "parallelism": f"replicas x{world}"},
+            "fwd_tflops": round(fwd_flops / 1e9 / fwd_ms, 1),
+            "fwd_frac_of_peak": round(fwd_flops / 1e9 / fwd_ms / peaks["bf16"], 4),
+            "fwd_fused_tflops": round(fwd_flops / 1e9 / fused_ms, 1),
+            "fwd_fused_frac_of_peak": round(fwd_flops / 1e9 / fused_ms / peaks["bf16"], 4),
+            "step_frac_of_peak": round(value / world / peaks["bf16_sustained"], 4),
+            "peak_source": peaks["source"],
+            "pairs": pairs,
+            "kernels": kernels,
+            "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": None},
+            "e2e": {"value": round(step_flops * world / 1e9 / e2e_ms, 2), "unit": "TFLOPS",
+                    "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": base,
+        }
+    if dist is not None:
+        dist_barrier(dist, device)
+        dist.destroy_process_group()
+    return out
+
+
+# --------------------------------------------------------------------- reference arm (oracle)
+
+def run_reference(args, w, rank, world):
+    """The oracle timed on the host cores; rank 0 only."""
+    if rank != 0:
+        return None
+    base, _ = cpu_baseline(w)           # warm-up / first call builds the oracle
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline(w, budget_tokens=1024)
+    for _ in range(args.steps):
+        b, dt = cpu_baseline(w, budget_tokens=1536)
+        vals.append((b, dt))
+    tot_flops = sum(b["value"] * dt for b, dt in vals) * 1e12
+    tot_t = sum(dt for _, dt in vals)
+    value = tot_flops / tot_t / 1e12
+    return {
+        "impl": "reference",
+        "metric": "causal CP-attention TFLOPS fwd+bwd on 1 B200",
+        "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(tot_t / len(vals) * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "sample": vals[0][0]["sample"]},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": base["cores"],
+                         "kind": "oracle", "sample": vals[0][0]["sample"]},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="long128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--rotate", default=None, choices=["allgather", "ring"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local_rank = dist_env()
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        out = run_reference(args, w, rank, world)
+    else:
+        out = run_native(args, w, rank, world, local_rank)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,265 @@
+"""Zigzag context-parallel causal attention on one B200.
+
+A thin binding over libcpattn (include/cp_attn.h): every step of the path
+(plan, gather, forward, merge, backward) runs in the library's CUDA kernels;
+this module only marshals torch tensors (device memory and streams) into the
+C ABI.  There is no CPU fallback: without the built library every call raises.
+
+Typical use (all tensors on one CUDA device, bf16 BHSD in original order):
+
+    prob = Problem(batch=1, seq_len=S, cp=8, num_heads=32, num_kv_heads=8, head_dim=128,
+                   rotate="ring")
+    plan = Plan(prob)
+    qs, ks, vs = plan.shard([q, k, v])            # original -> shard order
+    o, lse = attn_fwd(prob, plan, qs, ks, vs)     # shard order
+    dq, dk, dv = attn_bwd(prob, plan, qs, ks, vs, o, lse, plan.shard([do])[0])
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import CpPlan, CpProblem, STATUS_NAMES
+
+__all__ = ["CPError", "Problem", "Plan", "attn_fwd", "attn_bwd", "lse_merge",
+           "fwd_workspace_bytes", "bwd_workspace_bytes", "get_device_status",
+           "set_wait_limit_ns", "selftest_wait_timeout", "version", "lib", "launch_count",
+           "LaunchTrace"]
+
+
+class CPError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise CPError(status, what)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def version() -> int:
+    return int(lib().cp_version())
+
+
+class Problem:
+    """cp_problem_t.  ``cu_seqlens`` (int32, original order, device) turns on the
+    packed-document mask."""
+
+    def __init__(self, batch: int, seq_len: int, cp: int, num_heads: int, num_kv_heads: int,
+                 head_dim: int, rotate: str = "allgather", cu_seqlens: torch.Tensor | None = None,
+                 merge: str = "fused", softmax_scale: float = 0.0):
+        self.cu_seqlens = cu_seqlens
+        self.batch, self.seq_len, self.cp = batch, seq_len, cp
+        self.num_heads, self.num_kv_heads, self.head_dim = num_heads, num_kv_heads, head_dim
+        self.rotate, self.merge = rotate, merge
+        self.num_docs = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+        self.c = CpProblem(batch, seq_len, cp, num_heads, num_kv_heads, head_dim,
+                           _lib.ROTATE[rotate], _lib.MASK["causal" if cu_seqlens is None else "doc"],
+                           _lib.MERGE[merge], float(softmax_scale), self.num_docs, 0,
+                           None if cu_seqlens is None else cu_seqlens.data_ptr())
+
+    def with_merge(self, merge: str) -> "Problem":
+        return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
+                       self.head_dim, self.rotate, self.cu_seqlens, merge,
+                       self.c.softmax_scale)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+class Plan:
+    """Caller-owned plan buffers (cp_plan_t) filled by cp_plan_shards."""
+
+    def __init__(self, prob: Problem, device=None, stream=None):
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        S, cp = prob.seq_len, prob.cp
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.prob = prob
+        self.perm = torch.empty(S, **i32)
+        self.inv_perm = torch.empty(S, **i32)
+        self.src = torch.empty(cp * cp, **i32)
+        self.doc_start = torch.empty(S, **i32)
+        self.rank_cu_off = torch.empty(cp + 1, **i32)
+        self.rank_cu = torch.empty(3 * cp + max(prob.num_docs, 1), **i32)
+        self.pairs = torch.empty(cp, dtype=torch.int64, device=dev)
+        self.c = CpPlan(*(t.data_ptr() for t in (self.perm, self.inv_perm, self.src,
+                                                  self.doc_start, self.rank_cu_off,
+                                                  self.rank_cu, self.pairs)))
+        self.build(stream=stream)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+    def _bufs(self, tensors):
+        n = len(tensors)
+        for t in tensors:
+            if t.dim() < 2 or t.shape[-2] != self.prob.seq_len or not t.is_contiguous():
+                raise ValueError("buffers must be contiguous [..., seq_len, row] tensors")
+        outer = (ctypes.c_int64 * max(n, 1))(*[t[..., 0, 0].numel() for t in tensors])
+        row = (ctypes.c_int64 * max(n, 1))(*[t.shape[-1] * t.element_size() for t in tensors])
+        return n, outer, row
+
+    def build(self, bufs_in=(), bufs_out=(), stream=None):
+        n, outer, row = self._bufs(list(bufs_in))
+        pin = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in bufs_in])
+        pout = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in bufs_out])
+        _check(lib().cp_plan_shards(self.prob.ref, self.ref, n, pin, pout, outer, row, None,
+                                    None, _stream(stream)), "cp_plan_shards")
+
+    def shard(self, tensors, stream=None):
+        """Gather tensors [..., S, row] from original into shard order (new tensors)."""
+        outs = [torch.empty_like(t) for t in tensors]
+        self.build(tensors, outs, stream)
+        return outs
+
+    def unshard(self, tensors, stream=None):
+        """Scatter tensors [..., S, row] from shard back into original order."""
+        outs = [torch.empty_like(t) for t in tensors]
+        n, outer, row = self._bufs(list(tensors))
+        pin = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in tensors])
+        pout = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in outs])
+        _check(lib().cp_unshard(self.prob.ref, self.ref, n, pin, pout, outer, row,
+                                _stream(stream)), "cp_unshard")
+        return outs
+
+
+def fwd_workspace_bytes(prob: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    dummy = ctypes.c_void_p(256)
+    plan = CpPlan(256, 256, 256, 256, 256, 256, 256)
+    _check(lib().cp_attn_fwd(prob.ref, ctypes.byref(plan), dummy, dummy, dummy, dummy, dummy,
+                             None, ctypes.byref(n), None), "cp_attn_fwd(workspace query)")
+    return n.value
+
+
+def bwd_workspace_bytes(prob: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    d = ctypes.c_void_p(256)
+    plan = CpPlan(256, 256, 256, 256, 256, 256, 256)
+    _check(lib().cp_attn_bwd(prob.ref, ctypes.byref(plan), d, d, d, d, d, d, d, d, d, None,
+                             ctypes.byref(n), None), "cp_attn_bwd(workspace query)")
+    return n.value
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def attn_fwd(prob: Problem, plan: Plan, q, k, v, o=None, lse=None, ws=None, stream=None):
+    """cp_attn_fwd on shard-order q [B,Hq,S,D], k/v [B,Hkv,S,D]; returns (o, lse)."""
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    nbytes = fwd_workspace_bytes(prob)
+    w = _workspace(nbytes, q.device, ws)
+    n = ctypes.c_size_t(nbytes)
+    _check(lib().cp_attn_fwd(prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                             _ptr(w), ctypes.byref(n) if w is not None else None,
+                             _stream(stream)), "cp_attn_fwd")
+    return o, lse
+
+
+def attn_bwd(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq=None, dk=None, dv=None,
+             ws=None, stream=None):
+    """cp_attn_bwd; returns (dq, dk, dv) in shard order."""
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = bwd_workspace_bytes(prob)
+    w = _workspace(nbytes, q.device, ws)
+    n = ctypes.c_size_t(nbytes)
+    _check(lib().cp_attn_bwd(prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                             _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(w),
+                             ctypes.byref(n) if w is not None else None, _stream(stream)),
+           "cp_attn_bwd")
+    return dq, dk, dv
+
+
+def lse_merge(o_parts, lse_parts, o_out=None, lse_out=None, stream=None):
+    """cp_lse_merge on o_parts fp32 [n, rows, D], lse_parts fp32 [n, rows]."""
+    n, rows, D = o_parts.shape
+    if o_out is None:
+        o_out = torch.empty((rows, D), dtype=torch.bfloat16, device=o_parts.device)
+    if lse_out is None:
+        lse_out = torch.empty(rows, dtype=torch.float32, device=o_parts.device)
+    _check(lib().cp_lse_merge(rows, D, n, _ptr(o_parts), _ptr(lse_parts), _ptr(o_out),
+                              _ptr(lse_out), _stream(stream)), "cp_lse_merge")
+    return o_out, lse_out
+
+
+def get_device_status(stream=None) -> int:
+    st = ctypes.c_int32(0)
+    _check(lib().cp_get_device_status(ctypes.byref(st), _stream(stream)), "cp_get_device_status")
+    return st.value
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    _check(lib().cp_set_wait_limit_ns(int(limit_ns)), "cp_set_wait_limit_ns")
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(lib().cp_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "cp_selftest_wait_timeout")
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().cp_launch_count())
+
+
+class LaunchTrace:
+    """Context manager around cp_trace_begin / cp_trace_end: CUDA events recorded
+    on the launching stream just before and after each library kernel launch."""
+
+    def __init__(self, capacity: int = 512):
+        self.cap = capacity
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.events:          # torch creates the CUDA event on first record
+            e.record()
+        torch.cuda.synchronize()
+        self._handles = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.events])
+        self._ids = (ctypes.c_int32 * capacity)()
+        self.n = 0
+
+    def __enter__(self):
+        _check(lib().cp_trace_begin(self._handles, self.cap), "cp_trace_begin")
+        return self
+
+    def __exit__(self, *exc):
+        n = ctypes.c_int32(0)
+        _check(lib().cp_trace_end(ctypes.byref(n), self._ids), "cp_trace_end")
+        self.n = n.value
+        return False
+
+    def launches(self):
+        """[(kernel name, milliseconds)] for the traced launches (synchronises)."""
+        torch.cuda.synchronize()
+        out = []
+        for i in range(min(self.n, self.cap)):
+            name = _lib.KERNEL_NAMES.get(self._ids[i], str(self._ids[i]))
+            out.append((name, self.events[2 * i].elapsed_time(self.events[2 * i + 1])))
+        return out

@@ -1,0 +1,666 @@
+// Backward kernels.  Gradients of causal (optionally packed-document) attention
+// from the saved final LSE, with P = exp(scale q.k - LSE_q) recomputed on the
+// fly:  D_q = dO_q . O_q,  dV_k = sum_q P dO_q,  dS = P (dO_q . v_k - D_q),
+// dQ_q = scale sum_k dS k_k,  dK_k = scale sum_q dS q_q.
+//
+// Two deterministic passes, no atomics:
+//   * bwd_prep_kernel: D (fp32) and LSE * log2(e) per row.
+//   * cp_bwd_dkdv_kernel (KV-tile major): one CTA owns a 128-key tile of KV
+//     head j and loops over every query head of its group and every virtual
+//     rank's query tile that attends to it (the single-GPU form of handing
+//     dK_j / dV_j back around the ring), accumulating dK and dV in tensor
+//     memory:  S^T = K Q^T,  dP^T = V dO^T  ->  P^T, dS^T (bf16, tensor memory)
+//     ->  dV += P^T dO,  dK += dS^T Q.
+//   * cp_bwd_dq_kernel (query-tile major, visiting the K/V shards in the plan's
+//     order like the forward):  S = Q K^T,  dP = dO V^T  ->  dS (bf16, tensor
+//     memory)  ->  dQ += dS K.
+// Each 128-row tile lives in one zigzag chunk, so original positions are
+// linear inside a tile and the causal / document tests are per-tile ranges.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+#include "zigzag.cuh"
+#include "fwd.cuh"
+
+namespace cpattn {
+
+// ----------------------------------------------------------------------------
+// Preprocess: delta[row] = sum_d dO*O, lse2[row] = LSE * log2(e).  One warp
+// per row; lane l reads 4 consecutive elements (head_dim <= 128).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                const float* __restrict__ lse, float* __restrict__ delta,
+                float* __restrict__ lse2, int64_t rows, int D)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t row = warp_g; row < rows; row += nwarps) {
+        float acc = 0.f;
+        if (lane * 4 < D) {
+            const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + row * D) + lane);
+            const uint2 b = __ldg(reinterpret_cast<const uint2*>(dout + row * D) + lane);
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float2 x = __bfloat1622float2(a2[i]), y = __bfloat1622float2(b2[i]);
+                acc = fmaf(x.x, y.x, acc);
+                acc = fmaf(x.y, y.y, acc);
+            }
+        }
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+            delta[row] = acc;
+            lse2[row] = __ldg(lse + row) * 1.4426950408889634f;
+        }
+    }
+}
+
+struct BwdParams {
+    int32_t B, Hq, Hkv, S, cp, C;
+    int32_t docs;
+    float scale;             // softmax scale
+    float scale_log2;        // softmax scale * log2(e)
+    int32_t n_items;
+    const int32_t* src;      // [cp*cp]
+    const int32_t* doc_start;  // [S] shard order
+    const float* lse2;       // [B*Hq][S]
+    const float* delta;      // [B*Hq][S]
+    __nv_bfloat16* dq;       // [B*Hq][S][D]
+    __nv_bfloat16* dk;       // [B*Hkv][S][D]
+    __nv_bfloat16* dv;
+};
+
+// ============================================================================
+// dK / dV pass
+// ============================================================================
+template <int D>
+struct DkdvCfg {
+    static constexpr int TILE = 128 * D * 2;
+    static constexpr int NST = (D == 128) ? 2 : 4;            // Q/dO stages
+    static constexpr int ST_STRIDE = 2 * TILE + 2048;          // Q | dO | lse2 | delta | ds
+    static constexpr int K_OFF = 0, V_OFF = TILE;
+    static constexpr int ST_OFF = 2 * TILE;
+    static constexpr int BAR_OFF = ST_OFF + NST * ST_STRIDE;
+    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full, acc_full, drain
+    static constexpr int NBAR = 6 + 2 * NST;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
+    static constexpr int THREADS = 192;
+};
+
+struct DkdvItem {
+    int bkv, b, hk, kpos, ko;
+};
+
+__device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int w)
+{
+    DkdvItem it;
+    const int BHkv = P.B * P.Hkv;
+    it.bkv = w % BHkv;
+    const int t = w / BHkv;                  // key tile by ascending original position
+    it.b = it.bkv / P.Hkv;
+    it.hk = it.bkv - it.b * P.Hkv;
+    it.ko = t * 128;
+    it.kpos = shard_of_orig(it.ko, P.C, P.cp);
+    return it;
+}
+
+// Iterates the (query head, query tile) pairs that attend to a key tile, in the
+// same order for every role.  Query tiles are visited rank by rank.
+struct QTileWalk {
+    int g, nqt;   // heads per group, query tiles per rank
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                   const BwdParams P)
+{
+    using Cfg = DkdvCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sK = sbase + Cfg::K_OFF, sV = sbase + Cfg::V_OFF, sST = sbase + Cfg::ST_OFF;
+    const uint32_t bars = sbase + Cfg::BAR_OFF;
+    const uint32_t bar_kv_full = bars, bar_kv_empty = bars + 8;
+    const uint32_t bar_st_full = bars + 16, bar_st_empty = bars + 16 + 8 * Cfg::NST;
+    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST, bar_p_full = bar_s_full + 8;
+    const uint32_t bar_acc_full = bar_s_full + 16, bar_drain = bar_s_full + 24;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = P.Hq / P.Hkv;
+    const int n2c = 2 * P.C;
+    const int nqt = n2c / 128;
+    const uint32_t st_bytes = 2 * Cfg::TILE + 1024 + (P.docs ? 512 : 0);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar_kv_full, 1);
+        mbar_init(bar_kv_empty, 1);
+        for (int i = 0; i < Cfg::NST; ++i) {
+            mbar_init(bar_st_full + 8 * i, 1);
+            mbar_init(bar_st_empty + 8 * i, 1);
+        }
+        mbar_init(bar_s_full, 1);
+        mbar_init(bar_p_full, 4);
+        mbar_init(bar_acc_full, 1);
+        mbar_init(bar_drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(smem_u32(tmem_slot), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmdO);
+            uint32_t nst = 0, iter = 0;
+            bool ok = true, kv_issued = false;
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+                const DkdvItem it = decode_dkdv(P, w);
+                ok = mbar_wait(bar_kv_empty, (iter & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                kv_issued = true;
+                mbar_arrive_expect_tx(bar_kv_full, 2 * Cfg::TILE);
+                for (int h = 0; h < D / 64; ++h) {
+                    tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
+                    tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
+                }
+                for (int hq = 0; hq < g && ok; ++hq) {
+                    const int bh = it.b * P.Hq + it.hk * g + hq;
+                    for (int qt = 0; qt < P.cp * nqt && ok; ++qt) {
+                        const int qpos = qt * 128;
+                        const int qo = orig_of_shard(qpos, P.C, P.cp);
+                        const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
+                        const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                        if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                        const uint32_t slot = nst % Cfg::NST, par = (nst / Cfg::NST) & 1;
+                        ++nst;
+                        ok = mbar_wait(bar_st_empty + 8 * slot, par ^ 1, abort_flag);
+                        if (!ok) break;
+                        const uint32_t st = sST + slot * Cfg::ST_STRIDE;
+                        const size_t row = static_cast<size_t>(bh) * P.S + qpos;
+                        mbar_arrive_expect_tx(bar_st_full + 8 * slot, st_bytes);
+                        for (int h = 0; h < D / 64; ++h) {
+                            tma_load_2d(st + h * 16384, &tmQ, h * 64, static_cast<int>(row), bar_st_full + 8 * slot);
+                            tma_load_2d(st + Cfg::TILE + h * 16384, &tmdO, h * 64, static_cast<int>(row),
+                                        bar_st_full + 8 * slot);
+                        }
+                        bulk_load(st + 2 * Cfg::TILE, P.lse2 + row, 512, bar_st_full + 8 * slot);
+                        bulk_load(st + 2 * Cfg::TILE + 512, P.delta + row, 512, bar_st_full + 8 * slot);
+                        if (P.docs)
+                            bulk_load(st + 2 * Cfg::TILE + 1024, P.doc_start + qpos, 512, bar_st_full + 8 * slot);
+                    }
+                }
+            }
+            if (!ok) {
+                for (uint32_t n = (nst > Cfg::NST ? nst - Cfg::NST : 0); n < nst; ++n)
+                    mbar_wait_drain(bar_st_full + 8 * (n % Cfg::NST), (n / Cfg::NST) & 1);
+                // the K/V load of the item that was in progress (if it was issued)
+                if (kv_issued) mbar_wait_drain(bar_kv_full, (iter & 1));
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);   // K-major A and B
+            constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A tmem, B MN-major
+            const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+            uint32_t nst = 0, iter = 0, p_phase = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+                const DkdvItem it = decode_dkdv(P, w);
+                ok = mbar_wait(bar_kv_full, iter & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                bool first = true;
+                for (int hq = 0; hq < g && ok; ++hq) {
+                    for (int qt = 0; qt < P.cp * nqt && ok; ++qt) {
+                        const int qpos = qt * 128;
+                        const int qo = orig_of_shard(qpos, P.C, P.cp);
+                        const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
+                        const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                        if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                        const uint32_t slot = nst % Cfg::NST, par = (nst / Cfg::NST) & 1;
+                        ++nst;
+                        ok = mbar_wait(bar_st_full + 8 * slot, par, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sQ = sST + slot * Cfg::ST_STRIDE, sdO = sQ + Cfg::TILE;
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+                            mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
+                                   IDESC_S, k > 0 ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+                            mma_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024),
+                                   IDESC_S, k > 0 ? 1u : 0u);
+                        }
+                        mma_commit(bar_s_full);
+                        ok = mbar_wait(bar_p_full, p_phase, abort_flag);
+                        if (!ok) break;
+                        p_phase ^= 1;
+                        tc_fence_after();
+                        // dV += P^T dO ; dK += dS^T Q   (K dimension = 128 query rows)
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tdV, tS + k * 8, sdesc_sw128(sdO + k * 2048, 16384, 1024), IDESC_G,
+                                   (!first || k > 0) ? 1u : 0u);
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tdK, tdP + k * 8, sdesc_sw128(sQ + k * 2048, 16384, 1024), IDESC_G,
+                                   (!first || k > 0) ? 1u : 0u);
+                        mma_commit(bar_st_empty + 8 * slot);
+                        first = false;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(bar_kv_empty);
+                if (!first) mma_commit(bar_acc_full);   // the softmax group waits only if it had a tile
+            }
+            mma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax group (key rows)
+        const int row = warp * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_off, tdP = tmem + lane_off + 128;
+        const uint32_t tdV = tmem + lane_off + 256, tdK = tmem + lane_off + 384;
+        uint32_t nst = 0, s_phase = 0, a_phase = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
+            const DkdvItem it = decode_dkdv(P, w);
+            const int k_orig = it.ko + row;
+            bool had = false;
+            for (int hq = 0; hq < g && ok; ++hq) {
+                for (int qt = 0; qt < P.cp * nqt && ok; ++qt) {
+                    const int qpos = qt * 128;
+                    const int qo = orig_of_shard(qpos, P.C, P.cp);
+                    const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
+                    const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                    const int cls = classify_tile(qo, dsf, dsl, it.ko);
+                    if (cls == TILE_SKIP) continue;
+                    const uint32_t slot = nst % Cfg::NST;
+                    ++nst;
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));
+                    if (!ok) break;
+                    s_phase ^= 1;
+                    tc_fence_after();
+                    const uint8_t* st = smem + Cfg::ST_OFF + slot * Cfg::ST_STRIDE;
+                    const float* s_lse2 = reinterpret_cast<const float*>(st + 2 * Cfg::TILE);
+                    const float* s_delta = reinterpret_cast<const float*>(st + 2 * Cfg::TILE + 512);
+                    const int* s_ds = reinterpret_cast<const int*>(st + 2 * Cfg::TILE + 1024);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < 128; c0 += 32) {
+                        float sv[32], dp[32];
+                        tmem_ld32f(tS + c0, sv);
+                        tmem_ld32f(tdP + c0, dp);
+                        tmem_wait_ld();
+                        reg_fence32f(sv);
+                        reg_fence32f(dp);
+                        uint32_t pk[16], dk[16];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float p2[2], d2[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = c0 + i + e;
+                                float pv = ex2_approx(fmaf(sv[i + e], P.scale_log2, -s_lse2[c]));
+                                if (cls == TILE_PARTIAL) {
+                                    const int q_orig = qo + c;
+                                    const int dsq = P.docs ? s_ds[c] : 0;
+                                    if (k_orig > q_orig || k_orig < dsq) pv = 0.f;
+                                }
+                                p2[e] = pv;
+                                d2[e] = pv * (dp[i + e] - s_delta[c]);
+                            }
+                            pk[i / 2] = pack_bf16(p2[0], p2[1]);
+                            dk[i / 2] = pack_bf16(d2[0], d2[1]);
+                        }
+                        tmem_st16(tS + c0 / 2, pk);
+                        tmem_st16(tdP + c0 / 2, dk);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_p_full);
+                    had = true;
+                }
+            }
+            if (!ok) break;
+            // ---- epilogue: dK (scaled) and dV of this key tile
+            const size_t orow = static_cast<size_t>(it.bkv) * P.S + it.kpos + row;
+            if (had) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_acc_full, a_phase, abort_flag));
+                if (!ok) break;
+                a_phase ^= 1;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float a[32], b[32];
+                    tmem_ld32f(tdV + c0, a);
+                    tmem_ld32f(tdK + c0, b);
+                    tmem_wait_ld();
+                    reg_fence32f(a);
+                    reg_fence32f(b);
+                    uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + c0);
+                    uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        dv[i] = make_uint4(pack_bf16(a[8 * i], a[8 * i + 1]), pack_bf16(a[8 * i + 2], a[8 * i + 3]),
+                                           pack_bf16(a[8 * i + 4], a[8 * i + 5]), pack_bf16(a[8 * i + 6], a[8 * i + 7]));
+                        dk[i] = make_uint4(pack_bf16(b[8 * i] * P.scale, b[8 * i + 1] * P.scale),
+                                           pack_bf16(b[8 * i + 2] * P.scale, b[8 * i + 3] * P.scale),
+                                           pack_bf16(b[8 * i + 4] * P.scale, b[8 * i + 5] * P.scale),
+                                           pack_bf16(b[8 * i + 6] * P.scale, b[8 * i + 7] * P.scale));
+                    }
+                }
+            } else {
+                uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D);
+                uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D);
+                for (int i = 0; i < D / 8; ++i) { dv[i] = make_uint4(0, 0, 0, 0); dk[i] = make_uint4(0, 0, 0, 0); }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_relinquish();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ============================================================================
+// dQ pass
+// ============================================================================
+template <int D>
+struct DqCfg {
+    static constexpr int TILE = 128 * D * 2;
+    static constexpr int NSLOT = (D == 128) ? 4 : 8;
+    static constexpr int Q_OFF = 0, DO_OFF = TILE, KV_OFF = 2 * TILE;
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE;
+    // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, p_full, acc_full, drain
+    static constexpr int NBAR = 6 + 2 * NSLOT;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
+    static constexpr int THREADS = 192;
+};
+
+struct DqItem {
+    int bh, bkv, r, qpos, qo;
+};
+
+__device__ __forceinline__ DqItem decode_dq(const BwdParams& P, int w)
+{
+    DqItem it;
+    const int BH = P.B * P.Hq;
+    it.bh = w % BH;
+    const int t = w / BH;
+    const int ntiles = P.S / 128;
+    it.qo = (ntiles - 1 - t) * 128;          // descending original position
+    it.qpos = shard_of_orig(it.qo, P.C, P.cp);
+    it.r = it.qpos / (2 * P.C);
+    const int g = P.Hq / P.Hkv;
+    const int b = it.bh / P.Hq, h = it.bh - b * P.Hq;
+    it.bkv = b * P.Hkv + h / g;
+    return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                 const BwdParams P)
+{
+    using Cfg = DqCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + Cfg::Q_OFF, sdO = sbase + Cfg::DO_OFF, sKV = sbase + Cfg::KV_OFF;
+    const uint32_t bars = sbase + Cfg::BAR_OFF;
+    const uint32_t bar_q_full = bars, bar_q_empty = bars + 8;
+    const uint32_t bar_kv_full = bars + 16, bar_kv_empty = bars + 16 + 8 * Cfg::NSLOT;
+    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT, bar_p_full = bar_s_full + 8;
+    const uint32_t bar_acc_full = bar_s_full + 16, bar_drain = bar_s_full + 24;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n2c = 2 * P.C;
+    const int ktiles = n2c / 128;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
+        for (int i = 0; i < Cfg::NSLOT; ++i) {
+            mbar_init(bar_kv_full + 8 * i, 1);
+            mbar_init(bar_kv_empty + 8 * i, 1);
+        }
+        mbar_init(bar_s_full, 1);
+        mbar_init(bar_p_full, 4);
+        mbar_init(bar_acc_full, 1);
+        mbar_init(bar_drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(smem_u32(tmem_slot), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmdO);
+            uint32_t nload = 0, iter = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+                const DqItem it = decode_dq(P, w);
+                const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
+                const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
+                ok = mbar_wait(bar_q_empty, (iter & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_q_full, 2 * Cfg::TILE);
+                for (int h = 0; h < D / 64; ++h) {
+                    tma_load_2d(sQ + h * 16384, &tmQ, h * 64, it.bh * P.S + it.qpos, bar_q_full);
+                    tma_load_2d(sdO + h * 16384, &tmdO, h * 64, it.bh * P.S + it.qpos, bar_q_full);
+                }
+                for (int s = 0; s < P.cp && ok; ++s) {
+                    const int j = __ldg(P.src + it.r * P.cp + s);
+                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                        const int kpos = j * n2c + kt * 128;
+                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
+                        for (int kv = 0; kv < 2 && ok; ++kv, ++nload) {
+                            const uint32_t slot = nload % Cfg::NSLOT, par = (nload / Cfg::NSLOT) & 1;
+                            ok = mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, abort_flag);
+                            if (!ok) break;
+                            mbar_arrive_expect_tx(bar_kv_full + 8 * slot, Cfg::TILE);
+                            for (int h = 0; h < D / 64; ++h)
+                                tma_load_2d(sKV + slot * Cfg::TILE + h * 16384,
+                                            kv == 0 ? (const void*)&tmK : (const void*)&tmV, h * 64,
+                                            it.bkv * P.S + kpos, bar_kv_full + 8 * slot);
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                for (uint32_t n = (nload > Cfg::NSLOT ? nload - Cfg::NSLOT : 0); n < nload; ++n)
+                    mbar_wait_drain(bar_kv_full + 8 * (n % Cfg::NSLOT), (n / Cfg::NSLOT) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);
+            const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+            uint32_t nload = 0, iter = 0, p_phase = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+                const DqItem it = decode_dq(P, w);
+                const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
+                const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
+                ok = mbar_wait(bar_q_full, iter & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                bool first = true;
+                for (int s = 0; s < P.cp && ok; ++s) {
+                    const int j = __ldg(P.src + it.r * P.cp + s);
+                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                        const int kpos = j * n2c + kt * 128;
+                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
+                        const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
+                        const uint32_t vslot = (nload + 1) % Cfg::NSLOT, vpar = ((nload + 1) / Cfg::NSLOT) & 1;
+                        nload += 2;
+                        ok = mbar_wait(bar_kv_full + 8 * kslot, kpar, abort_flag) &&
+                             mbar_wait(bar_kv_full + 8 * vslot, vpar, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sk = sKV + kslot * Cfg::TILE, sv = sKV + vslot * Cfg::TILE;
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+                            mma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024),
+                                   IDESC_S, k > 0 ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+                            mma_ss(tdP, sdesc_sw128(sdO + off, 16, 1024), sdesc_sw128(sv + off, 16, 1024),
+                                   IDESC_S, k > 0 ? 1u : 0u);
+                        }
+                        mma_commit(bar_s_full);
+                        mma_commit(bar_kv_empty + 8 * vslot);
+                        ok = mbar_wait(bar_p_full, p_phase, abort_flag);
+                        if (!ok) break;
+                        p_phase ^= 1;
+                        tc_fence_after();
+                        // dQ += dS K   (K dimension = 128 keys)
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tdQ, tS + k * 8, sdesc_sw128(sk + k * 2048, 16384, 1024), IDESC_G,
+                                   (!first || k > 0) ? 1u : 0u);
+                        mma_commit(bar_kv_empty + 8 * kslot);
+                        first = false;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(bar_q_empty);
+                if (!first) mma_commit(bar_acc_full);   // the softmax group waits only if it had a tile
+            }
+            mma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax group (query rows)
+        const int row = warp * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_off, tdP = tmem + lane_off + 128, tdQ = tmem + lane_off + 256;
+        uint32_t s_phase = 0, a_phase = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
+            const DqItem it = decode_dq(P, w);
+            const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
+            const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
+            const size_t rowi = static_cast<size_t>(it.bh) * P.S + it.qpos + row;
+            const float lse2 = __ldg(P.lse2 + rowi);
+            const float dlt = __ldg(P.delta + rowi);
+            const int q_orig = it.qo + row;
+            const int ds_row = P.docs ? __ldg(P.doc_start + it.qpos + row) : 0;
+            bool had = false;
+            for (int s = 0; s < P.cp && ok; ++s) {
+                const int j = __ldg(P.src + it.r * P.cp + s);
+                for (int kt = 0; kt < ktiles && ok; ++kt) {
+                    const int kpos = j * n2c + kt * 128;
+                    const int ko = orig_of_shard(kpos, P.C, P.cp);
+                    const int cls = classify_tile(it.qo, dsf, dsl, ko);
+                    if (cls == TILE_SKIP) continue;
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));
+                    if (!ok) break;
+                    s_phase ^= 1;
+                    tc_fence_after();
+                    const int lo = ds_row - ko, hi = q_orig - ko;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < 128; c0 += 32) {
+                        float sv[32], dp[32];
+                        tmem_ld32f(tS + c0, sv);
+                        tmem_ld32f(tdP + c0, dp);
+                        tmem_wait_ld();
+                        reg_fence32f(sv);
+                        reg_fence32f(dp);
+                        uint32_t dk[16];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float d2[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = c0 + i + e;
+                                float pv = ex2_approx(fmaf(sv[i + e], P.scale_log2, -lse2));
+                                if (cls == TILE_PARTIAL && (c < lo || c > hi)) pv = 0.f;
+                                d2[e] = pv * (dp[i + e] - dlt);
+                            }
+                            dk[i / 2] = pack_bf16(d2[0], d2[1]);
+                        }
+                        tmem_st16(tS + c0 / 2, dk);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_p_full);
+                    had = true;
+                }
+            }
+            if (!ok) break;
+            if (had) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_acc_full, a_phase, abort_flag));
+                if (!ok) break;
+                a_phase ^= 1;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float a[32];
+                    tmem_ld32f(tdQ + c0, a);
+                    tmem_wait_ld();
+                    reg_fence32f(a);
+                    uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dq[i] = make_uint4(pack_bf16(a[8 * i] * P.scale, a[8 * i + 1] * P.scale),
+                                           pack_bf16(a[8 * i + 2] * P.scale, a[8 * i + 3] * P.scale),
+                                           pack_bf16(a[8 * i + 4] * P.scale, a[8 * i + 5] * P.scale),
+                                           pack_bf16(a[8 * i + 6] * P.scale, a[8 * i + 7] * P.scale));
+                }
+            } else {
+                uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D);
+                for (int i = 0; i < D / 8; ++i) dq[i] = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_relinquish();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace cpattn

@@ -1,0 +1,499 @@
+// libcpattn: the C ABI declared in include/cp_attn.h.  Host-side argument
+// checks, workspace accounting, tensor-map encoding and kernel launches.  The
+// library is one translation unit; the kernels live in the included headers.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "cp_attn.h"
+#include "ptx.cuh"
+#include "tmap.h"
+#include "zigzag.cuh"
+#include "plan.cuh"
+#include "merge.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+using namespace cpattn;
+
+namespace {
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    }
+    return n;
+}
+
+// Checks shared by every call that takes a cp_problem_t.
+cp_status_t check_problem(const cp_problem_t* p)
+{
+    if (!p) return CP_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->seq_len < 1 || p->cp_size < 1 || p->num_heads < 1 ||
+        p->num_kv_heads < 1 || p->head_dim < 1)
+        return CP_ERR_INVALID_ARG;
+    if (p->seq_len % (2 * p->cp_size) != 0) return CP_ERR_INVALID_ARG;
+    if (p->num_heads % p->num_kv_heads != 0) return CP_ERR_INVALID_ARG;
+    if (p->rotate != CP_ROTATE_ALLGATHER && p->rotate != CP_ROTATE_RING) return CP_ERR_INVALID_ARG;
+    if (p->mask != CP_MASK_CAUSAL && p->mask != CP_MASK_DOC_CAUSAL) return CP_ERR_INVALID_ARG;
+    if (p->merge != CP_MERGE_SEPARATE && p->merge != CP_MERGE_FUSED) return CP_ERR_INVALID_ARG;
+    if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return CP_ERR_INVALID_ARG;
+    if (p->mask == CP_MASK_DOC_CAUSAL) {
+        if (!p->cu_seqlens || p->num_docs < 1 || p->num_docs > p->seq_len) return CP_ERR_INVALID_ARG;
+    }
+    if (p->cp_size > PLAN_MAX_CP) return CP_ERR_UNSUPPORTED;
+    // every flat row index (batch*heads*seq) and element offset must fit the kernels' types
+    const int64_t rows = static_cast<int64_t>(p->batch) * p->num_heads * p->seq_len;
+    if (rows > (int64_t(1) << 31) - 1) return CP_ERR_UNSUPPORTED;
+    return CP_OK;
+}
+
+cp_status_t check_attention(const cp_problem_t* p)
+{
+    cp_status_t st = check_problem(p);
+    if (st != CP_OK) return st;
+    if (p->head_dim != 64 && p->head_dim != 128) return CP_ERR_UNSUPPORTED;
+    const int C = p->seq_len / (2 * p->cp_size);
+    if (C % 128 != 0) return CP_ERR_UNSUPPORTED;
+    return CP_OK;
+}
+
+cp_status_t check_plan(const cp_plan_t* pl, bool need_all)
+{
+    if (!pl) return CP_ERR_INVALID_ARG;
+    if (!pl->src || !pl->doc_start) return CP_ERR_INVALID_ARG;
+    if (need_all && (!pl->perm || !pl->inv_perm || !pl->rank_cu_off || !pl->rank_cu || !pl->pairs))
+        return CP_ERR_INVALID_ARG;
+    return CP_OK;
+}
+
+inline float softmax_scale(const cp_problem_t* p)
+{
+    return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
+}
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace handshake shared by every call that takes (ws, ws_bytes).
+// Returns true when the caller should return `out` right away.
+inline bool workspace_gate(size_t need, void* ws, size_t* ws_bytes, cp_status_t* out)
+{
+    if (ws_bytes && !ws) { *ws_bytes = need; *out = CP_OK; return true; }
+    if (need == 0) return false;
+    if (!ws || !ws_bytes) { *out = CP_ERR_INVALID_ARG; return true; }
+    if (*ws_bytes < need) { *out = CP_ERR_WORKSPACE; return true; }
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) { *out = CP_ERR_INVALID_ARG; return true; }
+    return false;
+}
+
+inline cp_status_t launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+// ---- launch counter and optional event trace (see cp_trace_begin)
+int64_t g_launches = 0;
+cudaEvent_t* g_trace_events = nullptr;
+int32_t g_trace_cap = 0, g_trace_n = 0;
+int32_t g_trace_ids[4096];
+constexpr int32_t kTraceMax = 4096;
+
+struct LaunchScope {
+    cudaStream_t s;
+    bool traced;
+    LaunchScope(int kernel, cudaStream_t stream) : s(stream), traced(false)
+    {
+        ++g_launches;
+        if (g_trace_events) {
+            if (g_trace_n < g_trace_cap) {
+                cudaEventRecord(g_trace_events[2 * g_trace_n], s);
+                traced = true;
+            }
+            if (g_trace_n < kTraceMax) g_trace_ids[g_trace_n] = kernel;
+        }
+    }
+    ~LaunchScope()
+    {
+        if (traced) cudaEventRecord(g_trace_events[2 * g_trace_n + 1], s);
+        if (g_trace_events) ++g_trace_n;
+    }
+};
+
+cp_status_t launch_gather(const cp_problem_t* p, int32_t n_bufs, const void* const* bufs_in,
+                          void* const* bufs_out, const int64_t* buf_outer,
+                          const int64_t* buf_row_bytes, int to_shard, cudaStream_t stream)
+{
+    const int C = p->seq_len / (2 * p->cp_size);
+    for (int i = 0; i < n_bufs; ++i) {
+        if (buf_outer[i] == 0) continue;
+        GatherParams G;
+        G.in = static_cast<const uint4*>(bufs_in[i]);
+        G.out = static_cast<uint4*>(bufs_out[i]);
+        G.rows = buf_outer[i] * p->seq_len;
+        G.vpr = static_cast<int32_t>(buf_row_bytes[i] / 16);
+        G.rpw = (G.vpr <= 32 && 32 % G.vpr == 0) ? 32 / G.vpr : 1;
+        G.S = p->seq_len;
+        G.C = C;
+        G.cp = p->cp_size;
+        G.to_shard = to_shard;
+        const int64_t warps_needed = (G.rows + G.rpw * 4 - 1) / (G.rpw * 4);
+        const int64_t blocks = std::min<int64_t>((warps_needed + 7) / 8, int64_t(num_sms()) * 8);
+        LaunchScope ls(CP_K_GATHER, stream);
+        gather_rows_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0, stream>>>(G);
+        if (launch_status() != CP_OK) return CP_ERR_CUDA;
+    }
+    return CP_OK;
+}
+
+cp_status_t check_bufs(const cp_problem_t* p, int32_t n_bufs, const void* const* bufs_in,
+                       void* const* bufs_out, const int64_t* buf_outer,
+                       const int64_t* buf_row_bytes)
+{
+    if (n_bufs < 0 || n_bufs > 16) return CP_ERR_INVALID_ARG;
+    if (n_bufs == 0) return CP_OK;
+    if (!bufs_in || !bufs_out || !buf_outer || !buf_row_bytes) return CP_ERR_INVALID_ARG;
+    for (int i = 0; i < n_bufs; ++i) {
+        if (buf_outer[i] < 0 || buf_row_bytes[i] <= 0 || buf_row_bytes[i] % 16 != 0)
+            return CP_ERR_INVALID_ARG;
+        if (buf_outer[i] == 0) continue;
+        if (!bufs_in[i] || !bufs_out[i] || !aligned16(bufs_in[i]) || !aligned16(bufs_out[i]))
+            return CP_ERR_INVALID_ARG;
+        if (buf_outer[i] * static_cast<int64_t>(p->seq_len) > (int64_t(1) << 40))
+            return CP_ERR_UNSUPPORTED;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(bufs_in[i]);
+        const uintptr_t b = reinterpret_cast<uintptr_t>(bufs_out[i]);
+        const uintptr_t n = static_cast<uintptr_t>(buf_outer[i] * p->seq_len * buf_row_bytes[i]);
+        if (a < b + n && b < a + n) return CP_ERR_INVALID_ARG;  // in/out overlap
+    }
+    return CP_OK;
+}
+
+template <int D>
+cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
+                       const void* v, void* o, float* lse, float* o_parts, float* lse_parts,
+                       cudaStream_t stream)
+{
+    using Cfg = FwdCfg<D>;
+    const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * S, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128))
+        return CP_ERR_CUDA;
+    FwdParams P;
+    P.BH = B * Hq;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.S = S;
+    P.cp = p->cp_size;
+    P.C = S / (2 * p->cp_size);
+    P.docs = p->mask == CP_MASK_DOC_CAUSAL;
+    P.fused = p->merge == CP_MERGE_FUSED;
+    P.scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+    P.ppc = (P.C + 255) / 256;
+    P.n_items = P.BH * 2 * P.cp * P.ppc;
+    P.src = pl->src;
+    P.doc_start = pl->doc_start;
+    P.o = static_cast<__nv_bfloat16*>(o);
+    P.lse = lse;
+    P.o_parts = o_parts;
+    P.lse_parts = lse_parts;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(cp_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        Cfg::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return CP_ERR_CUDA;
+    const int grid = std::min(P.n_items, num_sms());
+    LaunchScope ls(CP_K_FWD, stream);
+    cp_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, P);
+    return launch_status();
+}
+
+cp_status_t launch_merge(int64_t rows, int32_t D, int32_t n_parts, const float* o_parts,
+                         const float* lse_parts, void* o_out, float* lse_out, cudaStream_t stream)
+{
+    if (rows == 0) return CP_OK;
+    MergeParams M;
+    M.rows = rows;
+    M.D = D;
+    M.n_parts = n_parts;
+    M.o_parts = o_parts;
+    M.lse_parts = lse_parts;
+    M.o_out = static_cast<__nv_bfloat16*>(o_out);
+    M.lse_out = lse_out;
+    const int64_t blocks = std::min<int64_t>((rows + 7) / 8, int64_t(num_sms()) * 16);
+    LaunchScope ls(CP_K_MERGE, stream);
+    lse_merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(M);
+    return launch_status();
+}
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        fence_barrier_init();
+        // nothing ever arrives on this barrier: the bounded wait must give up
+        mbar_wait_limit(smem_u32(&bar), 0, &abort_flag, limit_ns);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t cp_version(void) { return kVersion; }
+
+int64_t cp_launch_count(void) { return g_launches; }
+
+cp_status_t cp_trace_begin(void* const* events, int32_t capacity)
+{
+    if (!events || capacity < 1) return CP_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < 2 * capacity; ++i)
+        if (!events[i]) return CP_ERR_INVALID_ARG;
+    g_trace_events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+    g_trace_cap = capacity;
+    g_trace_n = 0;
+    return CP_OK;
+}
+
+cp_status_t cp_trace_end(int32_t* n_launches, int32_t* kernel_ids)
+{
+    if (!n_launches) return CP_ERR_INVALID_ARG;
+    *n_launches = g_trace_n;
+    if (kernel_ids)
+        for (int32_t i = 0; i < std::min(g_trace_n, std::min(g_trace_cap, kTraceMax)); ++i)
+            kernel_ids[i] = g_trace_ids[i];
+    g_trace_events = nullptr;
+    g_trace_cap = 0;
+    g_trace_n = 0;
+    return CP_OK;
+}
+
+cp_status_t cp_plan_shards(const cp_problem_t* problem, const cp_plan_t* plan, int32_t n_bufs,
+                           const void* const* bufs_in, void* const* bufs_out,
+                           const int64_t* buf_outer, const int64_t* buf_row_bytes, void* ws,
+                           size_t* ws_bytes, void* stream)
+{
+    cp_status_t st = check_problem(problem);
+    if (st != CP_OK) return st;
+    if ((st = check_plan(plan, true)) != CP_OK) return st;
+    if ((st = check_bufs(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes)) != CP_OK)
+        return st;
+    if (workspace_gate(0, ws, ws_bytes, &st)) return st;
+    cudaStream_t s = as_stream(stream);
+    PlanParams P;
+    P.S = problem->seq_len;
+    P.cp = problem->cp_size;
+    P.C = P.S / (2 * P.cp);
+    P.docs = problem->mask == CP_MASK_DOC_CAUSAL;
+    P.num_docs = P.docs ? problem->num_docs : 1;
+    P.rotate = problem->rotate;
+    P.cu = problem->cu_seqlens;
+    P.perm = plan->perm;
+    P.inv_perm = plan->inv_perm;
+    P.src = plan->src;
+    P.doc_start = plan->doc_start;
+    P.rank_cu_off = plan->rank_cu_off;
+    P.rank_cu = plan->rank_cu;
+    P.pairs = plan->pairs;
+    {
+        LaunchScope ls(CP_K_PLAN_META, s);
+        plan_meta_kernel<<<1, 256, 0, s>>>(P);
+    }
+    if (launch_status() != CP_OK) return CP_ERR_CUDA;
+    const int blocks = std::min((P.S + 255) / 256, num_sms() * 8);
+    {
+        LaunchScope ls(CP_K_PLAN_INDEX, s);
+        plan_index_kernel<<<blocks, 256, 0, s>>>(P);
+    }
+    if (launch_status() != CP_OK) return CP_ERR_CUDA;
+    return launch_gather(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes, 1, s);
+}
+
+cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan, int32_t n_bufs,
+                       const void* const* bufs_in, void* const* bufs_out,
+                       const int64_t* buf_outer, const int64_t* buf_row_bytes, void* stream)
+{
+    cp_status_t st = check_problem(problem);
+    if (st != CP_OK) return st;
+    if (!plan) return CP_ERR_INVALID_ARG;
+    if ((st = check_bufs(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes)) != CP_OK)
+        return st;
+    return launch_gather(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes, 0,
+                         as_stream(stream));
+}
+
+cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                        const void* k, const void* v, void* o, float* lse, void* ws,
+                        size_t* ws_bytes, void* stream)
+{
+    cp_status_t st = check_attention(problem);
+    if (st != CP_OK) return st;
+    if ((st = check_plan(plan, false)) != CP_OK) return st;
+    if (!q || !k || !v || !o || !lse) return CP_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return CP_ERR_INVALID_ARG;
+    const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * problem->seq_len;
+    const bool separate = problem->merge == CP_MERGE_SEPARATE;
+    const size_t o_parts_bytes = separate ? round_up(size_t(problem->cp_size) * rows * problem->head_dim * 4, 256) : 0;
+    const size_t lse_parts_bytes = separate ? round_up(size_t(problem->cp_size) * rows * 4, 256) : 0;
+    if (workspace_gate(o_parts_bytes + lse_parts_bytes, ws, ws_bytes, &st)) return st;
+    float* o_parts = separate ? static_cast<float*>(ws) : nullptr;
+    float* lse_parts = separate ? reinterpret_cast<float*>(static_cast<char*>(ws) + o_parts_bytes) : nullptr;
+    cudaStream_t s = as_stream(stream);
+    st = problem->head_dim == 128 ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s)
+                                  : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s);
+    if (st != CP_OK || !separate) return st;
+    return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
+}
+
+cp_status_t cp_lse_merge(int64_t rows, int32_t head_dim, int32_t n_parts, const float* o_parts,
+                         const float* lse_parts, void* o_out, float* lse_out, void* stream)
+{
+    if (rows < 0 || head_dim < 4 || head_dim > 256 || head_dim % 4 != 0) return CP_ERR_INVALID_ARG;
+    if (n_parts < 1 || n_parts > MERGE_MAX_PARTS) return CP_ERR_INVALID_ARG;
+    if (rows == 0) return CP_OK;
+    if (!o_parts || !lse_parts || !o_out || !lse_out) return CP_ERR_INVALID_ARG;
+    if (!aligned16(o_parts) || !aligned16(o_out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+        (reinterpret_cast<uintptr_t>(lse_out) & 3u))
+        return CP_ERR_INVALID_ARG;
+    return launch_merge(rows, head_dim, n_parts, o_parts, lse_parts, o_out, lse_out, as_stream(stream));
+}
+
+cp_status_t cp_get_device_status(int32_t* status, void* stream)
+{
+    if (!status) return CP_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    int32_t v = 0;
+    const int32_t zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_cp_device_status, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return CP_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CP_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(g_cp_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return CP_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CP_ERR_CUDA;
+    *status = v;
+    return CP_OK;
+}
+
+cp_status_t cp_set_wait_limit_ns(uint64_t limit_ns)
+{
+    if (limit_ns == 0) return CP_ERR_INVALID_ARG;
+    const unsigned long long v = limit_ns;
+    if (cudaMemcpyToSymbol(g_cp_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return CP_ERR_CUDA;
+    return CP_OK;
+}
+
+cp_status_t cp_selftest_wait_timeout(uint64_t limit_ns, void* stream)
+{
+    if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return CP_ERR_INVALID_ARG;
+    LaunchScope ls(CP_K_SELFTEST, as_stream(stream));
+    selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns);
+    return launch_status();
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int D>
+cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
+                       const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                       void* dk, void* dv, float* delta, float* lse2, cudaStream_t stream)
+{
+    const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
+    const int64_t rows = static_cast<int64_t>(B) * Hq * S;
+    {
+        const int64_t blocks = std::min<int64_t>((rows + 7) / 8, int64_t(num_sms()) * 16);
+        LaunchScope ls(CP_K_BWD_PREP, stream);
+        bwd_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
+            lse2, rows, D);
+        if (launch_status() != CP_OK) return CP_ERR_CUDA;
+    }
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * S, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tdo, dout, D, static_cast<uint64_t>(B) * Hq * S, D * 2, 64, 128))
+        return CP_ERR_CUDA;
+    BwdParams P;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.S = S;
+    P.cp = p->cp_size;
+    P.C = S / (2 * p->cp_size);
+    P.docs = p->mask == CP_MASK_DOC_CAUSAL;
+    P.scale = softmax_scale(p);
+    P.scale_log2 = P.scale * 1.4426950408889634f;
+    P.src = pl->src;
+    P.doc_start = pl->doc_start;
+    P.lse2 = lse2;
+    P.delta = delta;
+    P.dq = static_cast<__nv_bfloat16*>(dq);
+    P.dk = static_cast<__nv_bfloat16*>(dk);
+    P.dv = static_cast<__nv_bfloat16*>(dv);
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        DkdvCfg<D>::SMEM_BYTES);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(cp_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            DqCfg<D>::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return CP_ERR_CUDA;
+    P.n_items = B * Hkv * (S / 128);
+    {
+    LaunchScope ls(CP_K_BWD_DKDV, stream);
+    cp_bwd_dkdv_kernel<D><<<std::min(P.n_items, num_sms()), DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES,
+                            stream>>>(tq, tk, tv, tdo, P);
+    }
+    if (launch_status() != CP_OK) return CP_ERR_CUDA;
+    P.n_items = B * Hq * (S / 128);
+    LaunchScope ls(CP_K_BWD_DQ, stream);
+    cp_bwd_dq_kernel<D><<<std::min(P.n_items, num_sms()), DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, P);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                                   const void* k, const void* v, const void* o, const float* lse,
+                                   const void* dout, void* dq, void* dk, void* dv, void* ws,
+                                   size_t* ws_bytes, void* stream)
+{
+    cp_status_t st = check_attention(problem);
+    if (st != CP_OK) return st;
+    if ((st = check_plan(plan, false)) != CP_OK) return st;
+    const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+    for (const void* x : ptrs)
+        if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
+    const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * problem->seq_len;
+    const size_t row_bytes = round_up(size_t(rows) * 4, 256);
+    if (workspace_gate(2 * row_bytes, ws, ws_bytes, &st)) return st;
+    float* delta = static_cast<float*>(ws);
+    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
+    cudaStream_t s = as_stream(stream);
+    return problem->head_dim == 128
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s);
+}

@@ -1,0 +1,483 @@
+// Forward kernel: causal (optionally packed-document) attention of every
+// virtual rank's query shard against the K/V shards in the plan's visit order.
+//
+// Work item = (batch*head, a pair of adjacent 128-row query tiles inside one
+// zigzag chunk).  Items are ordered by descending original query position, so
+// the longest items start first, and are dealt round-robin to one persistent
+// CTA per SM.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax group 0 (query tile 0): one TMEM lane = one query row
+//   warps 4-7  softmax group 1 (query tile 1)
+//   warp 8     TMA producer: Q tiles, then K and V tiles through a ring of
+//              shared-memory slots
+//   warp 9     MMA issuer (one thread) + tensor-memory owner
+// Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D),
+// O1 [384,384+D).  P is written back as bf16 over the first 64 columns of its
+// S region and used as the A operand of O += P V straight from tensor memory.
+//
+// Per KV tile t the MMA thread issues, for each query tile X that the tile
+// does not skip:  O_X += P_X(prev) V(prev)  then  S_X = Q_X K_t^T, so the
+// tensor core computes S for one query tile while the other group runs its
+// softmax (ping-pong between the two groups).
+//
+// Visit order: for virtual rank r the K/V shards are visited as src[r][s],
+// s = 0..cp-1 (all-gather: rank order; ring: (r - s) mod cp).  With
+// CP_MERGE_SEPARATE each step is one segment whose partial (O, LSE) is
+// written in fp32 and later combined by the merge kernel; with
+// CP_MERGE_FUSED the whole visit is one segment and the combine happens in the
+// running online-softmax state, step after step, in the same order.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+#include "zigzag.cuh"
+
+namespace cpattn {
+
+struct FwdParams {
+    int32_t BH, Hq, Hkv, S, cp, C;  // BH = batch * Hq
+    int32_t docs;                   // 1 = packed-document mask
+    int32_t fused;                  // 1 = CP_MERGE_FUSED
+    float scale_log2;               // softmax scale * log2(e)
+    int32_t n_items, ppc;           // items, query-tile pairs per chunk
+    const int32_t* src;             // [cp*cp]
+    const int32_t* doc_start;       // [S] shard order
+    __nv_bfloat16* o;               // [BH][S][D]  (fused)
+    float* lse;                     // [BH][S]     (fused)
+    float* o_parts;                 // [cp][BH][S][D] (separate)
+    float* lse_parts;               // [cp][BH][S]    (separate)
+};
+
+enum : int { TILE_SKIP = 0, TILE_FULL = 1, TILE_PARTIAL = 2 };
+
+// Query tile rows have original positions [qo, qo+127] and document starts
+// between dsf (first row) and dsl (last row); key tile keys [ko, ko+127].
+// A pair (q, k) is admitted when ds(q) <= k <= q.
+__device__ __forceinline__ int classify_tile(int qo, int dsf, int dsl, int ko)
+{
+    if (ko > qo + 127 || ko + 127 < dsf) return TILE_SKIP;
+    if (ko + 127 <= qo && ko >= dsl) return TILE_FULL;
+    return TILE_PARTIAL;
+}
+
+struct FwdItem {
+    int bh, bkv, r, p0, qo0, ntq;
+};
+
+__device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
+{
+    FwdItem it;
+    it.bh = w % P.BH;
+    const int t = w / P.BH;
+    const int u = P.ppc - 1 - t % P.ppc;
+    const int c = 2 * P.cp - 1 - t / P.ppc;  // original chunk, descending
+    int half;
+    if (c < P.cp) { it.r = c; half = 0; } else { it.r = 2 * P.cp - 1 - c; half = 1; }
+    it.p0 = it.r * 2 * P.C + half * P.C + u * 256;
+    it.qo0 = c * P.C + u * 256;
+    it.ntq = (u * 256 + 256 <= P.C) ? 2 : 1;
+    const int g = P.Hq / P.Hkv;
+    const int b = it.bh / P.Hq, h = it.bh - b * P.Hq;
+    it.bkv = b * P.Hkv + h / g;
+    return it;
+}
+
+template <int D>
+struct FwdCfg {
+    static constexpr int TILE_BYTES = 128 * D * 2;      // one 128-row bf16 tile
+    static constexpr int NSLOT = (D == 128) ? 4 : 8;    // K/V ring slots
+    static constexpr int Q_OFF = 0;                     // Q0, Q1
+    static constexpr int KV_OFF = 2 * TILE_BYTES;
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    // barriers: q_full, q_empty, s_full[2], p_full[2], o_full[2], kv_full[NSLOT], kv_empty[NSLOT], drain
+    static constexpr int NBAR = 9 + 2 * NSLOT;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;  // + alignment slack
+    static constexpr int THREADS = 320;
+};
+
+struct TileIter {
+    // per-item geometry shared by every role
+    int qo[2], dsf[2], dsl[2];
+};
+
+// Original start and document-start range of each query tile of an item; the
+// second tile exists only when it.ntq == 2 (no read past the item's rows).
+__device__ __forceinline__ TileIter load_tile_iter(const FwdParams& P, const FwdItem& it)
+{
+    TileIter ti;
+    for (int x = 0; x < 2; ++x) {
+        ti.qo[x] = it.qo0 + 128 * x;
+        ti.dsf[x] = 0;
+        ti.dsl[x] = 0;
+        if (P.docs && x < it.ntq) {
+            const int pr = it.p0 + 128 * x;
+            ti.dsf[x] = __ldg(P.doc_start + pr);
+            ti.dsl[x] = __ldg(P.doc_start + pr + 127);
+        }
+    }
+    return ti;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const FwdParams P)
+{
+    using Cfg = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ0 = sbase + Cfg::Q_OFF, sKV = sbase + Cfg::KV_OFF;
+    const uint32_t bars = sbase + Cfg::BAR_OFF;
+    const uint32_t bar_q_full = bars, bar_q_empty = bars + 8;
+    const uint32_t bar_s_full = bars + 16, bar_p_full = bars + 32, bar_o_full = bars + 48;
+    const uint32_t bar_kv_full = bars + 64, bar_kv_empty = bars + 64 + 8 * Cfg::NSLOT;
+    const uint32_t bar_drain = bars + 64 + 16 * Cfg::NSLOT;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n2c = 2 * P.C;
+    const int ktiles = n2c / 128;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar_s_full + 8 * x, 1);
+            mbar_init(bar_p_full + 8 * x, 4);
+            mbar_init(bar_o_full + 8 * x, 1);
+        }
+        for (int i = 0; i < Cfg::NSLOT; ++i) {
+            mbar_init(bar_kv_full + 8 * i, 1);
+            mbar_init(bar_kv_empty + 8 * i, 1);
+        }
+        mbar_init(bar_drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            uint32_t nload = 0, iter = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+                const FwdItem it = decode_item(P, w);
+                const TileIter ti = load_tile_iter(P, it);
+                ok = mbar_wait(bar_q_empty, (iter & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_q_full, it.ntq * Cfg::TILE_BYTES);
+                for (int x = 0; x < it.ntq; ++x)
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(sQ0 + x * Cfg::TILE_BYTES + h * 16384, &tmQ, h * 64,
+                                    it.bh * P.S + it.p0 + 128 * x, bar_q_full);
+                for (int s = 0; s < P.cp && ok; ++s) {
+                    const int j = __ldg(P.src + it.r * P.cp + s);
+                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                        const int kpos = j * n2c + kt * 128;
+                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
+                        const bool v1 = it.ntq == 2 &&
+                                        classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP;
+                        if (!v0 && !v1) continue;
+                        for (int kv = 0; kv < 2 && ok; ++kv, ++nload) {
+                            const uint32_t slot = nload % Cfg::NSLOT;
+                            const uint32_t par = (nload / Cfg::NSLOT) & 1;
+                            ok = mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, abort_flag);
+                            if (!ok) break;
+                            mbar_arrive_expect_tx(bar_kv_full + 8 * slot, Cfg::TILE_BYTES);
+                            for (int h = 0; h < D / 64; ++h)
+                                tma_load_2d(sKV + slot * Cfg::TILE_BYTES + h * 16384,
+                                            kv == 0 ? (const void*)&tmK : (const void*)&tmV, h * 64,
+                                            it.bkv * P.S + kpos, bar_kv_full + 8 * slot);
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                // abort path: let the copies already issued land before the CTA exits
+                for (uint32_t n = (nload > Cfg::NSLOT ? nload - Cfg::NSLOT : 0); n < nload; ++n)
+                    mbar_wait_drain(bar_kv_full + 8 * (n % Cfg::NSLOT), (n / Cfg::NSLOT) & 1);
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
+            const uint32_t tS[2] = {tmem + 0, tmem + 128};
+            const uint32_t tO[2] = {tmem + 256, tmem + 384};
+            uint32_t nload = 0, iter = 0;
+            uint32_t p_phase[2] = {0, 0};
+            bool ok = true;
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+                const FwdItem it = decode_item(P, w);
+                const TileIter ti = load_tile_iter(P, it);
+                ok = mbar_wait(bar_q_full, iter & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // pending PV per query tile: V slot/parity, users left on that slot
+                bool pend[2] = {false, false};
+                bool first[2] = {true, true};
+                bool seg_had[2] = {false, false};   // query tile x had a tile in this segment
+                uint32_t pend_slot[2] = {0, 0}, pend_par[2] = {0, 0};
+                int slot_users[Cfg::NSLOT];
+                for (int i = 0; i < Cfg::NSLOT; ++i) slot_users[i] = 0;
+
+                auto issue_pv = [&](int x) -> bool {
+                    if (!mbar_wait(bar_p_full + 8 * x, p_phase[x], abort_flag)) return false;
+                    p_phase[x] ^= 1;
+                    if (!mbar_wait(bar_kv_full + 8 * pend_slot[x], pend_par[x], abort_flag)) return false;
+                    tc_fence_after();
+                    const uint32_t sv = sKV + pend_slot[x] * Cfg::TILE_BYTES;
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tO[x], tS[x] + k * 8, sdesc_sw128(sv + k * 2048, 16384, 1024),
+                               IDESC_PV, (!first[x] || k > 0) ? 1u : 0u);
+                    first[x] = false;
+                    pend[x] = false;
+                    if (--slot_users[pend_slot[x]] == 0) mma_commit(bar_kv_empty + 8 * pend_slot[x]);
+                    return true;
+                };
+
+                for (int s = 0; s < P.cp && ok; ++s) {
+                    const int j = __ldg(P.src + it.r * P.cp + s);
+                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                        const int kpos = j * n2c + kt * 128;
+                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        const bool v[2] = {
+                            classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP,
+                            it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP};
+                        if (!v[0] && !v[1]) continue;
+                        const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
+                        const uint32_t vslot = (nload + 1) % Cfg::NSLOT,
+                                       vpar = ((nload + 1) / Cfg::NSLOT) & 1;
+                        nload += 2;
+                        ok = mbar_wait(bar_kv_full + 8 * kslot, kpar, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sk = sKV + kslot * Cfg::TILE_BYTES;
+                        slot_users[vslot] = (v[0] ? 1 : 0) + (v[1] ? 1 : 0);
+                        for (int x = 0; x < 2 && ok; ++x) {
+                            // A pending PV never outlives one tile: it is issued at the next
+                            // loaded tile whether or not that tile is valid for x, so a V slot
+                            // is held for at most one tile and the ring cannot stall.
+                            if (pend[x]) { ok = issue_pv(x); if (!ok) break; }
+                            if (!v[x]) continue;
+                            const uint32_t sq = sQ0 + x * Cfg::TILE_BYTES;
+#pragma unroll
+                            for (int k = 0; k < D / 16; ++k) {
+                                const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+                                mma_ss(tS[x], sdesc_sw128(sq + off, 16, 1024),
+                                       sdesc_sw128(sk + off, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
+                            }
+                            mma_commit(bar_s_full + 8 * x);
+                            pend[x] = true;
+                            seg_had[x] = true;
+                            pend_slot[x] = vslot;
+                            pend_par[x] = vpar;
+                        }
+                        if (!ok) break;
+                        mma_commit(bar_kv_empty + 8 * kslot);
+                    }
+                    // end of a segment: every step (separate) or the whole visit (fused)
+                    if (ok && (!P.fused || s == P.cp - 1)) {
+                        for (int x = 0; x < 2 && ok; ++x) {
+                            if (pend[x]) ok = issue_pv(x);
+                            // the softmax group of x waits for this whenever it had a tile in
+                            // the segment, even if its last PV was flushed at an earlier tile
+                            if (ok && seg_had[x]) mma_commit(bar_o_full + 8 * x);
+                            first[x] = true;
+                            seg_had[x] = false;
+                        }
+                    }
+                }
+                if (ok) mma_commit(bar_q_empty);
+            }
+            // drain: every MMA and commit issued above has completed
+            mma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax groups
+        const int X = warp >> 2;                 // query tile handled by this group
+        const int row = (warp & 3) * 32 + lane;  // TMEM lane == query row in the tile
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 128 * X;
+        const uint32_t tO = tmem + lane_off + 256 + 128 * X;
+        uint32_t s_phase = 0, o_phase = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
+            const FwdItem it = decode_item(P, w);
+            if (X >= it.ntq) continue;
+            const TileIter ti = load_tile_iter(P, it);
+            const int prow = it.p0 + 128 * X + row;      // shard position of my row
+            const int q_orig = ti.qo[X] + row;
+            const int ds_row = P.docs ? __ldg(P.doc_start + prow) : 0;
+            float m_used = -INFINITY, l_sum = 0.f;
+            bool first = true, had = false;
+            for (int s = 0; s < P.cp && ok; ++s) {
+                const int j = __ldg(P.src + it.r * P.cp + s);
+                for (int kt = 0; kt < ktiles && ok; ++kt) {
+                    const int kpos = j * n2c + kt * 128;
+                    const int ko = orig_of_shard(kpos, P.C, P.cp);
+                    const int cls = classify_tile(ti.qo[X], ti.dsf[X], ti.dsl[X], ko);
+                    if (cls == TILE_SKIP) continue;
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * X, s_phase, abort_flag));
+                    if (!ok) break;
+                    s_phase ^= 1;
+                    tc_fence_after();
+                    float sf[128];
+                    tmem_ld32f(tS + 0, sf + 0);
+                    tmem_ld32f(tS + 32, sf + 32);
+                    tmem_ld32f(tS + 64, sf + 64);
+                    tmem_ld32f(tS + 96, sf + 96);
+                    tmem_wait_ld();
+                    reg_fence32f(sf + 0);
+                    reg_fence32f(sf + 32);
+                    reg_fence32f(sf + 64);
+                    reg_fence32f(sf + 96);
+                    if (cls == TILE_PARTIAL) {
+                        const int lo = ds_row - ko, hi = q_orig - ko;
+#pragma unroll
+                        for (int c = 0; c < 128; ++c)
+                            if (c < lo || c > hi) sf[c] = -INFINITY;
+                    }
+                    float mx8[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(sf[i], sf[i + 8]);
+#pragma unroll
+                    for (int c = 16; c < 128; c += 16)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], fmaxf(sf[c + i], sf[c + 8 + i]));
+                    const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                    const float m_tile = mx * P.scale_log2;
+                    // lazy rescale: keep the reference max unless it is exceeded by more
+                    // than 8 (a factor 256 in the exponentials), or is still -inf
+                    const bool need = m_tile > m_used + 8.0f;
+                    float alpha = 1.f;
+                    if (need) {
+                        alpha = ex2_approx(m_used - m_tile);   // 0 when m_used = -inf
+                        m_used = m_tile;
+                    }
+                    if (!first && __any_sync(0xffffffffu, need)) {
+                        // O *= alpha for this row (the PV of the previous tile is complete)
+#pragma unroll 1
+                        for (int c0 = 0; c0 < D; c0 += 16) {
+                            float of[16];
+                            tmem_ld16f(tO + c0, of);
+                            tmem_wait_ld();
+                            reg_fence16f(of);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) of[i] *= alpha;
+                            tmem_st16f(tO + c0, of);
+                        }
+                    }
+                    const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+                    float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float a = ex2_approx(fmaf(sf[64 * h + 2 * i], P.scale_log2, -msub));
+                            const float b = ex2_approx(fmaf(sf[64 * h + 2 * i + 1], P.scale_log2, -msub));
+                            rs4[i & 3] += a + b;
+                            pk[i] = pack_bf16(a, b);
+                        }
+                        tmem_st32(tS + 32 * h, pk);
+                    }
+                    const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+                    l_sum = l_sum * alpha + rs;
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_p_full + 8 * X);
+                    first = false;
+                    had = true;
+                }
+                if (!ok) break;
+                if (!P.fused || s == P.cp - 1) {
+                    // ---- epilogue of the segment
+                    const size_t rowi = static_cast<size_t>(it.bh) * P.S + prow;
+                    if (had) {
+                        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + 8 * X, o_phase, abort_flag));
+                        if (!ok) break;
+                        o_phase ^= 1;
+                        tc_fence_after();
+                        const bool empty = !(l_sum > 0.f);
+                        const float inv_l = empty ? 0.f : 1.f / l_sum;
+                        const float lse_v = empty ? -INFINITY
+                                                  : (m_used + lg2_approx(l_sum)) * 0.69314718055994531f;
+#pragma unroll
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            float of[32];
+                            tmem_ld32f(tO + c0, of);
+                            tmem_wait_ld();
+                            reg_fence32f(of);
+                            uint32_t orr[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(of[i]);
+                            if (P.fused) {
+                                uint4* dst = reinterpret_cast<uint4*>(P.o + rowi * D + c0);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    uint4 u;
+                                    u.x = pack_bf16(__uint_as_float(orr[8 * i + 0]) * inv_l, __uint_as_float(orr[8 * i + 1]) * inv_l);
+                                    u.y = pack_bf16(__uint_as_float(orr[8 * i + 2]) * inv_l, __uint_as_float(orr[8 * i + 3]) * inv_l);
+                                    u.z = pack_bf16(__uint_as_float(orr[8 * i + 4]) * inv_l, __uint_as_float(orr[8 * i + 5]) * inv_l);
+                                    u.w = pack_bf16(__uint_as_float(orr[8 * i + 6]) * inv_l, __uint_as_float(orr[8 * i + 7]) * inv_l);
+                                    dst[i] = u;
+                                }
+                            } else {
+                                float4* dst = reinterpret_cast<float4*>(
+                                    P.o_parts + (static_cast<size_t>(s) * P.BH * P.S + rowi) * D + c0);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    dst[i] = make_float4(__uint_as_float(orr[4 * i + 0]) * inv_l,
+                                                         __uint_as_float(orr[4 * i + 1]) * inv_l,
+                                                         __uint_as_float(orr[4 * i + 2]) * inv_l,
+                                                         __uint_as_float(orr[4 * i + 3]) * inv_l);
+                            }
+                        }
+                        if (P.fused) P.lse[rowi] = lse_v;
+                        else P.lse_parts[static_cast<size_t>(s) * P.BH * P.S + rowi] = lse_v;
+                    } else if (!P.fused) {
+                        P.lse_parts[static_cast<size_t>(s) * P.BH * P.S + rowi] = -INFINITY;
+                    } else {
+                        // no admitted key anywhere (cannot happen for a valid mask): (0, -inf)
+                        uint4* dst = reinterpret_cast<uint4*>(P.o + rowi * D);
+                        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+                        P.lse[rowi] = -INFINITY;
+                    }
+                    m_used = -INFINITY;
+                    l_sum = 0.f;
+                    first = true;
+                    had = false;
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_relinquish();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace cpattn

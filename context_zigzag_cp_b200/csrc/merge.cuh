@@ -1,0 +1,77 @@
+// LSE merge: combine n partial attentions of the same query rows into the
+// attention over the union of their key sets (the concept guide's
+// "combine(attn)" step, read as the exact log-sum-exp merge).
+//
+// For a row with partials (O_i, L_i):  m = max_i L_i,  w_i = exp(L_i - m)
+// (0 for L_i = -inf), L = m + ln sum_i w_i, O = sum_i w_i O_i / sum_i w_i.
+// This is the closed form of folding the partials pairwise in order; a row
+// whose partials are all -inf stays (0, -inf).
+//
+// HBM-bound: each warp owns one row at a time; lane l reads columns
+// [4l, 4l+4) (and [128+4l, ...) for head_dim > 128) of each live partial with
+// 16-byte loads, so a warp reads 512 contiguous bytes per partial.  Partials
+// with L = -inf are not read.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace cpattn {
+
+constexpr int MERGE_MAX_PARTS = 64;
+
+struct MergeParams {
+    int64_t rows;
+    int32_t D, n_parts;
+    const float* o_parts;    // [n][rows][D]
+    const float* lse_parts;  // [n][rows]
+    __nv_bfloat16* o_out;    // [rows][D]
+    float* lse_out;          // [rows]
+};
+
+__global__ void __launch_bounds__(256) lse_merge_kernel(MergeParams M)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int nvec = M.D / 4;            // float4 per row
+    const bool two = nvec > 32;          // head_dim > 128: two vectors per lane
+    for (int64_t row = warp_g; row < M.rows; row += nwarps) {
+        // lane p holds L of parts p and p+32
+        float la = lane < M.n_parts ? __ldg(M.lse_parts + static_cast<int64_t>(lane) * M.rows + row) : -INFINITY;
+        float lb = lane + 32 < M.n_parts ? __ldg(M.lse_parts + static_cast<int64_t>(lane + 32) * M.rows + row) : -INFINITY;
+        float m = fmaxf(la, lb);
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+        float wsum = 0.f;
+        if (m != -INFINITY) {
+            const float wa = la == -INFINITY ? 0.f : expf(la - m);
+            const float wb = lb == -INFINITY ? 0.f : expf(lb - m);
+            float ws = wa + wb;
+            for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
+            wsum = ws;
+            for (int p = 0; p < M.n_parts; ++p) {
+                const float w = __shfl_sync(0xffffffffu, p < 32 ? wa : wb, p & 31);
+                if (w == 0.f) continue;  // warp-uniform
+                const float4* src = reinterpret_cast<const float4*>(
+                    M.o_parts + (static_cast<int64_t>(p) * M.rows + row) * M.D);
+                if (lane < nvec) {
+                    const float4 x = __ldg(src + lane);
+                    acc0.x += w * x.x; acc0.y += w * x.y; acc0.z += w * x.z; acc0.w += w * x.w;
+                }
+                if (two && lane + 32 < nvec) {
+                    const float4 x = __ldg(src + lane + 32);
+                    acc1.x += w * x.x; acc1.y += w * x.y; acc1.z += w * x.z; acc1.w += w * x.w;
+                }
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        uint2* dst = reinterpret_cast<uint2*>(M.o_out + row * M.D);
+        if (lane < nvec)
+            dst[lane] = make_uint2(pack_bf16(acc0.x * inv, acc0.y * inv), pack_bf16(acc0.z * inv, acc0.w * inv));
+        if (two && lane + 32 < nvec)
+            dst[lane + 32] = make_uint2(pack_bf16(acc1.x * inv, acc1.y * inv), pack_bf16(acc1.z * inv, acc1.w * inv));
+        if (lane == 0) M.lse_out[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+    }
+}
+
+}  // namespace cpattn

@@ -1,0 +1,201 @@
+// Shard planner / indexer and the shard gather.
+//
+// The sequence of S tokens is cut into 2*cp chunks of C = S/(2cp) tokens
+// (S % (2*cp) == 0: NeMo "Hierarchical Context Parallel Skill", "Required
+// constraints"); virtual rank r owns chunk r followed by chunk 2cp-1-r, so a
+// rank's early (cheap) causal rows are paired with late (expensive) ones and
+// every rank gets the same causal work.  K/V shards are visited in all-gather
+// order (s) or ring order ((r - s) mod cp) (Accelerate "Context Parallel"
+// concept guide, "all-to-all vs all-gather").
+//
+// All outputs are integers and bit-exact.
+#pragma once
+#include "ptx.cuh"
+#include "zigzag.cuh"
+
+namespace cpattn {
+
+constexpr int PLAN_MAX_CP = 1024;
+
+struct PlanParams {
+    int32_t S, cp, C, num_docs, docs, rotate;
+    const int32_t* cu;  // [num_docs+1] original order (docs only)
+    int32_t *perm, *inv_perm, *src, *doc_start, *rank_cu_off, *rank_cu;
+    int64_t* pairs;
+};
+
+// Largest d in [0, nd-1] with cu[d] <= x (cu[0] = 0 <= x for a valid list).
+__device__ __forceinline__ int doc_index(const int32_t* cu, int nd, int x)
+{
+    int lo = 0, hi = nd - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(cu + mid) <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Number of document starts strictly inside (a, a + len) (cu[1..nd-1]).
+__device__ __forceinline__ int doc_starts_inside(const int32_t* cu, int nd, int a, int len)
+{
+    if (nd <= 1) return 0;
+    int d = doc_index(cu, nd, a) + 1;  // first start > a (if cu valid)
+    int n = 0;
+    while (d < nd && __ldg(cu + d) < a + len) {
+        if (__ldg(cu + d) > a) ++n;
+        ++d;
+    }
+    return n;
+}
+
+// One block: validate cu_seqlens, zero the pair counters, write src and the
+// per-rank local segment lists.
+__global__ void __launch_bounds__(256) plan_meta_kernel(PlanParams P)
+{
+    __shared__ int32_t cnt[PLAN_MAX_CP + 1];
+    const int tid = threadIdx.x;
+    if (P.docs) {
+        bool bad = false;
+        if (tid == 0) bad = (__ldg(P.cu) != 0) || (__ldg(P.cu + P.num_docs) != P.S);
+        for (int d = tid; d < P.num_docs; d += blockDim.x)
+            if (__ldg(P.cu + d + 1) <= __ldg(P.cu + d)) bad = true;
+        if (bad) record_status(1 /* CP_ERR_INVALID_ARG */);
+    }
+    for (int i = tid; i < P.cp * P.cp; i += blockDim.x) {
+        const int r = i / P.cp, s = i - r * P.cp;
+        P.src[i] = P.rotate == 0 ? s : ((r - s) % P.cp + P.cp) % P.cp;
+    }
+    for (int r = tid; r < P.cp; r += blockDim.x) {
+        P.pairs[r] = 0;
+        int n = 3;  // local 0, chunk boundary C, end 2C
+        if (P.docs) {
+            n += doc_starts_inside(P.cu, P.num_docs, r * P.C, P.C);
+            n += doc_starts_inside(P.cu, P.num_docs, (2 * P.cp - 1 - r) * P.C, P.C);
+        }
+        cnt[r] = n;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int r = 0; r < P.cp; ++r) {
+            const int n = cnt[r];
+            cnt[r] = acc;
+            P.rank_cu_off[r] = acc;
+            acc += n;
+        }
+        P.rank_cu_off[P.cp] = acc;
+    }
+    __syncthreads();
+    for (int r = tid; r < P.cp; r += blockDim.x) {
+        int w = cnt[r];
+        for (int half = 0; half < 2; ++half) {
+            const int chunk = half == 0 ? r : 2 * P.cp - 1 - r;
+            const int a = chunk * P.C;
+            P.rank_cu[w++] = half * P.C;
+            if (P.docs && P.num_docs > 1) {
+                int d = doc_index(P.cu, P.num_docs, a) + 1;
+                while (d < P.num_docs && __ldg(P.cu + d) < a + P.C) {
+                    const int x = __ldg(P.cu + d);
+                    if (x > a) P.rank_cu[w++] = half * P.C + (x - a);
+                    ++d;
+                }
+            }
+        }
+        P.rank_cu[w++] = 2 * P.C;
+    }
+}
+
+// Grid over shard positions: perm, inv_perm, doc_start and the per-rank
+// unmasked pair counts (keys doc_start(o) .. o for the token at original o).
+__global__ void __launch_bounds__(256) plan_index_kernel(PlanParams P)
+{
+    const int n2c = 2 * P.C;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x; base < P.S;
+         base += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int p = static_cast<int>(base) + threadIdx.x;
+        int64_t cnt = 0;
+        int r = -1;
+        if (p < P.S) {
+            r = p / n2c;
+            const int t = p - r * n2c;
+            const int chunk = t < P.C ? r : 2 * P.cp - 1 - r;
+            const int o = chunk * P.C + (t < P.C ? t : t - P.C);
+            P.perm[p] = o;
+            P.inv_perm[o] = p;
+            const int ds = P.docs ? __ldg(P.cu + doc_index(P.cu, P.num_docs, o)) : 0;
+            P.doc_start[p] = ds;
+            cnt = static_cast<int64_t>(o) - ds + 1;
+        }
+        // warp-level sum when the whole warp belongs to one rank, else per thread
+        const int r0 = __shfl_sync(0xffffffffu, r, 0), r31 = __shfl_sync(0xffffffffu, r, 31);
+        if (r0 == r31 && r0 >= 0) {
+            for (int off = 16; off > 0; off >>= 1)
+                cnt += __shfl_down_sync(0xffffffffu, cnt, off);
+            if ((threadIdx.x & 31) == 0)
+                atomicAdd(reinterpret_cast<unsigned long long*>(P.pairs + r0),
+                          static_cast<unsigned long long>(cnt));
+        } else if (r >= 0) {
+            atomicAdd(reinterpret_cast<unsigned long long*>(P.pairs + r),
+                      static_cast<unsigned long long>(cnt));
+        }
+    }
+}
+
+// Row gather between original and shard order for one tensor
+// [outer][S][row_bytes] (row_bytes a multiple of 16).  to_shard = 1:
+// out[o][p] = in[o][orig(p)]; to_shard = 0: out[o][q] = in[o][shard(q)].
+struct GatherParams {
+    const uint4* in;
+    uint4* out;
+    int64_t rows;       // outer * S
+    int32_t vpr;        // 16-byte vectors per row
+    int32_t rpw;        // rows per warp pass (32 / vpr when vpr divides 32, else 1)
+    int32_t S, C, cp, to_shard;
+};
+
+__global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams G)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int sub = G.rpw > 1 ? lane / G.vpr : 0;
+    const int e0 = G.rpw > 1 ? lane - sub * G.vpr : lane;
+    constexpr int U = 4;
+    for (int64_t rb = warp_g * G.rpw * U; rb < G.rows; rb += nwarps * G.rpw * U) {
+        uint4 buf[U][1];
+        int64_t dst_row[U];
+        bool valid[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = rb + static_cast<int64_t>(u) * G.rpw + sub;
+            valid[u] = row < G.rows;
+            dst_row[u] = row;
+            if (valid[u]) {
+                const int64_t o = row / G.S;
+                const int p = static_cast<int>(row - o * G.S);
+                const int sp = G.to_shard ? orig_of_shard(p, G.C, G.cp) : shard_of_orig(p, G.C, G.cp);
+                const int64_t srow = o * G.S + sp;
+                if (e0 < G.vpr) buf[u][0] = __ldg(G.in + srow * G.vpr + e0);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (valid[u] && e0 < G.vpr) G.out[dst_row[u] * G.vpr + e0] = buf[u][0];
+        // rows wider than 32 vectors: remaining vectors of the same rows
+        if (G.rpw == 1 && G.vpr > 32) {
+            for (int e = e0 + 32; e < G.vpr; e += 32) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (!valid[u]) continue;
+                    const int64_t row = dst_row[u];
+                    const int64_t o = row / G.S;
+                    const int p = static_cast<int>(row - o * G.S);
+                    const int sp = G.to_shard ? orig_of_shard(p, G.C, G.cp) : shard_of_orig(p, G.C, G.cp);
+                    G.out[row * G.vpr + e] = __ldg(G.in + (o * G.S + sp) * G.vpr + e);
+                }
+            }
+        }
+    }
+}
+
+}  // namespace cpattn

@@ -1,0 +1,269 @@
+/*
+ * cp_attn.h -- C ABI of libcpattn: zigzag context-parallel causal attention on
+ * one B200 (sm_100a), with every context-parallel rank run as a virtual rank
+ * (a shard loop in HBM) on the same GPU.
+ *
+ * The problem, as the pages state it:
+ *   - Q, K and V are sharded along the sequence; rank i keeps its query shard
+ *     Q_i, attends it to its own K_i,V_i and then to every other rank's
+ *     K_j,V_j, and the partial attentions are combined
+ *     (Accelerate "Context Parallel" concept guide, "So how does it work?").
+ *     Each shard has the layout [batch, num_heads, seq_len/cp, head_dim].
+ *   - The K/V shards are visited in all-gather order (gather once, compute in
+ *     rank order) or ring order ("all-to-all": take the neighbour's shard
+ *     cp-1 times) (concept guide, "all-to-all vs all-gather";
+ *     "Configurable options": cp_size and cp_comm_strategy).
+ *   - seq_len must be divisible by 2*cp (NeMo "Hierarchical Context Parallel
+ *     Skill", "Required constraints"); the 2*cp chunks are paired head/tail
+ *     so every rank gets the same causal work.
+ *   - An invalid strategy or size is an error, not a silent fallback
+ *     (Accelerate FullyShardedDataParallelPlugin.__post_init__ checks).
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains memory.  Pointers must be 16-byte
+ *     aligned.
+ *   - Attention tensors are contiguous bf16 [batch][heads][seq][head_dim]
+ *     (BHSD) in SHARD order: position p = r*2C + t is local token t of virtual
+ *     rank r, C = seq_len/(2*cp).  LSE tensors are fp32 [batch][heads][seq],
+ *     natural log of the sum of exp(scaled scores).  cu_seqlens is in ORIGINAL
+ *     order.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Argument checks run on the host before any launch and
+ *     return an error without touching the GPU.  Errors found on the device
+ *     (a bounded wait that timed out) are recorded in a device status word that
+ *     cp_get_device_status() reads and clears.
+ *   - Workspace: calls that take (ws, ws_bytes) report the bytes they need in
+ *     *ws_bytes and launch nothing when ws == NULL.  Otherwise *ws_bytes must
+ *     be at least that size (else CP_ERR_WORKSPACE); ws must be 256-byte
+ *     aligned.  The workspace is scratch: its contents need not be preserved.
+ *   - No call is thread-safe with respect to another call on the same buffers.
+ */
+#ifndef CP_ATTN_H
+#define CP_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CP_API __attribute__((visibility("default")))
+#else
+#define CP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CP_OK = 0,
+    CP_ERR_INVALID_ARG = 1, /* bad size, null pointer, bad enum, bad cu_seqlens */
+    CP_ERR_UNSUPPORTED = 2, /* valid problem outside what the kernels cover   */
+    CP_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, no device)  */
+    CP_ERR_TIMEOUT = 4,     /* a bounded device wait gave up                  */
+    CP_ERR_WORKSPACE = 5    /* workspace smaller than required                */
+} cp_status_t;
+
+typedef enum { CP_ROTATE_ALLGATHER = 0, CP_ROTATE_RING = 1 } cp_rotate_t;
+typedef enum { CP_MASK_CAUSAL = 0, CP_MASK_DOC_CAUSAL = 1 } cp_mask_t;
+
+/* How cp_attn_fwd combines the per-step partial attentions.
+ *   CP_MERGE_SEPARATE: each (rank, step) unit writes its partial (O, LSE) in
+ *     fp32 to the workspace, then the cp_lse_merge kernel folds the cp
+ *     partials in visit order (the literal shard loop + combine).
+ *   CP_MERGE_FUSED: the forward kernel folds each step into the running
+ *     (O, LSE) in registers / tensor memory as it goes, in the same visit
+ *     order, and writes only the final result. */
+typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
+
+/* The problem.  Field meaning:
+ *   batch         >= 1
+ *   seq_len       S, tokens per sequence; S % (2*cp_size) == 0
+ *   cp_size       number of virtual ranks, >= 1
+ *   num_heads     query heads Hq; num_kv_heads Hkv divides Hq (GQA: query head
+ *                 h reads KV head h / (Hq/Hkv))
+ *   head_dim      D
+ *   rotate        cp_rotate_t
+ *   mask          cp_mask_t; CP_MASK_DOC_CAUSAL needs cu_seqlens
+ *   merge         cp_merge_t (forward only)
+ *   softmax_scale 0 => 1/sqrt(head_dim)
+ *   num_docs      documents in cu_seqlens (doc mask only)
+ *   cu_seqlens    DEVICE int32 [num_docs+1], 0 = cu[0] < cu[1] < ... <
+ *                 cu[num_docs] = S, original order; the same documents apply to
+ *                 every batch entry.  NULL for the plain causal mask.  Only
+ *                 cp_plan_shards reads it, on the device: a list that is not
+ *                 strictly increasing from 0 to S records CP_ERR_INVALID_ARG in
+ *                 the device status word (the host cannot see device memory
+ *                 without synchronising).  The forward/backward read the plan. */
+typedef struct {
+    int32_t batch;
+    int32_t seq_len;
+    int32_t cp_size;
+    int32_t num_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    int32_t rotate;
+    int32_t mask;
+    int32_t merge;
+    float softmax_scale;
+    int32_t num_docs;
+    int32_t reserved;
+    const int32_t* cu_seqlens;
+} cp_problem_t;
+
+/* The shard plan, written by cp_plan_shards into caller-owned DEVICE buffers:
+ *   perm        int32 [S]          original index of shard position p
+ *   inv_perm    int32 [S]          shard position of original index o
+ *   src         int32 [cp*cp]      K/V shard visited by rank r at step s:
+ *                                  s (all-gather) or (r - s) mod cp (ring)
+ *   doc_start   int32 [S]          original start of the document of token
+ *                                  perm[p] (0 everywhere for CP_MASK_CAUSAL)
+ *   rank_cu_off int32 [cp+1]       rank r's entries are rank_cu[off[r]..off[r+1])
+ *   rank_cu     int32 [3*cp + num_docs]  per rank, local offsets where a
+ *                                  segment starts (0, the chunk boundary C,
+ *                                  every document start inside the rank's
+ *                                  chunks), then 2C
+ *   pairs       int64 [cp]         unmasked (q, k) pairs whose query lives on
+ *                                  rank r (equal across ranks for the plain
+ *                                  causal mask) */
+typedef struct {
+    int32_t* perm;
+    int32_t* inv_perm;
+    int32_t* src;
+    int32_t* doc_start;
+    int32_t* rank_cu_off;
+    int32_t* rank_cu;
+    int64_t* pairs;
+} cp_plan_t;
+
+/*
+ * cp_plan_shards -- build the zigzag plan on the GPU and gather n_bufs tensors
+ * from ORIGINAL into SHARD order (rank r's chunk r then chunk 2cp-1-r), the
+ * counterpart of sharding the context buffers along their sequence dimension
+ * (concept guide, "Accelerate's interface": buffers / buffer_seq_dims).
+ *   bufs_in[i], bufs_out[i]  device tensors [outer_i][S][row_bytes_i]; in and
+ *                            out must not overlap
+ *   buf_outer[i]             outer extent (batch*heads) of buffer i
+ *   buf_row_bytes[i]         bytes per token row (head_dim*2 for bf16), a
+ *                            multiple of 16
+ *   n_bufs                   0..16; with 0 only the plan is built
+ * Reads problem->cu_seqlens for the doc mask.  Plan arrays and gathered
+ * tensors are complete when the stream reaches this point.
+ * Errors: CP_ERR_INVALID_ARG for the checks listed in cp_problem_t, a NULL
+ * plan array, bad buffer sizes; CP_ERR_CUDA on a launch failure.
+ */
+CP_API cp_status_t cp_plan_shards(const cp_problem_t* problem, const cp_plan_t* plan, int32_t n_bufs,
+                           const void* const* bufs_in, void* const* bufs_out,
+                           const int64_t* buf_outer, const int64_t* buf_row_bytes, void* ws,
+                           size_t* ws_bytes, void* stream);
+
+/*
+ * cp_unshard -- scatter n_bufs tensors from SHARD back to ORIGINAL order with
+ * the plan's perm (the "restore" of the sharded buffers).  Same buffer
+ * conventions as cp_plan_shards.
+ */
+CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan, int32_t n_bufs,
+                       const void* const* bufs_in, void* const* bufs_out,
+                       const int64_t* buf_outer, const int64_t* buf_row_bytes, void* stream);
+
+/*
+ * cp_attn_fwd -- causal (optionally packed-document) attention of every
+ * virtual rank's query shard against the K/V shards in the plan's visit order,
+ * combined into the exact unsharded result (concept guide, "So how does it
+ * work?": local attention, then every other shard, then combine).
+ *   q     bf16 [B][Hq][S][D]  shard order
+ *   k, v  bf16 [B][Hkv][S][D] shard order
+ *   o     bf16 [B][Hq][S][D]  output, shard order
+ *   lse   fp32 [B][Hq][S]     output, natural-log LSE of the scaled scores
+ * Supported: head_dim 64 or 128; C = S/(2cp) a multiple of 128.
+ * Workspace: CP_MERGE_SEPARATE needs cp fp32 partial (O, LSE) sets plus a
+ * small header; CP_MERGE_FUSED needs only the header.
+ * Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_WORKSPACE, CP_ERR_CUDA.
+ */
+CP_API cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                        const void* k, const void* v, void* o, float* lse, void* ws,
+                        size_t* ws_bytes, void* stream);
+
+/*
+ * cp_attn_bwd -- gradients of the attention output with respect to Q, K, V
+ * given the upstream gradient dO, from the saved final LSE (backward through
+ * the context-parallel attention; FLOPs counted as twice the forward, as the
+ * Accelerate example's model-FLOPs helper does).  dK_j and dV_j collect the
+ * contributions of every virtual rank that visits shard j.
+ *   q, k, v, o, dout  bf16, shard order (o and lse from cp_attn_fwd)
+ *   dq                bf16 [B][Hq][S][D]  output
+ *   dk, dv            bf16 [B][Hkv][S][D] output
+ * Workspace: an fp32 dQ accumulator, the per-row dot(dO, O), and a header.
+ * Errors: as cp_attn_fwd.
+ */
+CP_API cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                        const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* ws,
+                        size_t* ws_bytes, void* stream);
+
+/*
+ * cp_lse_merge -- combine n_parts partial attentions row by row, folding them
+ * in the given order: for running (O_a, L_a) and next (O_b, L_b),
+ * m = max(L_a, L_b); if m = -inf the row stays (0, -inf); else
+ * w = exp(L - m), L = m + ln(w_a + w_b), O = (w_a O_a + w_b O_b)/(w_a + w_b)
+ * (the concept guide's "combine(attn)", read as the exact log-sum-exp merge).
+ *   o_parts    fp32 [n_parts][rows][head_dim]
+ *   lse_parts  fp32 [n_parts][rows]; -inf marks a row with no key in that part
+ *              (its O part is not read)
+ *   o_out      bf16 [rows][head_dim] (round to nearest even)
+ *   lse_out    fp32 [rows]
+ * head_dim must be a positive multiple of 4 no larger than 256; 1 <= n_parts
+ * <= 64; rows >= 0.
+ * Errors: CP_ERR_INVALID_ARG, CP_ERR_CUDA.
+ */
+CP_API cp_status_t cp_lse_merge(int64_t rows, int32_t head_dim, int32_t n_parts, const float* o_parts,
+                         const float* lse_parts, void* o_out, float* lse_out, void* stream);
+
+/* Read and clear the device status word on `stream` (synchronises the stream).
+ * *status receives CP_OK or the first device-side error since the last read. */
+CP_API cp_status_t cp_get_device_status(int32_t* status, void* stream);
+
+/* Set the limit, in nanoseconds, after which a bounded device wait gives up
+ * (default 2 s).  Synchronous. */
+CP_API cp_status_t cp_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Self-test of the bounded-wait machinery: one CTA waits on an mbarrier that
+ * nothing will ever complete, gives up after limit_ns and records
+ * CP_ERR_TIMEOUT in the device status word.  The GPU context stays usable. */
+CP_API cp_status_t cp_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* Kernels of the library, as reported by the launch trace. */
+typedef enum {
+    CP_K_PLAN_META = 1,  /* plan: cu_seqlens check, src table, segment lists */
+    CP_K_PLAN_INDEX = 2, /* plan: perm, inv_perm, doc_start, pair counts     */
+    CP_K_GATHER = 3,     /* shard / unshard row gather                      */
+    CP_K_FWD = 4,        /* forward attention                               */
+    CP_K_MERGE = 5,      /* LSE merge                                       */
+    CP_K_BWD_PREP = 6,   /* backward: dot(dO, O), LSE * log2(e)             */
+    CP_K_BWD_DKDV = 7,   /* backward: dK, dV                                */
+    CP_K_BWD_DQ = 8,     /* backward: dQ                                    */
+    CP_K_SELFTEST = 9
+} cp_kernel_t;
+
+/* Number of kernels this library has launched in this process. */
+CP_API int64_t cp_launch_count(void);
+
+/* Launch trace.  cp_trace_begin hands the library `capacity` pairs of CUDA
+ * events (cudaEvent_t, created by the caller with timing enabled; 2*capacity
+ * handles).  Each later kernel launch k (k < capacity) records events[2k] on
+ * its stream just before the launch and events[2k+1] just after it, and notes
+ * its cp_kernel_t.  cp_trace_end stops recording and returns the number of
+ * launches seen (which may exceed capacity; only the first `capacity` carry
+ * events) and their kernel ids in kernel_ids[capacity].  Not thread-safe; the
+ * events stay owned by the caller. */
+CP_API cp_status_t cp_trace_begin(void* const* events, int32_t capacity);
+CP_API cp_status_t cp_trace_end(int32_t* n_launches, int32_t* kernel_ids);
+
+/* Library version, major*10000 + minor*100 + patch. */
+CP_API int32_t cp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CP_ATTN_H */
