@@ -185,6 +185,15 @@ def cpu_baseline(w: synth.Workload, budget_tokens: int = 3072):
                        f"head_dim {w.head_dim}), fp64 C oracle, {dt:.1f} s"), dt
 
 
+def config_dict(w: synth.Workload, rotate: str, world: int) -> dict:
+    q_mib = w.batch * w.num_heads * w.seq_len * w.head_dim * 2 / 2 ** 20
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "cp": w.cp,
+            "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+            "rotate": rotate, "mask": "doc" if w.docs else "causal", "merge": "separate",
+            "l2": "inputs larger than L2 (Q alone is %.0f MiB)" % q_mib,
+            "parallelism": f"replicas x{world}"}
+
+
 # --------------------------------------------------------------------- native arm
 
 KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_dkdv": 6.0, "bwd_dq": 2.0}   # x D*Hq*pairs
@@ -330,13 +339,7 @@ def run_native(args, w, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO)",
-            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "cp": w.cp,
-                       "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
-                       "head_dim": w.head_dim, "rotate": rotate,
-                       "mask": "doc" if w.docs else "causal", "merge": "separate",
-                       "l2": "inputs larger than L2 (Q alone is %.0f MiB)" % (
-                           q.numel() * 2 / 2 ** 20),
-                       "parallelism": f"replicas x{world}"},
+            "config": config_dict(w, rotate, world),
             "fwd_tflops": round(fwd_flops / 1e9 / fwd_ms, 1),
             "fwd_frac_of_peak": round(fwd_flops / 1e9 / fwd_ms / peaks["bf16"], 4),
             "fwd_fused_tflops": round(fwd_flops / 1e9 / fused_ms, 1),
@@ -383,7 +386,7 @@ def run_reference(args, w, rank, world):
         "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(tot_t / len(vals) * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name, "sample": vals[0][0]["sample"]},
+        "data": "synthetic", "config": config_dict(w, args.rotate or w.rotate, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": base["cores"],
                          "kind": "oracle", "sample": vals[0][0]["sample"]},
         "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,

@@ -226,6 +226,14 @@ def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
            "cp_selftest_wait_timeout")
 
 
+def selftest_exp2(x: torch.Tensor, stream=None):
+    """(software exp2, hardware ex2) of a float32 CUDA tensor."""
+    ys, yh = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().cp_selftest_exp2(_ptr(x), _ptr(ys), _ptr(yh), x.numel(), _stream(stream)),
+           "cp_selftest_exp2")
+    return ys, yh
+
+
 def launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(lib().cp_launch_count())

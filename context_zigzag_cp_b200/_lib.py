@@ -23,10 +23,11 @@ MERGE = {"separate": 0, "fused": 1}
 # Every function the header declares (checked against include/cp_attn.h by the tests).
 EXPORTED = ("cp_plan_shards", "cp_unshard", "cp_attn_fwd", "cp_attn_bwd", "cp_lse_merge",
             "cp_get_device_status", "cp_set_wait_limit_ns", "cp_selftest_wait_timeout",
-            "cp_launch_count", "cp_trace_begin", "cp_trace_end", "cp_version")
+            "cp_launch_count", "cp_trace_begin", "cp_trace_end", "cp_selftest_exp2",
+            "cp_version")
 
 KERNEL_NAMES = {1: "plan_meta", 2: "plan_index", 3: "gather", 4: "fwd", 5: "merge",
-                6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest"}
+                6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2"}
 
 
 class CpProblem(ctypes.Structure):
@@ -73,6 +74,7 @@ def load() -> ctypes.CDLL:
     lib.cp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.cp_version.argtypes = []
     lib.cp_launch_count.argtypes = []
+    lib.cp_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
     lib.cp_trace_begin.argtypes = [ctypes.POINTER(vp), ctypes.c_int32]
     lib.cp_trace_end.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     for name in EXPORTED:

@@ -8,6 +8,7 @@
 
 #include "cp_attn.h"
 #include "ptx.cuh"
+#include "exp2_poly.cuh"
 #include "tmap.h"
 #include "zigzag.cuh"
 #include "plan.cuh"
@@ -253,11 +254,31 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns)
     }
 }
 
+__global__ void selftest_exp2_kernel(const float* x, float* ys, float* yh, int64_t n)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        ys[i] = exp2_poly(x[i]);
+        yh[i] = ex2_approx(x[i]);
+    }
+}
+
 }  // namespace
 
 extern "C" {
 
 int32_t cp_version(void) { return kVersion; }
+
+cp_status_t cp_selftest_exp2(const float* x, float* y_soft, float* y_hw, int64_t n, void* stream)
+{
+    if (n < 0) return CP_ERR_INVALID_ARG;
+    if (n == 0) return CP_OK;
+    if (!x || !y_soft || !y_hw) return CP_ERR_INVALID_ARG;
+    LaunchScope ls(CP_K_SELFTEST_EXP2, as_stream(stream));
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, int64_t(num_sms()) * 8);
+    selftest_exp2_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(x, y_soft, y_hw, n);
+    return launch_status();
+}
 
 int64_t cp_launch_count(void) { return g_launches; }
 

@@ -6,12 +6,16 @@
 // the longest items start first, and are dealt round-robin to one persistent
 // CTA per SM.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads = three warpgroups):
 //   warps 0-3  softmax group 0 (query tile 0): one TMEM lane = one query row
 //   warps 4-7  softmax group 1 (query tile 1)
 //   warp 8     TMA producer: Q tiles, then K and V tiles through a ring of
 //              shared-memory slots
 //   warp 9     MMA issuer (one thread) + tensor-memory owner
+//   warps 10-11 idle
+// The block launches with 168 registers per thread; the softmax warpgroups
+// raise theirs to 208 and the producer/MMA warpgroup drops to 88
+// (2*128*208 + 128*88 = 384*168).
 // Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D),
 // O1 [384,384+D).  P is written back as bf16 over the first 64 columns of its
 // S region and used as the A operand of O += P V straight from tensor memory.
@@ -30,6 +34,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
+#include "exp2_poly.cuh"
 #include "zigzag.cuh"
 
 namespace cpattn {
@@ -92,7 +97,7 @@ struct FwdCfg {
     // barriers: q_full, q_empty, s_full[2], p_full[2], o_full[2], kv_full[NSLOT], kv_empty[NSLOT], drain
     static constexpr int NBAR = 9 + 2 * NSLOT;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;  // + alignment slack
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
 };
 
 struct TileIter {
@@ -118,8 +123,47 @@ __device__ __forceinline__ TileIter load_tile_iter(const FwdParams& P, const Fwd
     return ti;
 }
 
+// Exponentials of one query row's 128 scores (log2 domain, reference max msub),
+// packed to bf16 pairs and stored over the first 64 columns of the row's S
+// region; returns the fp32 row sum.  With SOFT, every fourth pair of columns
+// uses the software exp2 on the FMA pipe (only for unmasked tiles, whose
+// arguments are finite), the rest the hardware ex2.
+template <bool SOFT>
+__device__ __forceinline__ float exp_pack_store(const float* sf, float scale_log2, float msub,
+                                                uint32_t tS)
+{
+    const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
+    const uint64_t nm = f2_pack(-msub, -msub);
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const uint64_t x2 = f2_fma(f2_pack(sf[64 * h + 2 * i], sf[64 * h + 2 * i + 1]), sl2, nm);
+            uint64_t p2;
+            if (SOFT && (i & 3) == 3) {
+                p2 = exp2_poly2(x2);
+            } else {
+                float a, b;
+                f2_unpack(x2, a, b);
+                p2 = f2_pack(ex2_approx(a), ex2_approx(b));
+            }
+            acc[i & 3] = f2_add(acc[i & 3], p2);
+            float a, b;
+            f2_unpack(p2, a, b);
+            pk[i] = pack_bf16(a, b);
+        }
+        tmem_st32(tS + 32 * h, pk);
+    }
+    const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+    float a, b;
+    f2_unpack(t, a, b);
+    return a + b;
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const FwdParams P)
 {
@@ -162,8 +206,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 8) {
+    if (warp >= 8) {
+      regs_dec<88>();
+      if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
@@ -307,7 +352,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0);
         }
+      }
     } else {
+        regs_inc<208>();
         // ------------------------------------------------------------ softmax groups
         const int X = warp >> 2;                 // query tile handled by this group
         const int row = (warp & 3) * 32 + lane;  // TMEM lane == query row in the tile
@@ -352,15 +399,14 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         for (int c = 0; c < 128; ++c)
                             if (c < lo || c > hi) sf[c] = -INFINITY;
                     }
-                    float mx8[8];
+                    float mx4[4];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(sf[i], sf[i + 8]);
+                    for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(sf[i], sf[i + 4]);
 #pragma unroll
-                    for (int c = 16; c < 128; c += 16)
+                    for (int c = 8; c < 128; c += 8)
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], fmaxf(sf[c + i], sf[c + 8 + i]));
-                    const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                        for (int i = 0; i < 4; ++i) mx4[i] = fmax3(mx4[i], sf[c + i], sf[c + 4 + i]);
+                    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                     const float m_tile = mx * P.scale_log2;
                     // lazy rescale: keep the reference max unless it is exceeded by more
                     // than 8 (a factor 256 in the exponentials), or is still -inf
@@ -384,20 +430,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         }
                     }
                     const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-                    float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t pk[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float a = ex2_approx(fmaf(sf[64 * h + 2 * i], P.scale_log2, -msub));
-                            const float b = ex2_approx(fmaf(sf[64 * h + 2 * i + 1], P.scale_log2, -msub));
-                            rs4[i & 3] += a + b;
-                            pk[i] = pack_bf16(a, b);
-                        }
-                        tmem_st32(tS + 32 * h, pk);
-                    }
-                    const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+                    const float rs = (cls == TILE_FULL) ? exp_pack_store<true>(sf, P.scale_log2, msub, tS)
+                                                        : exp_pack_store<false>(sf, P.scale_log2, msub, tS);
                     l_sum = l_sum * alpha + rs;
                     tmem_wait_st();
                     tc_fence_before();

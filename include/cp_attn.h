@@ -242,7 +242,8 @@ typedef enum {
     CP_K_BWD_PREP = 6,   /* backward: dot(dO, O), LSE * log2(e)             */
     CP_K_BWD_DKDV = 7,   /* backward: dK, dV                                */
     CP_K_BWD_DQ = 8,     /* backward: dQ                                    */
-    CP_K_SELFTEST = 9
+    CP_K_SELFTEST = 9,
+    CP_K_SELFTEST_EXP2 = 10
 } cp_kernel_t;
 
 /* Number of kernels this library has launched in this process. */
@@ -258,6 +259,12 @@ CP_API int64_t cp_launch_count(void);
  * events stay owned by the caller. */
 CP_API cp_status_t cp_trace_begin(void* const* events, int32_t capacity);
 CP_API cp_status_t cp_trace_end(int32_t* n_launches, int32_t* kernel_ids);
+
+/* Self-test of the forward kernel's software exp2 (range reduction plus a
+ * polynomial on the FMA pipe): y_soft[i] = software 2^x[i], y_hw[i] = the
+ * hardware ex2.approx result, for n device floats (finite, <= 127). */
+CP_API cp_status_t cp_selftest_exp2(const float* x, float* y_soft, float* y_hw, int64_t n,
+                                    void* stream);
 
 /* Library version, major*10000 + minor*100 + patch. */
 CP_API int32_t cp_version(void);

@@ -362,3 +362,15 @@ def test_flop_convention_and_memory_estimate():
     assert oracle.flops(8, 128, 100, backward=True) == 3 * oracle.flops(8, 128, 100)
     # the concept guide's vanilla attention-matrix estimate: 128k*128k*2 B = 32 GiB per head
     assert 131072 * 131072 * 2 == 32 * 2 ** 30
+
+
+def test_bf16_ulp_helper():
+    """The tolerance helper's bf16 spacing: 2^-7 at 1, 2^-4 at 8..16, and exact for
+    values that bf16 represents."""
+    from helpers import bf16_ulp
+    assert bf16_ulp(np.array([1.0]))[0] == 2.0 ** -7
+    assert bf16_ulp(np.array([8.159]))[0] == 2.0 ** -4
+    assert bf16_ulp(np.array([-3.0]))[0] == 2.0 ** -6
+    x = torch.tensor([8.159, 1.2345, -0.3]).to(torch.bfloat16).double().numpy()
+    ref = np.array([8.159, 1.2345, -0.3])
+    assert (np.abs(x - ref) <= bf16_ulp(ref) / 2 + 1e-12).all()
