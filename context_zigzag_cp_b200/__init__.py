@@ -26,7 +26,7 @@ from ._lib import CpPlan, CpProblem, STATUS_NAMES
 __all__ = ["CPError", "Problem", "Plan", "attn_fwd", "attn_bwd", "lse_merge",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "get_device_status",
            "set_wait_limit_ns", "selftest_wait_timeout", "version", "lib", "launch_count",
-           "LaunchTrace"]
+           "LaunchTrace", "attn_bwd_noalloc"]
 
 
 class CPError(RuntimeError):
@@ -196,6 +196,19 @@ def attn_bwd(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq=None, dk=None, d
                              _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(w),
                              ctypes.byref(n) if w is not None else None, _stream(stream)),
            "cp_attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq, dk, dv, stream=None):
+    """cp_attn_bwd_noalloc: the backward without a workspace, for callers that cannot
+    allocate device memory at this point (inside a CUDA graph capture, or under an
+    allocator that hands out no scratch).  Its scratch lives in a fixed 32 MiB array
+    inside the library (batch * heads * seq_len <= 4,194,304 rows); calls that could
+    overlap on the GPU must be serialised, and the first call on a device must come
+    before any stream capture.  The caller passes every output; nothing is allocated."""
+    _check(lib().cp_attn_bwd_noalloc(prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                     _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _stream(stream)), "cp_attn_bwd_noalloc")
     return dq, dk, dv
 
 

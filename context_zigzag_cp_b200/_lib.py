@@ -24,7 +24,9 @@ MERGE = {"separate": 0, "fused": 1}
 EXPORTED = ("cp_plan_shards", "cp_unshard", "cp_attn_fwd", "cp_attn_bwd", "cp_lse_merge",
             "cp_get_device_status", "cp_set_wait_limit_ns", "cp_selftest_wait_timeout",
             "cp_launch_count", "cp_trace_begin", "cp_trace_end", "cp_selftest_exp2",
-            "cp_version")
+            "cp_attn_bwd_noalloc", "cp_version")
+
+NOALLOC_MAX_ROWS = 4194304
 
 KERNEL_NAMES = {1: "plan_meta", 2: "plan_index", 3: "gather", 4: "fwd", 5: "merge",
                 6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2"}
@@ -68,6 +70,7 @@ def load() -> ctypes.CDLL:
                                i64p, i64p, vp]
     lib.cp_attn_fwd.argtypes = [P, PL, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cp_attn_bwd.argtypes = [P, PL, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.cp_attn_bwd_noalloc.argtypes = [P, PL, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.cp_lse_merge.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp]
     lib.cp_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.cp_set_wait_limit_ns.argtypes = [ctypes.c_uint64]

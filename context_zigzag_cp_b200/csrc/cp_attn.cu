@@ -518,3 +518,58 @@ extern "C" cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t*
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s)
                : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s);
 }
+
+// ---------------------------------------------------------------------------
+// cp_attn_bwd_noalloc: the backward with its per-row scratch (dot(dO, O) and
+// LSE * log2(e), fp32 each) in a fixed device array instead of a caller
+// workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(2) * CP_NOALLOC_MAX_ROWS * sizeof(float);  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// The name g_noalloc_scratch is only a host-side handle; kernels need the
+// device address, looked up once per device.
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+cp_status_t noalloc_scratch(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CP_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CP_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return CP_OK;
+}
+
+}  // namespace
+
+extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp_plan_t* plan,
+                                           const void* q, const void* k, const void* v,
+                                           const void* o, const float* lse, const void* dout,
+                                           void* dq, void* dk, void* dv, void* stream)
+{
+    cp_status_t st = check_attention(problem);
+    if (st != CP_OK) return st;
+    if ((st = check_plan(plan, false)) != CP_OK) return st;
+    const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+    for (const void* x : ptrs)
+        if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
+    const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * problem->seq_len;
+    if (rows > CP_NOALLOC_MAX_ROWS) return CP_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != CP_OK) return st;
+    float* delta = static_cast<float*>(scratch);
+    float* lse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
+    cudaStream_t s = as_stream(stream);
+    return problem->head_dim == 128
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s);
+}

@@ -219,6 +219,38 @@ CP_API cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* pla
 CP_API cp_status_t cp_lse_merge(int64_t rows, int32_t head_dim, int32_t n_parts, const float* o_parts,
                          const float* lse_parts, void* o_out, float* lse_out, void* stream);
 
+/*
+ * cp_attn_bwd_noalloc -- cp_attn_bwd for callers that cannot hand the library a
+ * workspace.  Some callers cannot allocate device memory at the point where they
+ * run the backward: code that runs while a CUDA graph is being captured (device
+ * allocation is not allowed there), or a host program whose device memory is
+ * entirely pre-planned by a framework allocator that has no way to hand out
+ * scratch.  This entry point takes the same arguments as cp_attn_bwd minus the
+ * workspace and uses a fixed scratch array that the library holds in device
+ * memory instead (there is no counterpart of this entry point on the pages; it
+ * is a convenience of this library).
+ *   - Limit: batch * num_heads * seq_len <= CP_NOALLOC_MAX_ROWS (4,194,304
+ *     rows, e.g. 131072 tokens x 32 heads); larger problems get
+ *     CP_ERR_WORKSPACE and nothing is launched.
+ *   - Cost: every GPU that loads the library holds the 32 MiB array until the
+ *     process exits.
+ *   - The first call on each device looks up the array's device address (a
+ *     synchronous runtime query); make that first call before any stream
+ *     capture.  Later calls only launch kernels.
+ *   - Every call on a device shares the one array, and the array keeps the last
+ *     call's contents (nothing in it needs to start at zero: each call writes
+ *     every scratch value it reads).  Calls that can overlap on the GPU (two
+ *     streams, or two host threads) race on the array: serialise them.
+ *   - The library allocates and frees nothing in this call.
+ * Errors: as cp_attn_bwd, plus CP_ERR_WORKSPACE beyond the limit and
+ * CP_ERR_CUDA if the array's address cannot be obtained.
+ */
+#define CP_NOALLOC_MAX_ROWS 4194304
+CP_API cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp_plan_t* plan,
+                                       const void* q, const void* k, const void* v,
+                                       const void* o, const float* lse, const void* dout,
+                                       void* dq, void* dk, void* dv, void* stream);
+
 /* Read and clear the device status word on `stream` (synchronises the stream).
  * *status receives CP_OK or the first device-side error since the last read. */
 CP_API cp_status_t cp_get_device_status(int32_t* status, void* stream);

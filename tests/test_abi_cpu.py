@@ -158,3 +158,15 @@ def test_product_has_no_cpu_fallback():
         if fn.endswith(".py"):
             text = open(os.path.join(pkg, fn)).read()
             assert "import oracle" not in text and "from oracle" not in text, fn
+
+
+def test_noalloc_limit_checked_on_host(lib):
+    """Beyond the fixed scratch array the no-alloc backward refuses before any CUDA call."""
+    p = prob(seq_len=4096, cp=2, num_heads=_lib.NOALLOC_MAX_ROWS // 4096 + 1, num_kv_heads=1,
+             head_dim=128)
+    d = ctypes.c_void_p(256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256)
+    assert cz.lib().cp_attn_bwd_noalloc(p.ref, ctypes.byref(plan), d, d, d, d, d, d, d, d, d,
+                                        None) == _lib.CP_ERR_WORKSPACE
+    assert cz.lib().cp_attn_bwd_noalloc(p.ref, ctypes.byref(plan), None, d, d, d, d, d, d, d, d,
+                                        None) == _lib.CP_ERR_INVALID_ARG
