@@ -268,6 +268,23 @@ def run_native(args, w, rank, world, local_rank):
         if n in kernels:
             kernels[n]["tflops"] = round(share * w.head_dim * w.num_heads * pairs /
                                          (kernels[n]["ms"] / kernels[n]["launches"]) / 1e9, 1)
+    # HBM-bound kernels: achieved GB/s from their algorithmic bytes
+    rows = w.batch * w.num_heads * w.seq_len
+    row_bytes = w.head_dim * 2
+    n_q = w.batch * w.num_heads * w.seq_len * row_bytes
+    n_kv = w.batch * w.num_kv_heads * w.seq_len * row_bytes
+    lse_off = int(round(w.cp * rows * w.head_dim * 4 / 256 + 0.4999)) * 256
+    lse_parts = ws_f[lse_off:lse_off + w.cp * rows * 4].view(torch.float32)
+    live = int(torch.isfinite(lse_parts).sum().item())
+    hbm_bytes = {
+        "gather": 2 * (2 * n_q + 2 * n_kv),                       # read + write Q, dO, K, V
+        "merge": rows * w.cp * 4 + live * w.head_dim * 4 + rows * (row_bytes + 4),
+        "bwd_prep": rows * (2 * row_bytes + 4) + rows * 8,        # O, dO, LSE in; D, LSE2 out
+    }
+    for n, b in hbm_bytes.items():
+        if n in kernels and kernels[n]["ms"] > 0:
+            kernels[n]["gbs"] = round(b / (kernels[n]["ms"] * 1e-3) / 1e9, 1)
+            kernels[n]["frac_of_hbm_peak"] = round(kernels[n]["gbs"] / peaks["hbm"], 4)
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     dom_flops = KERNEL_FLOP_SHARE.get(dom, 0.0) * w.head_dim * w.num_heads * pairs
     dom_ms = kernels[dom]["ms"] / kernels[dom]["launches"]

@@ -14,6 +14,12 @@
 //   * cp_bwd_dq_kernel (query-tile major, visiting the K/V shards in the plan's
 //     order like the forward):  S = Q K^T,  dP = dO V^T  ->  dS (bf16, tensor
 //     memory)  ->  dQ += dS K.
+// In both passes the elementwise step is split by columns over four
+// warpgroups (32 columns each; a thread owns one TMEM lane = one row).  Each
+// warpgroup writes its bf16 results over the first 16 columns of its own
+// 32-column block, and the MMA thread issues the product for that block (a
+// 32-deep slice of the K dimension) as soon as that warpgroup is done, so the
+// four slices overlap with the remaining elementwise work.
 // Each 128-row tile lives in one zigzag chunk, so original positions are
 // linear inside a tile and the causal / document tests are per-tile ranges.
 #pragma once
@@ -76,6 +82,9 @@ struct BwdParams {
 // ============================================================================
 // dK / dV pass
 // ============================================================================
+constexpr int BWD_NWG = 4;                       // elementwise warpgroups
+constexpr int BWD_THREADS = (BWD_NWG + 1) * 128; // + producer / MMA warpgroup
+
 template <int D>
 struct DkdvCfg {
     static constexpr int TILE = 128 * D * 2;
@@ -84,22 +93,26 @@ struct DkdvCfg {
     static constexpr int K_OFF = 0, V_OFF = TILE;
     static constexpr int ST_OFF = 2 * TILE;
     static constexpr int BAR_OFF = ST_OFF + NST * ST_STRIDE;
-    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full, acc_full, drain
-    static constexpr int NBAR = 6 + 2 * NST;
+    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full[NWG], acc_full, drain
+    static constexpr int NBAR = 5 + 2 * NST + BWD_NWG;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = BWD_THREADS;
 };
 
 struct DkdvItem {
     int bkv, b, hk, kpos, ko;
 };
 
+// Items run KV head by KV head (key tiles by ascending original position, the
+// longest first): the CTAs in flight then own neighbouring key tiles of one KV
+// head and stream the same query tiles at about the same time, so those reads
+// hit in L2.
 __device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int w)
 {
     DkdvItem it;
-    const int BHkv = P.B * P.Hkv;
-    it.bkv = w % BHkv;
-    const int t = w / BHkv;                  // key tile by ascending original position
+    const int nkt = P.S / 128;
+    it.bkv = w / nkt;
+    const int t = w - it.bkv * nkt;
     it.b = it.bkv / P.Hkv;
     it.hk = it.bkv - it.b * P.Hkv;
     it.ko = t * 128;
@@ -107,14 +120,8 @@ __device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int w)
     return it;
 }
 
-// Iterates the (query head, query tile) pairs that attend to a key tile, in the
-// same order for every role.  Query tiles are visited rank by rank.
-struct QTileWalk {
-    int g, nqt;   // heads per group, query tiles per rank
-};
-
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
 cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                    const BwdParams P)
@@ -128,8 +135,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t bars = sbase + Cfg::BAR_OFF;
     const uint32_t bar_kv_full = bars, bar_kv_empty = bars + 8;
     const uint32_t bar_st_full = bars + 16, bar_st_empty = bars + 16 + 8 * Cfg::NST;
-    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST, bar_p_full = bar_s_full + 8;
-    const uint32_t bar_acc_full = bar_s_full + 16, bar_drain = bar_s_full + 24;
+    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST;
+    const uint32_t bar_p_full = bar_s_full + 8;                       // [NWG]
+    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NWG, bar_drain = bar_acc_full + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
 
@@ -138,6 +146,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int n2c = 2 * P.C;
     const int nqt = n2c / 128;
     const uint32_t st_bytes = 2 * Cfg::TILE + 1024 + (P.docs ? 512 : 0);
+    constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -148,18 +157,22 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mbar_init(bar_st_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_full, 4);
+        for (int i = 0; i < BWD_NWG; ++i) mbar_init(bar_p_full + 8 * i, 4);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_slot), 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp >= 4 * BWD_NWG) {
+      // producer / MMA warpgroup gives registers to the elementwise groups
+      // (4*128*104 + 128*64 = 640*96, the block's launch allotment)
+      regs_dec<64>();
+      if (warp == PROD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmdO);
@@ -205,17 +218,18 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (!ok) {
                 for (uint32_t n = (nst > Cfg::NST ? nst - Cfg::NST : 0); n < nst; ++n)
                     mbar_wait_drain(bar_st_full + 8 * (n % Cfg::NST), (n / Cfg::NST) & 1);
-                // the K/V load of the item that was in progress (if it was issued)
                 if (kv_issued) mbar_wait_drain(bar_kv_full, (iter & 1));
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);   // K-major A and B
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A tmem, B MN-major
             const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
-            uint32_t nst = 0, iter = 0, p_phase = 0;
+            uint32_t nst = 0, iter = 0;
+            uint32_t p_phase[BWD_NWG];
+            for (int i = 0; i < BWD_NWG; ++i) p_phase[i] = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DkdvItem it = decode_dkdv(P, w);
@@ -249,34 +263,43 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                    IDESC_S, k > 0 ? 1u : 0u);
                         }
                         mma_commit(bar_s_full);
-                        ok = mbar_wait(bar_p_full, p_phase, abort_flag);
+                        // dV += P^T dO ; dK += dS^T Q, one 32-deep slice of query rows per warpgroup
+                        for (int wg = 0; wg < BWD_NWG && ok; ++wg) {
+                            ok = mbar_wait(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
+                            if (!ok) break;
+                            p_phase[wg] ^= 1;
+                            tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 2; ++kk) {
+                                const uint32_t acc = (!first || wg > 0 || kk > 0) ? 1u : 0u;
+                                const uint32_t brow = (2 * wg + kk) * 2048;
+                                mma_ts(tdV, tS + 32 * wg + 8 * kk, sdesc_sw128(sdO + brow, 16384, 1024),
+                                       IDESC_G, acc);
+                                mma_ts(tdK, tdP + 32 * wg + 8 * kk, sdesc_sw128(sQ + brow, 16384, 1024),
+                                       IDESC_G, acc);
+                            }
+                        }
                         if (!ok) break;
-                        p_phase ^= 1;
-                        tc_fence_after();
-                        // dV += P^T dO ; dK += dS^T Q   (K dimension = 128 query rows)
-                        for (int k = 0; k < 8; ++k)
-                            mma_ts(tdV, tS + k * 8, sdesc_sw128(sdO + k * 2048, 16384, 1024), IDESC_G,
-                                   (!first || k > 0) ? 1u : 0u);
-                        for (int k = 0; k < 8; ++k)
-                            mma_ts(tdK, tdP + k * 8, sdesc_sw128(sQ + k * 2048, 16384, 1024), IDESC_G,
-                                   (!first || k > 0) ? 1u : 0u);
                         mma_commit(bar_st_empty + 8 * slot);
                         first = false;
                     }
                 }
                 if (!ok) break;
                 mma_commit(bar_kv_empty);
-                if (!first) mma_commit(bar_acc_full);   // the softmax group waits only if it had a tile
+                if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
             }
             mma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0);
         }
+      }
     } else {
-        // ------------------------------------------------------------ softmax group (key rows)
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_off, tdP = tmem + lane_off + 128;
-        const uint32_t tdV = tmem + lane_off + 256, tdK = tmem + lane_off + 384;
+        regs_inc<104>();
+        // ------------------------------------------------------------ elementwise groups (key rows)
+        const int wg = warp >> 2;                        // query columns [32wg, 32wg+32)
+        const int row = (warp & 3) * 32 + lane;          // key row of the tile (TMEM lane)
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 32 * wg, tdP = tmem + lane_off + 128 + 32 * wg;
+        const uint32_t tdV = tmem + lane_off + 256 + 32 * wg, tdK = tmem + lane_off + 384 + 32 * wg;
         uint32_t nst = 0, s_phase = 0, a_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
@@ -298,64 +321,61 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     s_phase ^= 1;
                     tc_fence_after();
                     const uint8_t* st = smem + Cfg::ST_OFF + slot * Cfg::ST_STRIDE;
-                    const float* s_lse2 = reinterpret_cast<const float*>(st + 2 * Cfg::TILE);
-                    const float* s_delta = reinterpret_cast<const float*>(st + 2 * Cfg::TILE + 512);
-                    const int* s_ds = reinterpret_cast<const int*>(st + 2 * Cfg::TILE + 1024);
-#pragma unroll 1
-                    for (int c0 = 0; c0 < 128; c0 += 32) {
-                        float sv[32], dp[32];
-                        tmem_ld32f(tS + c0, sv);
-                        tmem_ld32f(tdP + c0, dp);
-                        tmem_wait_ld();
-                        reg_fence32f(sv);
-                        reg_fence32f(dp);
-                        uint32_t pk[16], dk[16];
+                    const float* s_lse2 = reinterpret_cast<const float*>(st + 2 * Cfg::TILE) + 32 * wg;
+                    const float* s_delta = reinterpret_cast<const float*>(st + 2 * Cfg::TILE + 512) + 32 * wg;
+                    const int* s_ds = reinterpret_cast<const int*>(st + 2 * Cfg::TILE + 1024) + 32 * wg;
+                    float sv[32], dp[32];
+                    tmem_ld32f(tS, sv);
+                    tmem_ld32f(tdP, dp);
+                    tmem_wait_ld();
+                    reg_fence32f(sv);
+                    reg_fence32f(dp);
+                    uint32_t pk[16], dk[16];
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            float p2[2], d2[2];
+                    for (int i = 0; i < 32; i += 2) {
+                        float p2[2], d2[2];
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int c = c0 + i + e;
-                                float pv = ex2_approx(fmaf(sv[i + e], P.scale_log2, -s_lse2[c]));
-                                if (cls == TILE_PARTIAL) {
-                                    const int q_orig = qo + c;
-                                    const int dsq = P.docs ? s_ds[c] : 0;
-                                    if (k_orig > q_orig || k_orig < dsq) pv = 0.f;
-                                }
-                                p2[e] = pv;
-                                d2[e] = pv * (dp[i + e] - s_delta[c]);
+                        for (int e = 0; e < 2; ++e) {
+                            const int c = i + e;                       // column within the block
+                            float pv = ex2_approx(fmaf(sv[c], P.scale_log2, -s_lse2[c]));
+                            if (cls == TILE_PARTIAL) {
+                                const int q_orig = qo + 32 * wg + c;
+                                const int dsq = P.docs ? s_ds[c] : 0;
+                                if (k_orig > q_orig || k_orig < dsq) pv = 0.f;
                             }
-                            pk[i / 2] = pack_bf16(p2[0], p2[1]);
-                            dk[i / 2] = pack_bf16(d2[0], d2[1]);
+                            p2[e] = pv;
+                            d2[e] = pv * (dp[c] - s_delta[c]);
                         }
-                        tmem_st16(tS + c0 / 2, pk);
-                        tmem_st16(tdP + c0 / 2, dk);
+                        pk[i / 2] = pack_bf16(p2[0], p2[1]);
+                        dk[i / 2] = pack_bf16(d2[0], d2[1]);
                     }
+                    // this block's 32 score columns are read: overwrite its first 16
+                    tmem_st16(tS, pk);
+                    tmem_st16(tdP, dk);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_p_full);
+                    if (lane == 0) mbar_arrive(bar_p_full + 8 * wg);
                     had = true;
                 }
             }
             if (!ok) break;
-            // ---- epilogue: dK (scaled) and dV of this key tile
+            // ---- epilogue: this group's 32 columns of dK (scaled) and dV
             const size_t orow = static_cast<size_t>(it.bkv) * P.S + it.kpos + row;
             if (had) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_acc_full, a_phase, abort_flag));
                 if (!ok) break;
                 a_phase ^= 1;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                if (32 * wg < D) {
                     float a[32], b[32];
-                    tmem_ld32f(tdV + c0, a);
-                    tmem_ld32f(tdK + c0, b);
+                    tmem_ld32f(tdV, a);
+                    tmem_ld32f(tdK, b);
                     tmem_wait_ld();
                     reg_fence32f(a);
                     reg_fence32f(b);
-                    uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + c0);
-                    uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + c0);
+                    uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
+                    uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + 32 * wg);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         dv[i] = make_uint4(pack_bf16(a[8 * i], a[8 * i + 1]), pack_bf16(a[8 * i + 2], a[8 * i + 3]),
@@ -366,17 +386,17 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                            pack_bf16(b[8 * i + 6] * P.scale, b[8 * i + 7] * P.scale));
                     }
                 }
-            } else {
-                uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D);
-                uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D);
-                for (int i = 0; i < D / 8; ++i) { dv[i] = make_uint4(0, 0, 0, 0); dk[i] = make_uint4(0, 0, 0, 0); }
+            } else if (32 * wg < D) {
+                uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
+                uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + 32 * wg);
+                for (int i = 0; i < 4; ++i) { dv[i] = make_uint4(0, 0, 0, 0); dk[i] = make_uint4(0, 0, 0, 0); }
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == MMA_WARP) {
         __syncwarp();
         tc_fence_after();
         tmem_relinquish();
@@ -393,34 +413,38 @@ struct DqCfg {
     static constexpr int NSLOT = (D == 128) ? 4 : 8;
     static constexpr int Q_OFF = 0, DO_OFF = TILE, KV_OFF = 2 * TILE;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE;
-    // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, p_full, acc_full, drain
-    static constexpr int NBAR = 6 + 2 * NSLOT;
+    // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, p_full[NWG], acc_full, drain
+    static constexpr int NBAR = 5 + 2 * NSLOT + BWD_NWG;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = BWD_THREADS;
 };
 
 struct DqItem {
     int bh, bkv, r, qpos, qo;
 };
 
+// Items run GQA group by group; inside a group, query tiles by descending
+// original position (the longest first) with the group's query heads fastest,
+// so the CTAs in flight stream the same K/V tiles of one KV head.
 __device__ __forceinline__ DqItem decode_dq(const BwdParams& P, int w)
 {
     DqItem it;
-    const int BH = P.B * P.Hq;
-    it.bh = w % BH;
-    const int t = w / BH;
+    const int g = P.Hq / P.Hkv;
     const int ntiles = P.S / 128;
+    const int per_group = g * ntiles;
+    it.bkv = w / per_group;
+    const int rem = w - it.bkv * per_group;
+    const int t = rem / g, hq = rem - t * g;
+    const int b = it.bkv / P.Hkv, hk = it.bkv - b * P.Hkv;
+    it.bh = b * P.Hq + hk * g + hq;
     it.qo = (ntiles - 1 - t) * 128;          // descending original position
     it.qpos = shard_of_orig(it.qo, P.C, P.cp);
     it.r = it.qpos / (2 * P.C);
-    const int g = P.Hq / P.Hkv;
-    const int b = it.bh / P.Hq, h = it.bh - b * P.Hq;
-    it.bkv = b * P.Hkv + h / g;
     return it;
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
 cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                  const BwdParams P)
@@ -434,14 +458,16 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bars = sbase + Cfg::BAR_OFF;
     const uint32_t bar_q_full = bars, bar_q_empty = bars + 8;
     const uint32_t bar_kv_full = bars + 16, bar_kv_empty = bars + 16 + 8 * Cfg::NSLOT;
-    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT, bar_p_full = bar_s_full + 8;
-    const uint32_t bar_acc_full = bar_s_full + 16, bar_drain = bar_s_full + 24;
+    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT;
+    const uint32_t bar_p_full = bar_s_full + 8;                       // [NWG]
+    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NWG, bar_drain = bar_acc_full + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n2c = 2 * P.C;
     const int ktiles = n2c / 128;
+    constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -452,18 +478,22 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_kv_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_full, 4);
+        for (int i = 0; i < BWD_NWG; ++i) mbar_init(bar_p_full + 8 * i, 4);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_slot), 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp >= 4 * BWD_NWG) {
+      // producer / MMA warpgroup gives registers to the elementwise groups
+      // (4*128*104 + 128*64 = 640*96, the block's launch allotment)
+      regs_dec<64>();
+      if (warp == PROD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmdO);
@@ -504,13 +534,15 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     mbar_wait_drain(bar_kv_full + 8 * (n % Cfg::NSLOT), (n / Cfg::NSLOT) & 1);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);
             const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-            uint32_t nload = 0, iter = 0, p_phase = 0;
+            uint32_t nload = 0, iter = 0;
+            uint32_t p_phase[BWD_NWG];
+            for (int i = 0; i < BWD_NWG; ++i) p_phase[i] = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DqItem it = decode_dq(P, w);
@@ -548,30 +580,39 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         }
                         mma_commit(bar_s_full);
                         mma_commit(bar_kv_empty + 8 * vslot);
-                        ok = mbar_wait(bar_p_full, p_phase, abort_flag);
+                        // dQ += dS K, one 32-deep slice of keys per warpgroup
+                        for (int wg = 0; wg < BWD_NWG && ok; ++wg) {
+                            ok = mbar_wait(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
+                            if (!ok) break;
+                            p_phase[wg] ^= 1;
+                            tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 2; ++kk)
+                                mma_ts(tdQ, tS + 32 * wg + 8 * kk,
+                                       sdesc_sw128(sk + (2 * wg + kk) * 2048, 16384, 1024), IDESC_G,
+                                       (!first || wg > 0 || kk > 0) ? 1u : 0u);
+                        }
                         if (!ok) break;
-                        p_phase ^= 1;
-                        tc_fence_after();
-                        // dQ += dS K   (K dimension = 128 keys)
-                        for (int k = 0; k < 8; ++k)
-                            mma_ts(tdQ, tS + k * 8, sdesc_sw128(sk + k * 2048, 16384, 1024), IDESC_G,
-                                   (!first || k > 0) ? 1u : 0u);
                         mma_commit(bar_kv_empty + 8 * kslot);
                         first = false;
                     }
                 }
                 if (!ok) break;
                 mma_commit(bar_q_empty);
-                if (!first) mma_commit(bar_acc_full);   // the softmax group waits only if it had a tile
+                if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
             }
             mma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0);
         }
+      }
     } else {
-        // ------------------------------------------------------------ softmax group (query rows)
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_off, tdP = tmem + lane_off + 128, tdQ = tmem + lane_off + 256;
+        regs_inc<104>();
+        // ------------------------------------------------------------ elementwise groups (query rows)
+        const int wg = warp >> 2;                        // key columns [32wg, 32wg+32)
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 32 * wg, tdP = tmem + lane_off + 128 + 32 * wg;
+        const uint32_t tdQ = tmem + lane_off + 256 + 32 * wg;
         uint32_t s_phase = 0, a_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
@@ -595,34 +636,31 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     if (!ok) break;
                     s_phase ^= 1;
                     tc_fence_after();
-                    const int lo = ds_row - ko, hi = q_orig - ko;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < 128; c0 += 32) {
-                        float sv[32], dp[32];
-                        tmem_ld32f(tS + c0, sv);
-                        tmem_ld32f(tdP + c0, dp);
-                        tmem_wait_ld();
-                        reg_fence32f(sv);
-                        reg_fence32f(dp);
-                        uint32_t dk[16];
+                    const int lo = ds_row - ko - 32 * wg, hi = q_orig - ko - 32 * wg;
+                    float sv[32], dp[32];
+                    tmem_ld32f(tS, sv);
+                    tmem_ld32f(tdP, dp);
+                    tmem_wait_ld();
+                    reg_fence32f(sv);
+                    reg_fence32f(dp);
+                    uint32_t dk[16];
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            float d2[2];
+                    for (int i = 0; i < 32; i += 2) {
+                        float d2[2];
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int c = c0 + i + e;
-                                float pv = ex2_approx(fmaf(sv[i + e], P.scale_log2, -lse2));
-                                if (cls == TILE_PARTIAL && (c < lo || c > hi)) pv = 0.f;
-                                d2[e] = pv * (dp[i + e] - dlt);
-                            }
-                            dk[i / 2] = pack_bf16(d2[0], d2[1]);
+                        for (int e = 0; e < 2; ++e) {
+                            const int c = i + e;
+                            float pv = ex2_approx(fmaf(sv[c], P.scale_log2, -lse2));
+                            if (cls == TILE_PARTIAL && (c < lo || c > hi)) pv = 0.f;
+                            d2[e] = pv * (dp[c] - dlt);
                         }
-                        tmem_st16(tS + c0 / 2, dk);
+                        dk[i / 2] = pack_bf16(d2[0], d2[1]);
                     }
+                    tmem_st16(tS, dk);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_p_full);
+                    if (lane == 0) mbar_arrive(bar_p_full + 8 * wg);
                     had = true;
                 }
             }
@@ -632,13 +670,12 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 if (!ok) break;
                 a_phase ^= 1;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                if (32 * wg < D) {
                     float a[32];
-                    tmem_ld32f(tdQ + c0, a);
+                    tmem_ld32f(tdQ, a);
                     tmem_wait_ld();
                     reg_fence32f(a);
-                    uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + c0);
+                    uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 32 * wg);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         dq[i] = make_uint4(pack_bf16(a[8 * i] * P.scale, a[8 * i + 1] * P.scale),
@@ -646,16 +683,16 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                            pack_bf16(a[8 * i + 4] * P.scale, a[8 * i + 5] * P.scale),
                                            pack_bf16(a[8 * i + 6] * P.scale, a[8 * i + 7] * P.scale));
                 }
-            } else {
-                uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D);
-                for (int i = 0; i < D / 8; ++i) dq[i] = make_uint4(0, 0, 0, 0);
+            } else if (32 * wg < D) {
+                uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 32 * wg);
+                for (int i = 0; i < 4; ++i) dq[i] = make_uint4(0, 0, 0, 0);
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == MMA_WARP) {
         __syncwarp();
         tc_fence_after();
         tmem_relinquish();

@@ -268,6 +268,19 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const FwdItem it = decode_item(P, w);
                 const TileIter ti = load_tile_iter(P, it);
+                // number of loaded tiles of this item: Q is released to the producer
+                // right after the last S = Q K^T, before the item's final PVs
+                int n_tiles = 0;
+                for (int s = 0; s < P.cp; ++s) {
+                    const int j = __ldg(P.src + it.r * P.cp + s);
+                    for (int kt = 0; kt < ktiles; ++kt) {
+                        const int ko = orig_of_shard(j * n2c + kt * 128, P.C, P.cp);
+                        if (classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP ||
+                            (it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP))
+                            ++n_tiles;
+                    }
+                }
+                int tiles_done = 0;
                 ok = mbar_wait(bar_q_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -333,6 +346,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         }
                         if (!ok) break;
                         mma_commit(bar_kv_empty + 8 * kslot);
+                        if (++tiles_done == n_tiles) mma_commit(bar_q_empty);
                     }
                     // end of a segment: every step (separate) or the whole visit (fused)
                     if (ok && (!P.fused || s == P.cp - 1)) {
@@ -346,7 +360,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         }
                     }
                 }
-                if (ok) mma_commit(bar_q_empty);
+                if (ok && n_tiles == 0) mma_commit(bar_q_empty);
             }
             // drain: every MMA and commit issued above has completed
             mma_commit(bar_drain);

@@ -66,8 +66,9 @@ def test_gqa_docs_small(D):
 
 
 def test_batch2_cp3_scale():
-    case = make_case(2, 4, 2, 2304, 128, 3, 23, amp=1.5, with_dout=True)
-    check_full(case, 3, "ring", scale=0.07)
+    """Batch 2, cp 3 (three query tiles per chunk), GQA 4/2, a non-default scale."""
+    case = make_case(2, 4, 2, 2304, 128, 3, 23, with_dout=True)
+    check_full(case, 3, "ring", scale=0.07, emulate=True)
 
 
 # ----------------------------------------------------------------- full sizes, sampled
