@@ -145,6 +145,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int g = P.Hq / P.Hkv;
     const int n2c = 2 * P.C;
     const int nqt = n2c / 128;
+    const int half = P.C / 128;
     const uint32_t st_bytes = 2 * Cfg::TILE + 1024 + (P.docs ? 512 : 0);
     constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
@@ -190,9 +191,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
                 for (int hq = 0; hq < g && ok; ++hq) {
                     const int bh = it.b * P.Hq + it.hk * g + hq;
-                    for (int qt = 0; qt < P.cp * nqt && ok; ++qt) {
+                    for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
+                         ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
                         const int qpos = qt * 128;
-                        const int qo = orig_of_shard(qpos, P.C, P.cp);
+                        const int qo = key_tile_orig(qr, qlt, half, P.C, P.cp);
                         const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
                         const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
                         if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
@@ -226,7 +228,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);   // K-major A and B
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A tmem, B MN-major
+            constexpr uint32_t TILE16 = Cfg::TILE >> 4, ST16 = Cfg::ST_STRIDE >> 4;
             const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+            // descriptor bases; k-steps and stages are constant offsets in 16-byte units
+            const uint64_t dK = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
+            const uint64_t dST = sdesc_sw128(sST, 16, 1024), dSTmn = sdesc_sw128(sST, 16384, 1024);
             uint32_t nst = 0, iter = 0;
             uint32_t p_phase[BWD_NWG];
             for (int i = 0; i < BWD_NWG; ++i) p_phase[i] = 0;
@@ -238,9 +244,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_after();
                 bool first = true;
                 for (int hq = 0; hq < g && ok; ++hq) {
-                    for (int qt = 0; qt < P.cp * nqt && ok; ++qt) {
+                    for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
+                         ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
                         const int qpos = qt * 128;
-                        const int qo = orig_of_shard(qpos, P.C, P.cp);
+                        const int qo = key_tile_orig(qr, qlt, half, P.C, P.cp);
                         const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
                         const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
                         if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
@@ -249,18 +256,17 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         ok = mbar_wait(bar_st_full + 8 * slot, par, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t sQ = sST + slot * Cfg::ST_STRIDE, sdO = sQ + Cfg::TILE;
+                        const uint64_t bq = dST + slot * ST16, bdo = bq + TILE16;
+                        const uint64_t bq_mn = dSTmn + slot * ST16, bdo_mn = bq_mn + TILE16;
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-                            mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
-                                   IDESC_S, k > 0 ? 1u : 0u);
+                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                            mma_ss(tS, dK + off, bq + off, IDESC_S, k > 0 ? 1u : 0u);
                         }
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-                            mma_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024),
-                                   IDESC_S, k > 0 ? 1u : 0u);
+                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                            mma_ss(tdP, dVk + off, bdo + off, IDESC_S, k > 0 ? 1u : 0u);
                         }
                         mma_commit(bar_s_full);
                         // dV += P^T dO ; dK += dS^T Q, one 32-deep slice of query rows per warpgroup
@@ -272,11 +278,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
                             for (int kk = 0; kk < 2; ++kk) {
                                 const uint32_t acc = (!first || wg > 0 || kk > 0) ? 1u : 0u;
-                                const uint32_t brow = (2 * wg + kk) * 2048;
-                                mma_ts(tdV, tS + 32 * wg + 8 * kk, sdesc_sw128(sdO + brow, 16384, 1024),
-                                       IDESC_G, acc);
-                                mma_ts(tdK, tdP + 32 * wg + 8 * kk, sdesc_sw128(sQ + brow, 16384, 1024),
-                                       IDESC_G, acc);
+                                const uint32_t brow = ((2 * wg + kk) * 2048) >> 4;
+                                mma_ts(tdV, tS + 32 * wg + 8 * kk, bdo_mn + brow, IDESC_G, acc);
+                                mma_ts(tdK, tdP + 32 * wg + 8 * kk, bq_mn + brow, IDESC_G, acc);
                             }
                         }
                         if (!ok) break;
@@ -307,9 +311,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int k_orig = it.ko + row;
             bool had = false;
             for (int hq = 0; hq < g && ok; ++hq) {
-                for (int qt = 0; qt < P.cp * nqt && ok; ++qt) {
+                for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
+                     ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
                     const int qpos = qt * 128;
-                    const int qo = orig_of_shard(qpos, P.C, P.cp);
+                    const int qo = key_tile_orig(qr, qlt, half, P.C, P.cp);
                     const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
                     const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
                     const int cls = classify_tile(qo, dsf, dsl, it.ko);
@@ -467,6 +472,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n2c = 2 * P.C;
     const int ktiles = n2c / 128;
+    const int half = P.C / 128;
     constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
     if (threadIdx.x == 0) {
@@ -514,7 +520,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
                         const int kpos = j * n2c + kt * 128;
-                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
                         for (int kv = 0; kv < 2 && ok; ++kv, ++nload) {
                             const uint32_t slot = nload % Cfg::NSLOT, par = (nload / Cfg::NSLOT) & 1;
@@ -539,7 +545,10 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);
+            constexpr uint32_t TILE16 = Cfg::TILE >> 4;
             const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+            const uint64_t dQd = sdesc_sw128(sQ, 16, 1024), ddO = sdesc_sw128(sdO, 16, 1024);
+            const uint64_t dKV = sdesc_sw128(sKV, 16, 1024), dKVmn = sdesc_sw128(sKV, 16384, 1024);
             uint32_t nload = 0, iter = 0;
             uint32_t p_phase[BWD_NWG];
             for (int i = 0; i < BWD_NWG; ++i) p_phase[i] = 0;
@@ -556,7 +565,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
                         const int kpos = j * n2c + kt * 128;
-                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
                         const uint32_t vslot = (nload + 1) % Cfg::NSLOT, vpar = ((nload + 1) / Cfg::NSLOT) & 1;
@@ -565,18 +574,17 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                              mbar_wait(bar_kv_full + 8 * vslot, vpar, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t sk = sKV + kslot * Cfg::TILE, sv = sKV + vslot * Cfg::TILE;
+                        const uint64_t bk = dKV + kslot * TILE16, bv = dKV + vslot * TILE16;
+                        const uint64_t bk_mn = dKVmn + kslot * TILE16;
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-                            mma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024),
-                                   IDESC_S, k > 0 ? 1u : 0u);
+                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                            mma_ss(tS, dQd + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
                         }
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-                            mma_ss(tdP, sdesc_sw128(sdO + off, 16, 1024), sdesc_sw128(sv + off, 16, 1024),
-                                   IDESC_S, k > 0 ? 1u : 0u);
+                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                            mma_ss(tdP, ddO + off, bv + off, IDESC_S, k > 0 ? 1u : 0u);
                         }
                         mma_commit(bar_s_full);
                         mma_commit(bar_kv_empty + 8 * vslot);
@@ -588,9 +596,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             tc_fence_after();
 #pragma unroll
                             for (int kk = 0; kk < 2; ++kk)
-                                mma_ts(tdQ, tS + 32 * wg + 8 * kk,
-                                       sdesc_sw128(sk + (2 * wg + kk) * 2048, 16384, 1024), IDESC_G,
-                                       (!first || wg > 0 || kk > 0) ? 1u : 0u);
+                                mma_ts(tdQ, tS + 32 * wg + 8 * kk, bk_mn + (((2 * wg + kk) * 2048) >> 4),
+                                       IDESC_G, (!first || wg > 0 || kk > 0) ? 1u : 0u);
                         }
                         if (!ok) break;
                         mma_commit(bar_kv_empty + 8 * kslot);
@@ -628,8 +635,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
                 for (int kt = 0; kt < ktiles && ok; ++kt) {
-                    const int kpos = j * n2c + kt * 128;
-                    const int ko = orig_of_shard(kpos, P.C, P.cp);
+                    const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                     const int cls = classify_tile(it.qo, dsf, dsl, ko);
                     if (cls == TILE_SKIP) continue;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));

@@ -14,8 +14,8 @@
 //   warp 9     MMA issuer (one thread) + tensor-memory owner
 //   warps 10-11 idle
 // The block launches with 168 registers per thread; the softmax warpgroups
-// raise theirs to 208 and the producer/MMA warpgroup drops to 88
-// (2*128*208 + 128*88 = 384*168).
+// raise theirs to 200 and the producer/MMA warpgroup drops to 104
+// (2*128*200 + 128*104 = 384*168).
 // Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D),
 // O1 [384,384+D).  P is written back as bf16 over the first 64 columns of its
 // S region and used as the A operand of O += P V straight from tensor memory.
@@ -68,6 +68,14 @@ __device__ __forceinline__ int classify_tile(int qo, int dsf, int dsl, int ko)
 struct FwdItem {
     int bh, bkv, r, p0, qo0, ntq;
 };
+
+// Original start of key tile kt (0 <= kt < 2C/128) of shard j: the first C/128
+// tiles are chunk j, the rest chunk 2cp-1-j.  No division: every role calls
+// this once per key tile.
+__device__ __forceinline__ int key_tile_orig(int j, int kt, int half, int C, int cp)
+{
+    return kt < half ? j * C + kt * 128 : (2 * cp - 1 - j) * C + (kt - half) * 128;
+}
 
 __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
 {
@@ -184,6 +192,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n2c = 2 * P.C;
     const int ktiles = n2c / 128;
+    const int half = P.C / 128;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -207,7 +216,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (warp >= 8) {
-      regs_dec<88>();
+      regs_dec<104>();
       if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -230,7 +239,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
                         const int kpos = j * n2c + kt * 128;
-                        const int ko = orig_of_shard(kpos, P.C, P.cp);
+                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
                         const bool v1 = it.ntq == 2 &&
                                         classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP;
@@ -260,10 +269,14 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
-            const uint32_t tS[2] = {tmem + 0, tmem + 128};
-            const uint32_t tO[2] = {tmem + 256, tmem + 384};
-            uint32_t nload = 0, iter = 0;
-            uint32_t p_phase[2] = {0, 0};
+            constexpr uint32_t TILE16 = Cfg::TILE_BYTES >> 4;   // tile stride in descriptor units
+            // descriptors of Q tile 0 and KV slot 0; the others are constant offsets
+            const uint64_t dq0 = sdesc_sw128(sQ0, 16, 1024);
+            const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(sKV, 16384, 1024);
+            const uint32_t tS0 = tmem, tO0 = tmem + 256;
+            uint32_t ring_slot = 0, ring_par = 0, iter = 0;
+            uint32_t p_phase0 = 0, p_phase1 = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const FwdItem it = decode_item(P, w);
@@ -274,7 +287,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int s = 0; s < P.cp; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles; ++kt) {
-                        const int ko = orig_of_shard(j * n2c + kt * 128, P.C, P.cp);
+                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP ||
                             (it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP))
                             ++n_tiles;
@@ -284,80 +297,76 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 ok = mbar_wait(bar_q_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                // pending PV per query tile: V slot/parity, users left on that slot
-                bool pend[2] = {false, false};
-                bool first[2] = {true, true};
-                bool seg_had[2] = {false, false};   // query tile x had a tile in this segment
-                uint32_t pend_slot[2] = {0, 0}, pend_par[2] = {0, 0};
-                int slot_users[Cfg::NSLOT];
-                for (int i = 0; i < Cfg::NSLOT; ++i) slot_users[i] = 0;
+                bool pend0 = false, pend1 = false;       // a PV of the previous tile is due
+                bool first0 = true, first1 = true;       // next PV starts the accumulator
+                bool had0 = false, had1 = false;         // query tile had a tile in this segment
+                bool pv_live = false;                    // the previous tile's V slot is held
+                uint32_t pv_slot = 0, pv_par = 0;
 
-                auto issue_pv = [&](int x) -> bool {
-                    if (!mbar_wait(bar_p_full + 8 * x, p_phase[x], abort_flag)) return false;
-                    p_phase[x] ^= 1;
-                    if (!mbar_wait(bar_kv_full + 8 * pend_slot[x], pend_par[x], abort_flag)) return false;
+                // O_x += P_x V(previous tile), once softmax group x has written P_x
+                auto issue_pv = [&](int x, uint32_t& pph, bool& first) -> bool {
+                    if (!mbar_wait(bar_p_full + 8 * x, pph, abort_flag)) return false;
+                    pph ^= 1;
+                    if (!mbar_wait(bar_kv_full + 8 * pv_slot, pv_par, abort_flag)) return false;
                     tc_fence_after();
-                    const uint32_t sv = sKV + pend_slot[x] * Cfg::TILE_BYTES;
+                    const uint64_t bv = dv0 + pv_slot * TILE16;
+                    const uint32_t ts = tS0 + 128 * x, to = tO0 + 128 * x;
+#pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tO[x], tS[x] + k * 8, sdesc_sw128(sv + k * 2048, 16384, 1024),
-                               IDESC_PV, (!first[x] || k > 0) ? 1u : 0u);
-                    first[x] = false;
-                    pend[x] = false;
-                    if (--slot_users[pend_slot[x]] == 0) mma_commit(bar_kv_empty + 8 * pend_slot[x]);
+                        mma_ts(to, ts + 8 * k, bv + k * (2048 >> 4), IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                    first = false;
                     return true;
+                };
+                auto issue_s = [&](int x, uint32_t kslot) {
+                    const uint64_t aq = dq0 + x * TILE16, bk = dk0 + kslot * TILE16;
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                        mma_ss(tS0 + 128 * x, aq + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_s_full + 8 * x);
                 };
 
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
-                        const int kpos = j * n2c + kt * 128;
-                        const int ko = orig_of_shard(kpos, P.C, P.cp);
-                        const bool v[2] = {
-                            classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP,
-                            it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP};
-                        if (!v[0] && !v[1]) continue;
-                        const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
-                        const uint32_t vslot = (nload + 1) % Cfg::NSLOT,
-                                       vpar = ((nload + 1) / Cfg::NSLOT) & 1;
-                        nload += 2;
+                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                        const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
+                        const bool v1 = it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP;
+                        if (!v0 && !v1) continue;
+                        const uint32_t kslot = ring_slot, kpar = ring_par;
+                        if (++ring_slot == Cfg::NSLOT) { ring_slot = 0; ring_par ^= 1; }
+                        const uint32_t vslot = ring_slot, vpar = ring_par;
+                        if (++ring_slot == Cfg::NSLOT) { ring_slot = 0; ring_par ^= 1; }
                         ok = mbar_wait(bar_kv_full + 8 * kslot, kpar, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t sk = sKV + kslot * Cfg::TILE_BYTES;
-                        slot_users[vslot] = (v[0] ? 1 : 0) + (v[1] ? 1 : 0);
-                        for (int x = 0; x < 2 && ok; ++x) {
-                            // A pending PV never outlives one tile: it is issued at the next
-                            // loaded tile whether or not that tile is valid for x, so a V slot
-                            // is held for at most one tile and the ring cannot stall.
-                            if (pend[x]) { ok = issue_pv(x); if (!ok) break; }
-                            if (!v[x]) continue;
-                            const uint32_t sq = sQ0 + x * Cfg::TILE_BYTES;
-#pragma unroll
-                            for (int k = 0; k < D / 16; ++k) {
-                                const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-                                mma_ss(tS[x], sdesc_sw128(sq + off, 16, 1024),
-                                       sdesc_sw128(sk + off, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
-                            }
-                            mma_commit(bar_s_full + 8 * x);
-                            pend[x] = true;
-                            seg_had[x] = true;
-                            pend_slot[x] = vslot;
-                            pend_par[x] = vpar;
-                        }
+                        // A pending PV never outlives one tile: it is issued at the next loaded
+                        // tile whether or not that tile is valid for its query tile, so a V slot
+                        // is held for at most one tile and the ring cannot stall.
+                        if (pend0) { ok = issue_pv(0, p_phase0, first0); pend0 = false; }
+                        if (ok && v0) { issue_s(0, kslot); pend0 = true; had0 = true; }
+                        if (ok && pend1) { ok = issue_pv(1, p_phase1, first1); pend1 = false; }
+                        if (ok && v1) { issue_s(1, kslot); pend1 = true; had1 = true; }
                         if (!ok) break;
+                        if (pv_live) mma_commit(bar_kv_empty + 8 * pv_slot);   // every PV on it issued
                         mma_commit(bar_kv_empty + 8 * kslot);
+                        pv_live = true;
+                        pv_slot = vslot;
+                        pv_par = vpar;
                         if (++tiles_done == n_tiles) mma_commit(bar_q_empty);
                     }
                     // end of a segment: every step (separate) or the whole visit (fused)
                     if (ok && (!P.fused || s == P.cp - 1)) {
-                        for (int x = 0; x < 2 && ok; ++x) {
-                            if (pend[x]) ok = issue_pv(x);
-                            // the softmax group of x waits for this whenever it had a tile in
-                            // the segment, even if its last PV was flushed at an earlier tile
-                            if (ok && seg_had[x]) mma_commit(bar_o_full + 8 * x);
-                            first[x] = true;
-                            seg_had[x] = false;
-                        }
+                        if (pend0) { ok = issue_pv(0, p_phase0, first0); pend0 = false; }
+                        if (ok && pend1) { ok = issue_pv(1, p_phase1, first1); pend1 = false; }
+                        if (ok && pv_live) { mma_commit(bar_kv_empty + 8 * pv_slot); pv_live = false; }
+                        // each softmax group waits for this whenever it had a tile in the
+                        // segment, even if its last PV was issued at an earlier tile
+                        if (ok && had0) mma_commit(bar_o_full);
+                        if (ok && had1) mma_commit(bar_o_full + 8);
+                        first0 = first1 = true;
+                        had0 = had1 = false;
                     }
                 }
                 if (ok && n_tiles == 0) mma_commit(bar_q_empty);
@@ -368,7 +377,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     } else {
-        regs_inc<208>();
+        regs_inc<200>();
         // ------------------------------------------------------------ softmax groups
         const int X = warp >> 2;                 // query tile handled by this group
         const int row = (warp & 3) * 32 + lane;  // TMEM lane == query row in the tile
@@ -389,8 +398,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
                 for (int kt = 0; kt < ktiles && ok; ++kt) {
-                    const int kpos = j * n2c + kt * 128;
-                    const int ko = orig_of_shard(kpos, P.C, P.cp);
+                    const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                     const int cls = classify_tile(ti.qo[X], ti.dsf[X], ti.dsl[X], ko);
                     if (cls == TILE_SKIP) continue;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * X, s_phase, abort_flag));
@@ -444,8 +452,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         }
                     }
                     const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-                    const float rs = (cls == TILE_FULL) ? exp_pack_store<true>(sf, P.scale_log2, msub, tS)
-                                                        : exp_pack_store<false>(sf, P.scale_log2, msub, tS);
+                    const float rs = exp_pack_store<false>(sf, P.scale_log2, msub, tS);
                     l_sum = l_sum * alpha + rs;
                     tmem_wait_st();
                     tc_fence_before();
