@@ -225,7 +225,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the control flow; one elected lane issues each group
+        // of tensor-core instructions (cheaper than a single diverged lane).
+        {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);   // K-major A and B
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A tmem, B MN-major
             constexpr uint32_t TILE16 = Cfg::TILE >> 4, ST16 = Cfg::ST_STRIDE >> 4;
@@ -239,7 +241,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DkdvItem it = decode_dkdv(P, w);
-                ok = mbar_wait(bar_kv_full, iter & 1, abort_flag);
+                ok = mbar_wait_warp(bar_kv_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 bool first = true;
@@ -253,46 +255,57 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
                         const uint32_t slot = nst % Cfg::NST, par = (nst / Cfg::NST) & 1;
                         ++nst;
-                        ok = mbar_wait(bar_st_full + 8 * slot, par, abort_flag);
+                        ok = mbar_wait_warp(bar_st_full + 8 * slot, par, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         const uint64_t bq = dST + slot * ST16, bdo = bq + TILE16;
                         const uint64_t bq_mn = dSTmn + slot * ST16, bdo_mn = bq_mn + TILE16;
+                        if (elect_one()) {
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                            mma_ss(tS, dK + off, bq + off, IDESC_S, k > 0 ? 1u : 0u);
-                        }
+                            for (int k = 0; k < D / 16; ++k) {
+                                const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                                mma_ss(tS, dK + off, bq + off, IDESC_S, k > 0 ? 1u : 0u);
+                            }
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                            mma_ss(tdP, dVk + off, bdo + off, IDESC_S, k > 0 ? 1u : 0u);
+                            for (int k = 0; k < D / 16; ++k) {
+                                const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                                mma_ss(tdP, dVk + off, bdo + off, IDESC_S, k > 0 ? 1u : 0u);
+                            }
+                            mma_commit(bar_s_full);
                         }
-                        mma_commit(bar_s_full);
+                        __syncwarp();
                         // dV += P^T dO ; dK += dS^T Q, one 32-deep slice of query rows per warpgroup
                         for (int wg = 0; wg < BWD_NWG && ok; ++wg) {
-                            ok = mbar_wait(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
+                            ok = mbar_wait_warp(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
                             if (!ok) break;
                             p_phase[wg] ^= 1;
                             tc_fence_after();
+                            if (elect_one()) {
 #pragma unroll
-                            for (int kk = 0; kk < 2; ++kk) {
-                                const uint32_t acc = (!first || wg > 0 || kk > 0) ? 1u : 0u;
-                                const uint32_t brow = ((2 * wg + kk) * 2048) >> 4;
-                                mma_ts(tdV, tS + 32 * wg + 8 * kk, bdo_mn + brow, IDESC_G, acc);
-                                mma_ts(tdK, tdP + 32 * wg + 8 * kk, bq_mn + brow, IDESC_G, acc);
+                                for (int kk = 0; kk < 2; ++kk) {
+                                    const uint32_t acc = (!first || wg > 0 || kk > 0) ? 1u : 0u;
+                                    const uint32_t brow = ((2 * wg + kk) * 2048) >> 4;
+                                    mma_ts(tdV, tS + 32 * wg + 8 * kk, bdo_mn + brow, IDESC_G, acc);
+                                    mma_ts(tdK, tdP + 32 * wg + 8 * kk, bq_mn + brow, IDESC_G, acc);
+                                }
                             }
+                            __syncwarp();
                         }
                         if (!ok) break;
-                        mma_commit(bar_st_empty + 8 * slot);
+                        if (elect_one()) mma_commit(bar_st_empty + 8 * slot);
+                        __syncwarp();
                         first = false;
                     }
                 }
                 if (!ok) break;
-                mma_commit(bar_kv_empty);
-                if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
+                if (elect_one()) {
+                    mma_commit(bar_kv_empty);
+                    if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
+                }
+                __syncwarp();
             }
-            mma_commit(bar_drain);
+            if (elect_one()) mma_commit(bar_drain);
+            __syncwarp();
             mbar_wait_drain(bar_drain, 0);
         }
       }
@@ -542,7 +555,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the control flow; one elected lane issues each group
+        // of tensor-core instructions (cheaper than a single diverged lane).
+        {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);
             constexpr uint32_t TILE16 = Cfg::TILE >> 4;
@@ -557,7 +572,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const DqItem it = decode_dq(P, w);
                 const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
                 const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
-                ok = mbar_wait(bar_q_full, iter & 1, abort_flag);
+                ok = mbar_wait_warp(bar_q_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 bool first = true;
@@ -570,45 +585,56 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
                         const uint32_t vslot = (nload + 1) % Cfg::NSLOT, vpar = ((nload + 1) / Cfg::NSLOT) & 1;
                         nload += 2;
-                        ok = mbar_wait(bar_kv_full + 8 * kslot, kpar, abort_flag) &&
-                             mbar_wait(bar_kv_full + 8 * vslot, vpar, abort_flag);
+                        ok = mbar_wait_warp(bar_kv_full + 8 * kslot, kpar, abort_flag) &&
+                             mbar_wait_warp(bar_kv_full + 8 * vslot, vpar, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         const uint64_t bk = dKV + kslot * TILE16, bv = dKV + vslot * TILE16;
                         const uint64_t bk_mn = dKVmn + kslot * TILE16;
+                        if (elect_one()) {
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                            mma_ss(tS, dQd + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
-                        }
+                            for (int k = 0; k < D / 16; ++k) {
+                                const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                                mma_ss(tS, dQd + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
+                            }
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                            mma_ss(tdP, ddO + off, bv + off, IDESC_S, k > 0 ? 1u : 0u);
+                            for (int k = 0; k < D / 16; ++k) {
+                                const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                                mma_ss(tdP, ddO + off, bv + off, IDESC_S, k > 0 ? 1u : 0u);
+                            }
+                            mma_commit(bar_s_full);
+                            mma_commit(bar_kv_empty + 8 * vslot);
                         }
-                        mma_commit(bar_s_full);
-                        mma_commit(bar_kv_empty + 8 * vslot);
+                        __syncwarp();
                         // dQ += dS K, one 32-deep slice of keys per warpgroup
                         for (int wg = 0; wg < BWD_NWG && ok; ++wg) {
-                            ok = mbar_wait(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
+                            ok = mbar_wait_warp(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
                             if (!ok) break;
                             p_phase[wg] ^= 1;
                             tc_fence_after();
+                            if (elect_one()) {
 #pragma unroll
-                            for (int kk = 0; kk < 2; ++kk)
-                                mma_ts(tdQ, tS + 32 * wg + 8 * kk, bk_mn + (((2 * wg + kk) * 2048) >> 4),
-                                       IDESC_G, (!first || wg > 0 || kk > 0) ? 1u : 0u);
+                                for (int kk = 0; kk < 2; ++kk)
+                                    mma_ts(tdQ, tS + 32 * wg + 8 * kk, bk_mn + (((2 * wg + kk) * 2048) >> 4),
+                                           IDESC_G, (!first || wg > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            __syncwarp();
                         }
                         if (!ok) break;
-                        mma_commit(bar_kv_empty + 8 * kslot);
+                        if (elect_one()) mma_commit(bar_kv_empty + 8 * kslot);
+                        __syncwarp();
                         first = false;
                     }
                 }
                 if (!ok) break;
-                mma_commit(bar_q_empty);
-                if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
+                if (elect_one()) {
+                    mma_commit(bar_q_empty);
+                    if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
+                }
+                __syncwarp();
             }
-            mma_commit(bar_drain);
+            if (elect_one()) mma_commit(bar_drain);
+            __syncwarp();
             mbar_wait_drain(bar_drain, 0);
         }
       }

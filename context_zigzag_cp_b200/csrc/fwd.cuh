@@ -266,7 +266,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the control flow; one elected lane issues each group
+        // of tensor-core instructions (cheaper than a single diverged lane).
+        {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
             constexpr uint32_t TILE16 = Cfg::TILE_BYTES >> 4;   // tile stride in descriptor units
@@ -294,7 +296,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                 }
                 int tiles_done = 0;
-                ok = mbar_wait(bar_q_full, iter & 1, abort_flag);
+                ok = mbar_wait_warp(bar_q_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 bool pend0 = false, pend1 = false;       // a PV of the previous tile is due
@@ -305,26 +307,32 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
                 // O_x += P_x V(previous tile), once softmax group x has written P_x
                 auto issue_pv = [&](int x, uint32_t& pph, bool& first) -> bool {
-                    if (!mbar_wait(bar_p_full + 8 * x, pph, abort_flag)) return false;
+                    if (!mbar_wait_warp(bar_p_full + 8 * x, pph, abort_flag)) return false;
                     pph ^= 1;
-                    if (!mbar_wait(bar_kv_full + 8 * pv_slot, pv_par, abort_flag)) return false;
+                    if (!mbar_wait_warp(bar_kv_full + 8 * pv_slot, pv_par, abort_flag)) return false;
                     tc_fence_after();
                     const uint64_t bv = dv0 + pv_slot * TILE16;
                     const uint32_t ts = tS0 + 128 * x, to = tO0 + 128 * x;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ts(to, ts + 8 * k, bv + k * (2048 >> 4), IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(to, ts + 8 * k, bv + k * (2048 >> 4), IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                    }
+                    __syncwarp();
                     first = false;
                     return true;
                 };
                 auto issue_s = [&](int x, uint32_t kslot) {
                     const uint64_t aq = dq0 + x * TILE16, bk = dk0 + kslot * TILE16;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                        mma_ss(tS0 + 128 * x, aq + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
+                            mma_ss(tS0 + 128 * x, aq + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
+                        }
+                        mma_commit(bar_s_full + 8 * x);
                     }
-                    mma_commit(bar_s_full + 8 * x);
+                    __syncwarp();
                 };
 
                 for (int s = 0; s < P.cp && ok; ++s) {
@@ -338,7 +346,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (++ring_slot == Cfg::NSLOT) { ring_slot = 0; ring_par ^= 1; }
                         const uint32_t vslot = ring_slot, vpar = ring_par;
                         if (++ring_slot == Cfg::NSLOT) { ring_slot = 0; ring_par ^= 1; }
-                        ok = mbar_wait(bar_kv_full + 8 * kslot, kpar, abort_flag);
+                        ok = mbar_wait_warp(bar_kv_full + 8 * kslot, kpar, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         // A pending PV never outlives one tile: it is issued at the next loaded
@@ -349,30 +357,38 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (ok && pend1) { ok = issue_pv(1, p_phase1, first1); pend1 = false; }
                         if (ok && v1) { issue_s(1, kslot); pend1 = true; had1 = true; }
                         if (!ok) break;
-                        if (pv_live) mma_commit(bar_kv_empty + 8 * pv_slot);   // every PV on it issued
-                        mma_commit(bar_kv_empty + 8 * kslot);
+                        if (elect_one()) {
+                            if (pv_live) mma_commit(bar_kv_empty + 8 * pv_slot);   // every PV on it issued
+                            mma_commit(bar_kv_empty + 8 * kslot);
+                        }
+                        __syncwarp();
                         pv_live = true;
                         pv_slot = vslot;
                         pv_par = vpar;
-                        if (++tiles_done == n_tiles) mma_commit(bar_q_empty);
+                        if (++tiles_done == n_tiles) { if (elect_one()) mma_commit(bar_q_empty); __syncwarp(); }
                     }
                     // end of a segment: every step (separate) or the whole visit (fused)
                     if (ok && (!P.fused || s == P.cp - 1)) {
                         if (pend0) { ok = issue_pv(0, p_phase0, first0); pend0 = false; }
                         if (ok && pend1) { ok = issue_pv(1, p_phase1, first1); pend1 = false; }
-                        if (ok && pv_live) { mma_commit(bar_kv_empty + 8 * pv_slot); pv_live = false; }
-                        // each softmax group waits for this whenever it had a tile in the
-                        // segment, even if its last PV was issued at an earlier tile
-                        if (ok && had0) mma_commit(bar_o_full);
-                        if (ok && had1) mma_commit(bar_o_full + 8);
+                        if (ok && elect_one()) {
+                            if (pv_live) mma_commit(bar_kv_empty + 8 * pv_slot);
+                            // each softmax group waits for this whenever it had a tile in the
+                            // segment, even if its last PV was issued at an earlier tile
+                            if (had0) mma_commit(bar_o_full);
+                            if (had1) mma_commit(bar_o_full + 8);
+                        }
+                        __syncwarp();
+                        pv_live = false;
                         first0 = first1 = true;
                         had0 = had1 = false;
                     }
                 }
-                if (ok && n_tiles == 0) mma_commit(bar_q_empty);
+                if (ok && n_tiles == 0) { if (elect_one()) mma_commit(bar_q_empty); __syncwarp(); }
             }
             // drain: every MMA and commit issued above has completed
-            mma_commit(bar_drain);
+            if (elect_one()) mma_commit(bar_drain);
+            __syncwarp();
             mbar_wait_drain(bar_drain, 0);
         }
       }

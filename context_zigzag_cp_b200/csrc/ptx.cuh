@@ -106,6 +106,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     return mbar_wait_limit(bar, parity, abort, g_cp_wait_limit_ns);
 }
 
+// Warp-uniform bounded wait: every lane polls, and all lanes agree on the
+// outcome (a give-up on any lane is a give-up for the warp).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
 // Wait used while draining before exit: ignores the CTA's abort flag (so it
 // really waits for in-flight copies / MMAs) but is still bounded by the limit.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity)
