@@ -14,12 +14,13 @@
 //   * cp_bwd_dq_kernel (query-tile major, visiting the K/V shards in the plan's
 //     order like the forward):  S = Q K^T,  dP = dO V^T  ->  dS (bf16, tensor
 //     memory)  ->  dQ += dS K.
-// In both passes the elementwise step is split by columns over four
-// warpgroups (32 columns each; a thread owns one TMEM lane = one row).  Each
-// warpgroup writes its bf16 results over the first 16 columns of its own
-// 32-column block, and the MMA thread issues the product for that block (a
-// 32-deep slice of the K dimension) as soon as that warpgroup is done, so the
-// four slices overlap with the remaining elementwise work.
+// In both passes the elementwise step runs on four warpgroups (a thread owns
+// one TMEM lane = one row) over the 128 score columns in two 64-column slices:
+// in each slice warpgroup w takes 16 columns, reads them, and writes its bf16
+// results over the first 8 of them (only columns it has read itself, so no
+// warp overwrites another's input).  All four warpgroups finish slice 0 before
+// slice 1, and the MMA warp issues slice 0's products (a 64-deep part of the
+// K dimension) while slice 1 is computed.
 // Each 128-row tile lives in one zigzag chunk, so original positions are
 // linear inside a tile and the causal / document tests are per-tile ranges.
 #pragma once
@@ -84,6 +85,7 @@ struct BwdParams {
 // ============================================================================
 constexpr int BWD_NWG = 4;                       // elementwise warpgroups
 constexpr int BWD_THREADS = (BWD_NWG + 1) * 128; // + producer / MMA warpgroup
+constexpr int BWD_NSLICE = 2;                    // 64-column slices of a 128-column score tile
 
 template <int D>
 struct DkdvCfg {
@@ -93,8 +95,8 @@ struct DkdvCfg {
     static constexpr int K_OFF = 0, V_OFF = TILE;
     static constexpr int ST_OFF = 2 * TILE;
     static constexpr int BAR_OFF = ST_OFF + NST * ST_STRIDE;
-    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full[NWG], acc_full, drain
-    static constexpr int NBAR = 5 + 2 * NST + BWD_NWG;
+    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full[NSLICE], acc_full, drain, acc_empty
+    static constexpr int NBAR = 6 + 2 * NST + BWD_NSLICE;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
     static constexpr int THREADS = BWD_THREADS;
 };
@@ -136,8 +138,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t bar_kv_full = bars, bar_kv_empty = bars + 8;
     const uint32_t bar_st_full = bars + 16, bar_st_empty = bars + 16 + 8 * Cfg::NST;
     const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST;
-    const uint32_t bar_p_full = bar_s_full + 8;                       // [NWG]
-    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NWG, bar_drain = bar_acc_full + 8;
+    const uint32_t bar_p_full = bar_s_full + 8;                       // [NSLICE]
+    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
+    const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
 
@@ -158,9 +161,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mbar_init(bar_st_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
-        for (int i = 0; i < BWD_NWG; ++i) mbar_init(bar_p_full + 8 * i, 4);
+        for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_acc_empty, 4 * BWD_NWG);
         fence_barrier_init();
     }
     if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -236,9 +240,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const uint64_t dK = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
             const uint64_t dST = sdesc_sw128(sST, 16, 1024), dSTmn = sdesc_sw128(sST, 16384, 1024);
             uint32_t nst = 0, iter = 0;
-            uint32_t p_phase[BWD_NWG];
-            for (int i = 0; i < BWD_NWG; ++i) p_phase[i] = 0;
-            bool ok = true;
+            uint32_t p_phase[BWD_NSLICE];
+            for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
+            uint32_t ae_phase = 0;
+            bool ok = true, acc_busy = false;   // acc_busy: the last item's accumulators not yet read out
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DkdvItem it = decode_dkdv(P, w);
                 ok = mbar_wait_warp(bar_kv_full, iter & 1, abort_flag);
@@ -274,19 +279,27 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                             mma_commit(bar_s_full);
                         }
                         __syncwarp();
-                        // dV += P^T dO ; dK += dS^T Q, one 32-deep slice of query rows per warpgroup
-                        for (int wg = 0; wg < BWD_NWG && ok; ++wg) {
-                            ok = mbar_wait_warp(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
+                        // every group has stored the previous item's dK / dV
+                        if (first && acc_busy) {
+                            ok = mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag);
                             if (!ok) break;
-                            p_phase[wg] ^= 1;
+                            ae_phase ^= 1;
+                            acc_busy = false;
+                        }
+                        // dV += P^T dO ; dK += dS^T Q, one 64-deep slice of query rows at a time;
+                        // in slice j, warpgroup w's 16 query rows sit at columns 64j + 16w
+                        for (int j = 0; j < BWD_NSLICE && ok; ++j) {
+                            ok = mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag);
+                            if (!ok) break;
+                            p_phase[j] ^= 1;
                             tc_fence_after();
                             if (elect_one()) {
 #pragma unroll
-                                for (int kk = 0; kk < 2; ++kk) {
-                                    const uint32_t acc = (!first || wg > 0 || kk > 0) ? 1u : 0u;
-                                    const uint32_t brow = ((2 * wg + kk) * 2048) >> 4;
-                                    mma_ts(tdV, tS + 32 * wg + 8 * kk, bdo_mn + brow, IDESC_G, acc);
-                                    mma_ts(tdK, tdP + 32 * wg + 8 * kk, bq_mn + brow, IDESC_G, acc);
+                                for (int w4 = 0; w4 < BWD_NWG; ++w4) {
+                                    const uint32_t acc = (!first || j > 0 || w4 > 0) ? 1u : 0u;
+                                    const uint32_t brow = ((BWD_NWG * j + w4) * 2048) >> 4;
+                                    mma_ts(tdV, tS + 64 * j + 16 * w4, bdo_mn + brow, IDESC_G, acc);
+                                    mma_ts(tdK, tdP + 64 * j + 16 * w4, bq_mn + brow, IDESC_G, acc);
                                 }
                             }
                             __syncwarp();
@@ -303,6 +316,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
                 }
                 __syncwarp();
+                acc_busy = acc_busy || !first;
             }
             if (elect_one()) mma_commit(bar_drain);
             __syncwarp();
@@ -312,10 +326,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     } else {
         regs_inc<104>();
         // ------------------------------------------------------------ elementwise groups (key rows)
-        const int wg = warp >> 2;                        // query columns [32wg, 32wg+32)
+        const int wg = warp >> 2;                        // query columns [16wg, 16wg+16) of each slice
         const int row = (warp & 3) * 32 + lane;          // key row of the tile (TMEM lane)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_off + 32 * wg, tdP = tmem + lane_off + 128 + 32 * wg;
+        const uint32_t tS = tmem + lane_off + 16 * wg, tdP = tmem + lane_off + 128 + 16 * wg;
         const uint32_t tdV = tmem + lane_off + 256 + 32 * wg, tdK = tmem + lane_off + 384 + 32 * wg;
         uint32_t nst = 0, s_phase = 0, a_phase = 0;
         bool ok = true;
@@ -339,41 +353,51 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     s_phase ^= 1;
                     tc_fence_after();
                     const uint8_t* st = smem + Cfg::ST_OFF + slot * Cfg::ST_STRIDE;
-                    const float* s_lse2 = reinterpret_cast<const float*>(st + 2 * Cfg::TILE) + 32 * wg;
-                    const float* s_delta = reinterpret_cast<const float*>(st + 2 * Cfg::TILE + 512) + 32 * wg;
-                    const int* s_ds = reinterpret_cast<const int*>(st + 2 * Cfg::TILE + 1024) + 32 * wg;
+                    const float* s_lse2 = reinterpret_cast<const float*>(st + 2 * Cfg::TILE) + 16 * wg;
+                    const float* s_delta = reinterpret_cast<const float*>(st + 2 * Cfg::TILE + 512) + 16 * wg;
+                    const int* s_ds = reinterpret_cast<const int*>(st + 2 * Cfg::TILE + 1024) + 16 * wg;
                     float sv[32], dp[32];
-                    tmem_ld32f(tS, sv);
-                    tmem_ld32f(tdP, dp);
+                    tmem_ld16f(tS, sv);
+                    tmem_ld16f(tS + 64, sv + 16);
+                    tmem_ld16f(tdP, dp);
+                    tmem_ld16f(tdP + 64, dp + 16);
                     tmem_wait_ld();
                     reg_fence32f(sv);
                     reg_fence32f(dp);
-                    uint32_t pk[16], dk[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float p2[2], d2[2];
+                    for (int j = 0; j < BWD_NSLICE; ++j) {
+                        uint32_t pk[8], dk[8];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = i + e;                       // column within the block
-                            float pv = ex2_approx(fmaf(sv[c], P.scale_log2, -s_lse2[c]));
-                            if (cls == TILE_PARTIAL) {
-                                const int q_orig = qo + 32 * wg + c;
-                                const int dsq = P.docs ? s_ds[c] : 0;
-                                if (k_orig > q_orig || k_orig < dsq) pv = 0.f;
+                        for (int i = 0; i < 16; i += 4) {
+                            const float4 l4 = *reinterpret_cast<const float4*>(s_lse2 + 64 * j + i);
+                            const float4 d4 = *reinterpret_cast<const float4*>(s_delta + 64 * j + i);
+                            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                            float p4[4], g4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int c = i + e;                   // column within the block
+                                float pv = ex2_approx(fmaf(sv[16 * j + c], P.scale_log2, -lv[e]));
+                                if (cls == TILE_PARTIAL) {
+                                    const int q_orig = qo + 64 * j + 16 * wg + c;
+                                    const int dsq = P.docs ? s_ds[64 * j + c] : 0;
+                                    if (k_orig > q_orig || k_orig < dsq) pv = 0.f;
+                                }
+                                p4[e] = pv;
+                                g4[e] = pv * (dp[16 * j + c] - dv[e]);
                             }
-                            p2[e] = pv;
-                            d2[e] = pv * (dp[c] - s_delta[c]);
+                            pk[i / 2] = pack_bf16(p4[0], p4[1]);
+                            pk[i / 2 + 1] = pack_bf16(p4[2], p4[3]);
+                            dk[i / 2] = pack_bf16(g4[0], g4[1]);
+                            dk[i / 2 + 1] = pack_bf16(g4[2], g4[3]);
                         }
-                        pk[i / 2] = pack_bf16(p2[0], p2[1]);
-                        dk[i / 2] = pack_bf16(d2[0], d2[1]);
+                        // this warp's 16 score columns of the slice are read: overwrite the first 8
+                        tmem_st8(tS + 64 * j, pk);
+                        tmem_st8(tdP + 64 * j, dk);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_p_full + 8 * j);
                     }
-                    // this block's 32 score columns are read: overwrite its first 16
-                    tmem_st16(tS, pk);
-                    tmem_st16(tdP, dk);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_p_full + 8 * wg);
                     had = true;
                 }
             }
@@ -404,6 +428,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                            pack_bf16(b[8 * i + 6] * P.scale, b[8 * i + 7] * P.scale));
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_acc_empty);
             } else if (32 * wg < D) {
                 uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
                 uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + 32 * wg);
@@ -431,8 +458,8 @@ struct DqCfg {
     static constexpr int NSLOT = (D == 128) ? 4 : 8;
     static constexpr int Q_OFF = 0, DO_OFF = TILE, KV_OFF = 2 * TILE;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE;
-    // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, p_full[NWG], acc_full, drain
-    static constexpr int NBAR = 5 + 2 * NSLOT + BWD_NWG;
+    // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, p_full[NSLICE], acc_full, drain, acc_empty
+    static constexpr int NBAR = 6 + 2 * NSLOT + BWD_NSLICE;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
     static constexpr int THREADS = BWD_THREADS;
 };
@@ -477,8 +504,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bar_q_full = bars, bar_q_empty = bars + 8;
     const uint32_t bar_kv_full = bars + 16, bar_kv_empty = bars + 16 + 8 * Cfg::NSLOT;
     const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT;
-    const uint32_t bar_p_full = bar_s_full + 8;                       // [NWG]
-    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NWG, bar_drain = bar_acc_full + 8;
+    const uint32_t bar_p_full = bar_s_full + 8;                       // [NSLICE]
+    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
+    const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
 
@@ -497,9 +525,10 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_kv_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
-        for (int i = 0; i < BWD_NWG; ++i) mbar_init(bar_p_full + 8 * i, 4);
+        for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_acc_empty, 4 * BWD_NWG);
         fence_barrier_init();
     }
     if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -565,9 +594,10 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint64_t dQd = sdesc_sw128(sQ, 16, 1024), ddO = sdesc_sw128(sdO, 16, 1024);
             const uint64_t dKV = sdesc_sw128(sKV, 16, 1024), dKVmn = sdesc_sw128(sKV, 16384, 1024);
             uint32_t nload = 0, iter = 0;
-            uint32_t p_phase[BWD_NWG];
-            for (int i = 0; i < BWD_NWG; ++i) p_phase[i] = 0;
-            bool ok = true;
+            uint32_t p_phase[BWD_NSLICE];
+            for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
+            uint32_t ae_phase = 0;
+            bool ok = true, acc_busy = false;   // acc_busy: the last item's accumulators not yet read out
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DqItem it = decode_dq(P, w);
                 const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
@@ -579,7 +609,6 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
-                        const int kpos = j * n2c + kt * 128;
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
@@ -606,17 +635,25 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             mma_commit(bar_kv_empty + 8 * vslot);
                         }
                         __syncwarp();
-                        // dQ += dS K, one 32-deep slice of keys per warpgroup
-                        for (int wg = 0; wg < BWD_NWG && ok; ++wg) {
-                            ok = mbar_wait_warp(bar_p_full + 8 * wg, p_phase[wg], abort_flag);
+                        // every group has stored the previous item's dQ
+                        if (first && acc_busy) {
+                            ok = mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag);
                             if (!ok) break;
-                            p_phase[wg] ^= 1;
+                            ae_phase ^= 1;
+                            acc_busy = false;
+                        }
+                        // dQ += dS K, one 64-deep slice of keys at a time; in slice j,
+                        // warpgroup w's 16 keys sit at columns 64j + 16w
+                        for (int j = 0; j < BWD_NSLICE && ok; ++j) {
+                            ok = mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag);
+                            if (!ok) break;
+                            p_phase[j] ^= 1;
                             tc_fence_after();
                             if (elect_one()) {
 #pragma unroll
-                                for (int kk = 0; kk < 2; ++kk)
-                                    mma_ts(tdQ, tS + 32 * wg + 8 * kk, bk_mn + (((2 * wg + kk) * 2048) >> 4),
-                                           IDESC_G, (!first || wg > 0 || kk > 0) ? 1u : 0u);
+                                for (int w4 = 0; w4 < BWD_NWG; ++w4)
+                                    mma_ts(tdQ, tS + 64 * j + 16 * w4, bk_mn + (((BWD_NWG * j + w4) * 2048) >> 4),
+                                           IDESC_G, (!first || j > 0 || w4 > 0) ? 1u : 0u);
                             }
                             __syncwarp();
                         }
@@ -632,6 +669,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
                 }
                 __syncwarp();
+                acc_busy = acc_busy || !first;
             }
             if (elect_one()) mma_commit(bar_drain);
             __syncwarp();
@@ -641,10 +679,10 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     } else {
         regs_inc<104>();
         // ------------------------------------------------------------ elementwise groups (query rows)
-        const int wg = warp >> 2;                        // key columns [32wg, 32wg+32)
+        const int wg = warp >> 2;                        // key columns [16wg, 16wg+16) of each slice
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_off + 32 * wg, tdP = tmem + lane_off + 128 + 32 * wg;
+        const uint32_t tS = tmem + lane_off + 16 * wg, tdP = tmem + lane_off + 128 + 16 * wg;
         const uint32_t tdQ = tmem + lane_off + 256 + 32 * wg;
         uint32_t s_phase = 0, a_phase = 0;
         bool ok = true;
@@ -668,31 +706,36 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     if (!ok) break;
                     s_phase ^= 1;
                     tc_fence_after();
-                    const int lo = ds_row - ko - 32 * wg, hi = q_orig - ko - 32 * wg;
+                    const int lo = ds_row - ko - 16 * wg, hi = q_orig - ko - 16 * wg;
                     float sv[32], dp[32];
-                    tmem_ld32f(tS, sv);
-                    tmem_ld32f(tdP, dp);
+                    tmem_ld16f(tS, sv);
+                    tmem_ld16f(tS + 64, sv + 16);
+                    tmem_ld16f(tdP, dp);
+                    tmem_ld16f(tdP + 64, dp + 16);
                     tmem_wait_ld();
                     reg_fence32f(sv);
                     reg_fence32f(dp);
-                    uint32_t dk[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float d2[2];
+                    for (int j = 0; j < BWD_NSLICE; ++j) {
+                        uint32_t dk[8];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = i + e;
-                            float pv = ex2_approx(fmaf(sv[c], P.scale_log2, -lse2));
-                            if (cls == TILE_PARTIAL && (c < lo || c > hi)) pv = 0.f;
-                            d2[e] = pv * (dp[c] - dlt);
+                        for (int i = 0; i < 16; i += 2) {
+                            float d2[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = i + e;
+                                float pv = ex2_approx(fmaf(sv[16 * j + c], P.scale_log2, -lse2));
+                                if (cls == TILE_PARTIAL && (64 * j + c < lo || 64 * j + c > hi)) pv = 0.f;
+                                d2[e] = pv * (dp[16 * j + c] - dlt);
+                            }
+                            dk[i / 2] = pack_bf16(d2[0], d2[1]);
                         }
-                        dk[i / 2] = pack_bf16(d2[0], d2[1]);
+                        tmem_st8(tS + 64 * j, dk);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_p_full + 8 * j);
                     }
-                    tmem_st16(tS, dk);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_p_full + 8 * wg);
                     had = true;
                 }
             }
@@ -715,6 +758,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                            pack_bf16(a[8 * i + 4] * P.scale, a[8 * i + 5] * P.scale),
                                            pack_bf16(a[8 * i + 6] * P.scale, a[8 * i + 7] * P.scale));
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_acc_empty);
             } else if (32 * wg < D) {
                 uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 32 * wg);
                 for (int i = 0; i < 4; ++i) dq[i] = make_uint4(0, 0, 0, 0);
