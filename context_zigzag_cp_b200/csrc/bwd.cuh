@@ -75,10 +75,67 @@ struct BwdParams {
     const int32_t* doc_start;  // [S] shard order
     const float* lse2;       // [B*Hq][S]
     const float* delta;      // [B*Hq][S]
+    const __nv_bfloat16* q;  // [B*Hq][S][D]
+    const __nv_bfloat16* dout;  // [B*Hq][S][D]
     __nv_bfloat16* dq;       // [B*Hq][S][D]
     __nv_bfloat16* dk;       // [B*Hkv][S][D]
     __nv_bfloat16* dv;
 };
+
+// P^T and dS^T (bf16 pairs) for 16 query columns of one key row k in the dK/dV
+// pass.  MODE 0: every column admitted; 1: column c admitted when c >= thr
+// (thr = k - first query of the 16, the causal test); 2: also k >= ds[c].
+template <int MODE>
+__device__ __forceinline__ void dkdv_cols16(const float* sv, const float* dp, const float* s_lse2,
+                                            const float* s_delta, const int* s_ds, float scale_log2,
+                                            int thr, int k_orig, uint32_t* pk, uint32_t* dk)
+{
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(s_lse2 + i);
+        const float4 d4 = *reinterpret_cast<const float4*>(s_delta + i);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        int dsv[4] = {0, 0, 0, 0};
+        if (MODE == 2) {
+            const int4 q4 = *reinterpret_cast<const int4*>(s_ds + i);
+            dsv[0] = q4.x; dsv[1] = q4.y; dsv[2] = q4.z; dsv[3] = q4.w;
+        }
+        float p4[4], g4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int c = i + e;
+            float pv = ex2_approx(fmaf(sv[c], scale_log2, -lv[e]));
+            if (MODE >= 1 && c < thr) pv = 0.f;
+            if (MODE == 2 && k_orig < dsv[e]) pv = 0.f;
+            p4[e] = pv;
+            g4[e] = pv * (dp[c] - dv[e]);
+        }
+        pk[i / 2] = pack_bf16(p4[0], p4[1]);
+        pk[i / 2 + 1] = pack_bf16(p4[2], p4[3]);
+        dk[i / 2] = pack_bf16(g4[0], g4[1]);
+        dk[i / 2 + 1] = pack_bf16(g4[2], g4[3]);
+    }
+}
+
+// dS (bf16 pairs) for 16 key columns of one query row in the dQ pass; with
+// MASK, column c is admitted when lo <= c <= hi.
+template <bool MASK>
+__device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, float lse2, float dlt,
+                                          float scale_log2, int lo, int hi, uint32_t* dk)
+{
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        float d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int c = i + e;
+            float pv = ex2_approx(fmaf(sv[c], scale_log2, -lse2));
+            if (MASK && (c < lo || c > hi)) pv = 0.f;
+            d2[e] = pv * (dp[c] - dlt);
+        }
+        dk[i / 2] = pack_bf16(d2[0], d2[1]);
+    }
+}
 
 // ============================================================================
 // dK / dV pass
@@ -367,29 +424,16 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < BWD_NSLICE; ++j) {
                         uint32_t pk[8], dk[8];
-#pragma unroll
-                        for (int i = 0; i < 16; i += 4) {
-                            const float4 l4 = *reinterpret_cast<const float4*>(s_lse2 + 64 * j + i);
-                            const float4 d4 = *reinterpret_cast<const float4*>(s_delta + 64 * j + i);
-                            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                            float p4[4], g4[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int c = i + e;                   // column within the block
-                                float pv = ex2_approx(fmaf(sv[16 * j + c], P.scale_log2, -lv[e]));
-                                if (cls == TILE_PARTIAL) {
-                                    const int q_orig = qo + 64 * j + 16 * wg + c;
-                                    const int dsq = P.docs ? s_ds[64 * j + c] : 0;
-                                    if (k_orig > q_orig || k_orig < dsq) pv = 0.f;
-                                }
-                                p4[e] = pv;
-                                g4[e] = pv * (dp[16 * j + c] - dv[e]);
-                            }
-                            pk[i / 2] = pack_bf16(p4[0], p4[1]);
-                            pk[i / 2 + 1] = pack_bf16(p4[2], p4[3]);
-                            dk[i / 2] = pack_bf16(g4[0], g4[1]);
-                            dk[i / 2 + 1] = pack_bf16(g4[2], g4[3]);
-                        }
+                        const int thr = k_orig - (qo + 64 * j + 16 * wg);
+                        if (cls == TILE_FULL)
+                            dkdv_cols16<0>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
+                                           s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
+                        else if (!P.docs)
+                            dkdv_cols16<1>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
+                                           s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
+                        else
+                            dkdv_cols16<2>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
+                                           s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
                         // this warp's 16 score columns of the slice are read: overwrite the first 8
                         tmem_st8(tS + 64 * j, pk);
                         tmem_st8(tdP + 64 * j, dk);
@@ -452,14 +496,24 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 // ============================================================================
 // dQ pass
 // ============================================================================
+// The query tile's Q and dO rows sit in tensor memory (the A operands of S and
+// dP, written by the elementwise warps once per item), so shared memory holds
+// a deep K/V ring.  The elementwise warps copy S and dP out of tensor memory
+// first and release it (s_free), so the MMA warp computes the next key tile's
+// S and dP while dS of this one is formed.  dS goes to shared memory (bf16,
+// the K-major A operand of dQ += dS K), one 16 KB buffer per 64-key slice.
+// Tensor memory: S 0..127, dP 128..255, dQ 256..383, Q 384..447, dO 448..511.
 template <int D>
 struct DqCfg {
-    static constexpr int TILE = 128 * D * 2;
-    static constexpr int NSLOT = (D == 128) ? 4 : 8;
-    static constexpr int Q_OFF = 0, DO_OFF = TILE, KV_OFF = 2 * TILE;
-    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE;
-    // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, p_full[NSLICE], acc_full, drain, acc_empty
-    static constexpr int NBAR = 6 + 2 * NSLOT + BWD_NSLICE;
+    static constexpr int KTILE = 128 * D * 2;
+    static constexpr int NSLOT = (D == 128) ? 6 : 12;
+    static constexpr int DS_SLICE = 128 * 64 * 2;                // 128 query rows x 64 keys, bf16
+    static constexpr int KV_OFF = 0;
+    static constexpr int DS_OFF = KV_OFF + NSLOT * KTILE;
+    static constexpr int BAR_OFF = DS_OFF + BWD_NSLICE * DS_SLICE;
+    // qt_full, qt_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, s_free, p_full[NSLICE],
+    // ds_empty[NSLICE], acc_full, drain, acc_empty
+    static constexpr int NBAR = 7 + 2 * NSLOT + 2 * BWD_NSLICE;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
     static constexpr int THREADS = BWD_THREADS;
 };
@@ -499,13 +553,15 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sQ = sbase + Cfg::Q_OFF, sdO = sbase + Cfg::DO_OFF, sKV = sbase + Cfg::KV_OFF;
+    const uint32_t sKV = sbase + Cfg::KV_OFF;
+    const uint32_t sDS = sbase + Cfg::DS_OFF;
     const uint32_t bars = sbase + Cfg::BAR_OFF;
-    const uint32_t bar_q_full = bars, bar_q_empty = bars + 8;
+    const uint32_t bar_qt_full = bars, bar_qt_empty = bars + 8;
     const uint32_t bar_kv_full = bars + 16, bar_kv_empty = bars + 16 + 8 * Cfg::NSLOT;
-    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT;
-    const uint32_t bar_p_full = bar_s_full + 8;                       // [NSLICE]
-    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
+    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT, bar_s_free = bar_s_full + 8;
+    const uint32_t bar_p_full = bar_s_free + 8;                         // [NSLICE]
+    const uint32_t bar_ds_empty = bar_p_full + 8 * BWD_NSLICE;          // [NSLICE]
+    const uint32_t bar_acc_full = bar_ds_empty + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
@@ -518,14 +574,18 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_empty, 1);
+        mbar_init(bar_qt_full, 4 * BWD_NWG);
+        mbar_init(bar_qt_empty, 1);
         for (int i = 0; i < Cfg::NSLOT; ++i) {
             mbar_init(bar_kv_full + 8 * i, 1);
             mbar_init(bar_kv_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
-        for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
+        mbar_init(bar_s_free, 4 * BWD_NWG);
+        for (int i = 0; i < BWD_NSLICE; ++i) {
+            mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
+            mbar_init(bar_ds_empty + 8 * i, 1);
+        }
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
         mbar_init(bar_acc_empty, 4 * BWD_NWG);
@@ -544,20 +604,13 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (warp == PROD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmdO);
-            uint32_t nload = 0, iter = 0;
+            prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+            uint32_t nload = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
+            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
                 const DqItem it = decode_dq(P, w);
                 const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
                 const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
-                ok = mbar_wait(bar_q_empty, (iter & 1) ^ 1, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(bar_q_full, 2 * Cfg::TILE);
-                for (int h = 0; h < D / 64; ++h) {
-                    tma_load_2d(sQ + h * 16384, &tmQ, h * 64, it.bh * P.S + it.qpos, bar_q_full);
-                    tma_load_2d(sdO + h * 16384, &tmdO, h * 64, it.bh * P.S + it.qpos, bar_q_full);
-                }
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
@@ -568,9 +621,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             const uint32_t slot = nload % Cfg::NSLOT, par = (nload / Cfg::NSLOT) & 1;
                             ok = mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, abort_flag);
                             if (!ok) break;
-                            mbar_arrive_expect_tx(bar_kv_full + 8 * slot, Cfg::TILE);
+                            mbar_arrive_expect_tx(bar_kv_full + 8 * slot, Cfg::KTILE);
                             for (int h = 0; h < D / 64; ++h)
-                                tma_load_2d(sKV + slot * Cfg::TILE + h * 16384,
+                                tma_load_2d(sKV + slot * Cfg::KTILE + h * 16384,
                                             kv == 0 ? (const void*)&tmK : (const void*)&tmV, h * 64,
                                             it.bkv * P.S + kpos, bar_kv_full + 8 * slot);
                         }
@@ -582,30 +635,57 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     mbar_wait_drain(bar_kv_full + 8 * (n % Cfg::NSLOT), (n / Cfg::NSLOT) & 1);
             }
         }
-    } else if (warp == MMA_WARP) {
+      } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         // The whole warp runs the control flow; one elected lane issues each group
-        // of tensor-core instructions (cheaper than a single diverged lane).
+        // of tensor-core instructions.  Order per key tile i: S(i), dP(i) (once the
+        // elementwise warps have copied out tile i-1), then dQ += dS(i-1) K(i-1).
         {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);
-            constexpr uint32_t TILE16 = Cfg::TILE >> 4;
-            const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-            const uint64_t dQd = sdesc_sw128(sQ, 16, 1024), ddO = sdesc_sw128(sdO, 16, 1024);
+            constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);   // A K-major, B MN-major
+            constexpr uint32_t KT16 = Cfg::KTILE >> 4, DS16 = Cfg::DS_SLICE >> 4;
+            const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256, tQ = tmem + 384, tdO = tmem + 448;
             const uint64_t dKV = sdesc_sw128(sKV, 16, 1024), dKVmn = sdesc_sw128(sKV, 16384, 1024);
-            uint32_t nload = 0, iter = 0;
+            const uint64_t dDS = sdesc_sw128(sDS, 16, 1024);
+            uint32_t nload = 0, iter = 0, sf_phase = 0, ae_phase = 0;
             uint32_t p_phase[BWD_NSLICE];
             for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
-            uint32_t ae_phase = 0;
-            bool ok = true, acc_busy = false;   // acc_busy: the last item's accumulators not yet read out
+            bool ok = true, acc_busy = false, s_pending = false;
+            // dQ += dS K for one finished key tile, 64 keys per slice
+            auto issue_dq = [&](uint32_t kslot, bool& first) -> bool {
+                if (first && acc_busy) {   // every group has stored the previous item's dQ
+                    if (!mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag)) return false;
+                    ae_phase ^= 1;
+                    acc_busy = false;
+                }
+                const uint64_t bk_mn = dKVmn + kslot * KT16;
+                for (int j = 0; j < BWD_NSLICE; ++j) {
+                    if (!mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag)) return false;
+                    p_phase[j] ^= 1;
+                    tc_fence_after();
+                    if (elect_one()) {
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4)
+                            mma_ss(tdQ, dDS + j * DS16 + ((w4 * 32) >> 4), bk_mn + (((4 * j + w4) * 2048) >> 4),
+                                   IDESC_G, (!first || j > 0 || w4 > 0) ? 1u : 0u);
+                        mma_commit(bar_ds_empty + 8 * j);
+                    }
+                    __syncwarp();
+                }
+                first = false;
+                if (elect_one()) mma_commit(bar_kv_empty + 8 * kslot);
+                __syncwarp();
+                return true;
+            };
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DqItem it = decode_dq(P, w);
                 const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
                 const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
-                ok = mbar_wait_warp(bar_q_full, iter & 1, abort_flag);
+                ok = mbar_wait_warp(bar_qt_full, iter & 1, abort_flag);   // Q, dO rows in tensor memory
                 if (!ok) break;
                 tc_fence_after();
-                bool first = true;
+                bool first = true, prev_live = false;
+                uint32_t prev_kslot = 0;
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
@@ -617,56 +697,41 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         ok = mbar_wait_warp(bar_kv_full + 8 * kslot, kpar, abort_flag) &&
                              mbar_wait_warp(bar_kv_full + 8 * vslot, vpar, abort_flag);
                         if (!ok) break;
+                        if (s_pending) {   // S / dP of the previous tile are copied out
+                            ok = mbar_wait_warp(bar_s_free, sf_phase, abort_flag);
+                            if (!ok) break;
+                            sf_phase ^= 1;
+                        }
                         tc_fence_after();
-                        const uint64_t bk = dKV + kslot * TILE16, bv = dKV + vslot * TILE16;
-                        const uint64_t bk_mn = dKVmn + kslot * TILE16;
+                        const uint64_t bk = dKV + kslot * KT16, bv = dKV + vslot * KT16;
                         if (elect_one()) {
 #pragma unroll
                             for (int k = 0; k < D / 16; ++k) {
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                                mma_ss(tS, dQd + off, bk + off, IDESC_S, k > 0 ? 1u : 0u);
+                                mma_ts(tS, tQ + 8 * k, bk + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
 #pragma unroll
                             for (int k = 0; k < D / 16; ++k) {
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
-                                mma_ss(tdP, ddO + off, bv + off, IDESC_S, k > 0 ? 1u : 0u);
+                                mma_ts(tdP, tdO + 8 * k, bv + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
                             mma_commit(bar_s_full);
                             mma_commit(bar_kv_empty + 8 * vslot);
                         }
                         __syncwarp();
-                        // every group has stored the previous item's dQ
-                        if (first && acc_busy) {
-                            ok = mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag);
-                            if (!ok) break;
-                            ae_phase ^= 1;
-                            acc_busy = false;
-                        }
-                        // dQ += dS K, one 64-deep slice of keys at a time; in slice j,
-                        // warpgroup w's 16 keys sit at columns 64j + 16w
-                        for (int j = 0; j < BWD_NSLICE && ok; ++j) {
-                            ok = mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag);
-                            if (!ok) break;
-                            p_phase[j] ^= 1;
-                            tc_fence_after();
-                            if (elect_one()) {
-#pragma unroll
-                                for (int w4 = 0; w4 < BWD_NWG; ++w4)
-                                    mma_ts(tdQ, tS + 64 * j + 16 * w4, bk_mn + (((BWD_NWG * j + w4) * 2048) >> 4),
-                                           IDESC_G, (!first || j > 0 || w4 > 0) ? 1u : 0u);
-                            }
-                            __syncwarp();
-                        }
-                        if (!ok) break;
-                        if (elect_one()) mma_commit(bar_kv_empty + 8 * kslot);
-                        __syncwarp();
-                        first = false;
+                        s_pending = true;
+                        if (prev_live && !(ok = issue_dq(prev_kslot, first))) break;
+                        prev_live = true;
+                        prev_kslot = kslot;
                     }
                 }
                 if (!ok) break;
+                if (elect_one()) mma_commit(bar_qt_empty);   // the item's last S / dP are issued
+                __syncwarp();
+                if (prev_live) ok = issue_dq(prev_kslot, first);
+                if (!ok) break;
                 if (elect_one()) {
-                    mma_commit(bar_q_empty);
-                    if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
+                    if (!first) mma_commit(bar_acc_full);   // the elementwise groups wait only if they had a tile
                 }
                 __syncwarp();
                 acc_busy = acc_busy || !first;
@@ -684,17 +749,43 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + 16 * wg, tdP = tmem + lane_off + 128 + 16 * wg;
         const uint32_t tdQ = tmem + lane_off + 256 + 32 * wg;
-        uint32_t s_phase = 0, a_phase = 0;
+        // this row of a dS slice buffer (SW128 K-major: 16-byte chunk c of row r sits at chunk c ^ (r % 8))
+        const uint32_t ds_row = sDS + (row >> 3) * 1024 + (row & 7) * 128;
+        const uint32_t ds_c0 = ((2 * wg) ^ (row & 7)) * 16, ds_c1 = ((2 * wg + 1) ^ (row & 7)) * 16;
+        const uint32_t tQ = tmem + lane_off + 384 + 16 * wg, tdO = tmem + lane_off + 448 + 16 * wg;
+        uint32_t s_phase = 0, a_phase = 0, nstep = 0, iter = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
+        for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
             const DqItem it = decode_dq(P, w);
             const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
             const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
             const size_t rowi = static_cast<size_t>(it.bh) * P.S + it.qpos + row;
+            // this row's Q and dO (bf16 pairs, columns [32wg, 32wg+32)) into tensor memory once the
+            // previous item's S / dP have read the old ones
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_qt_empty, (iter & 1) ^ 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            if (32 * wg < D) {
+                const uint4* qsrc = reinterpret_cast<const uint4*>(P.q + rowi * D + 32 * wg);
+                const uint4* osrc = reinterpret_cast<const uint4*>(P.dout + rowi * D + 32 * wg);
+                uint32_t qa[16], oa[16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 x = __ldg(qsrc + i), y = __ldg(osrc + i);
+                    qa[4 * i] = x.x; qa[4 * i + 1] = x.y; qa[4 * i + 2] = x.z; qa[4 * i + 3] = x.w;
+                    oa[4 * i] = y.x; oa[4 * i + 1] = y.y; oa[4 * i + 2] = y.z; oa[4 * i + 3] = y.w;
+                }
+                tmem_st16(tQ, qa);
+                tmem_st16(tdO, oa);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_qt_full);
             const float lse2 = __ldg(P.lse2 + rowi);
             const float dlt = __ldg(P.delta + rowi);
             const int q_orig = it.qo + row;
-            const int ds_row = P.docs ? __ldg(P.doc_start + it.qpos + row) : 0;
+            const int ds_q = P.docs ? __ldg(P.doc_start + it.qpos + row) : 0;
             bool had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
@@ -706,7 +797,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     if (!ok) break;
                     s_phase ^= 1;
                     tc_fence_after();
-                    const int lo = ds_row - ko - 16 * wg, hi = q_orig - ko - 16 * wg;
+                    const int lo = ds_q - ko - 16 * wg, hi = q_orig - ko - 16 * wg;
                     float sv[32], dp[32];
                     tmem_ld16f(tS, sv);
                     tmem_ld16f(tS + 64, sv + 16);
@@ -715,27 +806,31 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     tmem_wait_ld();
                     reg_fence32f(sv);
                     reg_fence32f(dp);
+                    // S and dP of this tile are in registers: the MMA warp may overwrite them
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_s_free);
 #pragma unroll
-                    for (int j = 0; j < BWD_NSLICE; ++j) {
+                    for (int jj = 0; jj < BWD_NSLICE; ++jj) {
                         uint32_t dk[8];
-#pragma unroll
-                        for (int i = 0; i < 16; i += 2) {
-                            float d2[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int c = i + e;
-                                float pv = ex2_approx(fmaf(sv[16 * j + c], P.scale_log2, -lse2));
-                                if (cls == TILE_PARTIAL && (64 * j + c < lo || 64 * j + c > hi)) pv = 0.f;
-                                d2[e] = pv * (dp[16 * j + c] - dlt);
-                            }
-                            dk[i / 2] = pack_bf16(d2[0], d2[1]);
-                        }
-                        tmem_st8(tS + 64 * j, dk);
-                        tmem_wait_st();
-                        tc_fence_before();
+                        if (cls == TILE_FULL)
+                            dq_cols16<false>(sv + 16 * jj, dp + 16 * jj, lse2, dlt, P.scale_log2, 0, 0, dk);
+                        else
+                            dq_cols16<true>(sv + 16 * jj, dp + 16 * jj, lse2, dlt, P.scale_log2, lo - 64 * jj,
+                                            hi - 64 * jj, dk);
+                        // the previous tile's products have read this slice buffer
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(bar_ds_empty + 8 * jj, (nstep & 1) ^ 1, abort_flag));
+                        if (!ok) break;
+                        const uint32_t dst = ds_row + jj * Cfg::DS_SLICE;
+                        st_shared_v4(dst + ds_c0, dk[0], dk[1], dk[2], dk[3]);
+                        st_shared_v4(dst + ds_c1, dk[4], dk[5], dk[6], dk[7]);
+                        fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bar_p_full + 8 * j);
+                        if (lane == 0) mbar_arrive(bar_p_full + 8 * jj);
                     }
+                    if (!ok) break;
+                    ++nstep;
                     had = true;
                 }
             }

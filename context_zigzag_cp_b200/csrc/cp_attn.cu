@@ -468,6 +468,8 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.doc_start = pl->doc_start;
     P.lse2 = lse2;
     P.delta = delta;
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.dout = static_cast<const __nv_bfloat16*>(dout);
     P.dq = static_cast<__nv_bfloat16*>(dq);
     P.dk = static_cast<__nv_bfloat16*>(dk);
     P.dv = static_cast<__nv_bfloat16*>(dv);
