@@ -152,8 +152,9 @@ struct DkdvCfg {
     static constexpr int K_OFF = 0, V_OFF = TILE;
     static constexpr int ST_OFF = 2 * TILE;
     static constexpr int BAR_OFF = ST_OFF + NST * ST_STRIDE;
-    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full[NSLICE], acc_full, drain, acc_empty
-    static constexpr int NBAR = 6 + 2 * NST + BWD_NSLICE;
+    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, s_free, p_full[NSLICE], acc_full, drain,
+    // acc_empty
+    static constexpr int NBAR = 7 + 2 * NST + BWD_NSLICE;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
     static constexpr int THREADS = BWD_THREADS;
 };
@@ -194,8 +195,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t bars = sbase + Cfg::BAR_OFF;
     const uint32_t bar_kv_full = bars, bar_kv_empty = bars + 8;
     const uint32_t bar_st_full = bars + 16, bar_st_empty = bars + 16 + 8 * Cfg::NST;
-    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST;
-    const uint32_t bar_p_full = bar_s_full + 8;                       // [NSLICE]
+    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST, bar_s_free = bar_s_full + 8;
+    const uint32_t bar_p_full = bar_s_free + 8;                       // [NSLICE]
     const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
@@ -218,6 +219,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mbar_init(bar_st_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
+        mbar_init(bar_s_free, 4 * BWD_NWG);
         for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
@@ -296,17 +298,48 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             // descriptor bases; k-steps and stages are constant offsets in 16-byte units
             const uint64_t dK = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
             const uint64_t dST = sdesc_sw128(sST, 16, 1024), dSTmn = sdesc_sw128(sST, 16384, 1024);
-            uint32_t nst = 0, iter = 0;
+            uint32_t nst = 0, iter = 0, sf_phase = 0, ae_phase = 0;
             uint32_t p_phase[BWD_NSLICE];
             for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
-            uint32_t ae_phase = 0;
-            bool ok = true, acc_busy = false;   // acc_busy: the last item's accumulators not yet read out
+            // acc_busy: the last item's accumulators not yet read out; s_pending: S^T / dP^T of the
+            // last issued tile not yet copied out by the elementwise warps
+            bool ok = true, acc_busy = false, s_pending = false;
+            // dV += P^T dO, dK += dS^T Q for one finished query tile.  P^T and dS^T (bf16) sit in
+            // the dP^T columns: slice j at 64j (P^T) and 64j + 32 (dS^T), 16 query rows per 8 columns.
+            auto issue_products = [&](uint32_t slot, bool& first) -> bool {
+                if (first && acc_busy) {   // every group has stored the previous item's dK / dV
+                    if (!mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag)) return false;
+                    ae_phase ^= 1;
+                    acc_busy = false;
+                }
+                const uint64_t bq_mn = dSTmn + slot * ST16, bdo_mn = bq_mn + TILE16;
+                for (int j = 0; j < BWD_NSLICE; ++j) {
+                    if (!mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag)) return false;
+                    p_phase[j] ^= 1;
+                    tc_fence_after();
+                    if (elect_one()) {
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            const uint32_t acc = (!first || j > 0 || w4 > 0) ? 1u : 0u;
+                            const uint32_t brow = ((4 * j + w4) * 2048) >> 4;
+                            mma_ts(tdV, tdP + 64 * j + 8 * w4, bdo_mn + brow, IDESC_G, acc);
+                            mma_ts(tdK, tdP + 64 * j + 32 + 8 * w4, bq_mn + brow, IDESC_G, acc);
+                        }
+                    }
+                    __syncwarp();
+                }
+                first = false;
+                if (elect_one()) mma_commit(bar_st_empty + 8 * slot);
+                __syncwarp();
+                return true;
+            };
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DkdvItem it = decode_dkdv(P, w);
                 ok = mbar_wait_warp(bar_kv_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                bool first = true;
+                bool first = true, prev_live = false;
+                uint32_t prev_slot = 0;
                 for (int hq = 0; hq < g && ok; ++hq) {
                     for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
                          ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
@@ -319,15 +352,26 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         ++nst;
                         ok = mbar_wait_warp(bar_st_full + 8 * slot, par, abort_flag);
                         if (!ok) break;
+                        if (s_pending) {   // the previous tile's S^T / dP^T are copied out
+                            ok = mbar_wait_warp(bar_s_free, sf_phase, abort_flag);
+                            if (!ok) break;
+                            sf_phase ^= 1;
+                        }
                         tc_fence_after();
                         const uint64_t bq = dST + slot * ST16, bdo = bq + TILE16;
-                        const uint64_t bq_mn = dSTmn + slot * ST16, bdo_mn = bq_mn + TILE16;
+                        // S^T of this tile while the elementwise warps still work on the previous one
                         if (elect_one()) {
 #pragma unroll
                             for (int k = 0; k < D / 16; ++k) {
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
                                 mma_ss(tS, dK + off, bq + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
+                        }
+                        __syncwarp();
+                        // the previous tile's products read P^T / dS^T from the dP^T columns ...
+                        if (prev_live && !(ok = issue_products(prev_slot, first))) break;
+                        // ... before this tile's dP^T overwrites them (the tensor pipe runs in order)
+                        if (elect_one()) {
 #pragma unroll
                             for (int k = 0; k < D / 16; ++k) {
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
@@ -336,37 +380,12 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                             mma_commit(bar_s_full);
                         }
                         __syncwarp();
-                        // every group has stored the previous item's dK / dV
-                        if (first && acc_busy) {
-                            ok = mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag);
-                            if (!ok) break;
-                            ae_phase ^= 1;
-                            acc_busy = false;
-                        }
-                        // dV += P^T dO ; dK += dS^T Q, one 64-deep slice of query rows at a time;
-                        // in slice j, warpgroup w's 16 query rows sit at columns 64j + 16w
-                        for (int j = 0; j < BWD_NSLICE && ok; ++j) {
-                            ok = mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag);
-                            if (!ok) break;
-                            p_phase[j] ^= 1;
-                            tc_fence_after();
-                            if (elect_one()) {
-#pragma unroll
-                                for (int w4 = 0; w4 < BWD_NWG; ++w4) {
-                                    const uint32_t acc = (!first || j > 0 || w4 > 0) ? 1u : 0u;
-                                    const uint32_t brow = ((BWD_NWG * j + w4) * 2048) >> 4;
-                                    mma_ts(tdV, tS + 64 * j + 16 * w4, bdo_mn + brow, IDESC_G, acc);
-                                    mma_ts(tdK, tdP + 64 * j + 16 * w4, bq_mn + brow, IDESC_G, acc);
-                                }
-                            }
-                            __syncwarp();
-                        }
-                        if (!ok) break;
-                        if (elect_one()) mma_commit(bar_st_empty + 8 * slot);
-                        __syncwarp();
-                        first = false;
+                        s_pending = true;
+                        prev_live = true;
+                        prev_slot = slot;
                     }
                 }
+                if (ok && prev_live) ok = issue_products(prev_slot, first);
                 if (!ok) break;
                 if (elect_one()) {
                     mma_commit(bar_kv_empty);
@@ -388,7 +407,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + 16 * wg, tdP = tmem + lane_off + 128 + 16 * wg;
         const uint32_t tdV = tmem + lane_off + 256 + 32 * wg, tdK = tmem + lane_off + 384 + 32 * wg;
-        uint32_t nst = 0, s_phase = 0, a_phase = 0;
+        // packed P^T / dS^T of slice j go to dP^T columns 64j + 8wg and 64j + 32 + 8wg
+        const uint32_t tPk = tmem + lane_off + 128 + 8 * wg, tDk = tPk + 32;
+        uint32_t nst = 0, s_phase = 0, a_phase = 0, sf_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
             const DkdvItem it = decode_dkdv(P, w);
@@ -421,6 +442,15 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tmem_wait_ld();
                     reg_fence32f(sv);
                     reg_fence32f(dp);
+                    // scores are in registers: the MMA warp may compute the next tile's S^T
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_s_free);
+                    // every elementwise warp has its dP^T columns before any packed result lands there
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_free, sf_phase, abort_flag));
+                    if (!ok) break;
+                    sf_phase ^= 1;
+                    tc_fence_after();
 #pragma unroll
                     for (int j = 0; j < BWD_NSLICE; ++j) {
                         uint32_t pk[8], dk[8];
@@ -434,9 +464,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         else
                             dkdv_cols16<2>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
                                            s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
-                        // this warp's 16 score columns of the slice are read: overwrite the first 8
-                        tmem_st8(tS + 64 * j, pk);
-                        tmem_st8(tdP + 64 * j, dk);
+                        tmem_st8(tPk + 64 * j, pk);
+                        tmem_st8(tDk + 64 * j, dk);
                         tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
