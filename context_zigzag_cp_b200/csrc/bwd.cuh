@@ -147,15 +147,20 @@ constexpr int BWD_NSLICE = 2;                    // 64-column slices of a 128-co
 template <int D>
 struct DkdvCfg {
     static constexpr int TILE = 128 * D * 2;
-    static constexpr int NST = (D == 128) ? 2 : 4;            // Q/dO stages
-    static constexpr int ST_STRIDE = 2 * TILE + 2048;          // Q | dO | lse2 | delta | ds
+    // Q tiles are needed early (S^T of the next tile is issued while the current one is
+    // still in the elementwise step), dO tiles later: three Q slots, two dO slots; each dO
+    // slot carries the tile's lse2 and delta rows (512 B each).
+    static constexpr int NQ = 3, NDO = 2;
     static constexpr int K_OFF = 0, V_OFF = TILE;
-    static constexpr int ST_OFF = 2 * TILE;
-    static constexpr int BAR_OFF = ST_OFF + NST * ST_STRIDE;
-    // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, s_free, p_full[NSLICE], acc_full, drain,
-    // acc_empty
-    static constexpr int NBAR = 7 + 2 * NST + BWD_NSLICE;
-    static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
+    static constexpr int Q_OFF = 2 * TILE;
+    static constexpr int DO_OFF = Q_OFF + NQ * TILE;
+    static constexpr int LD_OFF = DO_OFF + NDO * TILE;
+    static constexpr int BAR_OFF = LD_OFF + NDO * 1024;
+    // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NDO], do_empty[NDO], s_full, s_free,
+    // p_full[NSLICE], acc_full, drain, acc_empty
+    static constexpr int NBAR = 7 + 2 * NQ + 2 * NDO + BWD_NSLICE;
+    // the dynamic shared window starts 1024-byte aligned (checked at run time), no slack
+    static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64;
     static constexpr int THREADS = BWD_THREADS;
 };
 
@@ -187,15 +192,20 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    const BwdParams P)
 {
     using Cfg = DkdvCfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if (smem_u32(smem_raw) & 1023u) {   // swizzled tiles need a 1024-byte aligned window
+        if (threadIdx.x == 0) record_status(3 /* CP_ERR_CUDA */);
+        return;
+    }
+    uint8_t* smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sK = sbase + Cfg::K_OFF, sV = sbase + Cfg::V_OFF, sST = sbase + Cfg::ST_OFF;
+    const uint32_t sK = sbase + Cfg::K_OFF, sV = sbase + Cfg::V_OFF;
+    const uint32_t sQ = sbase + Cfg::Q_OFF, sdO = sbase + Cfg::DO_OFF, sLD = sbase + Cfg::LD_OFF;
     const uint32_t bars = sbase + Cfg::BAR_OFF;
     const uint32_t bar_kv_full = bars, bar_kv_empty = bars + 8;
-    const uint32_t bar_st_full = bars + 16, bar_st_empty = bars + 16 + 8 * Cfg::NST;
-    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NST, bar_s_free = bar_s_full + 8;
+    const uint32_t bar_q_full = bars + 16, bar_q_empty = bar_q_full + 8 * Cfg::NQ;
+    const uint32_t bar_do_full = bar_q_empty + 8 * Cfg::NQ, bar_do_empty = bar_do_full + 8 * Cfg::NDO;
+    const uint32_t bar_s_full = bar_do_empty + 8 * Cfg::NDO, bar_s_free = bar_s_full + 8;
     const uint32_t bar_p_full = bar_s_free + 8;                       // [NSLICE]
     const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
@@ -207,16 +217,19 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int n2c = 2 * P.C;
     const int nqt = n2c / 128;
     const int half = P.C / 128;
-    const uint32_t st_bytes = 2 * Cfg::TILE + 1024 + (P.docs ? 512 : 0);
     constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         mbar_init(bar_kv_full, 1);
         mbar_init(bar_kv_empty, 1);
-        for (int i = 0; i < Cfg::NST; ++i) {
-            mbar_init(bar_st_full + 8 * i, 1);
-            mbar_init(bar_st_empty + 8 * i, 1);
+        for (int i = 0; i < Cfg::NQ; ++i) {
+            mbar_init(bar_q_full + 8 * i, 1);
+            mbar_init(bar_q_empty + 8 * i, 1);
+        }
+        for (int i = 0; i < Cfg::NDO; ++i) {
+            mbar_init(bar_do_full + 8 * i, 1);
+            mbar_init(bar_do_empty + 8 * i, 1);
         }
         mbar_init(bar_s_full, 1);
         mbar_init(bar_s_free, 4 * BWD_NWG);
@@ -261,28 +274,32 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
                         const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
                         if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
-                        const uint32_t slot = nst % Cfg::NST, par = (nst / Cfg::NST) & 1;
-                        ++nst;
-                        ok = mbar_wait(bar_st_empty + 8 * slot, par ^ 1, abort_flag);
-                        if (!ok) break;
-                        const uint32_t st = sST + slot * Cfg::ST_STRIDE;
                         const size_t row = static_cast<size_t>(bh) * P.S + qpos;
-                        mbar_arrive_expect_tx(bar_st_full + 8 * slot, st_bytes);
-                        for (int h = 0; h < D / 64; ++h) {
-                            tma_load_2d(st + h * 16384, &tmQ, h * 64, static_cast<int>(row), bar_st_full + 8 * slot);
-                            tma_load_2d(st + Cfg::TILE + h * 16384, &tmdO, h * 64, static_cast<int>(row),
-                                        bar_st_full + 8 * slot);
-                        }
-                        bulk_load(st + 2 * Cfg::TILE, P.lse2 + row, 512, bar_st_full + 8 * slot);
-                        bulk_load(st + 2 * Cfg::TILE + 512, P.delta + row, 512, bar_st_full + 8 * slot);
-                        if (P.docs)
-                            bulk_load(st + 2 * Cfg::TILE + 1024, P.doc_start + qpos, 512, bar_st_full + 8 * slot);
+                        const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
+                        const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
+                        ++nst;
+                        ok = mbar_wait(bar_q_empty + 8 * qs, qp ^ 1, abort_flag);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(bar_q_full + 8 * qs, Cfg::TILE);
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_2d(sQ + qs * Cfg::TILE + h * 16384, &tmQ, h * 64, static_cast<int>(row),
+                                        bar_q_full + 8 * qs);
+                        ok = mbar_wait(bar_do_empty + 8 * ds, dpar ^ 1, abort_flag);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(bar_do_full + 8 * ds, Cfg::TILE + 1024);
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_2d(sdO + ds * Cfg::TILE + h * 16384, &tmdO, h * 64, static_cast<int>(row),
+                                        bar_do_full + 8 * ds);
+                        bulk_load(sLD + ds * 1024, P.lse2 + row, 512, bar_do_full + 8 * ds);
+                        bulk_load(sLD + ds * 1024 + 512, P.delta + row, 512, bar_do_full + 8 * ds);
                     }
                 }
             }
-            if (!ok) {
-                for (uint32_t n = (nst > Cfg::NST ? nst - Cfg::NST : 0); n < nst; ++n)
-                    mbar_wait_drain(bar_st_full + 8 * (n % Cfg::NST), (n / Cfg::NST) & 1);
+            if (!ok) {   // let the copies in flight land before the CTA exits (bounded waits)
+                for (uint32_t n = (nst > Cfg::NQ ? nst - Cfg::NQ : 0); n < nst; ++n)
+                    mbar_wait_drain(bar_q_full + 8 * (n % Cfg::NQ), (n / Cfg::NQ) & 1);
+                for (uint32_t n = (nst > Cfg::NDO ? nst - Cfg::NDO : 0); n < nst; ++n)
+                    mbar_wait_drain(bar_do_full + 8 * (n % Cfg::NDO), (n / Cfg::NDO) & 1);
                 if (kv_issued) mbar_wait_drain(bar_kv_full, (iter & 1));
             }
         }
@@ -293,11 +310,12 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);   // K-major A and B
             constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A tmem, B MN-major
-            constexpr uint32_t TILE16 = Cfg::TILE >> 4, ST16 = Cfg::ST_STRIDE >> 4;
+            constexpr uint32_t TILE16 = Cfg::TILE >> 4;
             const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
             // descriptor bases; k-steps and stages are constant offsets in 16-byte units
             const uint64_t dK = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
-            const uint64_t dST = sdesc_sw128(sST, 16, 1024), dSTmn = sdesc_sw128(sST, 16384, 1024);
+            const uint64_t dQk = sdesc_sw128(sQ, 16, 1024), dQmn = sdesc_sw128(sQ, 16384, 1024);
+            const uint64_t dOk = sdesc_sw128(sdO, 16, 1024), dOmn = sdesc_sw128(sdO, 16384, 1024);
             uint32_t nst = 0, iter = 0, sf_phase = 0, ae_phase = 0;
             uint32_t p_phase[BWD_NSLICE];
             for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
@@ -306,13 +324,13 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             bool ok = true, acc_busy = false, s_pending = false;
             // dV += P^T dO, dK += dS^T Q for one finished query tile.  P^T and dS^T (bf16) sit in
             // the dP^T columns: slice j at 64j (P^T) and 64j + 32 (dS^T), 16 query rows per 8 columns.
-            auto issue_products = [&](uint32_t slot, bool& first) -> bool {
+            auto issue_products = [&](uint32_t qs, uint32_t ds, bool& first) -> bool {
                 if (first && acc_busy) {   // every group has stored the previous item's dK / dV
                     if (!mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag)) return false;
                     ae_phase ^= 1;
                     acc_busy = false;
                 }
-                const uint64_t bq_mn = dSTmn + slot * ST16, bdo_mn = bq_mn + TILE16;
+                const uint64_t bq_mn = dQmn + qs * TILE16, bdo_mn = dOmn + ds * TILE16;
                 for (int j = 0; j < BWD_NSLICE; ++j) {
                     if (!mbar_wait_warp(bar_p_full + 8 * j, p_phase[j], abort_flag)) return false;
                     p_phase[j] ^= 1;
@@ -329,7 +347,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     __syncwarp();
                 }
                 first = false;
-                if (elect_one()) mma_commit(bar_st_empty + 8 * slot);
+                if (elect_one()) {
+                    mma_commit(bar_q_empty + 8 * qs);
+                    mma_commit(bar_do_empty + 8 * ds);
+                }
                 __syncwarp();
                 return true;
             };
@@ -339,7 +360,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (!ok) break;
                 tc_fence_after();
                 bool first = true, prev_live = false;
-                uint32_t prev_slot = 0;
+                uint32_t prev_qs = 0, prev_ds = 0;
                 for (int hq = 0; hq < g && ok; ++hq) {
                     for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
                          ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
@@ -348,9 +369,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
                         const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
                         if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
-                        const uint32_t slot = nst % Cfg::NST, par = (nst / Cfg::NST) & 1;
+                        const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
+                        const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
                         ++nst;
-                        ok = mbar_wait_warp(bar_st_full + 8 * slot, par, abort_flag);
+                        ok = mbar_wait_warp(bar_q_full + 8 * qs, qp, abort_flag);
                         if (!ok) break;
                         if (s_pending) {   // the previous tile's S^T / dP^T are copied out
                             ok = mbar_wait_warp(bar_s_free, sf_phase, abort_flag);
@@ -358,7 +380,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                             sf_phase ^= 1;
                         }
                         tc_fence_after();
-                        const uint64_t bq = dST + slot * ST16, bdo = bq + TILE16;
+                        const uint64_t bq = dQk + qs * TILE16, bdo = dOk + ds * TILE16;
                         // S^T of this tile while the elementwise warps still work on the previous one
                         if (elect_one()) {
 #pragma unroll
@@ -369,7 +391,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         }
                         __syncwarp();
                         // the previous tile's products read P^T / dS^T from the dP^T columns ...
-                        if (prev_live && !(ok = issue_products(prev_slot, first))) break;
+                        if (prev_live && !(ok = issue_products(prev_qs, prev_ds, first))) break;
+                        ok = mbar_wait_warp(bar_do_full + 8 * ds, dpar, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
                         // ... before this tile's dP^T overwrites them (the tensor pipe runs in order)
                         if (elect_one()) {
 #pragma unroll
@@ -382,10 +407,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         __syncwarp();
                         s_pending = true;
                         prev_live = true;
-                        prev_slot = slot;
+                        prev_qs = qs;
+                        prev_ds = ds;
                     }
                 }
-                if (ok && prev_live) ok = issue_products(prev_slot, first);
+                if (ok && prev_live) ok = issue_products(prev_qs, prev_ds, first);
                 if (!ok) break;
                 if (elect_one()) {
                     mma_commit(bar_kv_empty);
@@ -424,16 +450,16 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
                     const int cls = classify_tile(qo, dsf, dsl, it.ko);
                     if (cls == TILE_SKIP) continue;
-                    const uint32_t slot = nst % Cfg::NST;
+                    const uint32_t ds = nst % Cfg::NDO;
                     ++nst;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));
                     if (!ok) break;
                     s_phase ^= 1;
                     tc_fence_after();
-                    const uint8_t* st = smem + Cfg::ST_OFF + slot * Cfg::ST_STRIDE;
-                    const float* s_lse2 = reinterpret_cast<const float*>(st + 2 * Cfg::TILE) + 16 * wg;
-                    const float* s_delta = reinterpret_cast<const float*>(st + 2 * Cfg::TILE + 512) + 16 * wg;
-                    const int* s_ds = reinterpret_cast<const int*>(st + 2 * Cfg::TILE + 1024) + 16 * wg;
+                    const uint8_t* ld = smem + Cfg::LD_OFF + ds * 1024;
+                    const float* s_lse2 = reinterpret_cast<const float*>(ld) + 16 * wg;
+                    const float* s_delta = reinterpret_cast<const float*>(ld + 512) + 16 * wg;
+                    const int* s_ds = P.doc_start + qpos + 16 * wg;   // documents only (global, cached)
                     float sv[32], dp[32];
                     tmem_ld16f(tS, sv);
                     tmem_ld16f(tS + 64, sv + 16);
