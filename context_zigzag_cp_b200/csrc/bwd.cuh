@@ -214,9 +214,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.Hq / P.Hkv;
-    const int n2c = 2 * P.C;
-    const int nqt = n2c / 128;
-    const int half = P.C / 128;
+    const int ntq = P.S / 128;                 // query tiles, visited from the last original position down
     constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
     if (threadIdx.x == 0) {
@@ -265,15 +263,14 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                     tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                 }
-                for (int hq = 0; hq < g && ok; ++hq) {
-                    const int bh = it.b * P.Hq + it.hk * g + hq;
-                    for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
-                         ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
-                        const int qpos = qt * 128;
-                        const int qo = key_tile_orig(qr, qlt, half, P.C, P.cp);
-                        const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
-                        const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
-                        if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                for (int t = ntq - 1; t >= it.ko / 128 && ok; --t) {
+                    const int qo = t * 128;
+                    const int qpos = shard_of_orig(qo, P.C, P.cp);
+                    const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
+                    const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                    if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                    for (int hq = 0; hq < g && ok; ++hq) {
+                        const int bh = it.b * P.Hq + it.hk * g + hq;
                         const size_t row = static_cast<size_t>(bh) * P.S + qpos;
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
                         const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
@@ -361,14 +358,13 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0;
-                for (int hq = 0; hq < g && ok; ++hq) {
-                    for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
-                         ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
-                        const int qpos = qt * 128;
-                        const int qo = key_tile_orig(qr, qlt, half, P.C, P.cp);
-                        const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
-                        const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
-                        if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                for (int t = ntq - 1; t >= it.ko / 128 && ok; --t) {
+                    const int qo = t * 128;
+                    const int qpos = shard_of_orig(qo, P.C, P.cp);
+                    const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
+                    const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                    if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                    for (int hq = 0; hq < g && ok; ++hq) {
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
                         const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
                         ++nst;
@@ -441,15 +437,14 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const DkdvItem it = decode_dkdv(P, w);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int hq = 0; hq < g && ok; ++hq) {
-                for (int qt = 0, qr = 0, qlt = 0; qt < P.cp * nqt && ok;
-                     ++qt, qlt = (qlt + 1 == nqt) ? 0 : qlt + 1, qr += (qlt == 0) ? 1 : 0) {
-                    const int qpos = qt * 128;
-                    const int qo = key_tile_orig(qr, qlt, half, P.C, P.cp);
-                    const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
-                    const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
-                    const int cls = classify_tile(qo, dsf, dsl, it.ko);
-                    if (cls == TILE_SKIP) continue;
+            for (int t = ntq - 1; t >= it.ko / 128 && ok; --t) {
+                const int qo = t * 128;
+                const int qpos = shard_of_orig(qo, P.C, P.cp);
+                const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
+                const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                const int cls = classify_tile(qo, dsf, dsl, it.ko);
+                if (cls == TILE_SKIP) continue;
+                for (int hq = 0; hq < g && ok; ++hq) {
                     const uint32_t ds = nst % Cfg::NDO;
                     ++nst;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));
