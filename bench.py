@@ -158,7 +158,7 @@ class ClockSampler:
 
 # --------------------------------------------------------------------- CPU baseline (oracle)
 
-def cpu_baseline(w: synth.Workload, budget_tokens: int = 3072):
+def cpu_baseline(w: synth.Workload, budget_tokens: int = 5120):
     """The oracle, as it stands, on a bounded sample of the workload: forward and
     backward of the first `budget_tokens` tokens of one KV group (all its query
     heads), FLOPs by the same convention."""
