@@ -82,36 +82,47 @@ struct BwdParams {
     __nv_bfloat16* dv;
 };
 
-// P^T and dS^T (bf16 pairs) for 16 query columns of one key row k in the dK/dV
-// pass.  MODE 0: every column admitted; 1: column c admitted when c >= thr
-// (thr = k - first query of the 16, the causal test); 2: also k >= ds[c].
+// P^T for 16 query columns of one key row k in the dK/dV pass, in place over
+// the scores.  MODE 0: every column admitted; 1: column c admitted when
+// c >= thr (thr = k - first query of the 16, the causal test); 2: also
+// k >= ds[c] (documents).
 template <int MODE>
-__device__ __forceinline__ void dkdv_cols16(const float* sv, const float* dp, const float* s_lse2,
-                                            const float* s_delta, const int* s_ds, float scale_log2,
-                                            int thr, int k_orig, uint32_t* pk, uint32_t* dk)
+__device__ __forceinline__ void dkdv_p16(float* sv, const float* s_lse2, const int* s_ds, float scale_log2,
+                                         int thr, int k_orig)
 {
 #pragma unroll
     for (int i = 0; i < 16; i += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(s_lse2 + i);
-        const float4 d4 = *reinterpret_cast<const float4*>(s_delta + i);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
         int dsv[4] = {0, 0, 0, 0};
         if (MODE == 2) {
             const int4 q4 = *reinterpret_cast<const int4*>(s_ds + i);
             dsv[0] = q4.x; dsv[1] = q4.y; dsv[2] = q4.z; dsv[3] = q4.w;
         }
-        float p4[4], g4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int c = i + e;
             float pv = ex2_approx(fmaf(sv[c], scale_log2, -lv[e]));
             if (MODE >= 1 && c < thr) pv = 0.f;
             if (MODE == 2 && k_orig < dsv[e]) pv = 0.f;
-            p4[e] = pv;
-            g4[e] = pv * (dp[c] - dv[e]);
+            sv[c] = pv;
         }
-        pk[i / 2] = pack_bf16(p4[0], p4[1]);
-        pk[i / 2 + 1] = pack_bf16(p4[2], p4[3]);
+    }
+}
+
+// dS^T = P^T (dP^T - delta) for 16 query columns, and both packed to bf16 pairs.
+__device__ __forceinline__ void dkdv_ds16(const float* pv, const float* dp, const float* s_delta, uint32_t* pk,
+                                          uint32_t* dk)
+{
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(s_delta + i);
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float g4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) g4[e] = pv[i + e] * (dp[i + e] - dv[e]);
+        pk[i / 2] = pack_bf16(pv[i], pv[i + 1]);
+        pk[i / 2 + 1] = pack_bf16(pv[i + 2], pv[i + 3]);
         dk[i / 2] = pack_bf16(g4[0], g4[1]);
         dk[i / 2 + 1] = pack_bf16(g4[2], g4[3]);
     }
@@ -148,17 +159,18 @@ template <int D>
 struct DkdvCfg {
     static constexpr int TILE = 128 * D * 2;
     // Q tiles are needed early (S^T of the next tile is issued while the current one is
-    // still in the elementwise step), dO tiles later: three Q slots, two dO slots; each dO
-    // slot carries the tile's lse2 and delta rows (512 B each).
+    // still in the elementwise step), dO tiles later: three Q slots, each with the tile's
+    // lse2 row (512 B, used with S^T), and two dO slots, each with its delta row.
     static constexpr int NQ = 3, NDO = 2;
     static constexpr int K_OFF = 0, V_OFF = TILE;
     static constexpr int Q_OFF = 2 * TILE;
     static constexpr int DO_OFF = Q_OFF + NQ * TILE;
-    static constexpr int LD_OFF = DO_OFF + NDO * TILE;
-    static constexpr int BAR_OFF = LD_OFF + NDO * 1024;
-    // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NDO], do_empty[NDO], s_full, s_free,
-    // p_full[NSLICE], acc_full, drain, acc_empty
-    static constexpr int NBAR = 7 + 2 * NQ + 2 * NDO + BWD_NSLICE;
+    static constexpr int LQ_OFF = DO_OFF + NDO * TILE;           // lse2 rows [NQ]
+    static constexpr int LD_OFF = LQ_OFF + NQ * 512;              // delta rows [NDO]
+    static constexpr int BAR_OFF = LD_OFF + NDO * 512;
+    // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NDO], do_empty[NDO], st_ready, dp_ready,
+    // s_free, dp_free, p_full[NSLICE], acc_full, drain, acc_empty
+    static constexpr int NBAR = 9 + 2 * NQ + 2 * NDO + BWD_NSLICE;
     // the dynamic shared window starts 1024-byte aligned (checked at run time), no slack
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64;
     static constexpr int THREADS = BWD_THREADS;
@@ -200,13 +212,15 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint8_t* smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sK = sbase + Cfg::K_OFF, sV = sbase + Cfg::V_OFF;
-    const uint32_t sQ = sbase + Cfg::Q_OFF, sdO = sbase + Cfg::DO_OFF, sLD = sbase + Cfg::LD_OFF;
+    const uint32_t sQ = sbase + Cfg::Q_OFF, sdO = sbase + Cfg::DO_OFF;
+    const uint32_t sLQ = sbase + Cfg::LQ_OFF, sLD = sbase + Cfg::LD_OFF;
     const uint32_t bars = sbase + Cfg::BAR_OFF;
     const uint32_t bar_kv_full = bars, bar_kv_empty = bars + 8;
     const uint32_t bar_q_full = bars + 16, bar_q_empty = bar_q_full + 8 * Cfg::NQ;
     const uint32_t bar_do_full = bar_q_empty + 8 * Cfg::NQ, bar_do_empty = bar_do_full + 8 * Cfg::NDO;
-    const uint32_t bar_s_full = bar_do_empty + 8 * Cfg::NDO, bar_s_free = bar_s_full + 8;
-    const uint32_t bar_p_full = bar_s_free + 8;                       // [NSLICE]
+    const uint32_t bar_st_ready = bar_do_empty + 8 * Cfg::NDO, bar_dp_ready = bar_st_ready + 8;
+    const uint32_t bar_s_free = bar_dp_ready + 8, bar_dp_free = bar_s_free + 8;
+    const uint32_t bar_p_full = bar_dp_free + 8;                      // [NSLICE]
     const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
@@ -229,8 +243,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mbar_init(bar_do_full + 8 * i, 1);
             mbar_init(bar_do_empty + 8 * i, 1);
         }
-        mbar_init(bar_s_full, 1);
+        mbar_init(bar_st_ready, 1);
+        mbar_init(bar_dp_ready, 1);
         mbar_init(bar_s_free, 4 * BWD_NWG);
+        mbar_init(bar_dp_free, 4 * BWD_NWG);
         for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
@@ -277,18 +293,18 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         ++nst;
                         ok = mbar_wait(bar_q_empty + 8 * qs, qp ^ 1, abort_flag);
                         if (!ok) break;
-                        mbar_arrive_expect_tx(bar_q_full + 8 * qs, Cfg::TILE);
+                        mbar_arrive_expect_tx(bar_q_full + 8 * qs, Cfg::TILE + 512);
                         for (int h = 0; h < D / 64; ++h)
                             tma_load_2d(sQ + qs * Cfg::TILE + h * 16384, &tmQ, h * 64, static_cast<int>(row),
                                         bar_q_full + 8 * qs);
+                        bulk_load(sLQ + qs * 512, P.lse2 + row, 512, bar_q_full + 8 * qs);
                         ok = mbar_wait(bar_do_empty + 8 * ds, dpar ^ 1, abort_flag);
                         if (!ok) break;
-                        mbar_arrive_expect_tx(bar_do_full + 8 * ds, Cfg::TILE + 1024);
+                        mbar_arrive_expect_tx(bar_do_full + 8 * ds, Cfg::TILE + 512);
                         for (int h = 0; h < D / 64; ++h)
                             tma_load_2d(sdO + ds * Cfg::TILE + h * 16384, &tmdO, h * 64, static_cast<int>(row),
                                         bar_do_full + 8 * ds);
-                        bulk_load(sLD + ds * 1024, P.lse2 + row, 512, bar_do_full + 8 * ds);
-                        bulk_load(sLD + ds * 1024 + 512, P.delta + row, 512, bar_do_full + 8 * ds);
+                        bulk_load(sLD + ds * 512, P.delta + row, 512, bar_do_full + 8 * ds);
                     }
                 }
             }
@@ -384,6 +400,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
                                 mma_ss(tS, dK + off, bq + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
+                            mma_commit(bar_st_ready);
                         }
                         __syncwarp();
                         // the previous tile's products read P^T / dS^T from the dP^T columns ...
@@ -398,7 +415,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
                                 mma_ss(tdP, dVk + off, bdo + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
-                            mma_commit(bar_s_full);
+                            mma_commit(bar_dp_ready);
                         }
                         __syncwarp();
                         s_pending = true;
@@ -431,7 +448,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const uint32_t tdV = tmem + lane_off + 256 + 32 * wg, tdK = tmem + lane_off + 384 + 32 * wg;
         // packed P^T / dS^T of slice j go to dP^T columns 64j + 8wg and 64j + 32 + 8wg
         const uint32_t tPk = tmem + lane_off + 128 + 8 * wg, tDk = tPk + 32;
-        uint32_t nst = 0, s_phase = 0, a_phase = 0, sf_phase = 0;
+        uint32_t nst = 0, st_phase = 0, dp_phase = 0, a_phase = 0, df_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
             const DkdvItem it = decode_dkdv(P, w);
@@ -445,46 +462,54 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const int cls = classify_tile(qo, dsf, dsl, it.ko);
                 if (cls == TILE_SKIP) continue;
                 for (int hq = 0; hq < g && ok; ++hq) {
-                    const uint32_t ds = nst % Cfg::NDO;
+                    const uint32_t qs = nst % Cfg::NQ, ds = nst % Cfg::NDO;
                     ++nst;
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));
-                    if (!ok) break;
-                    s_phase ^= 1;
-                    tc_fence_after();
-                    const uint8_t* ld = smem + Cfg::LD_OFF + ds * 1024;
-                    const float* s_lse2 = reinterpret_cast<const float*>(ld) + 16 * wg;
-                    const float* s_delta = reinterpret_cast<const float*>(ld + 512) + 16 * wg;
+                    const float* s_lse2 = reinterpret_cast<const float*>(smem + Cfg::LQ_OFF + qs * 512) + 16 * wg;
+                    const float* s_delta = reinterpret_cast<const float*>(smem + Cfg::LD_OFF + ds * 512) + 16 * wg;
                     const int* s_ds = P.doc_start + qpos + 16 * wg;   // documents only (global, cached)
+                    // ---- S^T: copy out, release, and form P^T while dP^T is still being computed
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_st_ready, st_phase, abort_flag));
+                    if (!ok) break;
+                    st_phase ^= 1;
+                    tc_fence_after();
                     float sv[32], dp[32];
                     tmem_ld16f(tS, sv);
                     tmem_ld16f(tS + 64, sv + 16);
+                    tmem_wait_ld();
+                    reg_fence32f(sv);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_s_free);   // the MMA warp may compute the next S^T
+#pragma unroll
+                    for (int j = 0; j < BWD_NSLICE; ++j) {
+                        const int thr = k_orig - (qo + 64 * j + 16 * wg);
+                        if (cls == TILE_FULL)
+                            dkdv_p16<0>(sv + 16 * j, s_lse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                        else if (!P.docs)
+                            dkdv_p16<1>(sv + 16 * j, s_lse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                        else
+                            dkdv_p16<2>(sv + 16 * j, s_lse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                    }
+                    // ---- dP^T: copy out; every warp has its columns before packed results land there
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
+                    if (!ok) break;
+                    dp_phase ^= 1;
+                    tc_fence_after();
                     tmem_ld16f(tdP, dp);
                     tmem_ld16f(tdP + 64, dp + 16);
                     tmem_wait_ld();
-                    reg_fence32f(sv);
                     reg_fence32f(dp);
-                    // scores are in registers: the MMA warp may compute the next tile's S^T
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_s_free);
-                    // every elementwise warp has its dP^T columns before any packed result lands there
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_free, sf_phase, abort_flag));
+                    if (lane == 0) mbar_arrive(bar_dp_free);
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_free, df_phase, abort_flag));
                     if (!ok) break;
-                    sf_phase ^= 1;
+                    df_phase ^= 1;
                     tc_fence_after();
 #pragma unroll
                     for (int j = 0; j < BWD_NSLICE; ++j) {
                         uint32_t pk[8], dk[8];
-                        const int thr = k_orig - (qo + 64 * j + 16 * wg);
-                        if (cls == TILE_FULL)
-                            dkdv_cols16<0>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
-                                           s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
-                        else if (!P.docs)
-                            dkdv_cols16<1>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
-                                           s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
-                        else
-                            dkdv_cols16<2>(sv + 16 * j, dp + 16 * j, s_lse2 + 64 * j, s_delta + 64 * j,
-                                           s_ds + 64 * j, P.scale_log2, thr, k_orig, pk, dk);
+                        dkdv_ds16(sv + 16 * j, dp + 16 * j, s_delta + 64 * j, pk, dk);
                         tmem_st8(tPk + 64 * j, pk);
                         tmem_st8(tDk + 64 * j, dk);
                         tmem_wait_st();
