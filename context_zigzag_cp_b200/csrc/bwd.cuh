@@ -32,13 +32,13 @@
 namespace cpattn {
 
 // ----------------------------------------------------------------------------
-// Preprocess: delta[row] = sum_d dO*O, lse2[row] = LSE * log2(e).  One warp
+// Preprocess: delta[row] = sum_d dO*O, nlse2[row] = -LSE * log2(e).  One warp
 // per row; lane l reads 4 consecutive elements (head_dim <= 128).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                 const float* __restrict__ lse, float* __restrict__ delta,
-                float* __restrict__ lse2, int64_t rows, int D)
+                float* __restrict__ nlse2, int64_t rows, int D)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -60,7 +60,7 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __rest
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) {
             delta[row] = acc;
-            lse2[row] = __ldg(lse + row) * 1.4426950408889634f;
+            nlse2[row] = __ldg(lse + row) * -1.4426950408889634f;
         }
     }
 }
@@ -73,7 +73,7 @@ struct BwdParams {
     int32_t n_items;
     const int32_t* src;      // [cp*cp]
     const int32_t* doc_start;  // [S] shard order
-    const float* lse2;       // [B*Hq][S]
+    const float* nlse2;      // [B*Hq][S], -LSE * log2(e)
     const float* delta;      // [B*Hq][S]
     const __nv_bfloat16* q;  // [B*Hq][S][D]
     const __nv_bfloat16* dout;  // [B*Hq][S][D]
@@ -82,18 +82,54 @@ struct BwdParams {
     __nv_bfloat16* dv;
 };
 
+// Of every four column pairs in the dK/dV pass's P, this many take 2^x from
+// the FMA-pipe polynomial (exp2_poly.cuh) instead of ex2.approx.  Measured on
+// B200 (gqa32k / long128k): 0 of 4 is fastest (1 and 2 of 4 cost 2-4 %), so
+// the elementwise step is not bound by the special-function pipe.
+#ifndef CP_BWD_POLY_PAIRS
+#define CP_BWD_POLY_PAIRS 0
+#endif
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 2^x for a pair: ex2.approx, or the polynomial when poly (a constant once the
+// caller's loop is unrolled).
+__device__ __forceinline__ uint64_t exp2_pair(uint64_t x2, bool poly)
+{
+    if (poly) return exp2_poly2(x2);
+    float a, b;
+    f2_unpack(x2, a, b);
+    return f2_pack(ex2_approx(a), ex2_approx(b));
+}
+
 // P^T for 16 query columns of one key row k in the dK/dV pass, in place over
-// the scores.  MODE 0: every column admitted; 1: column c admitted when
-// c >= thr (thr = k - first query of the 16, the causal test); 2: also
-// k >= ds[c] (documents).
+// the scores: P = 2^(s * scale * log2(e) - LSE * log2(e)).  MODE 0: every
+// column admitted; 1: column c admitted when c >= thr (thr = k - first query
+// of the 16, the causal test); 2: also k >= ds[c] (documents).
 template <int MODE>
-__device__ __forceinline__ void dkdv_p16(float* sv, const float* s_lse2, const int* s_ds, float scale_log2,
+__device__ __forceinline__ void dkdv_p16(float* sv, const float* s_nlse2, const int* s_ds, float scale_log2,
                                          int thr, int k_orig)
 {
+    const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll
     for (int i = 0; i < 16; i += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(s_lse2 + i);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const uint2 l01 = *reinterpret_cast<const uint2*>(s_nlse2 + i);
+        const uint2 l23 = *reinterpret_cast<const uint2*>(s_nlse2 + i + 2);
+        const uint64_t x01 = f2_fma(f2_pack(sv[i], sv[i + 1]), sc2,
+                                    (static_cast<uint64_t>(l01.y) << 32) | l01.x);
+        const uint64_t x23 = f2_fma(f2_pack(sv[i + 2], sv[i + 3]), sc2,
+                                    (static_cast<uint64_t>(l23.y) << 32) | l23.x);
+        // pairs i/2 and i/2 + 1; pair k takes the polynomial when k % 4 < CP_BWD_POLY_PAIRS
+        const uint64_t p01 = exp2_pair(x01, ((i / 2) % 4) < CP_BWD_POLY_PAIRS);
+        const uint64_t p23 = exp2_pair(x23, ((i / 2 + 1) % 4) < CP_BWD_POLY_PAIRS);
+        float p4[4];
+        f2_unpack(p01, p4[0], p4[1]);
+        f2_unpack(p23, p4[2], p4[3]);
         int dsv[4] = {0, 0, 0, 0};
         if (MODE == 2) {
             const int4 q4 = *reinterpret_cast<const int4*>(s_ds + i);
@@ -101,11 +137,9 @@ __device__ __forceinline__ void dkdv_p16(float* sv, const float* s_lse2, const i
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const int c = i + e;
-            float pv = ex2_approx(fmaf(sv[c], scale_log2, -lv[e]));
-            if (MODE >= 1 && c < thr) pv = 0.f;
-            if (MODE == 2 && k_orig < dsv[e]) pv = 0.f;
-            sv[c] = pv;
+            if (MODE >= 1 && i + e < thr) p4[e] = 0.f;
+            if (MODE == 2 && k_orig < dsv[e]) p4[e] = 0.f;
+            sv[i + e] = p4[e];
         }
     }
 }
@@ -114,24 +148,24 @@ __device__ __forceinline__ void dkdv_p16(float* sv, const float* s_lse2, const i
 __device__ __forceinline__ void dkdv_ds16(const float* pv, const float* dp, const float* s_delta, uint32_t* pk,
                                           uint32_t* dk)
 {
+    const uint64_t m1 = f2_pack(-1.f, -1.f);
 #pragma unroll
-    for (int i = 0; i < 16; i += 4) {
-        const float4 d4 = *reinterpret_cast<const float4*>(s_delta + i);
-        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float g4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) g4[e] = pv[i + e] * (dp[i + e] - dv[e]);
+    for (int i = 0; i < 16; i += 2) {
+        const uint2 d2 = *reinterpret_cast<const uint2*>(s_delta + i);
+        const uint64_t p2 = f2_pack(pv[i], pv[i + 1]);
+        const uint64_t g2 = f2_mul(p2, f2_fma((static_cast<uint64_t>(d2.y) << 32) | d2.x, m1,
+                                              f2_pack(dp[i], dp[i + 1])));
+        float g0, g1;
+        f2_unpack(g2, g0, g1);
         pk[i / 2] = pack_bf16(pv[i], pv[i + 1]);
-        pk[i / 2 + 1] = pack_bf16(pv[i + 2], pv[i + 3]);
-        dk[i / 2] = pack_bf16(g4[0], g4[1]);
-        dk[i / 2 + 1] = pack_bf16(g4[2], g4[3]);
+        dk[i / 2] = pack_bf16(g0, g1);
     }
 }
 
 // dS (bf16 pairs) for 16 key columns of one query row in the dQ pass; with
 // MASK, column c is admitted when lo <= c <= hi.
 template <bool MASK>
-__device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, float lse2, float dlt,
+__device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, float nlse2, float dlt,
                                           float scale_log2, int lo, int hi, uint32_t* dk)
 {
 #pragma unroll
@@ -140,7 +174,7 @@ __device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, floa
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int c = i + e;
-            float pv = ex2_approx(fmaf(sv[c], scale_log2, -lse2));
+            float pv = ex2_approx(fmaf(sv[c], scale_log2, nlse2));
             if (MASK && (c < lo || c > hi)) pv = 0.f;
             d2[e] = pv * (dp[c] - dlt);
         }
@@ -160,12 +194,12 @@ struct DkdvCfg {
     static constexpr int TILE = 128 * D * 2;
     // Q tiles are needed early (S^T of the next tile is issued while the current one is
     // still in the elementwise step), dO tiles later: three Q slots, each with the tile's
-    // lse2 row (512 B, used with S^T), and two dO slots, each with its delta row.
+    // nlse2 row (512 B, used with S^T), and two dO slots, each with its delta row.
     static constexpr int NQ = 3, NDO = 2;
     static constexpr int K_OFF = 0, V_OFF = TILE;
     static constexpr int Q_OFF = 2 * TILE;
     static constexpr int DO_OFF = Q_OFF + NQ * TILE;
-    static constexpr int LQ_OFF = DO_OFF + NDO * TILE;           // lse2 rows [NQ]
+    static constexpr int LQ_OFF = DO_OFF + NDO * TILE;           // nlse2 rows [NQ]
     static constexpr int LD_OFF = LQ_OFF + NQ * 512;              // delta rows [NDO]
     static constexpr int BAR_OFF = LD_OFF + NDO * 512;
     // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NDO], do_empty[NDO], st_ready, dp_ready,
@@ -297,7 +331,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         for (int h = 0; h < D / 64; ++h)
                             tma_load_2d(sQ + qs * Cfg::TILE + h * 16384, &tmQ, h * 64, static_cast<int>(row),
                                         bar_q_full + 8 * qs);
-                        bulk_load(sLQ + qs * 512, P.lse2 + row, 512, bar_q_full + 8 * qs);
+                        bulk_load(sLQ + qs * 512, P.nlse2 + row, 512, bar_q_full + 8 * qs);
                         ok = mbar_wait(bar_do_empty + 8 * ds, dpar ^ 1, abort_flag);
                         if (!ok) break;
                         mbar_arrive_expect_tx(bar_do_full + 8 * ds, Cfg::TILE + 512);
@@ -464,7 +498,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 for (int hq = 0; hq < g && ok; ++hq) {
                     const uint32_t qs = nst % Cfg::NQ, ds = nst % Cfg::NDO;
                     ++nst;
-                    const float* s_lse2 = reinterpret_cast<const float*>(smem + Cfg::LQ_OFF + qs * 512) + 16 * wg;
+                    const float* s_nlse2 = reinterpret_cast<const float*>(smem + Cfg::LQ_OFF + qs * 512) + 16 * wg;
                     const float* s_delta = reinterpret_cast<const float*>(smem + Cfg::LD_OFF + ds * 512) + 16 * wg;
                     const int* s_ds = P.doc_start + qpos + 16 * wg;   // documents only (global, cached)
                     // ---- S^T: copy out, release, and form P^T while dP^T is still being computed
@@ -484,11 +518,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     for (int j = 0; j < BWD_NSLICE; ++j) {
                         const int thr = k_orig - (qo + 64 * j + 16 * wg);
                         if (cls == TILE_FULL)
-                            dkdv_p16<0>(sv + 16 * j, s_lse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                            dkdv_p16<0>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
                         else if (!P.docs)
-                            dkdv_p16<1>(sv + 16 * j, s_lse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                            dkdv_p16<1>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
                         else
-                            dkdv_p16<2>(sv + 16 * j, s_lse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                            dkdv_p16<2>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
                     }
                     // ---- dP^T: copy out; every warp has its columns before packed results land there
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
@@ -857,7 +891,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_qt_full);
-            const float lse2 = __ldg(P.lse2 + rowi);
+            const float nlse2 = __ldg(P.nlse2 + rowi);
             const float dlt = __ldg(P.delta + rowi);
             const int q_orig = it.qo + row;
             const int ds_q = P.docs ? __ldg(P.doc_start + it.qpos + row) : 0;
@@ -889,9 +923,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     for (int jj = 0; jj < BWD_NSLICE; ++jj) {
                         uint32_t dk[8];
                         if (cls == TILE_FULL)
-                            dq_cols16<false>(sv + 16 * jj, dp + 16 * jj, lse2, dlt, P.scale_log2, 0, 0, dk);
+                            dq_cols16<false>(sv + 16 * jj, dp + 16 * jj, nlse2, dlt, P.scale_log2, 0, 0, dk);
                         else
-                            dq_cols16<true>(sv + 16 * jj, dp + 16 * jj, lse2, dlt, P.scale_log2, lo - 64 * jj,
+                            dq_cols16<true>(sv + 16 * jj, dp + 16 * jj, nlse2, dlt, P.scale_log2, lo - 64 * jj,
                                             hi - 64 * jj, dk);
                         // the previous tile's products have read this slice buffer
                         ok = __all_sync(0xffffffffu,

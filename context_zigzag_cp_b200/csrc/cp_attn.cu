@@ -436,7 +436,7 @@ namespace {
 template <int D>
 cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, const void* o, const float* lse, const void* dout, void* dq,
-                       void* dk, void* dv, float* delta, float* lse2, cudaStream_t stream)
+                       void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream)
 {
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
     const int64_t rows = static_cast<int64_t>(B) * Hq * S;
@@ -445,7 +445,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
         LaunchScope ls(CP_K_BWD_PREP, stream);
         bwd_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
-            lse2, rows, D);
+            nlse2, rows, D);
         if (launch_status() != CP_OK) return CP_ERR_CUDA;
     }
     CUtensorMap tq, tk, tv, tdo;
@@ -466,7 +466,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.scale_log2 = P.scale * 1.4426950408889634f;
     P.src = pl->src;
     P.doc_start = pl->doc_start;
-    P.lse2 = lse2;
+    P.nlse2 = nlse2;
     P.delta = delta;
     P.q = static_cast<const __nv_bfloat16*>(q);
     P.dout = static_cast<const __nv_bfloat16*>(dout);
@@ -514,16 +514,16 @@ extern "C" cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t*
     const size_t row_bytes = round_up(size_t(rows) * 4, 256);
     if (workspace_gate(2 * row_bytes, ws, ws_bytes, &st)) return st;
     float* delta = static_cast<float*>(ws);
-    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
+    float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     cudaStream_t s = as_stream(stream);
     return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s);
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s);
 }
 
 // ---------------------------------------------------------------------------
 // cp_attn_bwd_noalloc: the backward with its per-row scratch (dot(dO, O) and
-// LSE * log2(e), fp32 each) in a fixed device array instead of a caller
+// -LSE * log2(e), fp32 each) in a fixed device array instead of a caller
 // workspace.
 // ---------------------------------------------------------------------------
 namespace {
@@ -569,9 +569,9 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != CP_OK) return st;
     float* delta = static_cast<float*>(scratch);
-    float* lse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
+    float* nlse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
     cudaStream_t s = as_stream(stream);
     return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, lse2, s);
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s);
 }

@@ -271,7 +271,7 @@ typedef enum {
     CP_K_GATHER = 3,     /* shard / unshard row gather                      */
     CP_K_FWD = 4,        /* forward attention                               */
     CP_K_MERGE = 5,      /* LSE merge                                       */
-    CP_K_BWD_PREP = 6,   /* backward: dot(dO, O), LSE * log2(e)             */
+    CP_K_BWD_PREP = 6,   /* backward: dot(dO, O), -LSE * log2(e)            */
     CP_K_BWD_DKDV = 7,   /* backward: dK, dV                                */
     CP_K_BWD_DQ = 8,     /* backward: dQ                                    */
     CP_K_SELFTEST = 9,
