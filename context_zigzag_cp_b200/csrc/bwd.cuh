@@ -214,16 +214,23 @@ struct DkdvItem {
     int bkv, b, hk, kpos, ko;
 };
 
-// Items run KV head by KV head (key tiles by ascending original position, the
-// longest first): the CTAs in flight then own neighbouring key tiles of one KV
-// head and stream the same query tiles at about the same time, so those reads
-// hit in L2.
-__device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int w)
+// A work unit is a pair of key tiles of one KV head, original tiles p and
+// nkt - 1 - p (the backward's form of the zigzag pairing): under the causal
+// mask the pair attends to nkt + 1 query tiles whatever p is, so every CTA
+// gets the same work.  A CTA takes unit blockIdx.x + i * gridDim.x and does its
+// two key tiles one after the other (half 0, then half 1); for each it visits
+// the attending query tiles by ascending original position.  The CTAs of one
+// wave then read query tiles that lie within a window of about gridDim.x tiles
+// (first halves) or are the same tile (second halves), so each query tile comes
+// from DRAM about once per wave instead of once per CTA.
+__device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int unit, int half)
 {
     DkdvItem it;
     const int nkt = P.S / 128;
-    it.bkv = w / nkt;
-    const int t = w - it.bkv * nkt;
+    const int npair = nkt / 2;
+    it.bkv = unit / npair;
+    const int pidx = unit - it.bkv * npair;
+    const int t = half ? nkt - 1 - pidx : pidx;
     it.b = it.bkv / P.Hkv;
     it.hk = it.bkv - it.b * P.Hkv;
     it.ko = t * 128;
@@ -262,7 +269,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.Hq / P.Hkv;
-    const int ntq = P.S / 128;                 // query tiles, visited from the last original position down
+    const int ntq = P.S / 128;                 // query tiles, visited by ascending original position
     constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
     if (threadIdx.x == 0) {
@@ -303,8 +310,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmdO);
             uint32_t nst = 0, iter = 0;
             bool ok = true, kv_issued = false;
-            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
-                const DkdvItem it = decode_dkdv(P, w);
+            for (int w = blockIdx.x; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
+                const DkdvItem it = decode_dkdv(P, w, iter & 1);
                 ok = mbar_wait(bar_kv_empty, (iter & 1) ^ 1, abort_flag);
                 if (!ok) break;
                 kv_issued = true;
@@ -313,7 +320,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                     tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                 }
-                for (int t = ntq - 1; t >= it.ko / 128 && ok; --t) {
+                for (int t = it.ko / 128; t < ntq && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
@@ -401,14 +408,14 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 __syncwarp();
                 return true;
             };
-            for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
-                const DkdvItem it = decode_dkdv(P, w);
+            for (int w = blockIdx.x; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
+                const DkdvItem it = decode_dkdv(P, w, iter & 1);
                 ok = mbar_wait_warp(bar_kv_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0;
-                for (int t = ntq - 1; t >= it.ko / 128 && ok; --t) {
+                for (int t = it.ko / 128; t < ntq && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
@@ -484,11 +491,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const uint32_t tPk = tmem + lane_off + 128 + 8 * wg, tDk = tPk + 32;
         uint32_t nst = 0, st_phase = 0, dp_phase = 0, a_phase = 0, df_phase = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
-            const DkdvItem it = decode_dkdv(P, w);
+        for (int w = blockIdx.x, iter = 0; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
+            const DkdvItem it = decode_dkdv(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = ntq - 1; t >= it.ko / 128 && ok; --t) {
+            for (int t = it.ko / 128; t < ntq && ok; ++t) {
                 const int qo = t * 128;
                 const int qpos = shard_of_orig(qo, P.C, P.cp);
                 const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;

@@ -483,7 +483,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
                                             DqCfg<D>::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return CP_ERR_CUDA;
-    P.n_items = B * Hkv * (S / 128);
+    P.n_items = B * Hkv * (S / 256);   // pairs of key tiles (S / 128 is even)
     {
     LaunchScope ls(CP_K_BWD_DKDV, stream);
     cp_bwd_dkdv_kernel<D><<<std::min(P.n_items, num_sms()), DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES,
