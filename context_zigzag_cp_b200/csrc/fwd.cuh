@@ -77,11 +77,20 @@ __device__ __forceinline__ int key_tile_orig(int j, int kt, int half, int C, int
     return kt < half ? j * C + kt * 128 : (2 * cp - 1 - j) * C + (kt - half) * 128;
 }
 
+// Items run GQA group by group (a group: one KV head and its g query heads);
+// inside a group, 256-row query units by descending original position (the
+// longest first) with the group's query heads fastest.  The CTAs in flight then
+// stream the K/V tiles of one KV head, which stay in L2.
 __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
 {
     FwdItem it;
-    it.bh = w % P.BH;
-    const int t = w / P.BH;
+    const int g = P.Hq / P.Hkv;
+    const int per_group = g * 2 * P.cp * P.ppc;
+    it.bkv = w / per_group;
+    const int rem = w - it.bkv * per_group;
+    const int t = rem / g, hq = rem - t * g;
+    const int b = it.bkv / P.Hkv, hk = it.bkv - b * P.Hkv;
+    it.bh = b * P.Hq + hk * g + hq;
     const int u = P.ppc - 1 - t % P.ppc;
     const int c = 2 * P.cp - 1 - t / P.ppc;  // original chunk, descending
     int half;
@@ -89,9 +98,6 @@ __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
     it.p0 = it.r * 2 * P.C + half * P.C + u * 256;
     it.qo0 = c * P.C + u * 256;
     it.ntq = (u * 256 + 256 <= P.C) ? 2 : 1;
-    const int g = P.Hq / P.Hkv;
-    const int b = it.bh / P.Hq, h = it.bh - b * P.Hq;
-    it.bkv = b * P.Hkv + h / g;
     return it;
 }
 
