@@ -60,25 +60,27 @@ def version() -> int:
 
 class Problem:
     """cp_problem_t.  ``cu_seqlens`` (int32, original order, device) turns on the
-    packed-document mask."""
+    packed-document mask; ``window`` > 0 adds a sliding window (the query at q
+    sees keys q - window < k <= q)."""
 
     def __init__(self, batch: int, seq_len: int, cp: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, rotate: str = "allgather", cu_seqlens: torch.Tensor | None = None,
-                 merge: str = "fused", softmax_scale: float = 0.0):
+                 merge: str = "fused", softmax_scale: float = 0.0, window: int = 0):
         self.cu_seqlens = cu_seqlens
+        self.window = window
         self.batch, self.seq_len, self.cp = batch, seq_len, cp
         self.num_heads, self.num_kv_heads, self.head_dim = num_heads, num_kv_heads, head_dim
         self.rotate, self.merge = rotate, merge
         self.num_docs = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
         self.c = CpProblem(batch, seq_len, cp, num_heads, num_kv_heads, head_dim,
                            _lib.ROTATE[rotate], _lib.MASK["causal" if cu_seqlens is None else "doc"],
-                           _lib.MERGE[merge], float(softmax_scale), self.num_docs, 0,
+                           _lib.MERGE[merge], float(softmax_scale), self.num_docs, int(window),
                            None if cu_seqlens is None else cu_seqlens.data_ptr())
 
     def with_merge(self, merge: str) -> "Problem":
         return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
                        self.head_dim, self.rotate, self.cu_seqlens, merge,
-                       self.c.softmax_scale)
+                       self.c.softmax_scale, self.window)
 
     @property
     def ref(self):

@@ -38,7 +38,7 @@ class CpProblem(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("rotate", ctypes.c_int32), ("mask", ctypes.c_int32), ("merge", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("num_docs", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p)]
+                ("window", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p)]
 
 
 class CpPlan(ctypes.Structure):

@@ -68,6 +68,7 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __rest
 struct BwdParams {
     int32_t B, Hq, Hkv, S, cp, C;
     int32_t docs;
+    int32_t wm1;             // sliding window - 1 (larger than S: no window)
     float scale;             // softmax scale
     float scale_log2;        // softmax scale * log2(e)
     int32_t n_items;
@@ -109,11 +110,12 @@ __device__ __forceinline__ uint64_t exp2_pair(uint64_t x2, bool poly)
 
 // P^T for 16 query columns of one key row k in the dK/dV pass, in place over
 // the scores: P = 2^(s * scale * log2(e) - LSE * log2(e)).  MODE 0: every
-// column admitted; 1: column c admitted when c >= thr (thr = k - first query
-// of the 16, the causal test); 2: also k >= ds[c] (documents).
+// column admitted; 1: column c admitted when thr <= c <= thr + wm1 (thr = k -
+// first query of the 16: the causal test and the sliding window); 2: also
+// k >= ds[c] (documents).
 template <int MODE>
 __device__ __forceinline__ void dkdv_p16(float* sv, const float* s_nlse2, const int* s_ds, float scale_log2,
-                                         int thr, int k_orig)
+                                         int thr, int wm1, int k_orig)
 {
     const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll
@@ -137,7 +139,7 @@ __device__ __forceinline__ void dkdv_p16(float* sv, const float* s_nlse2, const 
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            if (MODE >= 1 && i + e < thr) p4[e] = 0.f;
+            if (MODE >= 1 && (i + e < thr || i + e > thr + wm1)) p4[e] = 0.f;
             if (MODE == 2 && k_orig < dsv[e]) p4[e] = 0.f;
             sv[i + e] = p4[e];
         }
@@ -320,11 +322,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                     tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                 }
-                for (int t = it.ko / 128; t < ntq && ok; ++t) {
+                for (int t = it.ko / 128; t < min(ntq, (it.ko + 127 + P.wm1) / 128 + 1) && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
-                    const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
-                    const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                    const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
+                    const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
                     if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const int bh = it.b * P.Hq + it.hk * g + hq;
@@ -415,11 +417,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0;
-                for (int t = it.ko / 128; t < ntq && ok; ++t) {
+                for (int t = it.ko / 128; t < min(ntq, (it.ko + 127 + P.wm1) / 128 + 1) && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
-                    const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
-                    const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                    const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
+                    const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
                     if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
@@ -495,11 +497,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const DkdvItem it = decode_dkdv(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = it.ko / 128; t < ntq && ok; ++t) {
+            for (int t = it.ko / 128; t < min(ntq, (it.ko + 127 + P.wm1) / 128 + 1) && ok; ++t) {
                 const int qo = t * 128;
                 const int qpos = shard_of_orig(qo, P.C, P.cp);
-                const int dsf = P.docs ? __ldg(P.doc_start + qpos) : 0;
-                const int dsl = P.docs ? __ldg(P.doc_start + qpos + 127) : 0;
+                const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
+                const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
                 const int cls = classify_tile(qo, dsf, dsl, it.ko);
                 if (cls == TILE_SKIP) continue;
                 for (int hq = 0; hq < g && ok; ++hq) {
@@ -525,11 +527,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     for (int j = 0; j < BWD_NSLICE; ++j) {
                         const int thr = k_orig - (qo + 64 * j + 16 * wg);
                         if (cls == TILE_FULL)
-                            dkdv_p16<0>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                            dkdv_p16<0>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, P.wm1, k_orig);
                         else if (!P.docs)
-                            dkdv_p16<1>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                            dkdv_p16<1>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, P.wm1, k_orig);
                         else
-                            dkdv_p16<2>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, k_orig);
+                            dkdv_p16<2>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, P.wm1, k_orig);
                     }
                     // ---- dP^T: copy out; every warp has its columns before packed results land there
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
@@ -725,8 +727,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
                 const DqItem it = decode_dq(P, w);
-                const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
-                const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
+                const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
+                const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     for (int kt = 0; kt < ktiles && ok; ++kt) {
@@ -795,8 +797,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             };
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
                 const DqItem it = decode_dq(P, w);
-                const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
-                const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
+                const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
+                const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
                 ok = mbar_wait_warp(bar_qt_full, iter & 1, abort_flag);   // Q, dO rows in tensor memory
                 if (!ok) break;
                 tc_fence_after();
@@ -873,8 +875,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
             const DqItem it = decode_dq(P, w);
-            const int dsf = P.docs ? __ldg(P.doc_start + it.qpos) : 0;
-            const int dsl = P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0;
+            const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
+            const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
             const size_t rowi = static_cast<size_t>(it.bh) * P.S + it.qpos + row;
             // this row's Q and dO (bf16 pairs, columns [32wg, 32wg+32)) into tensor memory once the
             // previous item's S / dP have read the old ones
@@ -901,7 +903,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const float nlse2 = __ldg(P.nlse2 + rowi);
             const float dlt = __ldg(P.delta + rowi);
             const int q_orig = it.qo + row;
-            const int ds_q = P.docs ? __ldg(P.doc_start + it.qpos + row) : 0;
+            const int ds_q = max(P.docs ? __ldg(P.doc_start + it.qpos + row) : 0, q_orig - P.wm1);
             bool had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);

@@ -50,6 +50,7 @@ cp_status_t check_problem(const cp_problem_t* p)
     if (p->mask != CP_MASK_CAUSAL && p->mask != CP_MASK_DOC_CAUSAL) return CP_ERR_INVALID_ARG;
     if (p->merge != CP_MERGE_SEPARATE && p->merge != CP_MERGE_FUSED) return CP_ERR_INVALID_ARG;
     if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return CP_ERR_INVALID_ARG;
+    if (p->window < 0) return CP_ERR_INVALID_ARG;
     if (p->mask == CP_MASK_DOC_CAUSAL) {
         if (!p->cu_seqlens || p->num_docs < 1 || p->num_docs > p->seq_len) return CP_ERR_INVALID_ARG;
     }
@@ -77,6 +78,14 @@ cp_status_t check_plan(const cp_plan_t* pl, bool need_all)
     if (need_all && (!pl->perm || !pl->inv_perm || !pl->rank_cu_off || !pl->rank_cu || !pl->pairs))
         return CP_ERR_INVALID_ARG;
     return CP_OK;
+}
+
+// Keys visible to the query at original position q start at q - wm1 (window W:
+// wm1 = W - 1); without a window wm1 is larger than any position, so the bound
+// never binds.
+inline int32_t window_minus_one(const cp_problem_t* p)
+{
+    return p->window > 0 ? p->window - 1 : p->seq_len + 256;
 }
 
 inline float softmax_scale(const cp_problem_t* p)
@@ -200,6 +209,7 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.cp = p->cp_size;
     P.C = S / (2 * p->cp_size);
     P.docs = p->mask == CP_MASK_DOC_CAUSAL;
+    P.wm1 = window_minus_one(p);
     P.fused = p->merge == CP_MERGE_FUSED;
     P.scale_log2 = softmax_scale(p) * 1.4426950408889634f;
     P.ppc = (P.C + 255) / 256;
@@ -323,6 +333,7 @@ cp_status_t cp_plan_shards(const cp_problem_t* problem, const cp_plan_t* plan, i
     P.cp = problem->cp_size;
     P.C = P.S / (2 * P.cp);
     P.docs = problem->mask == CP_MASK_DOC_CAUSAL;
+    P.wm1 = window_minus_one(problem);
     P.num_docs = P.docs ? problem->num_docs : 1;
     P.rotate = problem->rotate;
     P.cu = problem->cu_seqlens;
@@ -462,6 +473,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.cp = p->cp_size;
     P.C = S / (2 * p->cp_size);
     P.docs = p->mask == CP_MASK_DOC_CAUSAL;
+    P.wm1 = window_minus_one(p);
     P.scale = softmax_scale(p);
     P.scale_log2 = P.scale * 1.4426950408889634f;
     P.src = pl->src;

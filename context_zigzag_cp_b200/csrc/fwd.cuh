@@ -42,6 +42,7 @@ namespace cpattn {
 struct FwdParams {
     int32_t BH, Hq, Hkv, S, cp, C;  // BH = batch * Hq
     int32_t docs;                   // 1 = packed-document mask
+    int32_t wm1;                    // sliding window - 1 (larger than S: no window)
     int32_t fused;                  // 1 = CP_MERGE_FUSED
     float scale_log2;               // softmax scale * log2(e)
     int32_t n_items, ppc;           // items, query-tile pairs per chunk
@@ -55,9 +56,10 @@ struct FwdParams {
 
 enum : int { TILE_SKIP = 0, TILE_FULL = 1, TILE_PARTIAL = 2 };
 
-// Query tile rows have original positions [qo, qo+127] and document starts
-// between dsf (first row) and dsl (last row); key tile keys [ko, ko+127].
-// A pair (q, k) is admitted when ds(q) <= k <= q.
+// Query tile rows have original positions [qo, qo+127] and first visible keys
+// (document start, raised to q - W + 1 under a sliding window) between dsf
+// (first row) and dsl (last row); key tile keys [ko, ko+127].  A pair (q, k)
+// is admitted when first(q) <= k <= q.
 __device__ __forceinline__ int classify_tile(int qo, int dsf, int dsl, int ko)
 {
     if (ko > qo + 127 || ko + 127 < dsf) return TILE_SKIP;
@@ -119,8 +121,10 @@ struct TileIter {
     int qo[2], dsf[2], dsl[2];
 };
 
-// Original start and document-start range of each query tile of an item; the
-// second tile exists only when it.ntq == 2 (no read past the item's rows).
+// Original start of each query tile of an item and the range of its rows'
+// first visible key, max(document start, q - wm1), over the tile (first row,
+// last row); the second tile exists only when it.ntq == 2 (no read past the
+// item's rows).
 __device__ __forceinline__ TileIter load_tile_iter(const FwdParams& P, const FwdItem& it)
 {
     TileIter ti;
@@ -133,6 +137,8 @@ __device__ __forceinline__ TileIter load_tile_iter(const FwdParams& P, const Fwd
             ti.dsf[x] = __ldg(P.doc_start + pr);
             ti.dsl[x] = __ldg(P.doc_start + pr + 127);
         }
+        ti.dsf[x] = max(ti.dsf[x], ti.qo[x] - P.wm1);
+        ti.dsl[x] = max(ti.dsl[x], ti.qo[x] + 127 - P.wm1);
     }
     return ti;
 }
@@ -414,7 +420,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const TileIter ti = load_tile_iter(P, it);
             const int prow = it.p0 + 128 * X + row;      // shard position of my row
             const int q_orig = ti.qo[X] + row;
-            const int ds_row = P.docs ? __ldg(P.doc_start + prow) : 0;
+            const int ds_row = max(P.docs ? __ldg(P.doc_start + prow) : 0, q_orig - P.wm1);
             float m_used = -INFINITY, l_sum = 0.f;
             bool first = true, had = false;
             for (int s = 0; s < P.cp && ok; ++s) {

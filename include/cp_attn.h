@@ -88,6 +88,10 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *   merge         cp_merge_t (forward only)
  *   softmax_scale 0 => 1/sqrt(head_dim)
  *   num_docs      documents in cu_seqlens (doc mask only)
+ *   window        0: no window.  W > 0: sliding window on top of the mask --
+ *                 the query at original position q sees only keys k with
+ *                 q - W < k <= q (and, with documents, k in q's document).
+ *                 Negative values are CP_ERR_INVALID_ARG.
  *   cu_seqlens    DEVICE int32 [num_docs+1], 0 = cu[0] < cu[1] < ... <
  *                 cu[num_docs] = S, original order; the same documents apply to
  *                 every batch entry.  NULL for the plain causal mask.  Only
@@ -107,7 +111,7 @@ typedef struct {
     int32_t merge;
     float softmax_scale;
     int32_t num_docs;
-    int32_t reserved;
+    int32_t window;
     const int32_t* cu_seqlens;
 } cp_problem_t;
 
@@ -125,7 +129,7 @@ typedef struct {
  *                                  chunks), then 2C
  *   pairs       int64 [cp]         unmasked (q, k) pairs whose query lives on
  *                                  rank r (equal across ranks for the plain
- *                                  causal mask) */
+ *                                  causal mask without a window) */
 typedef struct {
     int32_t* perm;
     int32_t* inv_perm;

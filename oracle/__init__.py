@@ -61,7 +61,7 @@ def _load():
         lib = ctypes.CDLL(build())
         I32, I64, F64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         lib.orc_doc_start.argtypes = [I32, I32, _i32p, _i32p]
-        lib.orc_plan.argtypes = [I32, I32, I32, I32, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p,
+        lib.orc_plan.argtypes = [I32, I32, I32, I32, _i32p, I32, _i32p, _i32p, _i32p, _i32p, _i32p,
                                  _i32p, _i64p]
         lib.orc_fwd_rows.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _i32p,
                                      I64, _i64p, _f64p, _f64p]
@@ -111,9 +111,10 @@ def doc_start(seq_len: int, cu_seqlens=None) -> np.ndarray:
     return ds
 
 
-def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None) -> dict:
+def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None, window: int = 0) -> dict:
     """The zigzag plan: perm, inv_perm, src, doc_start (shard order), rank_cu_off,
-    rank_cu and pairs (int64), exactly as the library's planner must produce them."""
+    rank_cu and pairs (int64), exactly as the library's planner must produce them.
+    ``window`` > 0 counts pairs under a sliding window (keys q-W < k <= q)."""
     lib = _load()
     cu = (np.zeros(1, dtype=np.int32) if cu_seqlens is None
           else np.ascontiguousarray(cu_seqlens, dtype=np.int32))
@@ -123,11 +124,22 @@ def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None) -> d
                src=np.zeros(cp * cp, np.int32), doc_start=np.zeros(S, np.int32),
                rank_cu_off=np.zeros(cp + 1, np.int32),
                rank_cu=np.zeros(3 * cp + max(nd, 1), np.int32), pairs=np.zeros(cp, np.int64))
-    _check(lib.orc_plan(S, cp, ROTATE[rotate], nd, cu, out["perm"], out["inv_perm"],
+    _check(lib.orc_plan(S, cp, ROTATE[rotate], nd, cu, int(window), out["perm"], out["inv_perm"],
                         out["src"], out["doc_start"], out["rank_cu_off"], out["rank_cu"],
                         out["pairs"]), "plan")
     out["rank_cu"] = out["rank_cu"][: out["rank_cu_off"][cp]].copy()
     return out
+
+
+def first_key(seq_len: int, cu_seqlens=None, window: int = 0) -> np.ndarray:
+    """Per original position q, the first key q attends to: its document's start,
+    raised to q - W + 1 under a sliding window of W keys (window 0: none).  Every
+    attention function here takes this array as ``ds_orig`` (keys
+    first(q) <= k <= q are unmasked)."""
+    ds = doc_start(seq_len, cu_seqlens)
+    if window and window > 0:
+        ds = np.maximum(ds, np.arange(seq_len, dtype=np.int64) - (window - 1)).astype(np.int32)
+    return ds
 
 
 def _dims(q, k):
@@ -188,14 +200,14 @@ def lse_merge(o_parts, lse_parts):
     return o, lse
 
 
-def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=None):
+def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=None, window=0):
     """The sharded computation: for every rank r, the partials against K/V shard
     src[r][s] for each step s (all steps unless ``steps`` limits them), merged in
     visit order.  Returns O [B,Hq,S,D] and LSE [B,Hq,S] in SHARD order."""
     q = _f64(q)
     B, Hq, S, D = q.shape
-    pl = plan(S, cp, rotate, cu_seqlens)
-    ds = doc_start(S, cu_seqlens)
+    pl = plan(S, cp, rotate, cu_seqlens, window)
+    ds = first_key(S, cu_seqlens, window)
     n2c = S // cp
     o = np.zeros((B * Hq, S, D), np.float64)
     lse = np.zeros((B * Hq, S), np.float64)
@@ -251,8 +263,12 @@ def bwd_dkv_keys(q, k, v, dout, keys, ds_orig=None, scale=None):
     return dk, dv
 
 
-def causal_pairs(seq_len: int, cu_seqlens=None) -> int:
-    """Number of unmasked (q, k) pairs per head: sum over documents of L(L+1)/2."""
+def causal_pairs(seq_len: int, cu_seqlens=None, window: int = 0) -> int:
+    """Number of unmasked (q, k) pairs per head: sum over documents of L(L+1)/2
+    (with a sliding window: sum over q of q - first_key(q) + 1)."""
+    if window and window > 0:
+        fk = first_key(seq_len, cu_seqlens, window).astype(np.int64)
+        return int((np.arange(seq_len, dtype=np.int64) - fk + 1).sum())
     if cu_seqlens is None:
         return seq_len * (seq_len + 1) // 2
     L = np.diff(np.asarray(cu_seqlens, dtype=np.int64))

@@ -77,14 +77,16 @@ int orc_doc_start(int32_t S, int32_t num_docs, const int32_t *cu, int32_t *ds_or
  *                     total entries.  rank r's list holds the local offsets
  *                     where a segment starts (local 0, the chunk boundary C,
  *                     and every document start inside its chunks), then 2C.
- *   pairs[r]        = number of unmasked (q, k) pairs whose query is on rank r
+ *   pairs[r]        = number of unmasked (q, k) pairs whose query is on rank r;
+ *                     with a sliding window W > 0 the query at o sees keys
+ *                     max(ds(o), o - W + 1) .. o (window 0: no window)
  * Returns ORC_EINVAL on a bad configuration.
  */
 int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int32_t *cu,
-             int32_t *perm, int32_t *inv_perm, int32_t *src, int32_t *doc_start,
+             int32_t window, int32_t *perm, int32_t *inv_perm, int32_t *src, int32_t *doc_start,
              int32_t *rank_cu_off, int32_t *rank_cu, int64_t *pairs)
 {
-    if (cp < 1 || S <= 0 || S % (2 * cp) != 0) return ORC_EINVAL;
+    if (cp < 1 || S <= 0 || S % (2 * cp) != 0 || window < 0) return ORC_EINVAL;
     if (rotate != 0 && rotate != 1) return ORC_EINVAL;
     int64_t C = S / (2 * cp);
     int32_t *ds_orig = (int32_t *)malloc(sizeof(int32_t) * (size_t)S);
@@ -110,7 +112,9 @@ int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int3
             int64_t o = orc_orig_of_local(C, cp, r, t);
             int is_start = (t == 0) || (t == C) || (ds_orig[o] == o);
             if (is_start) rank_cu[n++] = (int32_t)t;
-            cnt += o - ds_orig[o] + 1; /* keys ds(o)..o are unmasked */
+            int64_t first = ds_orig[o];
+            if (window > 0 && o - window + 1 > first) first = o - window + 1;
+            cnt += o - first + 1; /* keys first..o are unmasked */
         }
         rank_cu[n++] = (int32_t)(2 * C);
         pairs[r] = cnt;

@@ -80,6 +80,12 @@ def test_bad_enums_and_scale(lib):
     p = prob()
     p.c.merge = 5
     assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob()
+    p.c.window = -1                  # a sliding window is 0 (none) or positive
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob()
+    p.c.window = 37
+    assert fwd_query(p)[0] == _lib.CP_OK
 
 
 def test_workspace_query(lib):

@@ -374,3 +374,95 @@ def test_bf16_ulp_helper():
     x = torch.tensor([8.159, 1.2345, -0.3]).to(torch.bfloat16).double().numpy()
     ref = np.array([8.159, 1.2345, -0.3])
     assert (np.abs(x - ref) <= bf16_ulp(ref) / 2 + 1e-12).all()
+
+
+# ------------------------------------------------------------- sliding-window pins
+# A sliding window of W keys on top of the causal (and document) mask: the query
+# at q sees keys q - W < k <= q.  The oracle takes it as first_key(q) = max(doc
+# start, q - W + 1); these pins check that array and everything built on it
+# against the band mask written out directly.
+
+def band_brute_force(q, k, v, cu, window, scale):
+    """Explicit softmax over the mask k <= q, k > q - W, k in q's document."""
+    B, Hq, S, D = q.shape
+    g = Hq // k.shape[1]
+    qi = np.arange(S)[:, None]
+    ki = np.arange(S)[None, :]
+    doc = np.zeros(S, np.int64) if cu is None else np.searchsorted(np.asarray(cu), np.arange(S), side="right") - 1
+    mask = (ki <= qi) & (ki > qi - window) & (doc[ki] == doc[qi])
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, S))
+    for b in range(B):
+        for h in range(Hq):
+            s = np.where(mask, scale * q[b, h] @ k[b, h // g].T, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            o[b, h] = (e / e.sum(axis=1, keepdims=True)) @ v[b, h // g]
+            lse[b, h] = m[:, 0] + np.log(e.sum(axis=1))
+    return o, lse, int(mask.sum())
+
+
+@pytest.mark.parametrize("Hq,Hkv,S,D,W,docs", [(2, 2, 32, 8, 5, None), (4, 2, 48, 4, 13, [0, 9, 10, 48]),
+                                               (3, 1, 33, 5, 1, [0, 20, 33]), (2, 1, 40, 8, 40, None)])
+def test_window_brute_force(Hq, Hkv, S, D, W, docs):
+    q, k, v = rnd((1, Hq, S, D), 41), rnd((1, Hkv, S, D), 42), rnd((1, Hkv, S, D), 43)
+    cu = None if docs is None else np.array(docs, np.int32)
+    o, lse = oracle.fwd(q, k, v, oracle.first_key(S, cu, W))
+    bo, bl, npairs = band_brute_force(q, k, v, cu, W, 1 / math.sqrt(D))
+    np.testing.assert_allclose(o, bo, atol=1e-12)
+    np.testing.assert_allclose(lse, bl, atol=1e-12)
+    assert oracle.causal_pairs(S, cu, W) == npairs
+    if S % 2 == 0:   # the zigzag plan needs S divisible by 2 * cp
+        assert int(oracle.plan(S, 1, "allgather", cu, W)["pairs"].sum()) == npairs
+
+
+def test_window_one_closed_form():
+    """W = 1: every query sees only itself, so O = V[q] and LSE = scale * q.k_q."""
+    S, D = 64, 16
+    q, k, v = rnd((1, 4, S, D), 44), rnd((1, 2, S, D), 45), rnd((1, 2, S, D), 46)
+    o, lse = oracle.fwd(q, k, v, oracle.first_key(S, None, 1))
+    sc = 1 / math.sqrt(D)
+    for h in range(4):
+        np.testing.assert_allclose(o[0, h], v[0, h // 2], atol=1e-14)
+        np.testing.assert_allclose(lse[0, h], sc * (q[0, h] * k[0, h // 2]).sum(-1), atol=1e-13)
+
+
+def test_window_wider_than_sequence_is_causal():
+    cu = np.array([0, 100, 256], np.int32)
+    assert np.array_equal(oracle.first_key(256, cu, 256), oracle.doc_start(256, cu))
+    assert np.array_equal(oracle.plan(256, 4, "ring", cu, 300)["pairs"], oracle.plan(256, 4, "ring", cu)["pairs"])
+
+
+@pytest.mark.parametrize("cp,rotate,W", [(2, "allgather", 37), (4, "ring", 100)])
+def test_window_sharded_equals_unsharded(cp, rotate, W):
+    S, D = 256, 8
+    cu = np.array([0, 70, 71, 256], np.int32)
+    q, k, v = rnd((1, 4, S, D), 47), rnd((1, 2, S, D), 48), rnd((1, 2, S, D), 49)
+    o, lse = oracle.fwd(q, k, v, oracle.first_key(S, cu, W))
+    so, sl = oracle.cp_fwd(q, k, v, cp, rotate, cu, window=W)
+    perm = oracle.plan(S, cp, rotate, cu, W)["perm"]
+    np.testing.assert_allclose(so, o[:, :, perm], atol=1e-12)
+    np.testing.assert_allclose(sl, lse[:, :, perm], atol=1e-12)
+
+
+def test_window_bwd_finite_differences():
+    B, Hq, Hkv, S, D, W = 1, 2, 1, 16, 8, 4
+    q, k, v = rnd((B, Hq, S, D), 51), rnd((B, Hkv, S, D), 52), rnd((B, Hkv, S, D), 53)
+    dout = rnd((B, Hq, S, D), 54)
+    ds = oracle.first_key(S, [0, 9, 16], W)
+    o, lse = oracle.fwd(q, k, v, ds)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds)
+    eps = 1e-6
+    g = np.random.default_rng(55)
+    for name, x, gx in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(10):
+            idx = tuple(int(g.integers(0, n)) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], dout, ds)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], dout, ds)
+            assert abs((lp - lm) / (2 * eps) - gx[idx]) < 1e-6, (name, idx)
