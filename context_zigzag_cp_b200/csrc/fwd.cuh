@@ -143,12 +143,20 @@ __device__ __forceinline__ TileIter load_tile_iter(const FwdParams& P, const Fwd
     return ti;
 }
 
+// Of every four column pairs of an unmasked tile, this many take 2^x from the
+// software exp2 on the FMA pipe (exp2_poly.cuh), the rest from ex2.approx.
+// Measured on B200 (gqa32k, long128k): 0 is fastest; 1 of 4 costs 1-2 %, 2 of
+// 4 costs 3-5 %, so the special-function pipe does not set the forward's pace.
+#ifndef CP_FWD_POLY_PAIRS
+#define CP_FWD_POLY_PAIRS 0
+#endif
+
 // Exponentials of one query row's 128 scores (log2 domain, reference max msub),
 // packed to bf16 pairs and stored over the first 64 columns of the row's S
-// region; returns the fp32 row sum.  With SOFT, every fourth pair of columns
-// uses the software exp2 on the FMA pipe (only for unmasked tiles, whose
-// arguments are finite), the rest the hardware ex2.
-template <bool SOFT>
+// region; returns the fp32 row sum.  NSOFT of every four pairs of columns use
+// the software exp2 on the FMA pipe (only for unmasked tiles, whose arguments
+// are finite), the rest the hardware ex2.
+template <int NSOFT>
 __device__ __forceinline__ float exp_pack_store(const float* sf, float scale_log2, float msub,
                                                 uint32_t tS)
 {
@@ -162,7 +170,7 @@ __device__ __forceinline__ float exp_pack_store(const float* sf, float scale_log
         for (int i = 0; i < 32; ++i) {
             const uint64_t x2 = f2_fma(f2_pack(sf[64 * h + 2 * i], sf[64 * h + 2 * i + 1]), sl2, nm);
             uint64_t p2;
-            if (SOFT && (i & 3) == 3) {
+            if ((i & 3) >= 4 - NSOFT) {
                 p2 = exp2_poly2(x2);
             } else {
                 float a, b;
@@ -480,7 +488,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         }
                     }
                     const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-                    const float rs = exp_pack_store<false>(sf, P.scale_log2, msub, tS);
+                    const float rs = cls == TILE_FULL
+                                         ? exp_pack_store<CP_FWD_POLY_PAIRS>(sf, P.scale_log2, msub, tS)
+                                         : exp_pack_store<0>(sf, P.scale_log2, msub, tS);
                     l_sum = l_sum * alpha + rs;
                     tmem_wait_st();
                     tc_fence_before();
