@@ -164,23 +164,28 @@ __device__ __forceinline__ void dkdv_ds16(const float* pv, const float* dp, cons
     }
 }
 
-// dS (bf16 pairs) for 16 key columns of one query row in the dQ pass; with
-// MASK, column c is admitted when lo <= c <= hi.
+// dS (bf16 pairs) for 16 key columns of one query row in the dQ pass, with
+// packed f32x2 arithmetic; with MASK, column c is admitted when lo <= c <= hi.
 template <bool MASK>
 __device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, float nlse2, float dlt,
                                           float scale_log2, int lo, int hi, uint32_t* dk)
 {
+    const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nl2 = f2_pack(nlse2, nlse2);
+    const uint64_t nd2 = f2_pack(-dlt, -dlt);
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-        float d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int c = i + e;
-            float pv = ex2_approx(fmaf(sv[c], scale_log2, nlse2));
-            if (MASK && (c < lo || c > hi)) pv = 0.f;
-            d2[e] = pv * (dp[c] - dlt);
+        const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sc2, nl2);
+        float a, b;
+        f2_unpack(x2, a, b);
+        a = ex2_approx(a);
+        b = ex2_approx(b);
+        if (MASK) {
+            if (i < lo || i > hi) a = 0.f;
+            if (i + 1 < lo || i + 1 > hi) b = 0.f;
         }
-        dk[i / 2] = pack_bf16(d2[0], d2[1]);
+        const uint64_t g2 = f2_mul(f2_pack(a, b), f2_add(f2_pack(dp[i], dp[i + 1]), nd2));
+        f2_unpack(g2, a, b);
+        dk[i / 2] = pack_bf16(a, b);
     }
 }
 
