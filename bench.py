@@ -200,12 +200,14 @@ KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_dkdv": 6.0, "bwd_dq": 2.0}   # x D*Hq*pair
 
 # DRAM bytes (read + write) per launch from one ncu capture of the full-size workload
 # (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass; profiles/dram_bytes_long128k.md).
-# A figure is reported only while the kernel's source is the one it was taken on
-# (first 16 hex digits of the file's sha256); after any change it reads as null.
+# A figure is reported only while the kernel's source is the one it was taken on:
+# first 16 hex digits of the sha256 of the file's code lines (text after "//" and
+# blank lines dropped, so comment edits keep it); after any code change it reads
+# as null.
 MEASURED_TRAFFIC = {
     ("long128k", "allgather", "bwd_dkdv"): {"bytes": 85.58e9 + 0.548e9,
                                              "src": "context_zigzag_cp_b200/csrc/bwd.cuh",
-                                             "sha256_16": "54c0db54196ff756"},
+                                             "sha256_16": "d78ed47e4722ddef"},
 }
 
 
@@ -216,11 +218,19 @@ def measured_traffic(workload: str, rotate: str, kernel: str):
         return None
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), rec["src"])
     try:
-        with open(path, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        digest = code_digest(path)
     except OSError:
         return None
     return rec["bytes"] if digest == rec["sha256_16"] else None
+
+
+def code_digest(path: str) -> str:
+    """sha256 (16 hex digits) of a source file's code: each line cut at "//" and
+    stripped, empty lines dropped."""
+    import hashlib
+    with open(path, encoding="utf-8") as f:
+        lines = [ln.split("//", 1)[0].strip() for ln in f]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()[:16]
 
 
 def run_native(args, w, rank, world, local_rank):

@@ -1,28 +1,29 @@
-// Backward kernels.  Gradients of causal (optionally packed-document) attention
-// from the saved final LSE, with P = exp(scale q.k - LSE_q) recomputed on the
-// fly:  D_q = dO_q . O_q,  dV_k = sum_q P dO_q,  dS = P (dO_q . v_k - D_q),
-// dQ_q = scale sum_k dS k_k,  dK_k = scale sum_q dS q_q.
+// Backward kernels.  Gradients of causal (optionally packed-document, optionally
+// sliding-window) attention from the saved final LSE, with P = exp(scale q.k -
+// LSE_q) recomputed on the fly:  D_q = dO_q . O_q,  dV_k = sum_q P dO_q,
+// dS = P (dO_q . v_k - D_q),  dQ_q = scale sum_k dS k_k,  dK_k = scale sum_q dS q_q.
 //
 // Two deterministic passes, no atomics:
-//   * bwd_prep_kernel: D (fp32) and LSE * log2(e) per row.
-//   * cp_bwd_dkdv_kernel (KV-tile major): one CTA owns a 128-key tile of KV
-//     head j and loops over every query head of its group and every virtual
-//     rank's query tile that attends to it (the single-GPU form of handing
-//     dK_j / dV_j back around the ring), accumulating dK and dV in tensor
-//     memory:  S^T = K Q^T,  dP^T = V dO^T  ->  P^T, dS^T (bf16, tensor memory)
-//     ->  dV += P^T dO,  dK += dS^T Q.
+//   * bwd_prep_kernel: D (fp32) and -LSE * log2(e) per row.
+//   * cp_bwd_dkdv_kernel (KV-tile major): a CTA takes a zigzag pair of 128-key
+//     tiles of one KV head and, for each, visits every query head of its group
+//     and every virtual rank's query tile that attends to it (the single-GPU
+//     form of handing dK_j / dV_j back around the ring), accumulating dK and dV
+//     in tensor memory:  S^T = K Q^T,  dP^T = V dO^T  ->  P^T, dS^T (bf16,
+//     written into the dP^T columns)  ->  dV += P^T dO,  dK += dS^T Q.
 //   * cp_bwd_dq_kernel (query-tile major, visiting the K/V shards in the plan's
-//     order like the forward):  S = Q K^T,  dP = dO V^T  ->  dS (bf16, tensor
-//     memory)  ->  dQ += dS K.
+//     order like the forward; Q and dO rows held in tensor memory):  S = Q K^T,
+//     dP = dO V^T  ->  dS (bf16, shared memory)  ->  dQ += dS K.
 // In both passes the elementwise step runs on four warpgroups (a thread owns
-// one TMEM lane = one row) over the 128 score columns in two 64-column slices:
-// in each slice warpgroup w takes 16 columns, reads them, and writes its bf16
-// results over the first 8 of them (only columns it has read itself, so no
-// warp overwrites another's input).  All four warpgroups finish slice 0 before
-// slice 1, and the MMA warp issues slice 0's products (a 64-deep part of the
-// K dimension) while slice 1 is computed.
+// one TMEM lane = one row), each taking 16 columns of each 64-column slice of
+// the 128 score columns.  The warps copy their scores out of tensor memory and
+// release it at once, so the MMA warp computes the next tile's scores while
+// this tile's elementwise step runs; all four warpgroups finish slice 0 before
+// slice 1, and the MMA warp issues slice 0's products (a 64-deep part of the K
+// dimension) while slice 1 is computed.
 // Each 128-row tile lives in one zigzag chunk, so original positions are
-// linear inside a tile and the causal / document tests are per-tile ranges.
+// linear inside a tile and the causal / document / window tests are per-tile
+// ranges.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -476,7 +477,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (!ok) break;
                 if (elect_one()) {
                     mma_commit(bar_kv_empty);
-                    if (!first) mma_commit(bar_acc_full);   // the softmax groups wait only if they had a tile
+                    if (!first) mma_commit(bar_acc_full);   // the elementwise groups wait only if they had a tile
                 }
                 __syncwarp();
                 acc_busy = acc_busy || !first;

@@ -1,17 +1,18 @@
-// Forward kernel: causal (optionally packed-document) attention of every
-// virtual rank's query shard against the K/V shards in the plan's visit order.
+// Forward kernel: causal (optionally packed-document, optionally sliding-window)
+// attention of every virtual rank's query shard against the K/V shards in the
+// plan's visit order.
 //
 // Work item = (batch*head, a pair of adjacent 128-row query tiles inside one
-// zigzag chunk).  Items are ordered by descending original query position, so
-// the longest items start first, and are dealt round-robin to one persistent
-// CTA per SM.
+// zigzag chunk).  Items run GQA group by group; inside a group by descending
+// original query position (the longest items start first) with the group's
+// query heads fastest, dealt round-robin to one persistent CTA per SM.
 //
 // Warp roles (384 threads = three warpgroups):
 //   warps 0-3  softmax group 0 (query tile 0): one TMEM lane = one query row
 //   warps 4-7  softmax group 1 (query tile 1)
 //   warp 8     TMA producer: Q tiles, then K and V tiles through a ring of
 //              shared-memory slots
-//   warp 9     MMA issuer (one thread) + tensor-memory owner
+//   warp 9     MMA issuer (one elected lane per group of MMAs) + tensor-memory owner
 //   warps 10-11 idle
 // The block launches with 168 registers per thread; the softmax warpgroups
 // raise theirs to 200 and the producer/MMA warpgroup drops to 104
@@ -20,7 +21,7 @@
 // O1 [384,384+D).  P is written back as bf16 over the first 64 columns of its
 // S region and used as the A operand of O += P V straight from tensor memory.
 //
-// Per KV tile t the MMA thread issues, for each query tile X that the tile
+// Per KV tile t the MMA warp issues, for each query tile X that the tile
 // does not skip:  O_X += P_X(prev) V(prev)  then  S_X = Q_X K_t^T, so the
 // tensor core computes S for one query tile while the other group runs its
 // softmax (ping-pong between the two groups).
