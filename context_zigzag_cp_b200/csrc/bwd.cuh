@@ -692,7 +692,6 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n2c = 2 * P.C;
-    const int ktiles = n2c / 128;
     const int half = P.C / 128;
     constexpr int PROD_WARP = 4 * BWD_NWG, MMA_WARP = 4 * BWD_NWG + 1;
 
@@ -737,7 +736,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                    const KtSpan ks = kt_span(j, dsf, it.qo + 127, half, P.C, P.cp);
+                    for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int kpos = j * n2c + kt * 128;
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
@@ -812,7 +812,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 uint32_t prev_kslot = 0;
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                    const KtSpan ks = kt_span(j, dsf, it.qo + 127, half, P.C, P.cp);
+                    for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
@@ -913,7 +914,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             bool had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
-                for (int kt = 0; kt < ktiles && ok; ++kt) {
+                const KtSpan ks = kt_span(j, dsf, it.qo + 127, half, P.C, P.cp);
+                for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                     const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                     const int cls = classify_tile(it.qo, dsf, dsl, ko);
                     if (cls == TILE_SKIP) continue;

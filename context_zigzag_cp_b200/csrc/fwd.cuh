@@ -84,6 +84,32 @@ __device__ __forceinline__ int key_tile_orig(int j, int kt, int half, int C, int
 // inside a group, 256-row query units by descending original position (the
 // longest first) with the group's query heads fastest.  The CTAs in flight then
 // stream the K/V tiles of one KV head, which stay in L2.
+// The key tiles of shard j (kt < 2C/128: the first C/128 tiles are chunk j,
+// the rest chunk 2cp-1-j) that can hold a key in [lo, hi]: kt in [a0, b0) or
+// [a1, b1).  Loops visit only these (for (kt = kt_first(r); kt < r.b1;
+// kt = kt_next(r, kt))); the tiles outside are skip tiles under every mask, so
+// walking them one by one would only cost time (much of it under a sliding
+// window).  An empty first range is [0, 0), an empty second one [half, half).
+struct KtSpan {
+    int a0, b0, a1, b1;
+};
+
+__device__ __forceinline__ KtSpan kt_span(int j, int lo, int hi, int half, int C, int cp)
+{
+    KtSpan r;
+    const int c0 = j * C, c1 = (2 * cp - 1 - j) * C;
+    r.a0 = max(0, (lo - c0) >> 7);                 // arithmetic shift: floor division by 128
+    r.b0 = min(half, ((hi - c0) >> 7) + 1);
+    if (r.a0 >= r.b0) r.a0 = r.b0 = 0;
+    r.a1 = half + max(0, (lo - c1) >> 7);
+    r.b1 = half + min(half, ((hi - c1) >> 7) + 1);
+    if (r.a1 >= r.b1) r.a1 = r.b1 = half;
+    return r;
+}
+
+__device__ __forceinline__ int kt_first(const KtSpan& r) { return r.a0 < r.b0 ? r.a0 : r.a1; }
+__device__ __forceinline__ int kt_next(const KtSpan& r, int kt) { return kt + 1 == r.b0 ? r.a1 : kt + 1; }
+
 __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
 {
     FwdItem it;
@@ -212,7 +238,6 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n2c = 2 * P.C;
-    const int ktiles = n2c / 128;
     const int half = P.C / 128;
 
     if (threadIdx.x == 0) {
@@ -258,7 +283,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                     it.bh * P.S + it.p0 + 128 * x, bar_q_full);
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1, half, P.C, P.cp);
+                    for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int kpos = j * n2c + kt * 128;
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
@@ -309,7 +335,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 int n_tiles = 0;
                 for (int s = 0; s < P.cp; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    for (int kt = 0; kt < ktiles; ++kt) {
+                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1, half, P.C, P.cp);
+                    for (int kt = kt_first(ks); kt < ks.b1; kt = kt_next(ks, kt)) {
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         if (classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP ||
                             (it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP))
@@ -358,7 +385,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    for (int kt = 0; kt < ktiles && ok; ++kt) {
+                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1, half, P.C, P.cp);
+                    for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                         const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
                         const bool v1 = it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP;
@@ -434,7 +462,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool first = true, had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
-                for (int kt = 0; kt < ktiles && ok; ++kt) {
+                const KtSpan ks = kt_span(j, ti.dsf[X], ti.qo[X] + 127, half, P.C, P.cp);
+                for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                     const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                     const int cls = classify_tile(ti.qo[X], ti.dsf[X], ti.dsl[X], ko);
                     if (cls == TILE_SKIP) continue;
