@@ -29,6 +29,7 @@
 #include "ptx.cuh"
 #include "zigzag.cuh"
 #include "fwd.cuh"
+#include "plan.cuh"
 
 namespace cpattn {
 
@@ -75,6 +76,8 @@ struct BwdParams {
     int32_t n_items;
     const int32_t* src;      // [cp*cp]
     const int32_t* doc_start;  // [S] shard order
+    const int32_t* cu;       // [num_docs+1] document offsets, original order (documents only)
+    int32_t num_docs;
     const float* nlse2;      // [B*Hq][S], -LSE * log2(e)
     const float* delta;      // [B*Hq][S]
     const __nv_bfloat16* q;  // [B*Hq][S][D]
@@ -193,6 +196,18 @@ __device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, floa
 // ============================================================================
 // dK / dV pass
 // ============================================================================
+// One past the last query tile that can attend to the key tile at original ko:
+// queries come at or after the key (the loop starts at ko's tile), no later than
+// the window allows, and inside the document of the tile's last key.
+__device__ __forceinline__ int dkdv_last_tile(const BwdParams& P, int ko, int ntq)
+{
+    int t_end = min(ntq, (ko + 127 + P.wm1) / 128 + 1);
+    if (P.docs) {
+        const int de = __ldg(P.cu + doc_index(P.cu, P.num_docs, ko + 127) + 1);
+        t_end = min(t_end, (de - 1) / 128 + 1);
+    }
+    return t_end;
+}
 constexpr int BWD_NWG = 4;                       // elementwise warpgroups
 constexpr int BWD_THREADS = (BWD_NWG + 1) * 128; // + producer / MMA warpgroup
 constexpr int BWD_NSLICE = 2;                    // 64-column slices of a 128-column score tile
@@ -328,7 +343,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                     tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                 }
-                for (int t = it.ko / 128; t < min(ntq, (it.ko + 127 + P.wm1) / 128 + 1) && ok; ++t) {
+                for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
@@ -423,7 +438,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0;
-                for (int t = it.ko / 128; t < min(ntq, (it.ko + 127 + P.wm1) / 128 + 1) && ok; ++t) {
+                for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
@@ -503,7 +518,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const DkdvItem it = decode_dkdv(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = it.ko / 128; t < min(ntq, (it.ko + 127 + P.wm1) / 128 + 1) && ok; ++t) {
+            for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                 const int qo = t * 128;
                 const int qpos = shard_of_orig(qo, P.C, P.cp);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);

@@ -478,6 +478,8 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.scale_log2 = P.scale * 1.4426950408889634f;
     P.src = pl->src;
     P.doc_start = pl->doc_start;
+    P.cu = p->cu_seqlens;
+    P.num_docs = P.docs ? p->num_docs : 0;
     P.nlse2 = nlse2;
     P.delta = delta;
     P.q = static_cast<const __nv_bfloat16*>(q);
