@@ -268,7 +268,11 @@ def run_native(args, w, rank, world, local_rank):
     st = cz.get_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
-    pairs = int(plan.pairs.sum().item()) * w.batch
+    pairs_rank = plan.pairs.cpu().to(torch.float64)
+    pairs = int(pairs_rank.sum().item()) * w.batch
+    # unmasked pairs per virtual rank, max over mean: 1 for the plain causal zigzag;
+    # packed documents leave the sequence-level zigzag unbalanced
+    rank_imbalance = float(pairs_rank.max() / pairs_rank.mean())
     fwd_flops = 4.0 * w.head_dim * w.num_heads * pairs
     step_flops = 3.0 * fwd_flops
 
@@ -398,6 +402,7 @@ def run_native(args, w, rank, world, local_rank):
             "step_frac_of_peak": round(value / world / peaks["bf16_sustained"], 4),
             "peak_source": peaks["source"],
             "pairs": pairs,
+            "rank_pairs_max_over_mean": round(rank_imbalance, 4),
             "kernels": kernels,
             "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
