@@ -130,10 +130,16 @@ __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
     return it;
 }
 
+// K/V ring slots of the forward at head_dim 128: 5 (Q tiles 64 KB + ring 160 KB
+// fit the 227 KB a CTA may use); measured 3.5 % faster than 4 at gqa32k.
+#ifndef CP_FWD_NSLOT128
+#define CP_FWD_NSLOT128 5
+#endif
+
 template <int D>
 struct FwdCfg {
     static constexpr int TILE_BYTES = 128 * D * 2;      // one 128-row bf16 tile
-    static constexpr int NSLOT = (D == 128) ? 4 : 8;    // K/V ring slots
+    static constexpr int NSLOT = (D == 128) ? CP_FWD_NSLOT128 : 8;   // K/V ring slots
     static constexpr int Q_OFF = 0;                     // Q0, Q1
     static constexpr int KV_OFF = 2 * TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
