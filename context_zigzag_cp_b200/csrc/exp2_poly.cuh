@@ -1,5 +1,7 @@
-// Software 2^x on the FMA pipe, used for a share of the forward kernel's
-// exponentials so that the special-function unit is not the bottleneck.
+// Software 2^x on the FMA pipe, for moving a share of the attention kernels'
+// exponentials off the special-function unit (build knobs CP_FWD_POLY_PAIRS and
+// CP_BWD_POLY_PAIRS, off by default: on B200 that share measured slower), and
+// checked against the hardware ex2 by cp_selftest_exp2.
 //
 // Method: Cody & Waite range reduction, x = j + f with j = round(x) and
 // f in [-1/2, 1/2], then 2^x = 2^j * p(f), where p is the degree-3 polynomial

@@ -171,8 +171,9 @@ CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan
                        const int64_t* buf_outer, const int64_t* buf_row_bytes, void* stream);
 
 /*
- * cp_attn_fwd -- causal (optionally packed-document) attention of every
- * virtual rank's query shard against the K/V shards in the plan's visit order,
+ * cp_attn_fwd -- causal (optionally packed-document, optionally sliding-window)
+ * attention of every virtual rank's query shard against the K/V shards in the
+ * plan's visit order,
  * combined into the exact unsharded result (concept guide, "So how does it
  * work?": local attention, then every other shard, then combine).
  *   q     bf16 [B][Hq][S][D]  shard order
@@ -180,8 +181,8 @@ CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan
  *   o     bf16 [B][Hq][S][D]  output, shard order
  *   lse   fp32 [B][Hq][S]     output, natural-log LSE of the scaled scores
  * Supported: head_dim 64 or 128; C = S/(2cp) a multiple of 128.
- * Workspace: CP_MERGE_SEPARATE needs cp fp32 partial (O, LSE) sets plus a
- * small header; CP_MERGE_FUSED needs only the header.
+ * Workspace: CP_MERGE_SEPARATE needs cp fp32 partial (O, LSE) sets (each
+ * region rounded up to 256 bytes); CP_MERGE_FUSED needs none (0 bytes).
  * Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_WORKSPACE, CP_ERR_CUDA.
  */
 CP_API cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
@@ -197,7 +198,9 @@ CP_API cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* pla
  *   q, k, v, o, dout  bf16, shard order (o and lse from cp_attn_fwd)
  *   dq                bf16 [B][Hq][S][D]  output
  *   dk, dv            bf16 [B][Hkv][S][D] output
- * Workspace: an fp32 dQ accumulator, the per-row dot(dO, O), and a header.
+ * Workspace: two fp32 values per query row, dot(dO, O) and -LSE * log2(e)
+ * (each array rounded up to 256 bytes); dQ needs no accumulator, the
+ * backward runs as two deterministic passes.
  * Errors: as cp_attn_fwd.
  */
 CP_API cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
