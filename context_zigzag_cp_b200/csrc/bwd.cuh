@@ -168,27 +168,36 @@ __device__ __forceinline__ void dkdv_ds16(const float* pv, const float* dp, cons
     }
 }
 
-// dS (bf16 pairs) for 16 key columns of one query row in the dQ pass, with
-// packed f32x2 arithmetic; with MASK, column c is admitted when lo <= c <= hi.
+// P for 16 key columns of one query row in the dQ pass, in place over the
+// scores, with packed f32x2 arithmetic; with MASK, column c is admitted when
+// lo <= c <= hi.
 template <bool MASK>
-__device__ __forceinline__ void dq_cols16(const float* sv, const float* dp, float nlse2, float dlt,
-                                          float scale_log2, int lo, int hi, uint32_t* dk)
+__device__ __forceinline__ void dq_p16(float* sv, float nlse2, float scale_log2, int lo, int hi)
 {
     const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nl2 = f2_pack(nlse2, nlse2);
-    const uint64_t nd2 = f2_pack(-dlt, -dlt);
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-        const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sc2, nl2);
         float a, b;
-        f2_unpack(x2, a, b);
+        f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), sc2, nl2), a, b);
         a = ex2_approx(a);
         b = ex2_approx(b);
         if (MASK) {
             if (i < lo || i > hi) a = 0.f;
             if (i + 1 < lo || i + 1 > hi) b = 0.f;
         }
-        const uint64_t g2 = f2_mul(f2_pack(a, b), f2_add(f2_pack(dp[i], dp[i + 1]), nd2));
-        f2_unpack(g2, a, b);
+        sv[i] = a;
+        sv[i + 1] = b;
+    }
+}
+
+// dS = P (dP - delta) for 16 key columns, packed to bf16 pairs.
+__device__ __forceinline__ void dq_ds16(const float* pv, const float* dp, float dlt, uint32_t* dk)
+{
+    const uint64_t nd2 = f2_pack(-dlt, -dlt);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        float a, b;
+        f2_unpack(f2_mul(f2_pack(pv[i], pv[i + 1]), f2_add(f2_pack(dp[i], dp[i + 1]), nd2)), a, b);
         dk[i / 2] = pack_bf16(a, b);
     }
 }
@@ -637,22 +646,22 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 // ============================================================================
 // The query tile's Q and dO rows sit in tensor memory (the A operands of S and
 // dP, written by the elementwise warps once per item), so shared memory holds
-// a deep K/V ring.  The elementwise warps copy S and dP out of tensor memory
-// first and release it (s_free), so the MMA warp computes the next key tile's
-// S and dP while dS of this one is formed.  dS goes to shared memory (bf16,
-// the K-major A operand of dQ += dS K), one 16 KB buffer per 64-key slice.
+// a deep K/V ring.  Same schedule as the dK/dV pass: the elementwise warps copy
+// S out and release it (s_free), so the MMA warp computes the next key tile's S
+// at once; they form P while the previous tile's products and this tile's dP
+// are on the tensor core, copy dP out, and write dS (bf16) into the dP columns
+// once every warp has (dp_free), in two 64-key slices; slice 0's
+// dQ += dS K (A from tensor memory) runs while slice 1 is formed.
 // Tensor memory: S 0..127, dP 128..255, dQ 256..383, Q 384..447, dO 448..511.
 template <int D>
 struct DqCfg {
     static constexpr int KTILE = 128 * D * 2;
     static constexpr int NSLOT = (D == 128) ? 6 : 12;
-    static constexpr int DS_SLICE = 128 * 64 * 2;                // 128 query rows x 64 keys, bf16
     static constexpr int KV_OFF = 0;
-    static constexpr int DS_OFF = KV_OFF + NSLOT * KTILE;
-    static constexpr int BAR_OFF = DS_OFF + BWD_NSLICE * DS_SLICE;
-    // qt_full, qt_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full, s_free, p_full[NSLICE],
-    // ds_empty[NSLICE], acc_full, drain, acc_empty
-    static constexpr int NBAR = 7 + 2 * NSLOT + 2 * BWD_NSLICE;
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * KTILE;
+    // qt_full, qt_empty, kv_full[NSLOT], kv_empty[NSLOT], st_ready, dp_ready, s_free, dp_free,
+    // p_full[NSLICE], acc_full, drain, acc_empty
+    static constexpr int NBAR = 9 + 2 * NSLOT + BWD_NSLICE;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
     static constexpr int THREADS = BWD_THREADS;
 };
@@ -693,14 +702,13 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sKV = sbase + Cfg::KV_OFF;
-    const uint32_t sDS = sbase + Cfg::DS_OFF;
     const uint32_t bars = sbase + Cfg::BAR_OFF;
     const uint32_t bar_qt_full = bars, bar_qt_empty = bars + 8;
     const uint32_t bar_kv_full = bars + 16, bar_kv_empty = bars + 16 + 8 * Cfg::NSLOT;
-    const uint32_t bar_s_full = bars + 16 + 16 * Cfg::NSLOT, bar_s_free = bar_s_full + 8;
-    const uint32_t bar_p_full = bar_s_free + 8;                         // [NSLICE]
-    const uint32_t bar_ds_empty = bar_p_full + 8 * BWD_NSLICE;          // [NSLICE]
-    const uint32_t bar_acc_full = bar_ds_empty + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
+    const uint32_t bar_st_ready = bars + 16 + 16 * Cfg::NSLOT, bar_dp_ready = bar_st_ready + 8;
+    const uint32_t bar_s_free = bar_dp_ready + 8, bar_dp_free = bar_s_free + 8;
+    const uint32_t bar_p_full = bar_dp_free + 8;                        // [NSLICE]
+    const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
@@ -718,12 +726,11 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_kv_full + 8 * i, 1);
             mbar_init(bar_kv_empty + 8 * i, 1);
         }
-        mbar_init(bar_s_full, 1);
+        mbar_init(bar_st_ready, 1);
+        mbar_init(bar_dp_ready, 1);
         mbar_init(bar_s_free, 4 * BWD_NWG);
-        for (int i = 0; i < BWD_NSLICE; ++i) {
-            mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
-            mbar_init(bar_ds_empty + 8 * i, 1);
-        }
+        mbar_init(bar_dp_free, 4 * BWD_NWG);
+        for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
         mbar_init(bar_acc_empty, 4 * BWD_NWG);
@@ -777,20 +784,21 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         // The whole warp runs the control flow; one elected lane issues each group
-        // of tensor-core instructions.  Order per key tile i: S(i), dP(i) (once the
-        // elementwise warps have copied out tile i-1), then dQ += dS(i-1) K(i-1).
+        // of tensor-core instructions.  Order per key tile i: S(i) (once the
+        // elementwise warps have copied out S(i-1)), dQ += dS(i-1) K(i-1) (dS sits
+        // in the dP columns), then dP(i) over them (the tensor pipe runs in order).
         {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);   // A K-major, B MN-major
-            constexpr uint32_t KT16 = Cfg::KTILE >> 4, DS16 = Cfg::DS_SLICE >> 4;
+            constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);   // A tmem, B MN-major
+            constexpr uint32_t KT16 = Cfg::KTILE >> 4;
             const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256, tQ = tmem + 384, tdO = tmem + 448;
             const uint64_t dKV = sdesc_sw128(sKV, 16, 1024), dKVmn = sdesc_sw128(sKV, 16384, 1024);
-            const uint64_t dDS = sdesc_sw128(sDS, 16, 1024);
             uint32_t nload = 0, iter = 0, sf_phase = 0, ae_phase = 0;
             uint32_t p_phase[BWD_NSLICE];
             for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
             bool ok = true, acc_busy = false, s_pending = false;
-            // dQ += dS K for one finished key tile, 64 keys per slice
+            // dQ += dS K for one finished key tile; dS of slice j (64 keys) sits at dP
+            // columns 64j + 8w, 16 keys per 8 columns
             auto issue_dq = [&](uint32_t kslot, bool& first) -> bool {
                 if (first && acc_busy) {   // every group has stored the previous item's dQ
                     if (!mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag)) return false;
@@ -805,9 +813,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     if (elect_one()) {
 #pragma unroll
                         for (int w4 = 0; w4 < 4; ++w4)
-                            mma_ss(tdQ, dDS + j * DS16 + ((w4 * 32) >> 4), bk_mn + (((4 * j + w4) * 2048) >> 4),
-                                   IDESC_G, (!first || j > 0 || w4 > 0) ? 1u : 0u);
-                        mma_commit(bar_ds_empty + 8 * j);
+                            mma_ts(tdQ, tdP + 64 * j + 8 * w4, bk_mn + (((4 * j + w4) * 2048) >> 4), IDESC_G,
+                                   (!first || j > 0 || w4 > 0) ? 1u : 0u);
                     }
                     __syncwarp();
                 }
@@ -834,10 +841,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
                         const uint32_t vslot = (nload + 1) % Cfg::NSLOT, vpar = ((nload + 1) / Cfg::NSLOT) & 1;
                         nload += 2;
-                        ok = mbar_wait_warp(bar_kv_full + 8 * kslot, kpar, abort_flag) &&
-                             mbar_wait_warp(bar_kv_full + 8 * vslot, vpar, abort_flag);
+                        ok = mbar_wait_warp(bar_kv_full + 8 * kslot, kpar, abort_flag);
                         if (!ok) break;
-                        if (s_pending) {   // S / dP of the previous tile are copied out
+                        if (s_pending) {   // S of the previous tile is copied out
                             ok = mbar_wait_warp(bar_s_free, sf_phase, abort_flag);
                             if (!ok) break;
                             sf_phase ^= 1;
@@ -850,17 +856,26 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
                                 mma_ts(tS, tQ + 8 * k, bk + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
+                            mma_commit(bar_st_ready);
+                        }
+                        __syncwarp();
+                        s_pending = true;
+                        // the previous tile's products read dS from the dP columns ...
+                        if (prev_live && !(ok = issue_dq(prev_kslot, first))) break;
+                        // ... before this tile's dP overwrites them
+                        ok = mbar_wait_warp(bar_kv_full + 8 * vslot, vpar, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (elect_one()) {
 #pragma unroll
                             for (int k = 0; k < D / 16; ++k) {
                                 const uint32_t off = ((k / 4) * 16384 + (k % 4) * 32) >> 4;
                                 mma_ts(tdP, tdO + 8 * k, bv + off, IDESC_S, k > 0 ? 1u : 0u);
                             }
-                            mma_commit(bar_s_full);
+                            mma_commit(bar_dp_ready);
                             mma_commit(bar_kv_empty + 8 * vslot);
                         }
                         __syncwarp();
-                        s_pending = true;
-                        if (prev_live && !(ok = issue_dq(prev_kslot, first))) break;
                         prev_live = true;
                         prev_kslot = kslot;
                     }
@@ -889,11 +904,10 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + 16 * wg, tdP = tmem + lane_off + 128 + 16 * wg;
         const uint32_t tdQ = tmem + lane_off + 256 + 32 * wg;
-        // this row of a dS slice buffer (SW128 K-major: 16-byte chunk c of row r sits at chunk c ^ (r % 8))
-        const uint32_t ds_row = sDS + (row >> 3) * 1024 + (row & 7) * 128;
-        const uint32_t ds_c0 = ((2 * wg) ^ (row & 7)) * 16, ds_c1 = ((2 * wg + 1) ^ (row & 7)) * 16;
         const uint32_t tQ = tmem + lane_off + 384 + 16 * wg, tdO = tmem + lane_off + 448 + 16 * wg;
-        uint32_t s_phase = 0, a_phase = 0, nstep = 0, iter = 0;
+        // packed dS of slice j goes to dP columns 64j + 8wg
+        const uint32_t tDs = tmem + lane_off + 128 + 8 * wg;
+        uint32_t st_phase = 0, dp_phase = 0, df_phase = 0, a_phase = 0, iter = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
             const DqItem it = decode_dq(P, w);
@@ -934,44 +948,53 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
                     const int cls = classify_tile(it.qo, dsf, dsl, ko);
                     if (cls == TILE_SKIP) continue;
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, s_phase, abort_flag));
+                    // ---- S: copy out, release, and form P while dP is still being computed
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_st_ready, st_phase, abort_flag));
                     if (!ok) break;
-                    s_phase ^= 1;
+                    st_phase ^= 1;
                     tc_fence_after();
                     const int lo = ds_q - ko - 16 * wg, hi = q_orig - ko - 16 * wg;
                     float sv[32], dp[32];
                     tmem_ld16f(tS, sv);
                     tmem_ld16f(tS + 64, sv + 16);
+                    tmem_wait_ld();
+                    reg_fence32f(sv);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_s_free);   // the MMA warp may compute the next S
+#pragma unroll
+                    for (int jj = 0; jj < BWD_NSLICE; ++jj) {
+                        if (cls == TILE_FULL)
+                            dq_p16<false>(sv + 16 * jj, nlse2, P.scale_log2, 0, 0);
+                        else
+                            dq_p16<true>(sv + 16 * jj, nlse2, P.scale_log2, lo - 64 * jj, hi - 64 * jj);
+                    }
+                    // ---- dP: copy out; every warp has its columns before dS lands there
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
+                    if (!ok) break;
+                    dp_phase ^= 1;
+                    tc_fence_after();
                     tmem_ld16f(tdP, dp);
                     tmem_ld16f(tdP + 64, dp + 16);
                     tmem_wait_ld();
-                    reg_fence32f(sv);
                     reg_fence32f(dp);
-                    // S and dP of this tile are in registers: the MMA warp may overwrite them
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_s_free);
+                    if (lane == 0) mbar_arrive(bar_dp_free);
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_free, df_phase, abort_flag));
+                    if (!ok) break;
+                    df_phase ^= 1;
+                    tc_fence_after();
 #pragma unroll
                     for (int jj = 0; jj < BWD_NSLICE; ++jj) {
                         uint32_t dk[8];
-                        if (cls == TILE_FULL)
-                            dq_cols16<false>(sv + 16 * jj, dp + 16 * jj, nlse2, dlt, P.scale_log2, 0, 0, dk);
-                        else
-                            dq_cols16<true>(sv + 16 * jj, dp + 16 * jj, nlse2, dlt, P.scale_log2, lo - 64 * jj,
-                                            hi - 64 * jj, dk);
-                        // the previous tile's products have read this slice buffer
-                        ok = __all_sync(0xffffffffu,
-                                        mbar_wait(bar_ds_empty + 8 * jj, (nstep & 1) ^ 1, abort_flag));
-                        if (!ok) break;
-                        const uint32_t dst = ds_row + jj * Cfg::DS_SLICE;
-                        st_shared_v4(dst + ds_c0, dk[0], dk[1], dk[2], dk[3]);
-                        st_shared_v4(dst + ds_c1, dk[4], dk[5], dk[6], dk[7]);
-                        fence_proxy_async_smem();
+                        dq_ds16(sv + 16 * jj, dp + 16 * jj, dlt, dk);
+                        tmem_st8(tDs + 64 * jj, dk);
+                        tmem_wait_st();
+                        tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar_p_full + 8 * jj);
                     }
-                    if (!ok) break;
-                    ++nstep;
                     had = true;
                 }
             }
