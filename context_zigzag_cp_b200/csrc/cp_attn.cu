@@ -66,6 +66,8 @@ cp_status_t check_attention(const cp_problem_t* p)
     cp_status_t st = check_problem(p);
     if (st != CP_OK) return st;
     if (p->head_dim != 64 && p->head_dim != 128) return CP_ERR_UNSUPPORTED;
+    // the kernels' tile bounds (key tile end + window or sequence length) stay in int32
+    if (p->seq_len > (1 << 29)) return CP_ERR_UNSUPPORTED;
     const int C = p->seq_len / (2 * p->cp_size);
     if (C % 128 != 0) return CP_ERR_UNSUPPORTED;
     return CP_OK;
