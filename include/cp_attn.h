@@ -180,7 +180,7 @@ CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan
  *   k, v  bf16 [B][Hkv][S][D] shard order
  *   o     bf16 [B][Hq][S][D]  output, shard order
  *   lse   fp32 [B][Hq][S]     output, natural-log LSE of the scaled scores
- * Supported: head_dim 64 or 128; C = S/(2cp) a multiple of 128.
+ * Supported: head_dim 64 or 128; C = S/(2cp) a multiple of 128; S <= 2^29.
  * Workspace: CP_MERGE_SEPARATE needs cp fp32 partial (O, LSE) sets (each
  * region rounded up to 256 bytes); CP_MERGE_FUSED needs none (0 bytes).
  * Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_WORKSPACE, CP_ERR_CUDA.
