@@ -48,6 +48,39 @@ def _ptr(t) -> ctypes.c_void_p:
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
 
+def _on_device(t, dev) -> bool:
+    """True when tensor t lives on CUDA device dev."""
+    return t.device.type == "cuda" and t.device == dev
+
+
+def _validate(*specs) -> None:
+    """Refuse tensors the kernels would read or write out of bounds before any
+    pointer reaches the library.  ``specs``: (tensor or None, shape, dtype, name);
+    None entries are outputs the binding allocates itself.  Shapes and dtypes are
+    checked first, then that every tensor is contiguous and on one CUDA device."""
+    given = [sp for sp in specs if sp[0] is not None]
+    for t, shape, dtype, name in given:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    dev = given[0][0].device
+    for t, _, _, name in given:
+        if not _on_device(t, dev):
+            raise ValueError(f"{name}: on {t.device}; every tensor must be on one CUDA device "
+                             f"(the first is on {dev})")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+
+
+def _attn_shapes(prob: "Problem"):
+    q = (prob.batch, prob.num_heads, prob.seq_len, prob.head_dim)
+    kv = (prob.batch, prob.num_kv_heads, prob.seq_len, prob.head_dim)
+    return q, kv, q[:-1]
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -111,17 +144,24 @@ class Plan:
     def ref(self):
         return ctypes.byref(self.c)
 
-    def _bufs(self, tensors):
+    def _bufs(self, tensors, outs):
         n = len(tensors)
-        for t in tensors:
-            if t.dim() < 2 or t.shape[-2] != self.prob.seq_len or not t.is_contiguous():
-                raise ValueError("buffers must be contiguous [..., seq_len, row] tensors")
+        if len(outs) != n:
+            raise ValueError(f"{n} input buffers but {len(outs)} output buffers")
+        for i, (t, u) in enumerate(zip(tensors, outs)):
+            if not isinstance(t, torch.Tensor) or not isinstance(u, torch.Tensor):
+                raise TypeError(f"buffer {i}: expected torch.Tensor inputs and outputs")
+            if t.dim() < 2 or t.shape[-2] != self.prob.seq_len:
+                raise ValueError(f"buffer {i}: shape {tuple(t.shape)} is not [..., seq_len, row]")
+            _validate((t, t.shape, t.dtype, f"buffer {i}"), (u, t.shape, t.dtype, f"output {i}"))
+            if not _on_device(t, self.perm.device):
+                raise ValueError(f"buffer {i}: on {t.device}, the plan is on {self.perm.device}")
         outer = (ctypes.c_int64 * max(n, 1))(*[t[..., 0, 0].numel() for t in tensors])
         row = (ctypes.c_int64 * max(n, 1))(*[t.shape[-1] * t.element_size() for t in tensors])
         return n, outer, row
 
     def build(self, bufs_in=(), bufs_out=(), stream=None):
-        n, outer, row = self._bufs(list(bufs_in))
+        n, outer, row = self._bufs(list(bufs_in), list(bufs_out))
         pin = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in bufs_in])
         pout = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in bufs_out])
         _check(lib().cp_plan_shards(self.prob.ref, self.ref, n, pin, pout, outer, row, None,
@@ -136,7 +176,7 @@ class Plan:
     def unshard(self, tensors, stream=None):
         """Scatter tensors [..., S, row] from shard back into original order."""
         outs = [torch.empty_like(t) for t in tensors]
-        n, outer, row = self._bufs(list(tensors))
+        n, outer, row = self._bufs(list(tensors), outs)
         pin = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in tensors])
         pout = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in outs])
         _check(lib().cp_unshard(self.prob.ref, self.ref, n, pin, pout, outer, row,
@@ -165,6 +205,8 @@ def bwd_workspace_bytes(prob: Problem) -> int:
 def _workspace(nbytes: int, device, ws):
     if nbytes == 0:
         return None
+    if ws is not None and (ws.device != device or not ws.is_contiguous()):
+        raise ValueError(f"ws: must be a contiguous tensor on {device}")
     if ws is not None and ws.numel() * ws.element_size() >= nbytes:
         return ws
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -172,6 +214,10 @@ def _workspace(nbytes: int, device, ws):
 
 def attn_fwd(prob: Problem, plan: Plan, q, k, v, o=None, lse=None, ws=None, stream=None):
     """cp_attn_fwd on shard-order q [B,Hq,S,D], k/v [B,Hkv,S,D]; returns (o, lse)."""
+    qs, kvs, ls = _attn_shapes(prob)
+    bf16 = torch.bfloat16
+    _validate((q, qs, bf16, "q"), (k, kvs, bf16, "k"), (v, kvs, bf16, "v"), (o, qs, bf16, "o"),
+              (lse, ls, torch.float32, "lse"))
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
@@ -185,9 +231,18 @@ def attn_fwd(prob: Problem, plan: Plan, q, k, v, o=None, lse=None, ws=None, stre
     return o, lse
 
 
+def _validate_bwd(prob, q, k, v, o, lse, do, dq, dk, dv):
+    qs, kvs, ls = _attn_shapes(prob)
+    bf16 = torch.bfloat16
+    _validate((q, qs, bf16, "q"), (k, kvs, bf16, "k"), (v, kvs, bf16, "v"), (o, qs, bf16, "o"),
+              (lse, ls, torch.float32, "lse"), (do, qs, bf16, "do"), (dq, qs, bf16, "dq"),
+              (dk, kvs, bf16, "dk"), (dv, kvs, bf16, "dv"))
+
+
 def attn_bwd(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq=None, dk=None, dv=None,
              ws=None, stream=None):
     """cp_attn_bwd; returns (dq, dk, dv) in shard order."""
+    _validate_bwd(prob, q, k, v, o, lse, do, dq, dk, dv)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -208,6 +263,9 @@ def attn_bwd_noalloc(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq, dk, dv,
     inside the library (batch * heads * seq_len <= 4,194,304 rows); calls that could
     overlap on the GPU must be serialised, and the first call on a device must come
     before any stream capture.  The caller passes every output; nothing is allocated."""
+    if dq is None or dk is None or dv is None:
+        raise ValueError("attn_bwd_noalloc: dq, dk and dv must be given")
+    _validate_bwd(prob, q, k, v, o, lse, do, dq, dk, dv)
     _check(lib().cp_attn_bwd_noalloc(prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                      _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                                      _stream(stream)), "cp_attn_bwd_noalloc")
@@ -216,7 +274,12 @@ def attn_bwd_noalloc(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq, dk, dv,
 
 def lse_merge(o_parts, lse_parts, o_out=None, lse_out=None, stream=None):
     """cp_lse_merge on o_parts fp32 [n, rows, D], lse_parts fp32 [n, rows]."""
+    if not isinstance(o_parts, torch.Tensor) or o_parts.dim() != 3:
+        raise ValueError("o_parts: expected a [n, rows, head_dim] tensor")
     n, rows, D = o_parts.shape
+    _validate((o_parts, (n, rows, D), torch.float32, "o_parts"),
+              (lse_parts, (n, rows), torch.float32, "lse_parts"),
+              (o_out, (rows, D), torch.bfloat16, "o_out"), (lse_out, (rows,), torch.float32, "lse_out"))
     if o_out is None:
         o_out = torch.empty((rows, D), dtype=torch.bfloat16, device=o_parts.device)
     if lse_out is None:
