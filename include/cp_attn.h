@@ -77,9 +77,10 @@ typedef enum { CP_MASK_CAUSAL = 0, CP_MASK_DOC_CAUSAL = 1 } cp_mask_t;
 typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
 
 /* The problem.  Field meaning:
- *   batch         >= 1
+ *   batch         >= 1; batch * num_heads * seq_len must stay below 2^31
+ *                 (CP_ERR_UNSUPPORTED otherwise: flat row indices are int32)
  *   seq_len       S, tokens per sequence; S % (2*cp_size) == 0
- *   cp_size       number of virtual ranks, >= 1
+ *   cp_size       number of virtual ranks, 1..1024 (CP_ERR_UNSUPPORTED above)
  *   num_heads     query heads Hq; num_kv_heads Hkv divides Hq (GQA: query head
  *                 h reads KV head h / (Hq/Hkv))
  *   head_dim      D

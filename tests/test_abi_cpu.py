@@ -60,6 +60,9 @@ def fwd_query(p):
     (dict(num_heads=3, num_kv_heads=2), _lib.CP_ERR_INVALID_ARG),
     (dict(head_dim=96), _lib.CP_ERR_UNSUPPORTED),
     (dict(seq_len=384, cp=3), _lib.CP_ERR_UNSUPPORTED),   # C = 64, not a multiple of 128
+    (dict(seq_len=2050, cp=1025), _lib.CP_ERR_UNSUPPORTED),  # more virtual ranks than the planner holds
+    (dict(batch=1024, num_heads=1024, num_kv_heads=1024, seq_len=4096),
+     _lib.CP_ERR_UNSUPPORTED),                            # 2^32 rows: beyond int32 row indices
     (dict(), _lib.CP_OK),
 ])
 def test_fwd_host_checks(lib, kw, status):
