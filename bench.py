@@ -198,8 +198,8 @@ def config_dict(w: synth.Workload, rotate: str, world: int) -> dict:
 
 KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_dkdv": 6.0, "bwd_dq": 2.0}   # x D*Hq*pairs
 
-# DRAM bytes (read + write) per launch from one ncu capture of the full-size workload
-# (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass; profiles/dram_bytes_long128k.md).
+# DRAM bytes (read + write) per launch of a kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum).
 # A figure is reported only while the kernel's source is the one it was taken on:
 # first 16 hex digits of the sha256 of the file's code lines (text after "//" and
 # blank lines dropped, so comment edits keep it); after any code change it reads
@@ -231,6 +231,43 @@ def code_digest(path: str) -> str:
     with open(path, encoding="utf-8") as f:
         lines = [ln.split("//", 1)[0].strip() for ln in f]
     return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()[:16]
+
+
+def forward_at(args, name, device, dist, peaks, reps=5):
+    """The forward alone (cp_attn_fwd, both merge modes) on another workload, so the
+    low end of the 32k-128k range is measured in the same run: device time per
+    call over `reps` calls after 3 warm-up calls, max over ranks."""
+    import torch
+    import context_zigzag_cp_b200 as cz
+    w = synth.WORKLOADS[name]
+    t = synth.workload_inputs(w, device=device, with_dout=False)
+    cu = None if t["cu_seqlens"] is None else torch.from_numpy(t["cu_seqlens"]).to(device)
+    out = {"workload": name, "rotate": w.rotate}
+    prob = cz.Problem(w.batch, w.seq_len, w.cp, w.num_heads, w.num_kv_heads, w.head_dim,
+                      w.rotate, cu, merge="separate")
+    plan = cz.Plan(prob)
+    qs, ks, vs = plan.shard([t["q"], t["k"], t["v"]])
+    o = torch.empty_like(qs)
+    lse = torch.empty(qs.shape[:-1], dtype=torch.float32, device=device)
+    ws = torch.empty(max(cz.fwd_workspace_bytes(prob), 256), dtype=torch.uint8, device=device)
+    flops = 4.0 * w.head_dim * w.num_heads * int(plan.pairs.sum().item()) * w.batch
+    for merge in ("separate", "fused"):
+        pr = prob.with_merge(merge)
+        for _ in range(3):
+            cz.attn_fwd(pr, plan, qs, ks, vs, o, lse, ws=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            cz.attn_fwd(pr, plan, qs, ks, vs, o, lse, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = dist_max(dist, e0.elapsed_time(e1) / reps, device)
+        out[merge] = {"ms": round(ms, 3), "tflops": round(flops / 1e9 / ms, 1),
+                      "frac_of_peak": round(flops / 1e9 / ms / peaks["bf16"], 4)}
+    if cz.get_device_status() != 0:
+        raise RuntimeError("device status after the 32k forward")
+    return out
 
 
 def run_native(args, w, rank, world, local_rank):
@@ -343,6 +380,7 @@ def run_native(args, w, rank, world, local_rank):
 
     fwd_ms = dist_max(dist, time_fwd(prob), device)
     fused_ms = dist_max(dist, time_fwd(prob_fused), device)
+    fwd_32k = forward_at(args, "gqa32k", device, dist, peaks) if w.name != "gqa32k" else None
 
     # ---- end to end through the public API with pinned host buffers
     hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
@@ -418,6 +456,7 @@ def run_native(args, w, rank, world, local_rank):
             "fwd_frac_of_peak": round(fwd_flops / 1e9 / fwd_ms / peaks["bf16"], 4),
             "fwd_fused_tflops": round(fwd_flops / 1e9 / fused_ms, 1),
             "fwd_fused_frac_of_peak": round(fwd_flops / 1e9 / fused_ms / peaks["bf16"], 4),
+            "fwd_32k": fwd_32k,
             "step_frac_of_peak": round(value / world / peaks["bf16_sustained"], 4),
             "peak_source": peaks["source"],
             "pairs": pairs,

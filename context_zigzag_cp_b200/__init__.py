@@ -75,6 +75,28 @@ def _validate(*specs) -> None:
             raise ValueError(f"{name}: must be contiguous")
 
 
+def _check_plan(prob: "Problem", plan: "Plan", dev) -> None:
+    """The plan's arrays are sized and filled for the problem it was built from;
+    the kernels index them by the problem's seq_len and cp, so a plan built for
+    another problem (or living on another device) is refused here."""
+    if not isinstance(plan, Plan):
+        raise TypeError(f"plan: expected a Plan, got {type(plan).__name__}")
+    pp = plan.prob
+    if (pp.seq_len, pp.cp, pp.rotate) != (prob.seq_len, prob.cp, prob.rotate):
+        raise ValueError(f"plan: built for seq_len {pp.seq_len}, cp {pp.cp}, {pp.rotate}; the "
+                         f"problem has seq_len {prob.seq_len}, cp {prob.cp}, {prob.rotate}")
+    if pp.cu_seqlens is not prob.cu_seqlens:
+        same = (pp.cu_seqlens is not None and prob.cu_seqlens is not None
+                and pp.cu_seqlens.shape == prob.cu_seqlens.shape
+                and bool(torch.equal(pp.cu_seqlens, prob.cu_seqlens)))
+        if not same:
+            raise ValueError("plan: built for other documents (cu_seqlens) than the problem's")
+    if not _on_device(plan.perm, dev):
+        raise ValueError(f"plan: on {plan.perm.device}, the tensors are on {dev}")
+    if prob.cu_seqlens is not None and not _on_device(prob.cu_seqlens, dev):
+        raise ValueError(f"cu_seqlens: on {prob.cu_seqlens.device}, the tensors are on {dev}")
+
+
 def _attn_shapes(prob: "Problem"):
     q = (prob.batch, prob.num_heads, prob.seq_len, prob.head_dim)
     kv = (prob.batch, prob.num_kv_heads, prob.seq_len, prob.head_dim)
@@ -99,6 +121,15 @@ class Problem:
     def __init__(self, batch: int, seq_len: int, cp: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, rotate: str = "allgather", cu_seqlens: torch.Tensor | None = None,
                  merge: str = "fused", softmax_scale: float = 0.0, window: int = 0):
+        if cu_seqlens is not None:
+            if not isinstance(cu_seqlens, torch.Tensor):
+                raise TypeError("cu_seqlens: expected a torch.Tensor")
+            if cu_seqlens.dtype != torch.int32 or cu_seqlens.device.type != "cuda":
+                raise ValueError(f"cu_seqlens: must be an int32 CUDA tensor, got "
+                                 f"{cu_seqlens.dtype} on {cu_seqlens.device}")
+            if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2 or not cu_seqlens.is_contiguous():
+                raise ValueError("cu_seqlens: must be a contiguous 1-D tensor of num_docs + 1 >= 2 "
+                                 "offsets")
         self.cu_seqlens = cu_seqlens
         self.window = window
         self.batch, self.seq_len, self.cp = batch, seq_len, cp
@@ -218,6 +249,7 @@ def attn_fwd(prob: Problem, plan: Plan, q, k, v, o=None, lse=None, ws=None, stre
     bf16 = torch.bfloat16
     _validate((q, qs, bf16, "q"), (k, kvs, bf16, "k"), (v, kvs, bf16, "v"), (o, qs, bf16, "o"),
               (lse, ls, torch.float32, "lse"))
+    _check_plan(prob, plan, q.device)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
@@ -231,18 +263,19 @@ def attn_fwd(prob: Problem, plan: Plan, q, k, v, o=None, lse=None, ws=None, stre
     return o, lse
 
 
-def _validate_bwd(prob, q, k, v, o, lse, do, dq, dk, dv):
+def _validate_bwd(prob, plan, q, k, v, o, lse, do, dq, dk, dv):
     qs, kvs, ls = _attn_shapes(prob)
     bf16 = torch.bfloat16
     _validate((q, qs, bf16, "q"), (k, kvs, bf16, "k"), (v, kvs, bf16, "v"), (o, qs, bf16, "o"),
               (lse, ls, torch.float32, "lse"), (do, qs, bf16, "do"), (dq, qs, bf16, "dq"),
               (dk, kvs, bf16, "dk"), (dv, kvs, bf16, "dv"))
+    _check_plan(prob, plan, q.device)
 
 
 def attn_bwd(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq=None, dk=None, dv=None,
              ws=None, stream=None):
     """cp_attn_bwd; returns (dq, dk, dv) in shard order."""
-    _validate_bwd(prob, q, k, v, o, lse, do, dq, dk, dv)
+    _validate_bwd(prob, plan, q, k, v, o, lse, do, dq, dk, dv)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -265,7 +298,7 @@ def attn_bwd_noalloc(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq, dk, dv,
     before any stream capture.  The caller passes every output; nothing is allocated."""
     if dq is None or dk is None or dv is None:
         raise ValueError("attn_bwd_noalloc: dq, dk and dv must be given")
-    _validate_bwd(prob, q, k, v, o, lse, do, dq, dk, dv)
+    _validate_bwd(prob, plan, q, k, v, o, lse, do, dq, dk, dv)
     _check(lib().cp_attn_bwd_noalloc(prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                      _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                                      _stream(stream)), "cp_attn_bwd_noalloc")

@@ -26,15 +26,49 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Per-device state.  Kernel attributes (the large dynamic shared-memory opt-in)
+// and the SM count belong to a device, not to the process: a process that drives
+// several GPUs sets them once on each, on first use with that device current.
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int g_num_sms[kMaxDevices] = {};
+uint32_t g_attr_done[kMaxDevices] = {};   // bit per kernel family (AttrSet)
+
+enum AttrSet : uint32_t { ATTR_FWD64 = 1, ATTR_FWD128 = 2, ATTR_BWD64 = 4, ATTR_BWD128 = 8 };
+
+inline int current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
+}
+
 int num_sms()
 {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    const int dev = current_device();
+    if (dev < 0) return 148;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_num_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return 148;
+        g_num_sms[dev] = n;
     }
-    return n;
+    return g_num_sms[dev];
+}
+
+// Run `set` (which applies cudaFuncSetAttribute to one kernel family) once per
+// device; a failure is reported and retried on the next call.
+template <typename F>
+cp_status_t ensure_attr(AttrSet which, F set)
+{
+    const int dev = current_device();
+    if (dev < 0) return CP_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_attr_done[dev] & which) return CP_OK;
+    if (set() != cudaSuccess) return CP_ERR_CUDA;
+    g_attr_done[dev] |= which;
+    return CP_OK;
 }
 
 // Checks shared by every call that takes a cp_problem_t.
@@ -222,13 +256,11 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.lse = lse;
     P.o_parts = o_parts;
     P.lse_parts = lse_parts;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(cp_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        Cfg::SMEM_BYTES);
+    const cp_status_t ast = ensure_attr(D == 128 ? ATTR_FWD128 : ATTR_FWD64, [] {
+        return cudaFuncSetAttribute(cp_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::SMEM_BYTES);
     });
-    if (attr_err != cudaSuccess) return CP_ERR_CUDA;
+    if (ast != CP_OK) return ast;
     const int grid = std::min(P.n_items, num_sms());
     LaunchScope ls(CP_K_FWD, stream);
     cp_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, P);
@@ -489,16 +521,16 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.dq = static_cast<__nv_bfloat16*>(dq);
     P.dk = static_cast<__nv_bfloat16*>(dk);
     P.dv = static_cast<__nv_bfloat16*>(dv);
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        DkdvCfg<D>::SMEM_BYTES);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(cp_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            DqCfg<D>::SMEM_BYTES);
+    const cp_status_t ast = ensure_attr(D == 128 ? ATTR_BWD128 : ATTR_BWD64, [] {
+        cudaError_t e = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             DkdvCfg<D>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(cp_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     DqCfg<D>::SMEM_BYTES);
+        return e;
     });
-    if (attr_err != cudaSuccess) return CP_ERR_CUDA;
+    if (ast != CP_OK) return ast;
     P.n_items = B * Hkv * (S / 256);   // pairs of key tiles (S / 128 is even)
     {
     LaunchScope ls(CP_K_BWD_DKDV, stream);
@@ -548,17 +580,22 @@ constexpr size_t kNoallocScratchBytes = size_t(2) * CP_NOALLOC_MAX_ROWS * sizeof
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 // The name g_noalloc_scratch is only a host-side handle; kernels need the
-// device address, looked up once per device.
-constexpr int kMaxDevices = 64;
+// device address.  It is looked up on every call made outside a stream capture
+// (so a context re-created after cudaDeviceReset gets its own address) and
+// cached per device for calls made while `stream` is being captured, where the
+// lookup is not made.
 void* g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-cp_status_t noalloc_scratch(void** out)
+cp_status_t noalloc_scratch(cudaStream_t stream, void** out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CP_ERR_CUDA;
+    const int dev = current_device();
+    if (dev < 0) return CP_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return CP_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone || !g_noalloc_ptr[dev]) {
+        if (cap != cudaStreamCaptureStatusNone) return CP_ERR_CUDA;   // never looked up before capture
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CP_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
@@ -582,11 +619,11 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
         if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
     const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * problem->seq_len;
     if (rows > CP_NOALLOC_MAX_ROWS) return CP_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
     void* scratch = nullptr;
-    if ((st = noalloc_scratch(&scratch)) != CP_OK) return st;
+    if ((st = noalloc_scratch(s, &scratch)) != CP_OK) return st;
     float* delta = static_cast<float*>(scratch);
     float* nlse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
-    cudaStream_t s = as_stream(stream);
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s)
                : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s);

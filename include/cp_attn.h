@@ -95,11 +95,15 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *                 Negative values are CP_ERR_INVALID_ARG.
  *   cu_seqlens    DEVICE int32 [num_docs+1], 0 = cu[0] < cu[1] < ... <
  *                 cu[num_docs] = S, original order; the same documents apply to
- *                 every batch entry.  NULL for the plain causal mask.  Only
- *                 cp_plan_shards reads it, on the device: a list that is not
+ *                 every batch entry.  NULL for the plain causal mask.
+ *                 cp_plan_shards checks it on the device: a list that is not
  *                 strictly increasing from 0 to S records CP_ERR_INVALID_ARG in
  *                 the device status word (the host cannot see device memory
- *                 without synchronising).  The forward/backward read the plan. */
+ *                 without synchronising).  cp_attn_bwd (and cp_attn_bwd_noalloc)
+ *                 read it again on the device, for the document end of each key
+ *                 tile, without checking it: the list must stay allocated and
+ *                 unchanged from cp_plan_shards until the backward has run.
+ *                 cp_attn_fwd reads only the plan. */
 typedef struct {
     int32_t batch;
     int32_t seq_len;
@@ -242,9 +246,12 @@ CP_API cp_status_t cp_lse_merge(int64_t rows, int32_t head_dim, int32_t n_parts,
  *     CP_ERR_WORKSPACE and nothing is launched.
  *   - Cost: every GPU that loads the library holds the 32 MiB array until the
  *     process exits.
- *   - The first call on each device looks up the array's device address (a
- *     synchronous runtime query); make that first call before any stream
- *     capture.  Later calls only launch kernels.
+ *   - A call made outside stream capture looks up the array's device address
+ *     (a runtime query) and remembers it for its device; a call made while
+ *     `stream` is being captured uses the remembered address, so the first
+ *     call on each device must come before any stream capture (a first call
+ *     inside a capture returns CP_ERR_CUDA).  Looking the address up again on
+ *     each uncaptured call keeps it right after cudaDeviceReset.
  *   - Every call on a device shares the one array, and the array keeps the last
  *     call's contents (nothing in it needs to start at zero: each call writes
  *     every scratch value it reads).  Calls that can overlap on the GPU (two

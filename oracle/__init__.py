@@ -77,9 +77,12 @@ def _load():
                                         _f64p, _i32p, I64, _i64p, _f64p]
         lib.orc_bwd_dkv_keys.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
                                          _f64p, _i32p, I64, _i64p, _f64p, _f64p]
+        lib.orc_bwd_dkv_keys_fwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
+                                             _f64p, _f64p, _f64p, _i32p, I64, _i64p, _f64p, _f64p]
         lib.orc_num_threads.argtypes = []
         for name in ("orc_doc_start", "orc_plan", "orc_fwd_rows", "orc_fwd", "orc_partial",
-                     "orc_bwd", "orc_bwd_dq_rows", "orc_bwd_dkv_keys", "orc_num_threads"):
+                     "orc_bwd", "orc_bwd_dq_rows", "orc_bwd_dkv_keys", "orc_bwd_dkv_keys_fwd",
+                     "orc_num_threads"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -260,6 +263,23 @@ def bwd_dkv_keys(q, k, v, dout, keys, ds_orig=None, scale=None):
     dv = np.zeros((len(keys), D), np.float64)
     _check(_load().orc_bwd_dkv_keys(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, dout, ds,
                                     len(keys), keys, dk, dv), "bwd_dkv_keys")
+    return dk, dv
+
+
+def bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds_orig=None, scale=None):
+    """dK, dV at selected flat keys (bkv*S + k_orig) from the oracle's own forward
+    results o [B,Hq,S,D] / lse [B,Hq,S] of every row: [n, D] each.  The same sums
+    as ``bwd``, restricted to the selected keys; each row's forward is read once
+    instead of being recomputed per key, so early keys (attended by almost every
+    row) cost O(S D) each."""
+    q, k, v, o, lse, dout = map(_f64, (q, k, v, o, lse, dout))
+    B, Hq, Hkv, S, D = _dims(q, k)
+    ds = np.zeros(S, np.int32) if ds_orig is None else np.ascontiguousarray(ds_orig, np.int32)
+    keys = np.ascontiguousarray(keys, np.int64)
+    dk = np.zeros((len(keys), D), np.float64)
+    dv = np.zeros((len(keys), D), np.float64)
+    _check(_load().orc_bwd_dkv_keys_fwd(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, o, lse,
+                                        dout, ds, len(keys), keys, dk, dv), "bwd_dkv_keys_fwd")
     return dk, dv
 
 

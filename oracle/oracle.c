@@ -339,6 +339,55 @@ int orc_bwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double sca
 }
 
 /*
+ * dK, dV for selected keys only (keys_sel[i] = bkv*S + k, original k), from the
+ * oracle's own forward results o / lse of every row (the arrays orc_fwd
+ * writes): the same sum as orc_bwd, restricted to the selected keys,
+ *   dV_k = sum_q P_qk dO_q,  dK_k = scale sum_q P_qk (dO_q.v_k - dO_q.O_q) q_q,
+ * over the admitted rows q >= k of the group's query heads.  Each row's O and
+ * LSE are read, not recomputed, so a key costs O(S D) instead of a forward per
+ * row.
+ */
+int orc_bwd_dkv_keys_fwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
+                         const double *q, const double *k, const double *v, const double *o,
+                         const double *lse, const double *dout, const int32_t *ds_orig,
+                         int64_t nkeys, const int64_t *keys_sel, double *dk, double *dv)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0) return ORC_EINVAL;
+    int64_t g = Hq / Hkv, SD = (int64_t)S * D;
+    for (int64_t i = 0; i < nkeys; ++i)
+        if (keys_sel[i] < 0 || keys_sel[i] >= (int64_t)B * Hkv * S) return ORC_EINVAL;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nkeys; ++i) {
+        int64_t bkv = keys_sel[i] / S, kk = keys_sel[i] % S;
+        int64_t b = bkv / Hkv, hk = bkv % Hkv;
+        const double *kv = k + bkv * SD + kk * D, *vv = v + bkv * SD + kk * D;
+        double *dkv = dk + i * D, *dvv = dv + i * D;
+        for (int64_t d = 0; d < D; ++d) { dkv[d] = 0.0; dvv[d] = 0.0; }
+        for (int64_t h = hk * g; h < (hk + 1) * g; ++h) {
+            int64_t bh = b * Hq + h;
+            for (int64_t qi = kk; qi < S; ++qi) {
+                if (!orc_mask(ds_orig, qi, kk)) continue;
+                const double *qv = q + (bh * S + qi) * D, *ov = o + (bh * S + qi) * D;
+                const double *dov = dout + (bh * S + qi) * D;
+                double Dq = 0.0, dot = 0.0, dP = 0.0;
+                for (int64_t d = 0; d < D; ++d) {
+                    Dq += dov[d] * ov[d];
+                    dot += qv[d] * kv[d];
+                    dP += dov[d] * vv[d];
+                }
+                double P = exp(scale * dot - lse[bh * S + qi]);
+                double dS = P * (dP - Dq);
+                for (int64_t d = 0; d < D; ++d) {
+                    dvv[d] += P * dov[d];
+                    dkv[d] += scale * dS * qv[d];
+                }
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/*
  * dQ for selected rows only (rows[i] = bh*S + q), each from its own forward:
  * the row's LSE and O are recomputed by the definition first.
  */

@@ -27,3 +27,19 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With CP_PARITY_REPORT=<path>, write every bf16 comparison the tests made
+    (name, max / mean error, elements beyond the plain 2e-2, worst element in
+    bf16 ulps) as JSON: the per-configuration error table."""
+    path = os.environ.get("CP_PARITY_REPORT")
+    if not path:
+        return
+    try:
+        import helpers
+    except Exception:  # pragma: no cover
+        return
+    import json
+    with open(path, "w") as f:
+        json.dump(helpers.PARITY_LOG, f, indent=1)

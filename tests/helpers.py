@@ -22,23 +22,45 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.exp2(np.floor(np.log2(ax)) - 7)
 
 
+# Every comparison made through assert_bf16_close, for the per-configuration
+# error report (written by conftest.py when CP_PARITY_REPORT names a file).
+PARITY_LOG: list = []
+
+
+def bf16_bound(ref: np.ndarray, max_abs: float = O_MAX) -> np.ndarray:
+    """Per-element bound: the stated 2e-2 plus half a bf16 ulp of the reference value.
+    A bf16 output cannot land closer to the exact value than half an ulp (its own
+    rounding), so this is the 2e-2 budget on top of what the output format forces,
+    and nothing more: 0.0217 at |ref| 0.5, 0.0278 at 3, 0.0513 at 8."""
+    return max_abs + 0.5 * bf16_ulp(ref)
+
+
+def parity_stats(gpu: np.ndarray, ref: np.ndarray, max_abs: float = O_MAX) -> dict:
+    """Error summary of one comparison: max / mean error, how many elements exceed the
+    plain 2e-2, and the worst element measured against its bound, in bf16 ulps of
+    the reference value."""
+    err = np.abs(gpu - ref)
+    bound = bf16_bound(ref, max_abs)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    return dict(n=int(err.size), max=float(err.max()), mean=float(err.mean()),
+                n_over_abs=int((err > max_abs).sum()), n_over_bound=int((err > bound).sum()),
+                worst_err=float(err[worst]), worst_ref=float(abs(ref[worst])),
+                worst_bound=float(bound[worst]),
+                worst_ulps=float(err[worst] / bf16_ulp(np.asarray(ref[worst]))))
+
+
 def assert_bf16_close(gpu: np.ndarray, ref: np.ndarray, what: str, max_abs=O_MAX, mean_abs=O_MEAN):
-    """Element bound: |err| <= max(max_abs, 2^-6 |ref|).  The absolute bound governs
-    every |ref| <= 1.28; above that the bound is four bf16 unit roundoffs of the
-    value: bf16 cannot hold such values closely (half an ulp is 0.0156 at 4 and
-    0.031 at 8), and the bf16 P / dS operands of any tensor-core attention add
-    errors of the same order (a numpy emulation of those roundings reproduces the
-    GPU's errors to four digits).  Mean bound: mean |err| <= mean_abs."""
+    """Element bound |err| <= 2e-2 + ulp_bf16(ref)/2 (bf16_bound); mean bound
+    mean |err| <= 2e-3."""
     assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
     assert np.isfinite(gpu).all(), f"{what}: non-finite values"
-    err = np.abs(gpu - ref)
-    bound = np.maximum(max_abs, np.abs(ref) * 2.0 ** -6)
-    worst = np.unravel_index(np.argmax(err - bound), err.shape)
-    mx, mn = float(err.max()), float(err.mean())
-    ok = bool((err <= bound).all()) and mn <= mean_abs
-    assert ok, (f"{what}: max {mx:.3e} mean {mn:.3e}; worst vs bound: err {err[worst]:.3e} "
-                f"at |ref| {abs(ref[worst]):.3f} (bound {bound[worst]:.3e})")
-    return mx, mn
+    st = parity_stats(gpu, ref, max_abs)
+    PARITY_LOG.append(dict(what=what, **st))
+    ok = st["n_over_bound"] == 0 and st["mean"] <= mean_abs
+    assert ok, (f"{what}: max {st['max']:.3e} mean {st['mean']:.3e}; {st['n_over_bound']} of "
+                f"{st['n']} over the bound; worst: err {st['worst_err']:.3e} at |ref| "
+                f"{st['worst_ref']:.3f} (bound {st['worst_bound']:.3e})")
+    return st["max"], st["mean"]
 
 
 def assert_lse_close(gpu: np.ndarray, ref: np.ndarray, what: str, tol=LSE_MAX):

@@ -176,3 +176,70 @@ def test_workspace_taken_when_large_enough():
     assert small is not ws and small.numel() == 1024
     with pytest.raises(ValueError, match="ws"):
         cz._workspace(100, torch.device("meta"), ws)              # on another device
+
+
+def test_problem_checks_cu_seqlens():
+    """cu_seqlens reaches the kernels as a raw int32 device pointer: anything else
+    (a host tensor, int64, strided, too short) is refused when the Problem is made."""
+    with pytest.raises(ValueError, match="int32 CUDA"):
+        cz.Problem(B, S, CP, Hq, Hkv, D, cu_seqlens=torch.tensor([0, S], dtype=torch.int32))
+    with pytest.raises(ValueError, match="int32 CUDA"):
+        cz.Problem(B, S, CP, Hq, Hkv, D, cu_seqlens=torch.tensor([0, S], dtype=torch.int64))
+    with pytest.raises(TypeError):
+        cz.Problem(B, S, CP, Hq, Hkv, D, cu_seqlens=[0, S])
+
+
+class _DevTensor:
+    """Just enough of a CUDA int32 tensor for Problem's checks (CPU machine)."""
+
+    def __init__(self, n):
+        self.t = torch.arange(n, dtype=torch.int32)
+        self.dtype, self.device = torch.int32, torch.device("cuda", 0)
+        self.shape = self.t.shape
+
+    def dim(self):
+        return 1
+
+    def numel(self):
+        return self.t.numel()
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return 0
+
+
+def test_problem_cu_seqlens_shape_checked(monkeypatch):
+    monkeypatch.setattr(torch, "Tensor", (torch.Tensor, _DevTensor))
+    with pytest.raises(ValueError, match="num_docs"):
+        cz.Problem(B, S, CP, Hq, Hkv, D, cu_seqlens=_DevTensor(1))
+
+
+def test_plan_must_fit_problem(cpu_binding):
+    """A plan built for another seq_len, cp, order or document list is refused
+    before the kernels index its arrays with the problem's sizes."""
+    t = tensors()
+    args = (t["q"], t["k"], t["v"], t["o"], t["lse"])
+    p = prob()
+    for other in (cz.Problem(B, 2 * S, CP, Hq, Hkv, D), cz.Problem(B, S, 2 * CP, Hq, Hkv, D),
+                  cz.Problem(B, S, CP, Hq, Hkv, D, rotate="ring")):
+        with pytest.raises(ValueError, match="plan: built for"):
+            cz.attn_fwd(p, _cpu_plan(other), *args)
+        with pytest.raises(ValueError, match="plan: built for"):
+            cz.attn_bwd(p, _cpu_plan(other), *args, t["do"], t["dq"], t["dk"], t["dv"])
+        with pytest.raises(ValueError, match="plan: built for"):
+            cz.attn_bwd_noalloc(p, _cpu_plan(other), *args, t["do"], t["dq"], t["dk"], t["dv"])
+    with pytest.raises(TypeError, match="Plan"):
+        cz.attn_fwd(p, None, *args)
+    # documents: a plan made without them does not serve a problem that has them
+    docs = object.__new__(cz.Problem)
+    docs.__dict__.update(p.__dict__)
+    docs.cu_seqlens = torch.tensor([0, 100, S], dtype=torch.int32)
+    with pytest.raises(ValueError, match="other documents"):
+        cz.attn_fwd(docs, _cpu_plan(p), *args)
+    # and a plan on another device
+    plan = _cpu_plan(p)
+    plan.perm = torch.zeros(S, dtype=torch.int32, device="meta")
+    with pytest.raises(ValueError, match="plan: on"):
+        cz.attn_fwd(p, plan, *args)

@@ -344,6 +344,27 @@ def test_bwd_sampled_equals_full():
     sk, sv = oracle.bwd_dkv_keys(q, k, v, dout, keys, ds)
     np.testing.assert_allclose(sk, dk.reshape(-1, D)[keys], atol=1e-13)
     np.testing.assert_allclose(sv, dv.reshape(-1, D)[keys], atol=1e-13)
+    # the keys-only form that reads the forward's O / LSE instead of recomputing rows
+    fk, fv = oracle.bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds)
+    np.testing.assert_allclose(fk, dk.reshape(-1, D)[keys], atol=1e-13)
+    np.testing.assert_allclose(fv, dv.reshape(-1, D)[keys], atol=1e-13)
+
+
+def test_bwd_keys_from_forward_batch2():
+    """bwd_dkv_keys_fwd indexes batch and KV head: batch 2, GQA 3:1, keys of every
+    (batch, KV head), against the full backward."""
+    B, Hq, Hkv, S, D = 2, 6, 2, 30, 8
+    q, k, v = rnd((B, Hq, S, D), 48), rnd((B, Hkv, S, D), 49), rnd((B, Hkv, S, D), 50)
+    dout = rnd((B, Hq, S, D), 51)
+    ds = oracle.first_key(S, [0, 7, 30], window=9)
+    o, lse = oracle.fwd(q, k, v, ds)
+    _, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds)
+    keys = np.array([0, 6, 7, S + 3, 2 * S + 29, 3 * S + 0, 3 * S + 15])
+    fk, fv = oracle.bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds)
+    np.testing.assert_allclose(fk, dk.reshape(-1, D)[keys], atol=1e-13)
+    np.testing.assert_allclose(fv, dv.reshape(-1, D)[keys], atol=1e-13)
+    with pytest.raises(ValueError):
+        oracle.bwd_dkv_keys_fwd(q, k, v, o, lse, dout, np.array([4 * S]), ds)
 
 
 # --------------------------------------------------------------- arithmetic pins
