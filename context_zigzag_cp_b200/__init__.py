@@ -26,7 +26,7 @@ from ._lib import CpPlan, CpProblem, STATUS_NAMES
 __all__ = ["CPError", "Problem", "Plan", "attn_fwd", "attn_bwd", "lse_merge",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "get_device_status",
            "set_wait_limit_ns", "selftest_wait_timeout", "version", "lib", "launch_count",
-           "LaunchTrace", "attn_bwd_noalloc"]
+           "LaunchTrace", "attn_bwd_noalloc", "selftest_stall"]
 
 
 class CPError(RuntimeError):
@@ -335,6 +335,31 @@ def set_wait_limit_ns(limit_ns: int) -> None:
 def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check(lib().cp_selftest_wait_timeout(int(limit_ns), _stream(stream)),
            "cp_selftest_wait_timeout")
+
+
+def selftest_stall(kernel: str, prob: Problem, plan: Plan, q, k, v, o, lse, do=None, dq=None,
+                   dk=None, dv=None, stream=None) -> None:
+    """cp_selftest_stall: run the forward (kernel "fwd") or the backward ("bwd_dkdv",
+    "bwd_dq") with CTA 0 of the named kernel never receiving its first K/V tile, so
+    that its bounded wait runs out (the test of the kernels' timeout teardown).
+    For "fwd", o and lse are outputs; for the backward they are inputs."""
+    kid = _lib.KERNEL_IDS.get(kernel, -1)
+    if kernel == "fwd":
+        qs, kvs, ls = _attn_shapes(prob)
+        _validate((q, qs, torch.bfloat16, "q"), (k, kvs, torch.bfloat16, "k"),
+                  (v, kvs, torch.bfloat16, "v"), (o, qs, torch.bfloat16, "o"),
+                  (lse, ls, torch.float32, "lse"))
+        _check_plan(prob, plan, q.device)
+        nbytes = fwd_workspace_bytes(prob)
+    else:
+        _validate_bwd(prob, plan, q, k, v, o, lse, do, dq, dk, dv)
+        nbytes = bwd_workspace_bytes(prob)
+    w = _workspace(nbytes, q.device, None)
+    n = ctypes.c_size_t(nbytes)
+    _check(lib().cp_selftest_stall(kid, prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                   _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(w),
+                                   ctypes.byref(n) if w is not None else None, _stream(stream)),
+           "cp_selftest_stall")
 
 
 def selftest_exp2(x: torch.Tensor, stream=None):

@@ -24,12 +24,13 @@ MERGE = {"separate": 0, "fused": 1}
 EXPORTED = ("cp_plan_shards", "cp_unshard", "cp_attn_fwd", "cp_attn_bwd", "cp_lse_merge",
             "cp_get_device_status", "cp_set_wait_limit_ns", "cp_selftest_wait_timeout",
             "cp_launch_count", "cp_trace_begin", "cp_trace_end", "cp_selftest_exp2",
-            "cp_attn_bwd_noalloc", "cp_version")
+            "cp_attn_bwd_noalloc", "cp_selftest_stall", "cp_version")
 
 NOALLOC_MAX_ROWS = 4194304
 
 KERNEL_NAMES = {1: "plan_meta", 2: "plan_index", 3: "gather", 4: "fwd", 5: "merge",
                 6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2"}
+KERNEL_IDS = {name: i for i, name in KERNEL_NAMES.items()}
 
 
 class CpProblem(ctypes.Structure):
@@ -80,6 +81,8 @@ def load() -> ctypes.CDLL:
     lib.cp_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
     lib.cp_trace_begin.argtypes = [ctypes.POINTER(vp), ctypes.c_int32]
     lib.cp_trace_end.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
+    lib.cp_selftest_stall.argtypes = [ctypes.c_int32, P, PL, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                      vp, sz, vp]
     for name in EXPORTED:
         getattr(lib, name).restype = ctypes.c_int32
     lib.cp_launch_count.restype = ctypes.c_int64

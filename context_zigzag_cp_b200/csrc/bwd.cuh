@@ -74,6 +74,7 @@ struct BwdParams {
     float scale;             // softmax scale
     float scale_log2;        // softmax scale * log2(e)
     int32_t n_items;
+    int32_t stall;           // test hook: the cp_kernel_t whose CTA 0 skips its first K/V load
     const int32_t* src;      // [cp*cp]
     const int32_t* doc_start;  // [S] shard order
     const int32_t* cu;       // [num_docs+1] document offsets, original order (documents only)
@@ -347,10 +348,13 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 ok = mbar_wait(bar_kv_empty, (iter & 1) ^ 1, abort_flag);
                 if (!ok) break;
                 kv_issued = true;
-                mbar_arrive_expect_tx(bar_kv_full, 2 * Cfg::TILE);
-                for (int h = 0; h < D / 64; ++h) {
-                    tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
-                    tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
+                // test hook (cp_selftest_stall): the first K/V tile of CTA 0 is never loaded
+                if (!(P.stall == 7 /* CP_K_BWD_DKDV */ && blockIdx.x == 0 && iter == 0)) {
+                    mbar_arrive_expect_tx(bar_kv_full, 2 * Cfg::TILE);
+                    for (int h = 0; h < D / 64; ++h) {
+                        tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
+                        tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
+                    }
                 }
                 for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
@@ -767,6 +771,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             const uint32_t slot = nload % Cfg::NSLOT, par = (nload / Cfg::NSLOT) & 1;
                             ok = mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, abort_flag);
                             if (!ok) break;
+                            // test hook (cp_selftest_stall): the tile is never loaded
+                            if (P.stall == 8 /* CP_K_BWD_DQ */ && blockIdx.x == 0 && nload == 0) continue;
                             mbar_arrive_expect_tx(bar_kv_full + 8 * slot, Cfg::KTILE);
                             for (int h = 0; h < D / 64; ++h)
                                 tma_load_2d(sKV + slot * Cfg::KTILE + h * 16384,

@@ -228,7 +228,7 @@ cp_status_t check_bufs(const cp_problem_t* p, int32_t n_bufs, const void* const*
 template <int D>
 cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, void* o, float* lse, float* o_parts, float* lse_parts,
-                       cudaStream_t stream)
+                       cudaStream_t stream, int stall)
 {
     using Cfg = FwdCfg<D>;
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
@@ -250,6 +250,7 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.scale_log2 = softmax_scale(p) * 1.4426950408889634f;
     P.ppc = (P.C + 255) / 256;
     P.n_items = P.BH * 2 * P.cp * P.ppc;
+    P.stall = stall;
     P.src = pl->src;
     P.doc_start = pl->doc_start;
     P.o = static_cast<__nv_bfloat16*>(o);
@@ -405,9 +406,13 @@ cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan, int32
                          as_stream(stream));
 }
 
-cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
-                        const void* k, const void* v, void* o, float* lse, void* ws,
-                        size_t* ws_bytes, void* stream)
+}  // extern "C"
+
+namespace {
+
+cp_status_t attn_fwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                          const void* k, const void* v, void* o, float* lse, void* ws,
+                          size_t* ws_bytes, void* stream, int stall)
 {
     cp_status_t st = check_attention(problem);
     if (st != CP_OK) return st;
@@ -423,10 +428,21 @@ cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, cons
     float* o_parts = separate ? static_cast<float*>(ws) : nullptr;
     float* lse_parts = separate ? reinterpret_cast<float*>(static_cast<char*>(ws) + o_parts_bytes) : nullptr;
     cudaStream_t s = as_stream(stream);
-    st = problem->head_dim == 128 ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s)
-                                  : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s);
+    st = problem->head_dim == 128 ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall)
+                                  : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall);
     if (st != CP_OK || !separate) return st;
     return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                        const void* k, const void* v, void* o, float* lse, void* ws,
+                        size_t* ws_bytes, void* stream)
+{
+    return attn_fwd_impl(problem, plan, q, k, v, o, lse, ws, ws_bytes, stream, 0);
 }
 
 cp_status_t cp_lse_merge(int64_t rows, int32_t head_dim, int32_t n_parts, const float* o_parts,
@@ -481,7 +497,8 @@ namespace {
 template <int D>
 cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, const void* o, const float* lse, const void* dout, void* dq,
-                       void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream)
+                       void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream,
+                       int stall = 0)
 {
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
     const int64_t rows = static_cast<int64_t>(B) * Hq * S;
@@ -521,6 +538,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.dq = static_cast<__nv_bfloat16*>(dq);
     P.dk = static_cast<__nv_bfloat16*>(dk);
     P.dv = static_cast<__nv_bfloat16*>(dv);
+    P.stall = stall;
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_BWD128 : ATTR_BWD64, [] {
         cudaError_t e = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -547,10 +565,12 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
 
 }  // namespace
 
-extern "C" cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
-                                   const void* k, const void* v, const void* o, const float* lse,
-                                   const void* dout, void* dq, void* dk, void* dv, void* ws,
-                                   size_t* ws_bytes, void* stream)
+namespace {
+
+cp_status_t attn_bwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                          const void* k, const void* v, const void* o, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, void* ws,
+                          size_t* ws_bytes, void* stream, int stall)
 {
     cp_status_t st = check_attention(problem);
     if (st != CP_OK) return st;
@@ -565,8 +585,32 @@ extern "C" cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t*
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     cudaStream_t s = as_stream(stream);
     return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s);
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall);
+}
+
+}  // namespace
+
+extern "C" cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
+                                   const void* k, const void* v, const void* o, const float* lse,
+                                   const void* dout, void* dq, void* dk, void* dv, void* ws,
+                                   size_t* ws_bytes, void* stream)
+{
+    return attn_bwd_impl(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, stream, 0);
+}
+
+extern "C" cp_status_t cp_selftest_stall(int32_t kernel, const cp_problem_t* problem,
+                                         const cp_plan_t* plan, const void* q, const void* k,
+                                         const void* v, void* o, float* lse, const void* dout,
+                                         void* dq, void* dk, void* dv, void* ws, size_t* ws_bytes,
+                                         void* stream)
+{
+    if (kernel == CP_K_FWD)
+        return attn_fwd_impl(problem, plan, q, k, v, o, lse, ws, ws_bytes, stream, 1);
+    if (kernel == CP_K_BWD_DKDV || kernel == CP_K_BWD_DQ)
+        return attn_bwd_impl(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, stream,
+                             kernel);
+    return CP_ERR_INVALID_ARG;
 }
 
 // ---------------------------------------------------------------------------

@@ -47,6 +47,7 @@ struct FwdParams {
     int32_t fused;                  // 1 = CP_MERGE_FUSED
     float scale_log2;               // softmax scale * log2(e)
     int32_t n_items, ppc;           // items, query-tile pairs per chunk
+    int32_t stall;                  // test hook: 1 = CTA 0 skips its first K/V load
     const int32_t* src;             // [cp*cp]
     const int32_t* doc_start;       // [S] shard order
     __nv_bfloat16* o;               // [BH][S][D]  (fused)
@@ -302,6 +303,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             const uint32_t par = (nload / Cfg::NSLOT) & 1;
                             ok = mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, abort_flag);
                             if (!ok) break;
+                            // test hook (cp_selftest_stall): the tile is never loaded, so the
+                            // MMA warp's bounded wait on it runs out and the CTA tears down
+                            if (P.stall && blockIdx.x == 0 && nload == 0) continue;
                             mbar_arrive_expect_tx(bar_kv_full + 8 * slot, Cfg::TILE_BYTES);
                             for (int h = 0; h < D / 64; ++h)
                                 tma_load_2d(sKV + slot * Cfg::TILE_BYTES + h * 16384,

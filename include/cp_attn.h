@@ -279,6 +279,26 @@ CP_API cp_status_t cp_set_wait_limit_ns(uint64_t limit_ns);
  * CP_ERR_TIMEOUT in the device status word.  The GPU context stays usable. */
 CP_API cp_status_t cp_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* Test hook of the bounded-wait teardown inside the attention kernels.  Runs
+ * cp_attn_fwd (kernel = CP_K_FWD) or cp_attn_bwd (kernel = CP_K_BWD_DKDV or
+ * CP_K_BWD_DQ) with the same arguments and checks as those calls (o and lse are
+ * the forward's outputs or the backward's inputs; dout, dq, dk, dv are unused by
+ * CP_K_FWD and may be NULL there), except that in the named kernel the producer
+ * warp of CTA 0 skips its first K/V tile load.  The MMA warp of that CTA then
+ * waits on a barrier nothing completes: once the wait limit (cp_set_wait_limit_ns)
+ * passes it records CP_ERR_TIMEOUT in the device status word, the CTA's other
+ * warps give up their waits, the copies and tensor-core work already issued
+ * drain, the CTA frees its tensor memory and exits; every other CTA runs its
+ * work normally.  The outputs of CTA 0's work items are left unwritten.  After
+ * the call (and cp_get_device_status) the context is usable and later calls are
+ * unaffected.  Errors: as the call it runs; CP_ERR_INVALID_ARG for another
+ * kernel id. */
+CP_API cp_status_t cp_selftest_stall(int32_t kernel, const cp_problem_t* problem,
+                                     const cp_plan_t* plan, const void* q, const void* k,
+                                     const void* v, void* o, float* lse, const void* dout,
+                                     void* dq, void* dk, void* dv, void* ws, size_t* ws_bytes,
+                                     void* stream);
+
 /* Kernels of the library, as reported by the launch trace. */
 typedef enum {
     CP_K_PLAN_META = 1,  /* plan: cu_seqlens check, src table, segment lists */
