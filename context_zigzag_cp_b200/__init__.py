@@ -85,6 +85,8 @@ def _check_plan(prob: "Problem", plan: "Plan", dev) -> None:
     if (pp.seq_len, pp.cp, pp.rotate) != (prob.seq_len, prob.cp, prob.rotate):
         raise ValueError(f"plan: built for seq_len {pp.seq_len}, cp {pp.cp}, {pp.rotate}; the "
                          f"problem has seq_len {prob.seq_len}, cp {prob.cp}, {prob.rotate}")
+    if getattr(pp, "causal", True) != getattr(prob, "causal", True):
+        raise ValueError("plan: built for the other mask (causal / no causal mask)")
     if pp.cu_seqlens is not prob.cu_seqlens:
         same = (pp.cu_seqlens is not None and prob.cu_seqlens is not None
                 and pp.cu_seqlens.shape == prob.cu_seqlens.shape
@@ -116,11 +118,15 @@ def version() -> int:
 class Problem:
     """cp_problem_t.  ``cu_seqlens`` (int32, original order, device) turns on the
     packed-document mask; ``window`` > 0 adds a sliding window (the query at q
-    sees keys q - window < k <= q)."""
+    sees keys q - window < k <= q); ``causal=False`` drops the causal mask (every
+    query sees every key; no documents or window then)."""
 
     def __init__(self, batch: int, seq_len: int, cp: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, rotate: str = "allgather", cu_seqlens: torch.Tensor | None = None,
-                 merge: str = "fused", softmax_scale: float = 0.0, window: int = 0):
+                 merge: str = "fused", softmax_scale: float = 0.0, window: int = 0,
+                 causal: bool = True):
+        if not causal and (cu_seqlens is not None or window):
+            raise ValueError("causal=False takes no cu_seqlens and no window")
         if cu_seqlens is not None:
             if not isinstance(cu_seqlens, torch.Tensor):
                 raise TypeError("cu_seqlens: expected a torch.Tensor")
@@ -134,17 +140,18 @@ class Problem:
         self.window = window
         self.batch, self.seq_len, self.cp = batch, seq_len, cp
         self.num_heads, self.num_kv_heads, self.head_dim = num_heads, num_kv_heads, head_dim
-        self.rotate, self.merge = rotate, merge
+        self.rotate, self.merge, self.causal = rotate, merge, causal
         self.num_docs = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+        mask = "full" if not causal else ("causal" if cu_seqlens is None else "doc")
         self.c = CpProblem(batch, seq_len, cp, num_heads, num_kv_heads, head_dim,
-                           _lib.ROTATE[rotate], _lib.MASK["causal" if cu_seqlens is None else "doc"],
+                           _lib.ROTATE[rotate], _lib.MASK[mask],
                            _lib.MERGE[merge], float(softmax_scale), self.num_docs, int(window),
                            None if cu_seqlens is None else cu_seqlens.data_ptr())
 
     def with_merge(self, merge: str) -> "Problem":
         return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
                        self.head_dim, self.rotate, self.cu_seqlens, merge,
-                       self.c.softmax_scale, self.window)
+                       self.c.softmax_scale, self.window, self.causal)
 
     @property
     def ref(self):

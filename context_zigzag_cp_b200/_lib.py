@@ -17,7 +17,7 @@ STATUS_NAMES = {0: "CP_OK", 1: "CP_ERR_INVALID_ARG", 2: "CP_ERR_UNSUPPORTED", 3:
                 4: "CP_ERR_TIMEOUT", 5: "CP_ERR_WORKSPACE"}
 
 ROTATE = {"allgather": 0, "ring": 1}
-MASK = {"causal": 0, "doc": 1}
+MASK = {"causal": 0, "doc": 1, "full": 2}
 MERGE = {"separate": 0, "fused": 1}
 
 # Every function the header declares (checked against include/cp_attn.h by the tests).

@@ -71,6 +71,7 @@ struct BwdParams {
     int32_t B, Hq, Hkv, S, cp, C;
     int32_t docs;
     int32_t wm1;             // sliding window - 1 (larger than S: no window)
+    int32_t nc;              // last visible key of query q is q + nc: 0 causal, S none
     float scale;             // softmax scale
     float scale_log2;        // softmax scale * log2(e)
     int32_t n_items;
@@ -207,7 +208,8 @@ __device__ __forceinline__ void dq_ds16(const float* pv, const float* dp, float 
 // dK / dV pass
 // ============================================================================
 // One past the last query tile that can attend to the key tile at original ko:
-// queries come at or after the key (the loop starts at ko's tile), no later than
+// queries come at or after the key under the causal mask (the loop starts at
+// tile (ko - nc) / 128, ko's own tile when causal, tile 0 when not), no later than
 // the window allows, and inside the document of the tile's last key.
 __device__ __forceinline__ int dkdv_last_tile(const BwdParams& P, int ko, int ntq)
 {
@@ -356,12 +358,12 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
                     }
                 }
-                for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
+                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP) continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const int bh = it.b * P.Hq + it.hk * g + hq;
                         const size_t row = static_cast<size_t>(bh) * P.S + qpos;
@@ -451,12 +453,12 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0;
-                for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
+                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko) == TILE_SKIP) continue;
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP) continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
                         const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
@@ -531,12 +533,12 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const DkdvItem it = decode_dkdv(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = it.ko / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
+            for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                 const int qo = t * 128;
                 const int qpos = shard_of_orig(qo, P.C, P.cp);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                const int cls = classify_tile(qo, dsf, dsl, it.ko);
+                const int cls = classify_tile(qo, dsf, dsl, it.ko, P.nc);
                 if (cls == TILE_SKIP) continue;
                 for (int hq = 0; hq < g && ok; ++hq) {
                     const uint32_t qs = nst % Cfg::NQ, ds = nst % Cfg::NDO;
@@ -559,13 +561,16 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     if (lane == 0) mbar_arrive(bar_s_free);   // the MMA warp may compute the next S^T
 #pragma unroll
                     for (int j = 0; j < BWD_NSLICE; ++j) {
-                        const int thr = k_orig - (qo + 64 * j + 16 * wg);
+                        // column c (query qo + 64j + 16wg + c) is admitted when k - nc <= q
+                        // and q <= k + wm1: thr - nc <= c <= thr + wm1
+                        const int thr = k_orig - (qo + 64 * j + 16 * wg) - P.nc;
+                        const int wsp = P.wm1 + P.nc;
                         if (cls == TILE_FULL)
-                            dkdv_p16<0>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, P.wm1, k_orig);
+                            dkdv_p16<0>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, wsp, k_orig);
                         else if (!P.docs)
-                            dkdv_p16<1>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, P.wm1, k_orig);
+                            dkdv_p16<1>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, wsp, k_orig);
                         else
-                            dkdv_p16<2>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, P.wm1, k_orig);
+                            dkdv_p16<2>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, wsp, k_orig);
                     }
                     // ---- dP^T: copy out; every warp has its columns before packed results land there
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
@@ -762,11 +767,11 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, dsf, it.qo + 127, half, P.C, P.cp);
+                    const KtSpan ks = kt_span(j, dsf, it.qo + 127 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int kpos = j * n2c + kt * 128;
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                        if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
+                        if (classify_tile(it.qo, dsf, dsl, ko, P.nc) == TILE_SKIP) continue;
                         for (int kv = 0; kv < 2 && ok; ++kv, ++nload) {
                             const uint32_t slot = nload % Cfg::NSLOT, par = (nload / Cfg::NSLOT) & 1;
                             ok = mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, abort_flag);
@@ -840,10 +845,10 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 uint32_t prev_kslot = 0;
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, dsf, it.qo + 127, half, P.C, P.cp);
+                    const KtSpan ks = kt_span(j, dsf, it.qo + 127 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                        if (classify_tile(it.qo, dsf, dsl, ko) == TILE_SKIP) continue;
+                        if (classify_tile(it.qo, dsf, dsl, ko, P.nc) == TILE_SKIP) continue;
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
                         const uint32_t vslot = (nload + 1) % Cfg::NSLOT, vpar = ((nload + 1) / Cfg::NSLOT) & 1;
                         nload += 2;
@@ -949,17 +954,17 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             bool had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
-                const KtSpan ks = kt_span(j, dsf, it.qo + 127, half, P.C, P.cp);
+                const KtSpan ks = kt_span(j, dsf, it.qo + 127 + P.nc, half, P.C, P.cp);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                     const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                    const int cls = classify_tile(it.qo, dsf, dsl, ko);
+                    const int cls = classify_tile(it.qo, dsf, dsl, ko, P.nc);
                     if (cls == TILE_SKIP) continue;
                     // ---- S: copy out, release, and form P while dP is still being computed
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_st_ready, st_phase, abort_flag));
                     if (!ok) break;
                     st_phase ^= 1;
                     tc_fence_after();
-                    const int lo = ds_q - ko - 16 * wg, hi = q_orig - ko - 16 * wg;
+                    const int lo = ds_q - ko - 16 * wg, hi = q_orig + P.nc - ko - 16 * wg;
                     float sv[32], dp[32];
                     tmem_ld16f(tS, sv);
                     tmem_ld16f(tS + 64, sv + 16);

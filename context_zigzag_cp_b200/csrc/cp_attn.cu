@@ -81,10 +81,14 @@ cp_status_t check_problem(const cp_problem_t* p)
     if (p->seq_len % (2 * p->cp_size) != 0) return CP_ERR_INVALID_ARG;
     if (p->num_heads % p->num_kv_heads != 0) return CP_ERR_INVALID_ARG;
     if (p->rotate != CP_ROTATE_ALLGATHER && p->rotate != CP_ROTATE_RING) return CP_ERR_INVALID_ARG;
-    if (p->mask != CP_MASK_CAUSAL && p->mask != CP_MASK_DOC_CAUSAL) return CP_ERR_INVALID_ARG;
+    if (p->mask != CP_MASK_CAUSAL && p->mask != CP_MASK_DOC_CAUSAL && p->mask != CP_MASK_FULL)
+        return CP_ERR_INVALID_ARG;
     if (p->merge != CP_MERGE_SEPARATE && p->merge != CP_MERGE_FUSED) return CP_ERR_INVALID_ARG;
     if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return CP_ERR_INVALID_ARG;
     if (p->window < 0) return CP_ERR_INVALID_ARG;
+    // without the causal mask: no documents, and a window (one-sided) is not defined
+    if (p->mask == CP_MASK_FULL && (p->cu_seqlens || p->num_docs != 0)) return CP_ERR_INVALID_ARG;
+    if (p->mask == CP_MASK_FULL && p->window != 0) return CP_ERR_UNSUPPORTED;
     if (p->mask == CP_MASK_DOC_CAUSAL) {
         if (!p->cu_seqlens || p->num_docs < 1 || p->num_docs > p->seq_len) return CP_ERR_INVALID_ARG;
     }
@@ -122,6 +126,13 @@ cp_status_t check_plan(const cp_plan_t* pl, bool need_all)
 inline int32_t window_minus_one(const cp_problem_t* p)
 {
     return p->window > 0 ? p->window - 1 : p->seq_len + 256;
+}
+
+// Last visible key of the query at original position q is q + nc: nc = 0 under
+// the causal mask; nc = S (beyond every key) without it.
+inline int32_t noncausal_shift(const cp_problem_t* p)
+{
+    return p->mask == CP_MASK_FULL ? p->seq_len : 0;
 }
 
 inline float softmax_scale(const cp_problem_t* p)
@@ -246,6 +257,7 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.C = S / (2 * p->cp_size);
     P.docs = p->mask == CP_MASK_DOC_CAUSAL;
     P.wm1 = window_minus_one(p);
+    P.nc = noncausal_shift(p);
     P.fused = p->merge == CP_MERGE_FUSED;
     P.scale_log2 = softmax_scale(p) * 1.4426950408889634f;
     P.ppc = (P.C + 255) / 256;
@@ -369,6 +381,7 @@ cp_status_t cp_plan_shards(const cp_problem_t* problem, const cp_plan_t* plan, i
     P.C = P.S / (2 * P.cp);
     P.docs = problem->mask == CP_MASK_DOC_CAUSAL;
     P.wm1 = window_minus_one(problem);
+    P.causal = problem->mask != CP_MASK_FULL;
     P.num_docs = P.docs ? problem->num_docs : 1;
     P.rotate = problem->rotate;
     P.cu = problem->cu_seqlens;
@@ -525,6 +538,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.C = S / (2 * p->cp_size);
     P.docs = p->mask == CP_MASK_DOC_CAUSAL;
     P.wm1 = window_minus_one(p);
+    P.nc = noncausal_shift(p);
     P.scale = softmax_scale(p);
     P.scale_log2 = P.scale * 1.4426950408889634f;
     P.src = pl->src;

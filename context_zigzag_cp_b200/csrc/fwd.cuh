@@ -44,6 +44,7 @@ struct FwdParams {
     int32_t BH, Hq, Hkv, S, cp, C;  // BH = batch * Hq
     int32_t docs;                   // 1 = packed-document mask
     int32_t wm1;                    // sliding window - 1 (larger than S: no window)
+    int32_t nc;                     // last visible key of query q is q + nc: 0 causal, S none
     int32_t fused;                  // 1 = CP_MERGE_FUSED
     float scale_log2;               // softmax scale * log2(e)
     int32_t n_items, ppc;           // items, query-tile pairs per chunk
@@ -61,11 +62,12 @@ enum : int { TILE_SKIP = 0, TILE_FULL = 1, TILE_PARTIAL = 2 };
 // Query tile rows have original positions [qo, qo+127] and first visible keys
 // (document start, raised to q - W + 1 under a sliding window) between dsf
 // (first row) and dsl (last row); key tile keys [ko, ko+127].  A pair (q, k)
-// is admitted when first(q) <= k <= q.
-__device__ __forceinline__ int classify_tile(int qo, int dsf, int dsl, int ko)
+// is admitted when first(q) <= k <= q + nc: nc = 0 is the causal mask, nc = S
+// (larger than any k - q) leaves keys unbounded above (no causal mask).
+__device__ __forceinline__ int classify_tile(int qo, int dsf, int dsl, int ko, int nc)
 {
-    if (ko > qo + 127 || ko + 127 < dsf) return TILE_SKIP;
-    if (ko + 127 <= qo && ko >= dsl) return TILE_FULL;
+    if (ko > qo + 127 + nc || ko + 127 < dsf) return TILE_SKIP;
+    if (ko + 127 <= qo + nc && ko >= dsl) return TILE_FULL;
     return TILE_PARTIAL;
 }
 
@@ -290,13 +292,13 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                     it.bh * P.S + it.p0 + 128 * x, bar_q_full);
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1, half, P.C, P.cp);
+                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int kpos = j * n2c + kt * 128;
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                        const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
+                        const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko, P.nc) != TILE_SKIP;
                         const bool v1 = it.ntq == 2 &&
-                                        classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP;
+                                        classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko, P.nc) != TILE_SKIP;
                         if (!v0 && !v1) continue;
                         for (int kv = 0; kv < 2 && ok; ++kv, ++nload) {
                             const uint32_t slot = nload % Cfg::NSLOT;
@@ -345,11 +347,11 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 int n_tiles = 0;
                 for (int s = 0; s < P.cp; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1, half, P.C, P.cp);
+                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1; kt = kt_next(ks, kt)) {
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                        if (classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP ||
-                            (it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP))
+                        if (classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko, P.nc) != TILE_SKIP ||
+                            (it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko, P.nc) != TILE_SKIP))
                             ++n_tiles;
                     }
                 }
@@ -395,11 +397,11 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1, half, P.C, P.cp);
+                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                        const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko) != TILE_SKIP;
-                        const bool v1 = it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko) != TILE_SKIP;
+                        const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko, P.nc) != TILE_SKIP;
+                        const bool v1 = it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko, P.nc) != TILE_SKIP;
                         if (!v0 && !v1) continue;
                         const uint32_t kslot = ring_slot, kpar = ring_par;
                         if (++ring_slot == Cfg::NSLOT) { ring_slot = 0; ring_par ^= 1; }
@@ -472,10 +474,10 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool first = true, had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
-                const KtSpan ks = kt_span(j, ti.dsf[X], ti.qo[X] + 127, half, P.C, P.cp);
+                const KtSpan ks = kt_span(j, ti.dsf[X], ti.qo[X] + 127 + P.nc, half, P.C, P.cp);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                     const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
-                    const int cls = classify_tile(ti.qo[X], ti.dsf[X], ti.dsl[X], ko);
+                    const int cls = classify_tile(ti.qo[X], ti.dsf[X], ti.dsl[X], ko, P.nc);
                     if (cls == TILE_SKIP) continue;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * X, s_phase, abort_flag));
                     if (!ok) break;
@@ -492,7 +494,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     reg_fence32f(sf + 64);
                     reg_fence32f(sf + 96);
                     if (cls == TILE_PARTIAL) {
-                        const int lo = ds_row - ko, hi = q_orig - ko;
+                        const int lo = ds_row - ko, hi = q_orig + P.nc - ko;
 #pragma unroll
                         for (int c = 0; c < 128; ++c)
                             if (c < lo || c > hi) sf[c] = -INFINITY;

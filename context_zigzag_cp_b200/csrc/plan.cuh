@@ -20,6 +20,7 @@ constexpr int PLAN_MAX_CP = 1024;
 struct PlanParams {
     int32_t S, cp, C, num_docs, docs, rotate;
     int32_t wm1;        // sliding window - 1 (larger than S: no window)
+    int32_t causal;     // 0: every query sees every key (no causal mask, no documents)
     const int32_t* cu;  // [num_docs+1] original order (docs only)
     int32_t *perm, *inv_perm, *src, *doc_start, *rank_cu_off, *rank_cu;
     int64_t* pairs;
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(256) plan_meta_kernel(PlanParams P)
 
 // Grid over shard positions: perm, inv_perm, doc_start and the per-rank
 // unmasked pair counts (keys max(doc_start(o), o - wm1) .. o for the token at
-// original o).
+// original o under the causal mask; all S keys without it).
 __global__ void __launch_bounds__(256) plan_index_kernel(PlanParams P)
 {
     const int n2c = 2 * P.C;
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(256) plan_index_kernel(PlanParams P)
             P.inv_perm[o] = p;
             const int ds = P.docs ? __ldg(P.cu + doc_index(P.cu, P.num_docs, o)) : 0;
             P.doc_start[p] = ds;
-            cnt = static_cast<int64_t>(min(o - ds, P.wm1)) + 1;
+            cnt = P.causal ? static_cast<int64_t>(min(o - ds, P.wm1)) + 1 : static_cast<int64_t>(P.S);
         }
         // warp-level sum when the whole warp belongs to one rank, else per thread
         const int r0 = __shfl_sync(0xffffffffu, r, 0), r31 = __shfl_sync(0xffffffffu, r, 31);

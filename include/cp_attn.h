@@ -65,7 +65,11 @@ typedef enum {
 } cp_status_t;
 
 typedef enum { CP_ROTATE_ALLGATHER = 0, CP_ROTATE_RING = 1 } cp_rotate_t;
-typedef enum { CP_MASK_CAUSAL = 0, CP_MASK_DOC_CAUSAL = 1 } cp_mask_t;
+/* Masks.  CP_MASK_CAUSAL: the query at original position q sees keys k <= q.
+ * CP_MASK_DOC_CAUSAL: additionally only keys of its own document (cu_seqlens).
+ * CP_MASK_FULL: no mask, every query sees every key (bidirectional attention);
+ * it takes no documents (cu_seqlens NULL, num_docs 0) and no window. */
+typedef enum { CP_MASK_CAUSAL = 0, CP_MASK_DOC_CAUSAL = 1, CP_MASK_FULL = 2 } cp_mask_t;
 
 /* How cp_attn_fwd combines the per-step partial attentions.
  *   CP_MERGE_SEPARATE: each (rank, step) unit writes its partial (O, LSE) in
@@ -92,7 +96,8 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *   window        0: no window.  W > 0: sliding window on top of the mask --
  *                 the query at original position q sees only keys k with
  *                 q - W < k <= q (and, with documents, k in q's document).
- *                 Negative values are CP_ERR_INVALID_ARG.
+ *                 Negative values are CP_ERR_INVALID_ARG; W > 0 with
+ *                 CP_MASK_FULL is CP_ERR_UNSUPPORTED.
  *   cu_seqlens    DEVICE int32 [num_docs+1], 0 = cu[0] < cu[1] < ... <
  *                 cu[num_docs] = S, original order; the same documents apply to
  *                 every batch entry.  NULL for the plain causal mask.
@@ -134,7 +139,8 @@ typedef struct {
  *                                  chunks), then 2C
  *   pairs       int64 [cp]         unmasked (q, k) pairs whose query lives on
  *                                  rank r (equal across ranks for the plain
- *                                  causal mask without a window) */
+ *                                  causal mask without a window; 2C * S each
+ *                                  for CP_MASK_FULL) */
 typedef struct {
     int32_t* perm;
     int32_t* inv_perm;
@@ -177,8 +183,8 @@ CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan
 
 /*
  * cp_attn_fwd -- causal (optionally packed-document, optionally sliding-window)
- * attention of every virtual rank's query shard against the K/V shards in the
- * plan's visit order,
+ * or unmasked (CP_MASK_FULL) attention of every virtual rank's query shard
+ * against the K/V shards in the plan's visit order,
  * combined into the exact unsharded result (concept guide, "So how does it
  * work?": local attention, then every other shard, then combine).
  *   q     bf16 [B][Hq][S][D]  shard order

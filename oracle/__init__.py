@@ -61,24 +61,25 @@ def _load():
         lib = ctypes.CDLL(build())
         I32, I64, F64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         lib.orc_doc_start.argtypes = [I32, I32, _i32p, _i32p]
-        lib.orc_plan.argtypes = [I32, I32, I32, I32, _i32p, I32, _i32p, _i32p, _i32p, _i32p, _i32p,
-                                 _i32p, _i64p]
+        lib.orc_plan.argtypes = [I32, I32, I32, I32, _i32p, I32, I32, _i32p, _i32p, _i32p, _i32p,
+                                 _i32p, _i32p, _i64p]
         lib.orc_fwd_rows.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _i32p,
-                                     I64, _i64p, _f64p, _f64p]
-        lib.orc_fwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _i32p,
+                                     _i32p, I64, _i64p, _f64p, _f64p]
+        lib.orc_fwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _i32p, _i32p,
                                 _f64p, _f64p]
         lib.orc_partial.argtypes = [I32, I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
-                                    _i32p, _i32p, I32, I32, _f64p, _f64p]
+                                    _i32p, _i32p, _i32p, I32, I32, _f64p, _f64p]
         lib.orc_lse_merge.argtypes = [I64, I32, I32, _f64p, _f64p, _f64p, _f64p]
         lib.orc_lse_merge.restype = None
         lib.orc_bwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _f64p,
-                                _f64p, _f64p, _i32p, _f64p, _f64p, _f64p]
+                                _f64p, _f64p, _i32p, _i32p, _f64p, _f64p, _f64p]
         lib.orc_bwd_dq_rows.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
-                                        _f64p, _i32p, I64, _i64p, _f64p]
+                                        _f64p, _i32p, _i32p, I64, _i64p, _f64p]
         lib.orc_bwd_dkv_keys.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
-                                         _f64p, _i32p, I64, _i64p, _f64p, _f64p]
+                                         _f64p, _i32p, _i32p, I64, _i64p, _f64p, _f64p]
         lib.orc_bwd_dkv_keys_fwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
-                                             _f64p, _f64p, _f64p, _i32p, I64, _i64p, _f64p, _f64p]
+                                             _f64p, _f64p, _f64p, _i32p, _i32p, I64, _i64p, _f64p,
+                                             _f64p]
         lib.orc_num_threads.argtypes = []
         for name in ("orc_doc_start", "orc_plan", "orc_fwd_rows", "orc_fwd", "orc_partial",
                      "orc_bwd", "orc_bwd_dq_rows", "orc_bwd_dkv_keys", "orc_bwd_dkv_keys_fwd",
@@ -114,10 +115,12 @@ def doc_start(seq_len: int, cu_seqlens=None) -> np.ndarray:
     return ds
 
 
-def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None, window: int = 0) -> dict:
+def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None, window: int = 0,
+         causal: bool = True) -> dict:
     """The zigzag plan: perm, inv_perm, src, doc_start (shard order), rank_cu_off,
     rank_cu and pairs (int64), exactly as the library's planner must produce them.
-    ``window`` > 0 counts pairs under a sliding window (keys q-W < k <= q)."""
+    ``window`` > 0 counts pairs under a sliding window (keys q-W < k <= q);
+    ``causal`` False counts every key of the query's document."""
     lib = _load()
     cu = (np.zeros(1, dtype=np.int32) if cu_seqlens is None
           else np.ascontiguousarray(cu_seqlens, dtype=np.int32))
@@ -127,7 +130,8 @@ def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None, wind
                src=np.zeros(cp * cp, np.int32), doc_start=np.zeros(S, np.int32),
                rank_cu_off=np.zeros(cp + 1, np.int32),
                rank_cu=np.zeros(3 * cp + max(nd, 1), np.int32), pairs=np.zeros(cp, np.int64))
-    _check(lib.orc_plan(S, cp, ROTATE[rotate], nd, cu, int(window), out["perm"], out["inv_perm"],
+    _check(lib.orc_plan(S, cp, ROTATE[rotate], nd, cu, int(window), int(bool(causal)),
+                        out["perm"], out["inv_perm"],
                         out["src"], out["doc_start"], out["rank_cu_off"], out["rank_cu"],
                         out["pairs"]), "plan")
     out["rank_cu"] = out["rank_cu"][: out["rank_cu_off"][cp]].copy()
@@ -145,6 +149,23 @@ def first_key(seq_len: int, cu_seqlens=None, window: int = 0) -> np.ndarray:
     return ds
 
 
+def last_key(seq_len: int, cu_seqlens=None, causal: bool = True) -> np.ndarray:
+    """Per original position q, the last key q attends to: q itself under the causal
+    mask; without it, the last position of q's document (S - 1 with one document).
+    Every attention function here takes this array as ``lk_orig`` (None: causal)."""
+    if causal:
+        return np.arange(seq_len, dtype=np.int32)
+    if cu_seqlens is None:
+        return np.full(seq_len, seq_len - 1, dtype=np.int32)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    return np.repeat(cu[1:] - 1, np.diff(cu)).astype(np.int32)
+
+
+def _lk(S, lk_orig):
+    return (np.arange(S, dtype=np.int32) if lk_orig is None
+            else np.ascontiguousarray(lk_orig, np.int32))
+
+
 def _dims(q, k):
     B, Hq, S, D = q.shape
     assert k.shape[0] == B and k.shape[2] == S and k.shape[3] == D
@@ -155,18 +176,19 @@ def _scale(D, scale):
     return 1.0 / math.sqrt(D) if not scale else float(scale)
 
 
-def fwd(q, k, v, ds_orig=None, scale=None):
+def fwd(q, k, v, ds_orig=None, scale=None, lk_orig=None):
     """Unsharded attention: O [B,Hq,S,D], LSE [B,Hq,S] (natural log), original order."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, S, D = _dims(q, k)
     ds = np.zeros(S, np.int32) if ds_orig is None else np.ascontiguousarray(ds_orig, np.int32)
     o = np.zeros(q.shape, np.float64)
     lse = np.zeros((B, Hq, S), np.float64)
-    _check(_load().orc_fwd(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, ds, o, lse), "fwd")
+    _check(_load().orc_fwd(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, ds, _lk(S, lk_orig), o,
+                           lse), "fwd")
     return o, lse
 
 
-def fwd_rows(q, k, v, rows, ds_orig=None, scale=None):
+def fwd_rows(q, k, v, rows, ds_orig=None, scale=None, lk_orig=None):
     """Unsharded attention at selected flat rows (bh*S + q_orig): O [n,D], LSE [n]."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, S, D = _dims(q, k)
@@ -174,12 +196,12 @@ def fwd_rows(q, k, v, rows, ds_orig=None, scale=None):
     rows = np.ascontiguousarray(rows, np.int64)
     o = np.zeros((len(rows), D), np.float64)
     lse = np.zeros(len(rows), np.float64)
-    _check(_load().orc_fwd_rows(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, ds, len(rows),
-                                rows, o, lse), "fwd_rows")
+    _check(_load().orc_fwd_rows(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, ds, _lk(S, lk_orig),
+                                len(rows), rows, o, lse), "fwd_rows")
     return o, lse
 
 
-def partial(q, k, v, perm, cp, r, j, ds_orig=None, scale=None):
+def partial(q, k, v, perm, cp, r, j, ds_orig=None, scale=None, lk_orig=None):
     """Partial attention of rank r's queries against rank j's keys:
     O [B*Hq, 2C, D], LSE [B*Hq, 2C] (rank-local shard order)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -189,7 +211,8 @@ def partial(q, k, v, perm, cp, r, j, ds_orig=None, scale=None):
     o = np.zeros((B * Hq, n2c, D), np.float64)
     lse = np.zeros((B * Hq, n2c), np.float64)
     _check(_load().orc_partial(B, Hq, Hkv, S, D, cp, _scale(D, scale), q, k, v, ds,
-                               np.ascontiguousarray(perm, np.int32), r, j, o, lse), "partial")
+                               _lk(S, lk_orig), np.ascontiguousarray(perm, np.int32), r, j, o, lse),
+           "partial")
     return o, lse
 
 
@@ -203,14 +226,16 @@ def lse_merge(o_parts, lse_parts):
     return o, lse
 
 
-def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=None, window=0):
+def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=None, window=0,
+           causal=True):
     """The sharded computation: for every rank r, the partials against K/V shard
     src[r][s] for each step s (all steps unless ``steps`` limits them), merged in
     visit order.  Returns O [B,Hq,S,D] and LSE [B,Hq,S] in SHARD order."""
     q = _f64(q)
     B, Hq, S, D = q.shape
-    pl = plan(S, cp, rotate, cu_seqlens, window)
+    pl = plan(S, cp, rotate, cu_seqlens, window, causal)
     ds = first_key(S, cu_seqlens, window)
+    lk = last_key(S, cu_seqlens, causal)
     n2c = S // cp
     o = np.zeros((B * Hq, S, D), np.float64)
     lse = np.zeros((B * Hq, S), np.float64)
@@ -219,7 +244,7 @@ def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=N
         parts_o, parts_l = [], []
         for s in range(nsteps):
             j = int(pl["src"][r * cp + s])
-            po, pl_ = partial(q, k, v, pl["perm"], cp, r, j, ds, scale)
+            po, pl_ = partial(q, k, v, pl["perm"], cp, r, j, ds, scale, lk)
             parts_o.append(po.reshape(-1, D))
             parts_l.append(pl_.reshape(-1))
         mo, ml = lse_merge(np.stack(parts_o), np.stack(parts_l))
@@ -228,7 +253,7 @@ def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=N
     return o.reshape(B, Hq, S, D), lse.reshape(B, Hq, S)
 
 
-def bwd(q, k, v, o, lse, dout, ds_orig=None, scale=None):
+def bwd(q, k, v, o, lse, dout, ds_orig=None, scale=None, lk_orig=None):
     """Explicit-P gradients: dQ [B,Hq,S,D], dK/dV [B,Hkv,S,D], original order."""
     q, k, v, o, lse, dout = map(_f64, (q, k, v, o, lse, dout))
     B, Hq, Hkv, S, D = _dims(q, k)
@@ -237,11 +262,11 @@ def bwd(q, k, v, o, lse, dout, ds_orig=None, scale=None):
     dk = np.zeros(k.shape, np.float64)
     dv = np.zeros(k.shape, np.float64)
     _check(_load().orc_bwd(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, o, lse, dout, ds,
-                           dq, dk, dv), "bwd")
+                           _lk(S, lk_orig), dq, dk, dv), "bwd")
     return dq, dk, dv
 
 
-def bwd_dq_rows(q, k, v, dout, rows, ds_orig=None, scale=None):
+def bwd_dq_rows(q, k, v, dout, rows, ds_orig=None, scale=None, lk_orig=None):
     """dQ at selected flat rows (bh*S + q_orig), each from its own forward: [n, D]."""
     q, k, v, dout = map(_f64, (q, k, v, dout))
     B, Hq, Hkv, S, D = _dims(q, k)
@@ -249,11 +274,11 @@ def bwd_dq_rows(q, k, v, dout, rows, ds_orig=None, scale=None):
     rows = np.ascontiguousarray(rows, np.int64)
     dq = np.zeros((len(rows), D), np.float64)
     _check(_load().orc_bwd_dq_rows(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, dout, ds,
-                                   len(rows), rows, dq), "bwd_dq_rows")
+                                   _lk(S, lk_orig), len(rows), rows, dq), "bwd_dq_rows")
     return dq
 
 
-def bwd_dkv_keys(q, k, v, dout, keys, ds_orig=None, scale=None):
+def bwd_dkv_keys(q, k, v, dout, keys, ds_orig=None, scale=None, lk_orig=None):
     """dK, dV at selected flat keys (bkv*S + k_orig): [n, D] each."""
     q, k, v, dout = map(_f64, (q, k, v, dout))
     B, Hq, Hkv, S, D = _dims(q, k)
@@ -262,11 +287,11 @@ def bwd_dkv_keys(q, k, v, dout, keys, ds_orig=None, scale=None):
     dk = np.zeros((len(keys), D), np.float64)
     dv = np.zeros((len(keys), D), np.float64)
     _check(_load().orc_bwd_dkv_keys(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, dout, ds,
-                                    len(keys), keys, dk, dv), "bwd_dkv_keys")
+                                    _lk(S, lk_orig), len(keys), keys, dk, dv), "bwd_dkv_keys")
     return dk, dv
 
 
-def bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds_orig=None, scale=None):
+def bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds_orig=None, scale=None, lk_orig=None):
     """dK, dV at selected flat keys (bkv*S + k_orig) from the oracle's own forward
     results o [B,Hq,S,D] / lse [B,Hq,S] of every row: [n, D] each.  The same sums
     as ``bwd``, restricted to the selected keys; each row's forward is read once
@@ -279,13 +304,19 @@ def bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds_orig=None, scale=None):
     dk = np.zeros((len(keys), D), np.float64)
     dv = np.zeros((len(keys), D), np.float64)
     _check(_load().orc_bwd_dkv_keys_fwd(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, o, lse,
-                                        dout, ds, len(keys), keys, dk, dv), "bwd_dkv_keys_fwd")
+                                        dout, ds, _lk(S, lk_orig), len(keys), keys, dk, dv),
+           "bwd_dkv_keys_fwd")
     return dk, dv
 
 
-def causal_pairs(seq_len: int, cu_seqlens=None, window: int = 0) -> int:
+def causal_pairs(seq_len: int, cu_seqlens=None, window: int = 0, causal: bool = True) -> int:
     """Number of unmasked (q, k) pairs per head: sum over documents of L(L+1)/2
-    (with a sliding window: sum over q of q - first_key(q) + 1)."""
+    (with a sliding window: sum over q of q - first_key(q) + 1); without the
+    causal mask, sum over documents of L^2."""
+    if not causal:
+        L = (np.array([seq_len], dtype=np.int64) if cu_seqlens is None
+             else np.diff(np.asarray(cu_seqlens, dtype=np.int64)))
+        return int((L * L).sum())
     if window and window > 0:
         fk = first_key(seq_len, cu_seqlens, window).astype(np.int64)
         return int((np.arange(seq_len, dtype=np.int64) - fk + 1).sum())

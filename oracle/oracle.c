@@ -78,15 +78,19 @@ int orc_doc_start(int32_t S, int32_t num_docs, const int32_t *cu, int32_t *ds_or
  *                     where a segment starts (local 0, the chunk boundary C,
  *                     and every document start inside its chunks), then 2C.
  *   pairs[r]        = number of unmasked (q, k) pairs whose query is on rank r;
- *                     with a sliding window W > 0 the query at o sees keys
- *                     max(ds(o), o - W + 1) .. o (window 0: no window)
+ *                     causal: the query at o sees keys ds(o) .. o, raised to
+ *                     max(ds(o), o - W + 1) under a sliding window W > 0
+ *                     (window 0: no window); without the causal mask
+ *                     (causal = 0) it sees its whole document, ds(o) ..
+ *                     de(o) - 1 (window: only 0 is accepted then)
  * Returns ORC_EINVAL on a bad configuration.
  */
 int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int32_t *cu,
-             int32_t window, int32_t *perm, int32_t *inv_perm, int32_t *src, int32_t *doc_start,
+             int32_t window, int32_t causal, int32_t *perm, int32_t *inv_perm, int32_t *src, int32_t *doc_start,
              int32_t *rank_cu_off, int32_t *rank_cu, int64_t *pairs)
 {
     if (cp < 1 || S <= 0 || S % (2 * cp) != 0 || window < 0) return ORC_EINVAL;
+    if (!causal && window != 0) return ORC_EINVAL;
     if (rotate != 0 && rotate != 1) return ORC_EINVAL;
     int64_t C = S / (2 * cp);
     int32_t *ds_orig = (int32_t *)malloc(sizeof(int32_t) * (size_t)S);
@@ -114,7 +118,13 @@ int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int3
             if (is_start) rank_cu[n++] = (int32_t)t;
             int64_t first = ds_orig[o];
             if (window > 0 && o - window + 1 > first) first = o - window + 1;
-            cnt += o - first + 1; /* keys first..o are unmasked */
+            int64_t last = o;
+            if (!causal) { /* the end of o's document: the next document's start, or S */
+                last = S - 1;
+                for (int64_t d = 0; d < num_docs; ++d)
+                    if (cu[d] > o) { last = cu[d] - 1; break; }
+            }
+            cnt += last - first + 1; /* keys first..last are unmasked */
         }
         rank_cu[n++] = (int32_t)(2 * C);
         pairs[r] = cnt;
@@ -128,11 +138,13 @@ int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int3
 /* Attention by the definition                                               */
 /* ------------------------------------------------------------------------ */
 
-/* mask(q, k) for original positions: causal (k <= q) and same document
- * (k >= doc start of q). */
-static int orc_mask(const int32_t *ds_orig, int64_t q, int64_t k)
+/* mask(q, k) for original positions: the query at q sees the keys
+ * ds_orig[q] <= k <= lk_orig[q].  Causal: lk_orig[q] = q; without the causal
+ * mask: the last key of q's document (S - 1 with one document).  ds_orig[q] is
+ * q's document start, raised to q - W + 1 under a sliding window of W keys. */
+static int orc_mask(const int32_t *ds_orig, const int32_t *lk_orig, int64_t q, int64_t k)
 {
-    return k <= q && k >= ds_orig[q];
+    return k <= lk_orig[q] && k >= ds_orig[q];
 }
 
 /*
@@ -144,12 +156,13 @@ static int orc_mask(const int32_t *ds_orig, int64_t q, int64_t k)
  */
 static void orc_row(int64_t D, double scale, const double *q_vec, int64_t q_orig,
                     const double *kmat, const double *vmat, const int64_t *keys, int64_t nk,
-                    const int32_t *ds_orig, double *sc, double *o, double *lse)
+                    const int32_t *ds_orig, const int32_t *lk_orig, double *sc, double *o,
+                    double *lse)
 {
     double m = -INFINITY;
     for (int64_t i = 0; i < nk; ++i) {
         int64_t k = keys[i];
-        if (!orc_mask(ds_orig, q_orig, k)) { sc[i] = -INFINITY; continue; }
+        if (!orc_mask(ds_orig, lk_orig, q_orig, k)) { sc[i] = -INFINITY; continue; }
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d) dot += q_vec[d] * kmat[k * D + d];
         sc[i] = scale * dot;
@@ -172,11 +185,12 @@ static void orc_row(int64_t D, double scale, const double *q_vec, int64_t q_orig
 /*
  * Unsharded attention for selected rows.  rows[i] = bh*S + q (original q).
  * GQA: query head h of batch b reads KV head h / (Hq/Hkv) of batch b.
- * Output o[i][D], lse[i].  Keys visited: 0..q (the mask trims the rest).
+ * Output o[i][D], lse[i].  Keys visited: 0..lk_orig[q] (the mask trims the rest).
  */
 int orc_fwd_rows(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
                  const double *q, const double *k, const double *v, const int32_t *ds_orig,
-                 int64_t nrows, const int64_t *rows, double *o, double *lse)
+                 const int32_t *lk_orig, int64_t nrows, const int64_t *rows, double *o,
+                 double *lse)
 {
     if (Hkv <= 0 || Hq % Hkv != 0) return ORC_EINVAL;
     int64_t g = Hq / Hkv;
@@ -196,7 +210,8 @@ int orc_fwd_rows(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, doubl
                 int64_t b = bh / Hq, h = bh % Hq;
                 int64_t bkv = b * Hkv + h / g;
                 orc_row(D, scale, q + (bh * S + qi) * D, qi, k + bkv * (int64_t)S * D,
-                        v + bkv * (int64_t)S * D, keys, qi + 1, ds_orig, sc, o + i * D, lse + i);
+                        v + bkv * (int64_t)S * D, keys, (int64_t)lk_orig[qi] + 1, ds_orig, lk_orig,
+                        sc, o + i * D, lse + i);
             }
         }
         free(sc);
@@ -209,13 +224,13 @@ int orc_fwd_rows(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, doubl
 /* Unsharded attention over every row: o[BH][S][D], lse[BH][S] (original order). */
 int orc_fwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
             const double *q, const double *k, const double *v, const int32_t *ds_orig,
-            double *o, double *lse)
+            const int32_t *lk_orig, double *o, double *lse)
 {
     int64_t n = (int64_t)B * Hq * S;
     int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
     if (!rows) return ORC_EINVAL;
     for (int64_t i = 0; i < n; ++i) rows[i] = i;
-    int rc = orc_fwd_rows(B, Hq, Hkv, S, D, scale, q, k, v, ds_orig, n, rows, o, lse);
+    int rc = orc_fwd_rows(B, Hq, Hkv, S, D, scale, q, k, v, ds_orig, lk_orig, n, rows, o, lse);
     free(rows);
     return rc;
 }
@@ -228,8 +243,8 @@ int orc_fwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double sca
  */
 int orc_partial(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, int32_t cp,
                 double scale, const double *q, const double *k, const double *v,
-                const int32_t *ds_orig, const int32_t *perm, int32_t r, int32_t j,
-                double *o_part, double *lse_part)
+                const int32_t *ds_orig, const int32_t *lk_orig, const int32_t *perm, int32_t r,
+                int32_t j, double *o_part, double *lse_part)
 {
     if (Hkv <= 0 || Hq % Hkv != 0 || S % (2 * cp) != 0) return ORC_EINVAL;
     int64_t g = Hq / Hkv, n2c = S / cp, BH = (int64_t)B * Hq;
@@ -245,7 +260,7 @@ int orc_partial(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, int32_
             int64_t b = bh / Hq, h = bh % Hq, bkv = b * Hkv + h / g;
             int64_t qi = perm[(int64_t)r * n2c + t];
             orc_row(D, scale, q + (bh * S + qi) * D, qi, k + bkv * (int64_t)S * D,
-                    v + bkv * (int64_t)S * D, keys, n2c, ds_orig, sc, o_part + i * D,
+                    v + bkv * (int64_t)S * D, keys, n2c, ds_orig, lk_orig, sc, o_part + i * D,
                     lse_part + i);
         }
         free(sc);
@@ -299,7 +314,7 @@ void orc_lse_merge(int64_t rows, int32_t D, int32_t n_parts, const double *o_par
 int orc_bwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
             const double *q, const double *k, const double *v, const double *o,
             const double *lse, const double *dout, const int32_t *ds_orig,
-            double *dq, double *dk, double *dv)
+            const int32_t *lk_orig, double *dq, double *dk, double *dv)
 {
     if (Hkv <= 0 || Hq % Hkv != 0) return ORC_EINVAL;
     int64_t g = Hq / Hkv, SD = (int64_t)S * D;
@@ -320,7 +335,7 @@ int orc_bwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double sca
                 double *dqv = dq + (bh * S + qi) * D;
                 double L = lse[bh * S + qi], Dq = 0.0;
                 for (int64_t d = 0; d < D; ++d) Dq += dov[d] * ov[d];
-                for (int64_t kk = ds_orig[qi]; kk <= qi; ++kk) {
+                for (int64_t kk = ds_orig[qi]; kk <= lk_orig[qi]; ++kk) {
                     const double *kv = kh + kk * D, *vv = vh + kk * D;
                     double dot = 0.0, dP = 0.0;
                     for (int64_t d = 0; d < D; ++d) { dot += qv[d] * kv[d]; dP += dov[d] * vv[d]; }
@@ -343,14 +358,15 @@ int orc_bwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double sca
  * oracle's own forward results o / lse of every row (the arrays orc_fwd
  * writes): the same sum as orc_bwd, restricted to the selected keys,
  *   dV_k = sum_q P_qk dO_q,  dK_k = scale sum_q P_qk (dO_q.v_k - dO_q.O_q) q_q,
- * over the admitted rows q >= k of the group's query heads.  Each row's O and
+ * over the rows q that admit key k, in every query head of the group.  Each row's O and
  * LSE are read, not recomputed, so a key costs O(S D) instead of a forward per
  * row.
  */
 int orc_bwd_dkv_keys_fwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
                          const double *q, const double *k, const double *v, const double *o,
                          const double *lse, const double *dout, const int32_t *ds_orig,
-                         int64_t nkeys, const int64_t *keys_sel, double *dk, double *dv)
+                         const int32_t *lk_orig, int64_t nkeys, const int64_t *keys_sel,
+                         double *dk, double *dv)
 {
     if (Hkv <= 0 || Hq % Hkv != 0) return ORC_EINVAL;
     int64_t g = Hq / Hkv, SD = (int64_t)S * D;
@@ -365,8 +381,8 @@ int orc_bwd_dkv_keys_fwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t 
         for (int64_t d = 0; d < D; ++d) { dkv[d] = 0.0; dvv[d] = 0.0; }
         for (int64_t h = hk * g; h < (hk + 1) * g; ++h) {
             int64_t bh = b * Hq + h;
-            for (int64_t qi = kk; qi < S; ++qi) {
-                if (!orc_mask(ds_orig, qi, kk)) continue;
+            for (int64_t qi = 0; qi < S; ++qi) {
+                if (!orc_mask(ds_orig, lk_orig, qi, kk)) continue;
                 const double *qv = q + (bh * S + qi) * D, *ov = o + (bh * S + qi) * D;
                 const double *dov = dout + (bh * S + qi) * D;
                 double Dq = 0.0, dot = 0.0, dP = 0.0;
@@ -393,7 +409,8 @@ int orc_bwd_dkv_keys_fwd(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t 
  */
 int orc_bwd_dq_rows(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
                     const double *q, const double *k, const double *v, const double *dout,
-                    const int32_t *ds_orig, int64_t nrows, const int64_t *rows, double *dq)
+                    const int32_t *ds_orig, const int32_t *lk_orig, int64_t nrows,
+                    const int64_t *rows, double *dq)
 {
     if (Hkv <= 0 || Hq % Hkv != 0) return ORC_EINVAL;
     int64_t g = Hq / Hkv, SD = (int64_t)S * D;
@@ -410,12 +427,13 @@ int orc_bwd_dq_rows(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, do
             const double *qv = q + (bh * S + qi) * D, *dov = dout + (bh * S + qi) * D;
             const double *kh = k + bkv * SD, *vh = v + bkv * SD;
             double L;
-            orc_row(D, scale, qv, qi, kh, vh, keys, qi + 1, ds_orig, sc, orow, &L);
+            orc_row(D, scale, qv, qi, kh, vh, keys, (int64_t)lk_orig[qi] + 1, ds_orig, lk_orig, sc,
+                    orow, &L);
             double Dq = 0.0;
             for (int64_t d = 0; d < D; ++d) Dq += dov[d] * orow[d];
             double *dqv = dq + i * D;
             for (int64_t d = 0; d < D; ++d) dqv[d] = 0.0;
-            for (int64_t kk = ds_orig[qi]; kk <= qi; ++kk) {
+            for (int64_t kk = ds_orig[qi]; kk <= lk_orig[qi]; ++kk) {
                 double dot = 0.0, dP = 0.0;
                 for (int64_t d = 0; d < D; ++d) { dot += qv[d] * kh[kk * D + d]; dP += dov[d] * vh[kk * D + d]; }
                 double P = exp(scale * dot - L);
@@ -436,7 +454,8 @@ int orc_bwd_dq_rows(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, do
  */
 int orc_bwd_dkv_keys(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, double scale,
                      const double *q, const double *k, const double *v, const double *dout,
-                     const int32_t *ds_orig, int64_t nkeys, const int64_t *keys_sel,
+                     const int32_t *ds_orig, const int32_t *lk_orig, int64_t nkeys,
+                     const int64_t *keys_sel,
                      double *dk, double *dv)
 {
     if (Hkv <= 0 || Hq % Hkv != 0) return ORC_EINVAL;
@@ -456,11 +475,12 @@ int orc_bwd_dkv_keys(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, d
             for (int64_t d = 0; d < D; ++d) { dkv[d] = 0.0; dvv[d] = 0.0; }
             for (int64_t h = hk * g; h < (hk + 1) * g; ++h) {
                 int64_t bh = b * Hq + h;
-                for (int64_t qi = kk; qi < S; ++qi) {
-                    if (!orc_mask(ds_orig, qi, kk)) continue;
+                for (int64_t qi = 0; qi < S; ++qi) {
+                    if (!orc_mask(ds_orig, lk_orig, qi, kk)) continue;
                     const double *qv = q + (bh * S + qi) * D, *dov = dout + (bh * S + qi) * D;
                     double L;
-                    orc_row(D, scale, qv, qi, kh, vh, keys, qi + 1, ds_orig, sc, orow, &L);
+                    orc_row(D, scale, qv, qi, kh, vh, keys, (int64_t)lk_orig[qi] + 1, ds_orig,
+                            lk_orig, sc, orow, &L);
                     double Dq = 0.0, dot = 0.0, dP = 0.0;
                     for (int64_t d = 0; d < D; ++d) {
                         Dq += dov[d] * orow[d];

@@ -77,13 +77,17 @@ def random_docs(seq_len: int, seed: int, median: float, lo: int = 1, hi: int | N
                                               (lo, hi or seq_len)))
 
 
-def make_case(B, Hq, Hkv, S, D, cp, seed, amp=1.0, cu=None, with_dout=False, window=0):
+def make_case(B, Hq, Hkv, S, D, cp, seed, amp=1.0, cu=None, with_dout=False, window=0,
+              causal=True):
     """Seeded inputs on the CPU (original order) plus, per original position, the
-    first key it attends to (document start, raised by a sliding window)."""
+    first key it attends to (document start, raised by a sliding window) and the
+    last (itself under the causal mask, else the end of its document)."""
     t = synth.attn_inputs(B, Hq, Hkv, S, D, seed, amp=amp, with_dout=with_dout)
     t["cu_seqlens"] = cu
     t["window"] = window
+    t["causal"] = causal
     t["ds"] = oracle.first_key(S, cu, window)
+    t["lk"] = oracle.last_key(S, cu, causal)
     return t
 
 
@@ -93,7 +97,8 @@ def run_fwd(cz, case, cp, rotate="allgather", merge="fused", scale=0.0, dev="cud
     q, k, v = (case[n].to(dev) for n in ("q", "k", "v"))
     B, Hq, S, D = q.shape
     cu = None if case["cu_seqlens"] is None else torch.from_numpy(case["cu_seqlens"]).to(dev)
-    prob = cz.Problem(B, S, cp, Hq, k.shape[1], D, rotate, cu, merge, scale, case.get("window", 0))
+    prob = cz.Problem(B, S, cp, Hq, k.shape[1], D, rotate, cu, merge, scale, case.get("window", 0),
+                      case.get("causal", True))
     plan = cz.Plan(prob)
     qs, ks, vs = plan.shard([q, k, v])
     o, lse = cz.attn_fwd(prob, plan, qs, ks, vs)

@@ -179,3 +179,22 @@ def test_noalloc_limit_checked_on_host(lib):
                                         None) == _lib.CP_ERR_WORKSPACE
     assert cz.lib().cp_attn_bwd_noalloc(p.ref, ctypes.byref(plan), None, d, d, d, d, d, d, d, d,
                                         None) == _lib.CP_ERR_INVALID_ARG
+
+
+def test_full_mask_host_checks(lib):
+    """CP_MASK_FULL (no causal mask) takes no documents and no window."""
+    p = prob(causal=False)
+    assert p.c.mask == 2 and fwd_query(p)[0] == _lib.CP_OK
+    p.c.window = 5
+    assert fwd_query(p)[0] == _lib.CP_ERR_UNSUPPORTED
+    p = prob(causal=False)
+    p.c.num_docs = 2
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob(causal=False)
+    p.c.cu_seqlens = 256
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob()
+    p.c.mask = 3                     # no such mask
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    with pytest.raises(ValueError, match="causal=False"):
+        prob(causal=False, window=4)

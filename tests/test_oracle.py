@@ -480,3 +480,137 @@ def test_window_bwd_finite_differences():
             args[name] = xm
             lm = _loss(args["q"], args["k"], args["v"], dout, ds)
             assert abs((lp - lm) / (2 * eps) - gx[idx]) < 1e-6, (name, idx)
+
+
+# ------------------------------------------------- attention without the causal mask
+# (the bidirectional variant: every query sees every key of its document)
+
+def full_brute_force(q, k, v, cu, scale):
+    """Materialised score matrix with only the block-diagonal document mask (or none)
+    and an explicit softmax, written out here without the oracle's key ranges."""
+    B, Hq, S, D = q.shape
+    g = Hq // k.shape[1]
+    doc = np.zeros(S, np.int64) if cu is None else np.repeat(np.arange(len(cu) - 1), np.diff(cu))
+    mask = doc[:, None] == doc[None, :]
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, S))
+    for b in range(B):
+        for h in range(Hq):
+            s = np.where(mask, scale * q[b, h] @ k[b, h // g].T, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            o[b, h] = (e / e.sum(axis=1, keepdims=True)) @ v[b, h // g]
+            lse[b, h] = m[:, 0] + np.log(e.sum(axis=1))
+    return o, lse
+
+
+def test_last_key():
+    assert np.array_equal(oracle.last_key(5), np.arange(5))
+    assert np.array_equal(oracle.last_key(5, causal=False), [4] * 5)
+    assert np.array_equal(oracle.last_key(7, [0, 2, 7], causal=False), [1, 1, 6, 6, 6, 6, 6])
+
+
+@pytest.mark.parametrize("Hq,Hkv,S,D,docs", [(2, 2, 16, 8, None), (4, 2, 24, 4, [0, 5, 6, 24])])
+def test_noncausal_fwd_brute_force(Hq, Hkv, S, D, docs):
+    q, k, v = rnd((2, Hq, S, D), 61), rnd((2, Hkv, S, D), 62), rnd((2, Hkv, S, D), 63)
+    ds, lk = oracle.first_key(S, docs), oracle.last_key(S, docs, causal=False)
+    o, lse = oracle.fwd(q, k, v, ds, None, lk)
+    ro, rl = full_brute_force(q, k, v, docs, 1 / np.sqrt(D))
+    np.testing.assert_allclose(o, ro, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, atol=1e-12)
+
+
+def test_noncausal_matches_torch_sdpa_and_closed_form():
+    B, Hq, Hkv, S, D = 1, 4, 2, 40, 8
+    q, k, v = rnd((B, Hq, S, D), 64), rnd((B, Hkv, S, D), 65), rnd((B, Hkv, S, D), 66)
+    o, lse = oracle.fwd(q, k, v, None, None, oracle.last_key(S, causal=False))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x) for x in (q, k, v)), is_causal=False, enable_gqa=True).numpy()
+    np.testing.assert_allclose(o, ref, atol=1e-12)
+    # K = 0: every row is the mean of all V and LSE = ln S
+    o0, l0 = oracle.fwd(q, np.zeros_like(k), v, None, None, oracle.last_key(S, causal=False))
+    np.testing.assert_allclose(o0[0, 0], np.broadcast_to(v[0, 0].mean(0), (S, D)), atol=1e-12)
+    np.testing.assert_allclose(l0, np.log(S), atol=1e-12)
+
+
+@pytest.mark.parametrize("cp,rotate,docs", [(2, "allgather", None), (3, "ring", None),
+                                            (2, "ring", [0, 7, 30, 48])])
+def test_noncausal_sharded_merged_equals_unsharded(cp, rotate, docs):
+    S = 48
+    q, k, v = rnd((1, 2, S, 8), 67), rnd((1, 2, S, 8), 68), rnd((1, 2, S, 8), 69)
+    so, sl = oracle.cp_fwd(q, k, v, cp, rotate, docs, causal=False)
+    o, lse = oracle.fwd(q, k, v, oracle.first_key(S, docs), None,
+                        oracle.last_key(S, docs, causal=False))
+    perm = oracle.plan(S, cp, rotate, docs, causal=False)["perm"]
+    np.testing.assert_allclose(so, o[:, :, perm], atol=1e-12)
+    np.testing.assert_allclose(sl, lse[:, :, perm], atol=1e-12)
+
+
+def test_noncausal_plan_pairs():
+    """Every rank's 2C queries see all S keys: 2C*S pairs each (the zigzag changes
+    nothing); with documents, the pairs are the sum of L^2 over each rank's rows."""
+    for S, cp in ((512, 2), (8192, 4)):
+        pl = oracle.plan(S, cp, causal=False)
+        assert (pl["pairs"] == (S // cp) * S).all()
+        assert pl["pairs"].sum() == oracle.causal_pairs(S, causal=False) == S * S
+    cu = [0, 7, 30, 48]
+    pl = oracle.plan(48, 2, "ring", cu, causal=False)
+    L = np.repeat(np.diff(cu), np.diff(cu))                 # document length per position
+    per_rank = [int(L[pl["perm"][r * 24:(r + 1) * 24]].sum()) for r in range(2)]
+    assert list(pl["pairs"]) == per_rank
+    with pytest.raises(ValueError):
+        oracle.plan(48, 2, "ring", None, window=4, causal=False)
+
+
+def test_noncausal_bwd_finite_differences_and_autograd():
+    B, Hq, Hkv, S, D = 1, 4, 2, 16, 8
+    q, k, v = rnd((B, Hq, S, D), 70), rnd((B, Hkv, S, D), 71), rnd((B, Hkv, S, D), 72)
+    dout = rnd((B, Hq, S, D), 73)
+    cu = [0, 6, 16]
+    ds, lk = oracle.first_key(S, cu), oracle.last_key(S, cu, causal=False)
+    o, lse = oracle.fwd(q, k, v, ds, None, lk)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds, None, lk)
+    eps = 1e-6
+    g = np.random.default_rng(74)
+    for name, x, gx in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(10):
+            idx = tuple(int(g.integers(0, n)) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = float((oracle.fwd(args["q"], args["k"], args["v"], ds, None, lk)[0] * dout).sum())
+            args[name] = xm
+            lm = float((oracle.fwd(args["q"], args["k"], args["v"], ds, None, lk)[0] * dout).sum())
+            assert abs((lp - lm) / (2 * eps) - gx[idx]) < 1e-6, (name, idx)
+    # one document: torch autograd of non-causal SDPA
+    o, lse = oracle.fwd(q, k, v, None, None, oracle.last_key(S, causal=False))
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, None, None, oracle.last_key(S, causal=False))
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+    torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=False,
+                                                     enable_gqa=True).backward(torch.from_numpy(dout))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+
+
+def test_noncausal_sampled_equals_full():
+    B, Hq, Hkv, S, D = 1, 4, 2, 30, 8
+    q, k, v = rnd((B, Hq, S, D), 75), rnd((B, Hkv, S, D), 76), rnd((B, Hkv, S, D), 77)
+    dout = rnd((B, Hq, S, D), 78)
+    cu = [0, 11, 30]
+    ds, lk = oracle.first_key(S, cu), oracle.last_key(S, cu, causal=False)
+    o, lse = oracle.fwd(q, k, v, ds, None, lk)
+    dq, dk, dv = oracle.bwd(q, k, v, o, lse, dout, ds, None, lk)
+    rows = np.array([0, 5, 29, S + 12, 3 * S + 2])
+    np.testing.assert_allclose(oracle.bwd_dq_rows(q, k, v, dout, rows, ds, None, lk),
+                               dq.reshape(-1, D)[rows], atol=1e-13)
+    ro, rl = oracle.fwd_rows(q, k, v, rows, ds, None, lk)
+    np.testing.assert_allclose(ro, o.reshape(-1, D)[rows], atol=1e-13)
+    keys = np.array([0, 10, 11, 29, S + 3])
+    for fn in (lambda: oracle.bwd_dkv_keys(q, k, v, dout, keys, ds, None, lk),
+               lambda: oracle.bwd_dkv_keys_fwd(q, k, v, o, lse, dout, keys, ds, None, lk)):
+        sk, sv = fn()
+        np.testing.assert_allclose(sk, dk.reshape(-1, D)[keys], atol=1e-13)
+        np.testing.assert_allclose(sv, dv.reshape(-1, D)[keys], atol=1e-13)
