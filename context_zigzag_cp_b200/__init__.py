@@ -26,7 +26,8 @@ from ._lib import CpPlan, CpProblem, STATUS_NAMES
 __all__ = ["CPError", "Problem", "Plan", "attn_fwd", "attn_bwd", "lse_merge",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "get_device_status",
            "set_wait_limit_ns", "selftest_wait_timeout", "version", "lib", "launch_count",
-           "LaunchTrace", "attn_bwd_noalloc", "selftest_stall"]
+           "LaunchTrace", "attn_bwd_noalloc", "selftest_stall", "attn_fwd_rank", "attn_fwd_step",
+           "attn_bwd_rank", "f32_to_bf16"]
 
 
 class CPError(RuntimeError):
@@ -310,6 +311,97 @@ def attn_bwd_noalloc(prob: Problem, plan: Plan, q, k, v, o, lse, do, dq, dk, dv,
                                      _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                                      _stream(stream)), "cp_attn_bwd_noalloc")
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------ per-rank calls
+# One process per GPU: rank r holds its local query shard (2C = S / cp rows per
+# head, local row t = shard position r*2C + t); the K/V shards of the other ranks
+# arrive by collectives run outside the library (see context_zigzag_cp_b200.dist).
+
+def _rank_shapes(prob: "Problem"):
+    n2c = prob.seq_len // prob.cp
+    q = (prob.batch, prob.num_heads, n2c, prob.head_dim)
+    kv_all = (prob.batch, prob.num_kv_heads, prob.seq_len, prob.head_dim)
+    kv_one = (prob.batch, prob.num_kv_heads, n2c, prob.head_dim)
+    return q, kv_all, kv_one, q[:-1]
+
+
+def _ws_query(fn, *args) -> int:
+    n = ctypes.c_size_t(0)
+    _check(fn(*args, None, ctypes.byref(n), None), "workspace query")
+    return n.value
+
+
+def attn_fwd_rank(prob: Problem, plan: Plan, rank: int, q, k, v, o=None, lse=None, ws=None,
+                  stream=None):
+    """cp_attn_fwd_rank: rank's local q [B,Hq,2C,D] against gathered k/v [B,Hkv,S,D]
+    (shard order); returns the rank's (o [B,Hq,2C,D] bf16, lse [B,Hq,2C] fp32)."""
+    qs, kva, _, ls = _rank_shapes(prob)
+    bf16 = torch.bfloat16
+    _validate((q, qs, bf16, "q"), (k, kva, bf16, "k"), (v, kva, bf16, "v"), (o, qs, bf16, "o"),
+              (lse, ls, torch.float32, "lse"))
+    _check_plan(prob, plan, q.device)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(ls, dtype=torch.float32, device=q.device) if lse is None else lse
+    d = ctypes.c_void_p(256)
+    nbytes = _ws_query(lib().cp_attn_fwd_rank, prob.ref, plan.ref, int(rank), d, d, d, d, d)
+    w = _workspace(nbytes, q.device, ws)
+    n = ctypes.c_size_t(nbytes)
+    _check(lib().cp_attn_fwd_rank(prob.ref, plan.ref, int(rank), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                  _ptr(lse), _ptr(w), ctypes.byref(n) if w is not None else None,
+                                  _stream(stream)), "cp_attn_fwd_rank")
+    return o, lse
+
+
+def attn_fwd_step(prob: Problem, plan: Plan, rank: int, step: int, q, k, v, o_part=None,
+                  lse_part=None, stream=None):
+    """cp_attn_fwd_step: rank's local q against the one K/V shard it holds at ring step
+    `step` (k/v [B,Hkv,2C,D]); returns the step's fp32 partial (o [B,Hq,2C,D],
+    lse [B,Hq,2C]; lse = -inf where no key of the shard is visible)."""
+    qs, _, kv1, ls = _rank_shapes(prob)
+    bf16, f32 = torch.bfloat16, torch.float32
+    _validate((q, qs, bf16, "q"), (k, kv1, bf16, "k"), (v, kv1, bf16, "v"),
+              (o_part, qs, f32, "o_part"), (lse_part, ls, f32, "lse_part"))
+    _check_plan(prob, plan, q.device)
+    o_part = torch.empty(qs, dtype=f32, device=q.device) if o_part is None else o_part
+    lse_part = torch.empty(ls, dtype=f32, device=q.device) if lse_part is None else lse_part
+    _check(lib().cp_attn_fwd_step(prob.ref, plan.ref, int(rank), int(step), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(o_part), _ptr(lse_part), _stream(stream)),
+           "cp_attn_fwd_step")
+    return o_part, lse_part
+
+
+def attn_bwd_rank(prob: Problem, plan: Plan, rank: int, q, k, v, o, lse, do, dq=None,
+                  dk_part=None, dv_part=None, ws=None, stream=None):
+    """cp_attn_bwd_rank: the rank's dQ [B,Hq,2C,D] and its fp32 share of dK/dV for every
+    key [B,Hkv,S,D] (to be summed over the ranks by a reduce-scatter)."""
+    qs, kva, _, ls = _rank_shapes(prob)
+    bf16, f32 = torch.bfloat16, torch.float32
+    _validate((q, qs, bf16, "q"), (k, kva, bf16, "k"), (v, kva, bf16, "v"), (o, qs, bf16, "o"),
+              (lse, ls, f32, "lse"), (do, qs, bf16, "do"), (dq, qs, bf16, "dq"),
+              (dk_part, kva, f32, "dk_part"), (dv_part, kva, f32, "dv_part"))
+    _check_plan(prob, plan, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk_part = torch.empty(kva, dtype=f32, device=q.device) if dk_part is None else dk_part
+    dv_part = torch.empty(kva, dtype=f32, device=q.device) if dv_part is None else dv_part
+    d = ctypes.c_void_p(256)
+    nbytes = _ws_query(lib().cp_attn_bwd_rank, prob.ref, plan.ref, int(rank), d, d, d, d, d, d, d,
+                       d, d)
+    w = _workspace(nbytes, q.device, ws)
+    n = ctypes.c_size_t(nbytes)
+    _check(lib().cp_attn_bwd_rank(prob.ref, plan.ref, int(rank), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk_part),
+                                  _ptr(dv_part), _ptr(w), ctypes.byref(n) if w is not None else None,
+                                  _stream(stream)), "cp_attn_bwd_rank")
+    return dq, dk_part, dv_part
+
+
+def f32_to_bf16(x, out=None, stream=None):
+    """cp_f32_to_bf16 on a contiguous fp32 CUDA tensor (numel a multiple of 4)."""
+    _validate((x, tuple(x.shape), torch.float32, "x"), (out, tuple(x.shape), torch.bfloat16, "out"))
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib().cp_f32_to_bf16(_ptr(x), _ptr(out), x.numel(), _stream(stream)), "cp_f32_to_bf16")
+    return out
 
 
 def lse_merge(o_parts, lse_parts, o_out=None, lse_out=None, stream=None):

@@ -24,12 +24,14 @@ MERGE = {"separate": 0, "fused": 1}
 EXPORTED = ("cp_plan_shards", "cp_unshard", "cp_attn_fwd", "cp_attn_bwd", "cp_lse_merge",
             "cp_get_device_status", "cp_set_wait_limit_ns", "cp_selftest_wait_timeout",
             "cp_launch_count", "cp_trace_begin", "cp_trace_end", "cp_selftest_exp2",
-            "cp_attn_bwd_noalloc", "cp_selftest_stall", "cp_version")
+            "cp_attn_bwd_noalloc", "cp_selftest_stall", "cp_attn_fwd_rank", "cp_attn_fwd_step",
+            "cp_attn_bwd_rank", "cp_f32_to_bf16", "cp_version")
 
 NOALLOC_MAX_ROWS = 4194304
 
 KERNEL_NAMES = {1: "plan_meta", 2: "plan_index", 3: "gather", 4: "fwd", 5: "merge",
-                6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2"}
+                6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2",
+                11: "cast"}
 KERNEL_IDS = {name: i for i, name in KERNEL_NAMES.items()}
 
 
@@ -83,6 +85,11 @@ def load() -> ctypes.CDLL:
     lib.cp_trace_end.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     lib.cp_selftest_stall.argtypes = [ctypes.c_int32, P, PL, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                       vp, sz, vp]
+    i32 = ctypes.c_int32
+    lib.cp_attn_fwd_rank.argtypes = [P, PL, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.cp_attn_fwd_step.argtypes = [P, PL, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.cp_attn_bwd_rank.argtypes = [P, PL, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.cp_f32_to_bf16.argtypes = [vp, vp, ctypes.c_int64, vp]
     for name in EXPORTED:
         getattr(lib, name).restype = ctypes.c_int32
     lib.cp_launch_count.restype = ctypes.c_int64

@@ -76,6 +76,13 @@ struct BwdParams {
     float scale_log2;        // softmax scale * log2(e)
     int32_t n_items;
     int32_t stall;           // test hook: the cp_kernel_t whose CTA 0 skips its first K/V load
+    // Row layouts (as in FwdParams): Q, dO, dQ and the per-row workspace hold q_rows
+    // rows per batch*head starting at shard position q_base; K, V hold kv_rows rows
+    // per batch*KV head starting at kv_base.  dK / dV always cover all S keys.
+    int32_t q_rows, q_base, kv_rows, kv_base;
+    int32_t rank;            // -1: every rank's query rows; r: only rank r's
+    float* dk32;             // non-null: dK / dV written as fp32 partials here instead of bf16
+    float* dv32;
     const int32_t* src;      // [cp*cp]
     const int32_t* doc_start;  // [S] shard order
     const int32_t* cu;       // [num_docs+1] document offsets, original order (documents only)
@@ -220,6 +227,15 @@ __device__ __forceinline__ int dkdv_last_tile(const BwdParams& P, int ko, int nt
     }
     return t_end;
 }
+// True when the query tile starting at original qo belongs to the rank the pass
+// runs for (always, for a whole-sequence pass).
+__device__ __forceinline__ bool q_tile_on_rank(const BwdParams& P, int qo)
+{
+    if (P.rank < 0) return true;
+    const int c = qo / P.C;
+    return (c < P.cp ? c : 2 * P.cp - 1 - c) == P.rank;
+}
+
 constexpr int BWD_NWG = 4;                       // elementwise warpgroups
 constexpr int BWD_THREADS = (BWD_NWG + 1) * 128; // + producer / MMA warpgroup
 constexpr int BWD_NSLICE = 2;                    // 64-column slices of a 128-column score tile
@@ -354,8 +370,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (!(P.stall == 7 /* CP_K_BWD_DKDV */ && blockIdx.x == 0 && iter == 0)) {
                     mbar_arrive_expect_tx(bar_kv_full, 2 * Cfg::TILE);
                     for (int h = 0; h < D / 64; ++h) {
-                        tma_load_2d(sK + h * 16384, &tmK, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
-                        tma_load_2d(sV + h * 16384, &tmV, h * 64, it.bkv * P.S + it.kpos, bar_kv_full);
+                        const int kvrow = it.bkv * P.kv_rows + (it.kpos - P.kv_base);
+                        tma_load_2d(sK + h * 16384, &tmK, h * 64, kvrow, bar_kv_full);
+                        tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);
                     }
                 }
                 for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
@@ -363,10 +380,11 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP) continue;
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qo))
+                        continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const int bh = it.b * P.Hq + it.hk * g + hq;
-                        const size_t row = static_cast<size_t>(bh) * P.S + qpos;
+                        const size_t row = static_cast<size_t>(bh) * P.q_rows + (qpos - P.q_base);
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
                         const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
                         ++nst;
@@ -458,7 +476,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     const int qpos = shard_of_orig(qo, P.C, P.cp);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP) continue;
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qo))
+                        continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
                         const uint32_t ds = nst % Cfg::NDO, dpar = (nst / Cfg::NDO) & 1;
@@ -539,7 +558,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
                 const int cls = classify_tile(qo, dsf, dsl, it.ko, P.nc);
-                if (cls == TILE_SKIP) continue;
+                if (cls == TILE_SKIP || !q_tile_on_rank(P, qo)) continue;
                 for (int hq = 0; hq < g && ok; ++hq) {
                     const uint32_t qs = nst % Cfg::NQ, ds = nst % Cfg::NDO;
                     ++nst;
@@ -617,6 +636,16 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tmem_wait_ld();
                     reg_fence32f(a);
                     reg_fence32f(b);
+                    if (P.dk32) {   // fp32 partials (one rank's share, summed across ranks later)
+                        float4* dv = reinterpret_cast<float4*>(P.dv32 + orow * D + 32 * wg);
+                        float4* dk = reinterpret_cast<float4*>(P.dk32 + orow * D + 32 * wg);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            dv[i] = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+                            dk[i] = make_float4(b[4 * i] * P.scale, b[4 * i + 1] * P.scale,
+                                                b[4 * i + 2] * P.scale, b[4 * i + 3] * P.scale);
+                        }
+                    } else {
                     uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
                     uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + 32 * wg);
 #pragma unroll
@@ -628,14 +657,21 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                            pack_bf16(b[8 * i + 4] * P.scale, b[8 * i + 5] * P.scale),
                                            pack_bf16(b[8 * i + 6] * P.scale, b[8 * i + 7] * P.scale));
                     }
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty);
             } else if (32 * wg < D) {
-                uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
-                uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + 32 * wg);
-                for (int i = 0; i < 4; ++i) { dv[i] = make_uint4(0, 0, 0, 0); dk[i] = make_uint4(0, 0, 0, 0); }
+                if (P.dk32) {
+                    float4* dv = reinterpret_cast<float4*>(P.dv32 + orow * D + 32 * wg);
+                    float4* dk = reinterpret_cast<float4*>(P.dk32 + orow * D + 32 * wg);
+                    for (int i = 0; i < 8; ++i) { dv[i] = make_float4(0.f, 0.f, 0.f, 0.f); dk[i] = dv[i]; }
+                } else {
+                    uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
+                    uint4* dk = reinterpret_cast<uint4*>(P.dk + orow * D + 32 * wg);
+                    for (int i = 0; i < 4; ++i) { dv[i] = make_uint4(0, 0, 0, 0); dk[i] = make_uint4(0, 0, 0, 0); }
+                }
             }
         }
     }
@@ -686,14 +722,20 @@ __device__ __forceinline__ DqItem decode_dq(const BwdParams& P, int w)
 {
     DqItem it;
     const int g = P.Hq / P.Hkv;
-    const int ntiles = P.S / 128;
+    const int ntiles = P.rank < 0 ? P.S / 128 : 2 * P.C / 128;   // every tile, or rank r's
     const int per_group = g * ntiles;
     it.bkv = w / per_group;
     const int rem = w - it.bkv * per_group;
     const int t = rem / g, hq = rem - t * g;
     const int b = it.bkv / P.Hkv, hk = it.bkv - b * P.Hkv;
     it.bh = b * P.Hq + hk * g + hq;
-    it.qo = (ntiles - 1 - t) * 128;          // descending original position
+    if (P.rank < 0) {
+        it.qo = (ntiles - 1 - t) * 128;      // descending original position
+    } else {                                 // rank r: its tail chunk, then its head chunk
+        const int half = P.C / 128;
+        it.qo = t < half ? (2 * P.cp - 1 - P.rank) * P.C + (half - 1 - t) * 128
+                         : P.rank * P.C + (2 * half - 1 - t) * 128;
+    }
     it.qpos = shard_of_orig(it.qo, P.C, P.cp);
     it.r = it.qpos / (2 * P.C);
     return it;
@@ -782,7 +824,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                             for (int h = 0; h < D / 64; ++h)
                                 tma_load_2d(sKV + slot * Cfg::KTILE + h * 16384,
                                             kv == 0 ? (const void*)&tmK : (const void*)&tmV, h * 64,
-                                            it.bkv * P.S + kpos, bar_kv_full + 8 * slot);
+                                            it.bkv * P.kv_rows + (kpos - (P.kv_base < 0 ? j * n2c : P.kv_base)),
+                                            bar_kv_full + 8 * slot);
                         }
                     }
                 }
@@ -924,7 +967,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const DqItem it = decode_dq(P, w);
             const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
             const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
-            const size_t rowi = static_cast<size_t>(it.bh) * P.S + it.qpos + row;
+            const size_t rowi = static_cast<size_t>(it.bh) * P.q_rows + (it.qpos - P.q_base) + row;
             // this row's Q and dO (bf16 pairs, columns [32wg, 32wg+32)) into tensor memory once the
             // previous item's S / dP have read the old ones
             ok = __all_sync(0xffffffffu, mbar_wait(bar_qt_empty, (iter & 1) ^ 1, abort_flag));

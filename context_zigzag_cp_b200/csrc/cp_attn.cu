@@ -236,17 +236,37 @@ cp_status_t check_bufs(const cp_problem_t* p, int32_t n_bufs, const void* const*
     return CP_OK;
 }
 
+// Which rows a launch covers and how its tensors are laid out: the whole
+// sequence (every rank, every step, tensors of S rows per head), or one rank's
+// local query shard (2C rows per head, first row at shard position r*2C) against
+// gathered K/V (S rows) or against the single K/V shard of one ring step (2C rows).
+struct Layout {
+    int32_t q_rows, q_base, kv_rows, kv_base, rank, s0, s1;
+};
+
+inline Layout whole_layout(const cp_problem_t* p)
+{
+    return Layout{p->seq_len, 0, p->seq_len, 0, -1, 0, p->cp_size};
+}
+
+inline Layout rank_layout(const cp_problem_t* p, int rank, int step)
+{
+    const int n2c = p->seq_len / p->cp_size;
+    if (step < 0) return Layout{n2c, rank * n2c, p->seq_len, 0, rank, 0, p->cp_size};
+    return Layout{n2c, rank * n2c, n2c, -1, rank, step, step + 1};
+}
+
 template <int D>
 cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, void* o, float* lse, float* o_parts, float* lse_parts,
-                       cudaStream_t stream, int stall)
+                       cudaStream_t stream, int stall, const Layout& L, bool fused)
 {
     using Cfg = FwdCfg<D>;
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
     CUtensorMap tq, tk, tv;
-    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * S, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128))
+    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128))
         return CP_ERR_CUDA;
     FwdParams P;
     P.BH = B * Hq;
@@ -258,11 +278,18 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.docs = p->mask == CP_MASK_DOC_CAUSAL;
     P.wm1 = window_minus_one(p);
     P.nc = noncausal_shift(p);
-    P.fused = p->merge == CP_MERGE_FUSED;
+    P.fused = fused;
     P.scale_log2 = softmax_scale(p) * 1.4426950408889634f;
     P.ppc = (P.C + 255) / 256;
-    P.n_items = P.BH * 2 * P.cp * P.ppc;
+    P.n_items = P.BH * (L.rank < 0 ? 2 * P.cp : 2) * P.ppc;
     P.stall = stall;
+    P.q_rows = L.q_rows;
+    P.q_base = L.q_base;
+    P.kv_rows = L.kv_rows;
+    P.kv_base = L.kv_base;
+    P.rank = L.rank;
+    P.s0 = L.s0;
+    P.s1 = L.s1;
     P.src = pl->src;
     P.doc_start = pl->doc_start;
     P.o = static_cast<__nv_bfloat16*>(o);
@@ -441,8 +468,11 @@ cp_status_t attn_fwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
     float* o_parts = separate ? static_cast<float*>(ws) : nullptr;
     float* lse_parts = separate ? reinterpret_cast<float*>(static_cast<char*>(ws) + o_parts_bytes) : nullptr;
     cudaStream_t s = as_stream(stream);
-    st = problem->head_dim == 128 ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall)
-                                  : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall);
+    const Layout L = whole_layout(problem);
+    const bool fused = problem->merge == CP_MERGE_FUSED;
+    st = problem->head_dim == 128
+             ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall, L, fused)
+             : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall, L, fused);
     if (st != CP_OK || !separate) return st;
     return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
 }
@@ -511,10 +541,10 @@ template <int D>
 cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, const void* o, const float* lse, const void* dout, void* dq,
                        void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream,
-                       int stall = 0)
+                       int stall, const Layout& L, float* dk32, float* dv32)
 {
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
-    const int64_t rows = static_cast<int64_t>(B) * Hq * S;
+    const int64_t rows = static_cast<int64_t>(B) * Hq * L.q_rows;
     {
         const int64_t blocks = std::min<int64_t>((rows + 7) / 8, int64_t(num_sms()) * 16);
         LaunchScope ls(CP_K_BWD_PREP, stream);
@@ -524,10 +554,10 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
         if (launch_status() != CP_OK) return CP_ERR_CUDA;
     }
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * S, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * S, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tdo, dout, D, static_cast<uint64_t>(B) * Hq * S, D * 2, 64, 128))
+    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128) ||
+        !make_tmap_bf16_2d(&tdo, dout, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128))
         return CP_ERR_CUDA;
     BwdParams P;
     P.B = B;
@@ -553,6 +583,13 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.dk = static_cast<__nv_bfloat16*>(dk);
     P.dv = static_cast<__nv_bfloat16*>(dv);
     P.stall = stall;
+    P.q_rows = L.q_rows;
+    P.q_base = L.q_base;
+    P.kv_rows = L.kv_rows;
+    P.kv_base = L.kv_base;
+    P.rank = L.rank;
+    P.dk32 = dk32;
+    P.dv32 = dv32;
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_BWD128 : ATTR_BWD64, [] {
         cudaError_t e = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -570,7 +607,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
                             stream>>>(tq, tk, tv, tdo, P);
     }
     if (launch_status() != CP_OK) return CP_ERR_CUDA;
-    P.n_items = B * Hq * (S / 128);
+    P.n_items = B * Hq * (L.q_rows / 128);
     LaunchScope ls(CP_K_BWD_DQ, stream);
     cp_bwd_dq_kernel<D><<<std::min(P.n_items, num_sms()), DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(
         tq, tk, tv, tdo, P);
@@ -599,8 +636,10 @@ cp_status_t attn_bwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     cudaStream_t s = as_stream(stream);
     return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall);
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
+                                 whole_layout(problem), nullptr, nullptr)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
+                                whole_layout(problem), nullptr, nullptr);
 }
 
 }  // namespace
@@ -683,6 +722,122 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
     float* delta = static_cast<float*>(scratch);
     float* nlse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
     return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s);
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
+                                 whole_layout(problem), nullptr, nullptr)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
+                                whole_layout(problem), nullptr, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// Per-rank entry points: context parallelism across GPUs, one process per GPU.
+// Each rank holds its local query shard (Q_r, O_r, dO_r, dQ_r: 2C rows per
+// head) and receives the K/V shards from the others (all-gather, or one shard
+// per ring step); the backward's dK/dV contributions of every rank are summed
+// across ranks by the caller (reduce-scatter) and cast with cp_f32_to_bf16.
+// ---------------------------------------------------------------------------
+namespace {
+
+cp_status_t check_rank_call(const cp_problem_t* p, const cp_plan_t* pl, int32_t rank, int32_t step,
+                            bool need_step)
+{
+    cp_status_t st = check_attention(p);
+    if (st != CP_OK) return st;
+    if ((st = check_plan(pl, false)) != CP_OK) return st;
+    if (rank < 0 || rank >= p->cp_size) return CP_ERR_INVALID_ARG;
+    if (need_step ? (step < 0 || step >= p->cp_size) : step != -1) return CP_ERR_INVALID_ARG;
+    return CP_OK;
+}
+
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ in,
+                                                          uint2* __restrict__ out, int64_t n4)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 x = __ldg(in + i);
+        out[i] = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+    }
+}
+
+}  // namespace
+
+extern "C" cp_status_t cp_attn_fwd_rank(const cp_problem_t* problem, const cp_plan_t* plan,
+                                        int32_t rank, const void* q, const void* k, const void* v,
+                                        void* o, float* lse, void* ws, size_t* ws_bytes, void* stream)
+{
+    cp_status_t st = check_rank_call(problem, plan, rank, -1, false);
+    if (st != CP_OK) return st;
+    const void* ptrs[] = {q, k, v, o, lse};
+    for (const void* x : ptrs)
+        if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
+    const int n2c = problem->seq_len / problem->cp_size;
+    const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * n2c;
+    const bool separate = problem->merge == CP_MERGE_SEPARATE;
+    const size_t o_parts_bytes = separate ? round_up(size_t(problem->cp_size) * rows * problem->head_dim * 4, 256) : 0;
+    const size_t lse_parts_bytes = separate ? round_up(size_t(problem->cp_size) * rows * 4, 256) : 0;
+    if (workspace_gate(o_parts_bytes + lse_parts_bytes, ws, ws_bytes, &st)) return st;
+    float* o_parts = separate ? static_cast<float*>(ws) : nullptr;
+    float* lse_parts = separate ? reinterpret_cast<float*>(static_cast<char*>(ws) + o_parts_bytes) : nullptr;
+    cudaStream_t s = as_stream(stream);
+    const Layout L = rank_layout(problem, rank, -1);
+    st = problem->head_dim == 128
+             ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, 0, L, !separate)
+             : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, 0, L, !separate);
+    if (st != CP_OK || !separate) return st;
+    return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
+}
+
+extern "C" cp_status_t cp_attn_fwd_step(const cp_problem_t* problem, const cp_plan_t* plan,
+                                        int32_t rank, int32_t step, const void* q, const void* k,
+                                        const void* v, float* o_part, float* lse_part, void* stream)
+{
+    cp_status_t st = check_rank_call(problem, plan, rank, step, true);
+    if (st != CP_OK) return st;
+    const void* ptrs[] = {q, k, v, o_part, lse_part};
+    for (const void* x : ptrs)
+        if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    const Layout L = rank_layout(problem, rank, step);
+    return problem->head_dim == 128
+               ? launch_fwd<128>(problem, plan, q, k, v, nullptr, nullptr, o_part, lse_part, s, 0, L, false)
+               : launch_fwd<64>(problem, plan, q, k, v, nullptr, nullptr, o_part, lse_part, s, 0, L, false);
+}
+
+extern "C" cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_plan_t* plan,
+                                        int32_t rank, const void* q, const void* k, const void* v,
+                                        const void* o, const float* lse, const void* dout, void* dq,
+                                        float* dk_part, float* dv_part, void* ws, size_t* ws_bytes,
+                                        void* stream)
+{
+    cp_status_t st = check_rank_call(problem, plan, rank, -1, false);
+    if (st != CP_OK) return st;
+    const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk_part, dv_part};
+    for (const void* x : ptrs)
+        if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
+    const int n2c = problem->seq_len / problem->cp_size;
+    const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * n2c;
+    const size_t row_bytes = round_up(size_t(rows) * 4, 256);
+    if (workspace_gate(2 * row_bytes, ws, ws_bytes, &st)) return st;
+    float* delta = static_cast<float*>(ws);
+    float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
+    cudaStream_t s = as_stream(stream);
+    const Layout L = rank_layout(problem, rank, -1);
+    return problem->head_dim == 128
+               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
+                                 s, 0, L, dk_part, dv_part)
+               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
+                                s, 0, L, dk_part, dv_part);
+}
+
+extern "C" cp_status_t cp_f32_to_bf16(const float* in, void* out, int64_t n, void* stream)
+{
+    if (n < 0 || n % 4 != 0) return CP_ERR_INVALID_ARG;
+    if (n == 0) return CP_OK;
+    if (!in || !out || !aligned16(in) || (reinterpret_cast<uintptr_t>(out) & 7u)) return CP_ERR_INVALID_ARG;
+    const int64_t n4 = n / 4;
+    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, int64_t(num_sms()) * 8);
+    cudaStream_t s = as_stream(stream);
+    LaunchScope ls(CP_K_CAST, s);
+    f32_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(reinterpret_cast<const float4*>(in),
+                                                                   static_cast<uint2*>(out), n4);
+    return launch_status();
 }

@@ -49,6 +49,14 @@ struct FwdParams {
     float scale_log2;               // softmax scale * log2(e)
     int32_t n_items, ppc;           // items, query-tile pairs per chunk
     int32_t stall;                  // test hook: 1 = CTA 0 skips its first K/V load
+    // Row layouts.  Q / O / LSE (and partials) hold q_rows rows per batch*head whose
+    // first row is shard position q_base (S and 0 for the whole sequence; 2C and
+    // r*2C for rank r's local shard).  K / V hold kv_rows rows per batch*KV head
+    // starting at shard position kv_base (S and 0 gathered); kv_base = -1: they hold
+    // only the shard being visited (2C rows: the one shard of a ring step).
+    int32_t q_rows, q_base, kv_rows, kv_base;
+    int32_t rank;                   // -1: the items of every rank; r: rank r's only
+    int32_t s0, s1;                 // visit steps s0 .. s1-1 (partials indexed s - s0)
     const int32_t* src;             // [cp*cp]
     const int32_t* doc_start;       // [S] shard order
     __nv_bfloat16* o;               // [BH][S][D]  (fused)
@@ -113,18 +121,22 @@ __device__ __forceinline__ KtSpan kt_span(int j, int lo, int hi, int half, int C
 __device__ __forceinline__ int kt_first(const KtSpan& r) { return r.a0 < r.b0 ? r.a0 : r.a1; }
 __device__ __forceinline__ int kt_next(const KtSpan& r, int kt) { return kt + 1 == r.b0 ? r.a1 : kt + 1; }
 
+// Chunks an item list covers: all 2cp, or rank r's two (its tail chunk first).
+__device__ __forceinline__ int fwd_nchunks(const FwdParams& P) { return P.rank < 0 ? 2 * P.cp : 2; }
+
 __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
 {
     FwdItem it;
     const int g = P.Hq / P.Hkv;
-    const int per_group = g * 2 * P.cp * P.ppc;
+    const int per_group = g * fwd_nchunks(P) * P.ppc;
     it.bkv = w / per_group;
     const int rem = w - it.bkv * per_group;
     const int t = rem / g, hq = rem - t * g;
     const int b = it.bkv / P.Hkv, hk = it.bkv - b * P.Hkv;
     it.bh = b * P.Hq + hk * g + hq;
     const int u = P.ppc - 1 - t % P.ppc;
-    const int c = 2 * P.cp - 1 - t / P.ppc;  // original chunk, descending
+    const int ci = t / P.ppc;                // original chunk, descending
+    const int c = P.rank < 0 ? 2 * P.cp - 1 - ci : (ci == 0 ? 2 * P.cp - 1 - P.rank : P.rank);
     int half;
     if (c < P.cp) { it.r = c; half = 0; } else { it.r = 2 * P.cp - 1 - c; half = 1; }
     it.p0 = it.r * 2 * P.C + half * P.C + u * 256;
@@ -289,8 +301,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int x = 0; x < it.ntq; ++x)
                     for (int h = 0; h < D / 64; ++h)
                         tma_load_2d(sQ0 + x * Cfg::TILE_BYTES + h * 16384, &tmQ, h * 64,
-                                    it.bh * P.S + it.p0 + 128 * x, bar_q_full);
-                for (int s = 0; s < P.cp && ok; ++s) {
+                                    it.bh * P.q_rows + (it.p0 - P.q_base) + 128 * x, bar_q_full);
+                for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -312,7 +324,8 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             for (int h = 0; h < D / 64; ++h)
                                 tma_load_2d(sKV + slot * Cfg::TILE_BYTES + h * 16384,
                                             kv == 0 ? (const void*)&tmK : (const void*)&tmV, h * 64,
-                                            it.bkv * P.S + kpos, bar_kv_full + 8 * slot);
+                                            it.bkv * P.kv_rows + (kpos - (P.kv_base < 0 ? j * n2c : P.kv_base)),
+                                            bar_kv_full + 8 * slot);
                         }
                     }
                 }
@@ -345,7 +358,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 // number of loaded tiles of this item: Q is released to the producer
                 // right after the last S = Q K^T, before the item's final PVs
                 int n_tiles = 0;
-                for (int s = 0; s < P.cp; ++s) {
+                for (int s = P.s0; s < P.s1; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1; kt = kt_next(ks, kt)) {
@@ -395,7 +408,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     __syncwarp();
                 };
 
-                for (int s = 0; s < P.cp && ok; ++s) {
+                for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -429,7 +442,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (++tiles_done == n_tiles) { if (elect_one()) mma_commit(bar_q_empty); __syncwarp(); }
                     }
                     // end of a segment: every step (separate) or the whole visit (fused)
-                    if (ok && (!P.fused || s == P.cp - 1)) {
+                    if (ok && (!P.fused || s == P.s1 - 1)) {
                         if (pend0) { ok = issue_pv(0, p_phase0, first0); pend0 = false; }
                         if (ok && pend1) { ok = issue_pv(1, p_phase1, first1); pend1 = false; }
                         if (ok && elect_one()) {
@@ -472,7 +485,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const int ds_row = max(P.docs ? __ldg(P.doc_start + prow) : 0, q_orig - P.wm1);
             float m_used = -INFINITY, l_sum = 0.f;
             bool first = true, had = false;
-            for (int s = 0; s < P.cp && ok; ++s) {
+            for (int s = P.s0; s < P.s1 && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
                 const KtSpan ks = kt_span(j, ti.dsf[X], ti.qo[X] + 127 + P.nc, half, P.C, P.cp);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -542,9 +555,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     had = true;
                 }
                 if (!ok) break;
-                if (!P.fused || s == P.cp - 1) {
+                if (!P.fused || s == P.s1 - 1) {
                     // ---- epilogue of the segment
-                    const size_t rowi = static_cast<size_t>(it.bh) * P.S + prow;
+                    const size_t rowi = static_cast<size_t>(it.bh) * P.q_rows + (prow - P.q_base);
                     if (had) {
                         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + 8 * X, o_phase, abort_flag));
                         if (!ok) break;
@@ -576,7 +589,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                 }
                             } else {
                                 float4* dst = reinterpret_cast<float4*>(
-                                    P.o_parts + (static_cast<size_t>(s) * P.BH * P.S + rowi) * D + c0);
+                                    P.o_parts + (static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi) * D + c0);
 #pragma unroll
                                 for (int i = 0; i < 8; ++i)
                                     dst[i] = make_float4(__uint_as_float(orr[4 * i + 0]) * inv_l,
@@ -586,9 +599,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             }
                         }
                         if (P.fused) P.lse[rowi] = lse_v;
-                        else P.lse_parts[static_cast<size_t>(s) * P.BH * P.S + rowi] = lse_v;
+                        else P.lse_parts[static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi] = lse_v;
                     } else if (!P.fused) {
-                        P.lse_parts[static_cast<size_t>(s) * P.BH * P.S + rowi] = -INFINITY;
+                        P.lse_parts[static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi] = -INFINITY;
                     } else {
                         // no admitted key anywhere (cannot happen for a valid mask): (0, -inf)
                         uint4* dst = reinterpret_cast<uint4*>(P.o + rowi * D);

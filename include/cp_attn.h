@@ -272,6 +272,73 @@ CP_API cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp_pla
                                        const void* o, const float* lse, const void* dout,
                                        void* dq, void* dk, void* dv, void* stream);
 
+/*
+ * Per-rank calls: context parallelism across GPUs, one process per GPU.  Rank r
+ * of cp_size holds its own query shard -- Q_r, O_r, LSE_r, dO_r, dQ_r, each
+ * [B][heads][2C][...] with 2C = seq_len / cp_size rows per head, local row t being
+ * shard position r*2C + t -- and gets the K/V shards of the other ranks over the
+ * interconnect, as the concept guide describes ("So how does it work?": Q_i stays,
+ * K_j/V_j travel; "all-to-all vs all-gather": gather them all at once, or take the
+ * neighbour's shard cp-1 times).  The plan is the same on every rank (built by
+ * cp_plan_shards from the same problem).  The library moves no data between
+ * GPUs: the caller runs the collectives (NCCL all-gather, send/recv,
+ * reduce-scatter) between these calls.
+ */
+
+/*
+ * cp_attn_fwd_rank -- rank r's attention against K/V of every shard, already
+ * gathered in shard order (all-gather):
+ *   q        bf16 [B][Hq][2C][D]   rank r's query shard
+ *   k, v     bf16 [B][Hkv][S][D]   every shard, shard order
+ *   o        bf16 [B][Hq][2C][D]   output, lse fp32 [B][Hq][2C]
+ * The cp steps are visited in the plan's order and combined as problem->merge
+ * says (fused in the kernel, or per-step fp32 partials in the workspace merged by
+ * the LSE-merge kernel).  Supported sizes as cp_attn_fwd.
+ * Errors: as cp_attn_fwd; CP_ERR_INVALID_ARG for rank outside [0, cp_size).
+ */
+CP_API cp_status_t cp_attn_fwd_rank(const cp_problem_t* problem, const cp_plan_t* plan,
+                                    int32_t rank, const void* q, const void* k, const void* v,
+                                    void* o, float* lse, void* ws, size_t* ws_bytes, void* stream);
+
+/*
+ * cp_attn_fwd_step -- one step of the ring: rank r's queries against the single
+ * K/V shard j = src[r][step] that it holds at that step:
+ *   q                 bf16 [B][Hq][2C][D]   rank r's query shard
+ *   k, v              bf16 [B][Hkv][2C][D]  shard j
+ *   o_part, lse_part  fp32 [B][Hq][2C][D] and [B][Hq][2C]: the step's partial
+ *                     attention, O normalised over the step's keys, LSE = -inf for
+ *                     rows with no visible key in shard j (their O is not written)
+ * After all cp steps, cp_lse_merge over the cp partials (in step order) gives
+ * rank r's O and LSE: the ring form of the shard loop and combine.
+ * Errors: as cp_attn_fwd; CP_ERR_INVALID_ARG for rank or step outside [0, cp_size).
+ */
+CP_API cp_status_t cp_attn_fwd_step(const cp_problem_t* problem, const cp_plan_t* plan,
+                                    int32_t rank, int32_t step, const void* q, const void* k,
+                                    const void* v, float* o_part, float* lse_part, void* stream);
+
+/*
+ * cp_attn_bwd_rank -- rank r's backward: dQ of its query shard, and the
+ * contribution of its queries to dK and dV of every key.
+ *   q, o, dout      bf16 [B][Hq][2C][D], lse fp32 [B][Hq][2C]   rank r's shard
+ *   k, v            bf16 [B][Hkv][S][D]                          every shard, gathered
+ *   dq              bf16 [B][Hq][2C][D]   output
+ *   dk_part, dv_part  fp32 [B][Hkv][S][D] output: rank r's share of dK / dV for
+ *                   every key (zero where none of its queries sees the key).
+ * The caller sums dk_part / dv_part over the ranks (a reduce-scatter hands rank
+ * j the sum for its own shard j) and casts with cp_f32_to_bf16.
+ * Workspace: two fp32 values per local query row (as cp_attn_bwd).
+ * Errors: as cp_attn_bwd; CP_ERR_INVALID_ARG for rank outside [0, cp_size).
+ */
+CP_API cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_plan_t* plan,
+                                    int32_t rank, const void* q, const void* k, const void* v,
+                                    const void* o, const float* lse, const void* dout, void* dq,
+                                    float* dk_part, float* dv_part, void* ws, size_t* ws_bytes,
+                                    void* stream);
+
+/* out[i] = bf16(in[i]) (round to nearest even) for n floats; n a multiple of 4, in
+ * 16-byte and out 8-byte aligned. */
+CP_API cp_status_t cp_f32_to_bf16(const float* in, void* out, int64_t n, void* stream);
+
 /* Read and clear the device status word on `stream` (synchronises the stream).
  * *status receives CP_OK or the first device-side error since the last read. */
 CP_API cp_status_t cp_get_device_status(int32_t* status, void* stream);
@@ -316,7 +383,8 @@ typedef enum {
     CP_K_BWD_DKDV = 7,   /* backward: dK, dV                                */
     CP_K_BWD_DQ = 8,     /* backward: dQ                                    */
     CP_K_SELFTEST = 9,
-    CP_K_SELFTEST_EXP2 = 10
+    CP_K_SELFTEST_EXP2 = 10,
+    CP_K_CAST = 11       /* fp32 -> bf16 cast of summed dK / dV partials    */
 } cp_kernel_t;
 
 /* Number of kernels this library has launched in this process. */

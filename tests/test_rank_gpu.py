@@ -1,0 +1,79 @@
+"""The per-rank calls (cp_attn_fwd_rank, cp_attn_fwd_step, cp_attn_bwd_rank,
+cp_f32_to_bf16) on one GPU: every rank of a cp group run one after another, the
+K/V exchange done by slicing (all-gather: the whole shard-order K/V; ring step
+s: shard src[r][s]) and the dK/dV reduce-scatter by a sum.  The ranks' results
+reassembled must equal the whole-sequence calls (the same kernels restricted to
+one rank's rows: bit for bit for the forward and dQ) and the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import context_zigzag_cp_b200 as cz
+import oracle
+from helpers import assert_bf16_close, assert_lse_close, f64, make_case, random_docs, run_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+def _local(x, r, n2c):
+    return x[:, :, r * n2c:(r + 1) * n2c].contiguous()
+
+
+@pytest.mark.parametrize("Hq,Hkv,S,D,cp,docs,causal", [
+    (8, 2, 4096, 128, 4, False, True), (4, 2, 2304, 128, 3, True, True),
+    (4, 4, 2048, 64, 2, False, True), (4, 2, 2048, 128, 4, False, False)])
+def test_ranks_reassemble_whole(Hq, Hkv, S, D, cp, docs, causal):
+    cu = random_docs(S, 95, 300.0) if docs else None
+    case = make_case(1, Hq, Hkv, S, D, cp, 96 + S, cu=cu, with_dout=True, causal=causal)
+    prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, cp, "ring", "fused")
+    (dos,) = plan.shard([case["do"].cuda()])
+    dq, dk, dv = cz.attn_bwd(prob, plan, qs, ks, vs, o, lse, dos)
+    prob_sep = prob.with_merge("separate")
+    o_sep, lse_sep = cz.attn_fwd(prob_sep, plan, qs, ks, vs)
+    n2c = S // cp
+    src = plan.src.cpu().numpy()
+    ro, rl, rq = [], [], []
+    dk_sum = torch.zeros(ks.shape, dtype=torch.float32, device="cuda")
+    dv_sum = torch.zeros_like(dk_sum)
+    for r in range(cp):
+        q_r, do_r = _local(qs, r, n2c), _local(dos, r, n2c)
+        # all-gather order: one call against every shard
+        o_r, l_r = cz.attn_fwd_rank(prob, plan, r, q_r, ks, vs)
+        assert torch.equal(o_r, _local(o, r, n2c)) and torch.equal(l_r, _local(lse, r, n2c))
+        o_r2, l_r2 = cz.attn_fwd_rank(prob_sep, plan, r, q_r, ks, vs)
+        assert torch.equal(o_r2, _local(o_sep, r, n2c)) and torch.equal(l_r2, _local(lse_sep, r, n2c))
+        # ring order: one partial per step against the shard held then, merged in step order
+        parts = [cz.attn_fwd_step(prob, plan, r, s, q_r, _local(ks, int(src[r * cp + s]), n2c),
+                                  _local(vs, int(src[r * cp + s]), n2c)) for s in range(cp)]
+        om, lm = cz.lse_merge(torch.stack([p[0] for p in parts]).view(cp, -1, D),
+                              torch.stack([p[1] for p in parts]).view(cp, -1))
+        assert torch.equal(om.view_as(o_r), _local(o_sep, r, n2c))
+        assert torch.equal(lm.view_as(l_r), _local(lse_sep, r, n2c))
+        # backward: dQ of the rank's rows, its fp32 share of dK / dV of every key
+        dq_r, dkp, dvp = cz.attn_bwd_rank(prob, plan, r, q_r, ks, vs, o_r, l_r, do_r)
+        assert torch.equal(dq_r, _local(dq, r, n2c))
+        dk_sum += dkp
+        dv_sum += dvp
+        ro.append(o_r); rl.append(l_r); rq.append(dq_r)
+    torch.cuda.synchronize()
+    assert cz.get_device_status() == 0
+    dk_r, dv_r = cz.f32_to_bf16(dk_sum), cz.f32_to_bf16(dv_sum)
+    assert torch.equal(dk_r, dk_sum.to(torch.bfloat16))        # the cast is round-to-nearest-even
+    # against the oracle, in original order
+    (dk_u, dv_u) = plan.unshard([dk_r, dv_r])
+    q, k, v, do = (f64(case[n]) for n in ("q", "k", "v", "do"))
+    ref_o, ref_l = oracle.fwd(q, k, v, case["ds"], None, case["lk"])
+    _, rk, rv = oracle.bwd(q, k, v, ref_o, ref_l, do, case["ds"], None, case["lk"])
+    tag = f"S={S} cp={cp} per-rank sum"
+    assert_bf16_close(f64(dk_u), rk, "dK " + tag)
+    assert_bf16_close(f64(dv_u), rv, "dV " + tag)
+
+
+def test_rank_calls_reject_bad_rank_and_step():
+    case = make_case(1, 2, 2, 512, 64, 2, 97)
+    prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, 2, "ring", "fused")
+    q0 = _local(qs, 0, 256)
+    with pytest.raises(cz.CPError):
+        cz.attn_fwd_rank(prob, plan, 2, q0, ks, vs)
+    with pytest.raises(cz.CPError):
+        cz.attn_fwd_step(prob, plan, 0, 2, q0, _local(ks, 0, 256), _local(vs, 0, 256))
