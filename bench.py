@@ -196,7 +196,10 @@ def config_dict(w: synth.Workload, rotate: str, world: int) -> dict:
 
 # --------------------------------------------------------------------- native arm
 
-KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_dkdv": 6.0, "bwd_dq": 2.0}   # x D*Hq*pairs
+# algorithmic FLOPs per unmasked pair and query head, x D: the forward's two products;
+# the one-pass backward's four (dV, dP, dK, dQ; S recomputed, not counted); the
+# two-pass backward's dK/dV pass (dP, dV, dK) and dQ pass (dQ)
+KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_fused": 8.0, "bwd_dkdv": 6.0, "bwd_dq": 2.0}
 
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum).
@@ -354,7 +357,9 @@ def run_native(args, w, rank, world, local_rank):
     hbm_bytes = {
         "gather": 2 * (2 * n_q + 2 * n_kv),                       # read + write Q, dO, K, V
         "merge": rows * w.cp * 4 + live * w.head_dim * 4 + rows * (row_bytes + 4),
-        "bwd_prep": rows * (2 * row_bytes + 4) + rows * 8,        # O, dO, LSE in; D, LSE2 out
+        # O, dO, LSE in; delta, -LSE*log2(e) out; the one-pass form's dQ accumulator zeroed
+        "bwd_prep": rows * (2 * row_bytes + 4) + rows * 8 + rows * w.head_dim * 4,
+        "dq_convert": rows * w.head_dim * (4 + 2),                # fp32 accumulator in, bf16 dQ out
     }
     for n, b in hbm_bytes.items():
         if n in kernels and kernels[n]["ms"] > 0:
@@ -380,6 +385,23 @@ def run_native(args, w, rank, world, local_rank):
 
     fwd_ms = dist_max(dist, time_fwd(prob), device)
     fused_ms = dist_max(dist, time_fwd(prob_fused), device)
+
+    # ---- the backward alone, both forms (one pass with dQ reductions; two passes)
+    def time_bwd(pr, n=3):
+        wb = torch.empty(max(cz.bwd_workspace_bytes(pr), 256), dtype=torch.uint8, device=device)
+        cz.attn_bwd(pr, plan, qs, ks, vs, o, lse, dos, dq, dk, dv, ws=wb)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            cz.attn_bwd(pr, plan, qs, ks, vs, o, lse, dos, dq, dk, dv, ws=wb)
+        e1.record()
+        torch.cuda.synchronize()
+        del wb
+        return e0.elapsed_time(e1) / n
+
+    bwd_ms = dist_max(dist, time_bwd(prob), device)
+    bwd1_ms = dist_max(dist, time_bwd(prob.with_one_pass(True)), device)
     fwd_32k = forward_at(args, "gqa32k", device, dist, peaks) if w.name != "gqa32k" else None
 
     # ---- end to end through the public API with pinned host buffers
@@ -457,6 +479,10 @@ def run_native(args, w, rank, world, local_rank):
             "fwd_fused_tflops": round(fwd_flops / 1e9 / fused_ms, 1),
             "fwd_fused_frac_of_peak": round(fwd_flops / 1e9 / fused_ms / peaks["bf16"], 4),
             "fwd_32k": fwd_32k,
+            "bwd_tflops": round(2.0 * fwd_flops / 1e9 / bwd_ms, 1),
+            "bwd_ms": round(bwd_ms, 3),
+            "bwd_one_pass_tflops": round(2.0 * fwd_flops / 1e9 / bwd1_ms, 1),
+            "bwd_one_pass_ms": round(bwd1_ms, 3),
             "step_frac_of_peak": round(value / world / peaks["bf16_sustained"], 4),
             "peak_source": peaks["source"],
             "pairs": pairs,

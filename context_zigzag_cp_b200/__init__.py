@@ -120,12 +120,14 @@ class Problem:
     """cp_problem_t.  ``cu_seqlens`` (int32, original order, device) turns on the
     packed-document mask; ``window`` > 0 adds a sliding window (the query at q
     sees keys q - window < k <= q); ``causal=False`` drops the causal mask (every
-    query sees every key; no documents or window then)."""
+    query sees every key; no documents or window then); ``bwd_one_pass=True``
+    selects the one-pass backward (dQ by fp32 atomic reductions; the default is the
+    two deterministic passes)."""
 
     def __init__(self, batch: int, seq_len: int, cp: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, rotate: str = "allgather", cu_seqlens: torch.Tensor | None = None,
                  merge: str = "fused", softmax_scale: float = 0.0, window: int = 0,
-                 causal: bool = True):
+                 causal: bool = True, bwd_one_pass: bool = False):
         if not causal and (cu_seqlens is not None or window):
             raise ValueError("causal=False takes no cu_seqlens and no window")
         if cu_seqlens is not None:
@@ -142,17 +144,24 @@ class Problem:
         self.batch, self.seq_len, self.cp = batch, seq_len, cp
         self.num_heads, self.num_kv_heads, self.head_dim = num_heads, num_kv_heads, head_dim
         self.rotate, self.merge, self.causal = rotate, merge, causal
+        self.bwd_one_pass = bwd_one_pass
         self.num_docs = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
         mask = "full" if not causal else ("causal" if cu_seqlens is None else "doc")
         self.c = CpProblem(batch, seq_len, cp, num_heads, num_kv_heads, head_dim,
                            _lib.ROTATE[rotate], _lib.MASK[mask],
                            _lib.MERGE[merge], float(softmax_scale), self.num_docs, int(window),
+                           int(bool(bwd_one_pass)),
                            None if cu_seqlens is None else cu_seqlens.data_ptr())
 
     def with_merge(self, merge: str) -> "Problem":
         return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
                        self.head_dim, self.rotate, self.cu_seqlens, merge,
-                       self.c.softmax_scale, self.window, self.causal)
+                       self.c.softmax_scale, self.window, self.causal, self.bwd_one_pass)
+
+    def with_one_pass(self, bwd_one_pass: bool) -> "Problem":
+        return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
+                       self.head_dim, self.rotate, self.cu_seqlens, self.merge,
+                       self.c.softmax_scale, self.window, self.causal, bwd_one_pass)
 
     @property
     def ref(self):
@@ -452,7 +461,9 @@ def selftest_stall(kernel: str, prob: Problem, plan: Plan, q, k, v, o, lse, do=N
         nbytes = fwd_workspace_bytes(prob)
     else:
         _validate_bwd(prob, plan, q, k, v, o, lse, do, dq, dk, dv)
-        nbytes = bwd_workspace_bytes(prob)
+        # the stalled kernel picks the backward form: the one-pass kernel needs its dQ
+        # accumulator whatever the problem's default form is
+        nbytes = bwd_workspace_bytes(prob.with_one_pass(kernel == "bwd_fused"))
     w = _workspace(nbytes, q.device, None)
     n = ctypes.c_size_t(nbytes)
     _check(lib().cp_selftest_stall(kid, prob.ref, plan.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),

@@ -31,7 +31,7 @@ NOALLOC_MAX_ROWS = 4194304
 
 KERNEL_NAMES = {1: "plan_meta", 2: "plan_index", 3: "gather", 4: "fwd", 5: "merge",
                 6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2",
-                11: "cast"}
+                11: "cast", 12: "bwd_fused", 13: "dq_convert"}
 KERNEL_IDS = {name: i for i, name in KERNEL_NAMES.items()}
 
 
@@ -41,7 +41,8 @@ class CpProblem(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("rotate", ctypes.c_int32), ("mask", ctypes.c_int32), ("merge", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("num_docs", ctypes.c_int32),
-                ("window", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p)]
+                ("window", ctypes.c_int32), ("bwd_one_pass", ctypes.c_int32),
+                ("cu_seqlens", ctypes.c_void_p)]
 
 
 class CpPlan(ctypes.Structure):

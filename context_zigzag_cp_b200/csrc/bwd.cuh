@@ -34,13 +34,14 @@
 namespace cpattn {
 
 // ----------------------------------------------------------------------------
-// Preprocess: delta[row] = sum_d dO*O, nlse2[row] = -LSE * log2(e).  One warp
+// Preprocess: delta[row] = sum_d dO*O, nlse2[row] = -LSE * log2(e), and (for the
+// one-pass backward) the row of the fp32 dQ accumulator set to zero.  One warp
 // per row; lane l reads 4 consecutive elements (head_dim <= 128).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                 const float* __restrict__ lse, float* __restrict__ delta,
-                float* __restrict__ nlse2, int64_t rows, int D)
+                float* __restrict__ nlse2, int64_t rows, int D, float* __restrict__ dq_acc)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -59,6 +60,8 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __rest
                 acc = fmaf(x.y, y.y, acc);
             }
         }
+        if (dq_acc && lane * 4 < D)
+            reinterpret_cast<float4*>(dq_acc + row * D)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) {
             delta[row] = acc;
@@ -83,6 +86,7 @@ struct BwdParams {
     int32_t rank;            // -1: every rank's query rows; r: only rank r's
     float* dk32;             // non-null: dK / dV written as fp32 partials here instead of bf16
     float* dv32;
+    float* dq_acc;           // one-pass backward: fp32 dQ accumulator [B*Hq][q_rows][D] (unscaled)
     const int32_t* src;      // [cp*cp]
     const int32_t* doc_start;  // [S] shard order
     const int32_t* cu;       // [num_docs+1] document offsets, original order (documents only)
@@ -254,7 +258,7 @@ struct DkdvCfg {
     static constexpr int LD_OFF = LQ_OFF + NQ * 512;              // delta rows [NDO]
     static constexpr int BAR_OFF = LD_OFF + NDO * 512;
     // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NDO], do_empty[NDO], st_ready, dp_ready,
-    // s_free, dp_free, p_full[NSLICE], acc_full, drain, acc_empty
+    // s_free, (a spare slot), p_full[NSLICE], acc_full, drain, acc_empty
     static constexpr int NBAR = 9 + 2 * NQ + 2 * NDO + BWD_NSLICE;
     // the dynamic shared window starts 1024-byte aligned (checked at run time), no slack
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64;
@@ -311,8 +315,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t bar_q_full = bars + 16, bar_q_empty = bar_q_full + 8 * Cfg::NQ;
     const uint32_t bar_do_full = bar_q_empty + 8 * Cfg::NQ, bar_do_empty = bar_do_full + 8 * Cfg::NDO;
     const uint32_t bar_st_ready = bar_do_empty + 8 * Cfg::NDO, bar_dp_ready = bar_st_ready + 8;
-    const uint32_t bar_s_free = bar_dp_ready + 8, bar_dp_free = bar_s_free + 8;
-    const uint32_t bar_p_full = bar_dp_free + 8;                      // [NSLICE]
+    const uint32_t bar_s_free = bar_dp_ready + 8;
+    const uint32_t bar_p_full = bar_s_free + 16;                      // [NSLICE]
     const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
@@ -338,7 +342,6 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_init(bar_st_ready, 1);
         mbar_init(bar_dp_ready, 1);
         mbar_init(bar_s_free, 4 * BWD_NWG);
-        mbar_init(bar_dp_free, 4 * BWD_NWG);
         for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
@@ -433,7 +436,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             // last issued tile not yet copied out by the elementwise warps
             bool ok = true, acc_busy = false, s_pending = false;
             // dV += P^T dO, dK += dS^T Q for one finished query tile.  P^T and dS^T (bf16) sit in
-            // the dP^T columns: slice j at 64j (P^T) and 64j + 32 (dS^T), 16 query rows per 8 columns.
+            // the dP^T columns: query rows 64j + 16w .. +15 of slice j at 64j + 16w (P^T) and
+            // 64j + 16w + 8 (dS^T), each warp's over the 16 columns of dP^T it read.
             auto issue_products = [&](uint32_t qs, uint32_t ds, bool& first) -> bool {
                 if (first && acc_busy) {   // every group has stored the previous item's dK / dV
                     if (!mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag)) return false;
@@ -450,8 +454,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         for (int w4 = 0; w4 < 4; ++w4) {
                             const uint32_t acc = (!first || j > 0 || w4 > 0) ? 1u : 0u;
                             const uint32_t brow = ((4 * j + w4) * 2048) >> 4;
-                            mma_ts(tdV, tdP + 64 * j + 8 * w4, bdo_mn + brow, IDESC_G, acc);
-                            mma_ts(tdK, tdP + 64 * j + 32 + 8 * w4, bq_mn + brow, IDESC_G, acc);
+                            mma_ts(tdV, tdP + 64 * j + 16 * w4, bdo_mn + brow, IDESC_G, acc);
+                            mma_ts(tdK, tdP + 64 * j + 16 * w4 + 8, bq_mn + brow, IDESC_G, acc);
                         }
                     }
                     __syncwarp();
@@ -545,8 +549,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const uint32_t tS = tmem + lane_off + 16 * wg, tdP = tmem + lane_off + 128 + 16 * wg;
         const uint32_t tdV = tmem + lane_off + 256 + 32 * wg, tdK = tmem + lane_off + 384 + 32 * wg;
         // packed P^T / dS^T of slice j go to dP^T columns 64j + 8wg and 64j + 32 + 8wg
-        const uint32_t tPk = tmem + lane_off + 128 + 8 * wg, tDk = tPk + 32;
-        uint32_t nst = 0, st_phase = 0, dp_phase = 0, a_phase = 0, df_phase = 0;
+        // packed P^T / dS^T of slice j go over this warp's own dP^T columns, already read:
+        // 64j + 16wg (P^T) and 64j + 16wg + 8 (dS^T)
+        const uint32_t tPk = tmem + lane_off + 128 + 16 * wg, tDk = tPk + 8;
+        uint32_t nst = 0, st_phase = 0, dp_phase = 0, a_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x, iter = 0; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
             const DkdvItem it = decode_dkdv(P, w, iter & 1);
@@ -591,7 +597,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         else
                             dkdv_p16<2>(sv + 16 * j, s_nlse2 + 64 * j, s_ds + 64 * j, P.scale_log2, thr, wsp, k_orig);
                     }
-                    // ---- dP^T: copy out; every warp has its columns before packed results land there
+                    // ---- dP^T: copy out; the packed results go over this warp's own columns
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
                     if (!ok) break;
                     dp_phase ^= 1;
@@ -600,13 +606,6 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tmem_ld16f(tdP + 64, dp + 16);
                     tmem_wait_ld();
                     reg_fence32f(dp);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_dp_free);
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_free, df_phase, abort_flag));
-                    if (!ok) break;
-                    df_phase ^= 1;
-                    tc_fence_after();
 #pragma unroll
                     for (int j = 0; j < BWD_NSLICE; ++j) {
                         uint32_t pk[8], dk[8];
@@ -694,8 +693,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 // a deep K/V ring.  Same schedule as the dK/dV pass: the elementwise warps copy
 // S out and release it (s_free), so the MMA warp computes the next key tile's S
 // at once; they form P while the previous tile's products and this tile's dP
-// are on the tensor core, copy dP out, and write dS (bf16) into the dP columns
-// once every warp has (dp_free), in two 64-key slices; slice 0's
+// are on the tensor core, copy dP out, and write dS (bf16) over the dP columns
+// each warp has just read, in two 64-key slices; slice 0's
 // dQ += dS K (A from tensor memory) runs while slice 1 is formed.
 // Tensor memory: S 0..127, dP 128..255, dQ 256..383, Q 384..447, dO 448..511.
 template <int D>
@@ -704,7 +703,7 @@ struct DqCfg {
     static constexpr int NSLOT = (D == 128) ? 6 : 12;
     static constexpr int KV_OFF = 0;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * KTILE;
-    // qt_full, qt_empty, kv_full[NSLOT], kv_empty[NSLOT], st_ready, dp_ready, s_free, dp_free,
+    // qt_full, qt_empty, kv_full[NSLOT], kv_empty[NSLOT], st_ready, dp_ready, s_free, (spare),
     // p_full[NSLICE], acc_full, drain, acc_empty
     static constexpr int NBAR = 9 + 2 * NSLOT + BWD_NSLICE;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;
@@ -757,8 +756,8 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bar_qt_full = bars, bar_qt_empty = bars + 8;
     const uint32_t bar_kv_full = bars + 16, bar_kv_empty = bars + 16 + 8 * Cfg::NSLOT;
     const uint32_t bar_st_ready = bars + 16 + 16 * Cfg::NSLOT, bar_dp_ready = bar_st_ready + 8;
-    const uint32_t bar_s_free = bar_dp_ready + 8, bar_dp_free = bar_s_free + 8;
-    const uint32_t bar_p_full = bar_dp_free + 8;                        // [NSLICE]
+    const uint32_t bar_s_free = bar_dp_ready + 8;
+    const uint32_t bar_p_full = bar_s_free + 16;                        // [NSLICE]
     const uint32_t bar_acc_full = bar_p_full + 8 * BWD_NSLICE, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
@@ -780,7 +779,6 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_init(bar_st_ready, 1);
         mbar_init(bar_dp_ready, 1);
         mbar_init(bar_s_free, 4 * BWD_NWG);
-        mbar_init(bar_dp_free, 4 * BWD_NWG);
         for (int i = 0; i < BWD_NSLICE; ++i) mbar_init(bar_p_full + 8 * i, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
@@ -852,7 +850,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             for (int i = 0; i < BWD_NSLICE; ++i) p_phase[i] = 0;
             bool ok = true, acc_busy = false, s_pending = false;
             // dQ += dS K for one finished key tile; dS of slice j (64 keys) sits at dP
-            // columns 64j + 8w, 16 keys per 8 columns
+            // columns 64j + 16w (keys 64j + 16w .. +15, over the dP columns that warp read)
             auto issue_dq = [&](uint32_t kslot, bool& first) -> bool {
                 if (first && acc_busy) {   // every group has stored the previous item's dQ
                     if (!mbar_wait_warp(bar_acc_empty, ae_phase, abort_flag)) return false;
@@ -867,7 +865,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     if (elect_one()) {
 #pragma unroll
                         for (int w4 = 0; w4 < 4; ++w4)
-                            mma_ts(tdQ, tdP + 64 * j + 8 * w4, bk_mn + (((4 * j + w4) * 2048) >> 4), IDESC_G,
+                            mma_ts(tdQ, tdP + 64 * j + 16 * w4, bk_mn + (((4 * j + w4) * 2048) >> 4), IDESC_G,
                                    (!first || j > 0 || w4 > 0) ? 1u : 0u);
                     }
                     __syncwarp();
@@ -960,8 +958,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t tdQ = tmem + lane_off + 256 + 32 * wg;
         const uint32_t tQ = tmem + lane_off + 384 + 16 * wg, tdO = tmem + lane_off + 448 + 16 * wg;
         // packed dS of slice j goes to dP columns 64j + 8wg
-        const uint32_t tDs = tmem + lane_off + 128 + 8 * wg;
-        uint32_t st_phase = 0, dp_phase = 0, df_phase = 0, a_phase = 0, iter = 0;
+        // packed dS of slice j goes over this warp's own dP columns, already read: 64j + 16wg
+        const uint32_t tDs = tmem + lane_off + 128 + 16 * wg;
+        uint32_t st_phase = 0, dp_phase = 0, a_phase = 0, iter = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
             const DqItem it = decode_dq(P, w);
@@ -1023,7 +1022,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         else
                             dq_p16<true>(sv + 16 * jj, nlse2, P.scale_log2, lo - 64 * jj, hi - 64 * jj);
                     }
-                    // ---- dP: copy out; every warp has its columns before dS lands there
+                    // ---- dP: copy out; the packed dS goes over this warp's own columns
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_ready, dp_phase, abort_flag));
                     if (!ok) break;
                     dp_phase ^= 1;
@@ -1032,13 +1031,6 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     tmem_ld16f(tdP + 64, dp + 16);
                     tmem_wait_ld();
                     reg_fence32f(dp);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_dp_free);
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_free, df_phase, abort_flag));
-                    if (!ok) break;
-                    df_phase ^= 1;
-                    tc_fence_after();
 #pragma unroll
                     for (int jj = 0; jj < BWD_NSLICE; ++jj) {
                         uint32_t dk[8];

@@ -15,6 +15,7 @@
 #include "merge.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "bwd_fused.cuh"
 
 using namespace cpattn;
 
@@ -34,7 +35,9 @@ std::mutex g_dev_mu;
 int g_num_sms[kMaxDevices] = {};
 uint32_t g_attr_done[kMaxDevices] = {};   // bit per kernel family (AttrSet)
 
-enum AttrSet : uint32_t { ATTR_FWD64 = 1, ATTR_FWD128 = 2, ATTR_BWD64 = 4, ATTR_BWD128 = 8 };
+enum AttrSet : uint32_t {
+    ATTR_FWD64 = 1, ATTR_FWD128 = 2, ATTR_BWD64 = 4, ATTR_BWD128 = 8, ATTR_FUSED64 = 16, ATTR_FUSED128 = 32
+};
 
 inline int current_device()
 {
@@ -541,8 +544,10 @@ template <int D>
 cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, const void* o, const float* lse, const void* dout, void* dq,
                        void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream,
-                       int stall, const Layout& L, float* dk32, float* dv32)
+                       int stall, const Layout& L, float* dk32, float* dv32, float* dq_acc)
 {
+    // dq_acc non-null: the one-pass backward (cp_bwd_fused_kernel + dq_convert_kernel);
+    // null: the two deterministic passes (cp_bwd_dkdv_kernel, cp_bwd_dq_kernel)
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
     const int64_t rows = static_cast<int64_t>(B) * Hq * L.q_rows;
     {
@@ -550,7 +555,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
         LaunchScope ls(CP_K_BWD_PREP, stream);
         bwd_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
-            nlse2, rows, D);
+            nlse2, rows, D, dq_acc);
         if (launch_status() != CP_OK) return CP_ERR_CUDA;
     }
     CUtensorMap tq, tk, tv, tdo;
@@ -590,6 +595,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.rank = L.rank;
     P.dk32 = dk32;
     P.dv32 = dv32;
+    P.dq_acc = dq_acc;
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_BWD128 : ATTR_BWD64, [] {
         cudaError_t e = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -601,6 +607,25 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     });
     if (ast != CP_OK) return ast;
     P.n_items = B * Hkv * (S / 256);   // pairs of key tiles (S / 128 is even)
+    if (dq_acc) {
+        const cp_status_t fst = ensure_attr(D == 128 ? ATTR_FUSED128 : ATTR_FUSED64, [] {
+            return cudaFuncSetAttribute(cp_bwd_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        FusedCfg<D>::SMEM_BYTES);
+        });
+        if (fst != CP_OK) return fst;
+        {
+            LaunchScope ls(CP_K_BWD_FUSED, stream);
+            cp_bwd_fused_kernel<D><<<std::min(P.n_items, num_sms()), FusedCfg<D>::THREADS,
+                                     FusedCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, P);
+        }
+        if (launch_status() != CP_OK) return CP_ERR_CUDA;
+        const int64_t n8 = rows * D / 8;
+        const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, int64_t(num_sms()) * 8);
+        LaunchScope ls(CP_K_DQ_CONVERT, stream);
+        dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq), n8, P.scale);
+        return launch_status();
+    }
     {
     LaunchScope ls(CP_K_BWD_DKDV, stream);
     cp_bwd_dkdv_kernel<D><<<std::min(P.n_items, num_sms()), DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES,
@@ -631,15 +656,20 @@ cp_status_t attn_bwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
         if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
     const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * problem->seq_len;
     const size_t row_bytes = round_up(size_t(rows) * 4, 256);
-    if (workspace_gate(2 * row_bytes, ws, ws_bytes, &st)) return st;
+    // the two deterministic passes unless the caller asks for the one-pass form (the
+    // stall hook picks the form of the kernel it targets)
+    const bool one_pass = stall == CP_K_BWD_FUSED || (problem->bwd_one_pass && stall == 0);
+    const size_t acc_bytes = one_pass ? round_up(size_t(rows) * problem->head_dim * 4, 256) : 0;
+    if (workspace_gate(2 * row_bytes + acc_bytes, ws, ws_bytes, &st)) return st;
     float* delta = static_cast<float*>(ws);
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
+    float* dq_acc = one_pass ? reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * row_bytes) : nullptr;
     cudaStream_t s = as_stream(stream);
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
-                                 whole_layout(problem), nullptr, nullptr)
+                                 whole_layout(problem), nullptr, nullptr, dq_acc)
                : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
-                                whole_layout(problem), nullptr, nullptr);
+                                whole_layout(problem), nullptr, nullptr, dq_acc);
 }
 
 }  // namespace
@@ -660,7 +690,7 @@ extern "C" cp_status_t cp_selftest_stall(int32_t kernel, const cp_problem_t* pro
 {
     if (kernel == CP_K_FWD)
         return attn_fwd_impl(problem, plan, q, k, v, o, lse, ws, ws_bytes, stream, 1);
-    if (kernel == CP_K_BWD_DKDV || kernel == CP_K_BWD_DQ)
+    if (kernel == CP_K_BWD_DKDV || kernel == CP_K_BWD_DQ || kernel == CP_K_BWD_FUSED)
         return attn_bwd_impl(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, stream,
                              kernel);
     return CP_ERR_INVALID_ARG;
@@ -723,9 +753,9 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
     float* nlse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
-                                 whole_layout(problem), nullptr, nullptr)
+                                 whole_layout(problem), nullptr, nullptr, nullptr)
                : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
-                                whole_layout(problem), nullptr, nullptr);
+                                whole_layout(problem), nullptr, nullptr, nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -823,9 +853,9 @@ extern "C" cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_pl
     const Layout L = rank_layout(problem, rank, -1);
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
-                                 s, 0, L, dk_part, dv_part)
+                                 s, 0, L, dk_part, dv_part, nullptr)
                : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
-                                s, 0, L, dk_part, dv_part);
+                                s, 0, L, dk_part, dv_part, nullptr);
 }
 
 extern "C" cp_status_t cp_f32_to_bf16(const float* in, void* out, int64_t n, void* stream)

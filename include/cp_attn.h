@@ -98,6 +98,12 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *                 q - W < k <= q (and, with documents, k in q's document).
  *                 Negative values are CP_ERR_INVALID_ARG; W > 0 with
  *                 CP_MASK_FULL is CP_ERR_UNSUPPORTED.
+ *   bwd_one_pass  backward only.  0 (default): two passes, a dK/dV pass and a
+ *                 dQ pass that recomputes S and dP; bit-for-bit reproducible,
+ *                 and the faster form on B200 (128k: 438 vs 475 ms).
+ *                 1: one pass, dK, dV and dQ from one recomputation of S and dP,
+ *                 dQ summed in an fp32 accumulator by atomic reductions (its
+ *                 last bits depend on their order); bound by those reductions.
  *   cu_seqlens    DEVICE int32 [num_docs+1], 0 = cu[0] < cu[1] < ... <
  *                 cu[num_docs] = S, original order; the same documents apply to
  *                 every batch entry.  NULL for the plain causal mask.
@@ -122,6 +128,7 @@ typedef struct {
     float softmax_scale;
     int32_t num_docs;
     int32_t window;
+    int32_t bwd_one_pass;
     const int32_t* cu_seqlens;
 } cp_problem_t;
 
@@ -210,8 +217,9 @@ CP_API cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* pla
  *   dq                bf16 [B][Hq][S][D]  output
  *   dk, dv            bf16 [B][Hkv][S][D] output
  * Workspace: two fp32 values per query row, dot(dO, O) and -LSE * log2(e)
- * (each array rounded up to 256 bytes); dQ needs no accumulator, the
- * backward runs as two deterministic passes.
+ * (each array rounded up to 256 bytes), and for the one-pass backward
+ * (problem->bwd_one_pass == 1) an fp32 dQ accumulator of head_dim values per
+ * query row (rounded up to 256 bytes).
  * Errors: as cp_attn_fwd.
  */
 CP_API cp_status_t cp_attn_bwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
@@ -354,7 +362,9 @@ CP_API cp_status_t cp_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* Test hook of the bounded-wait teardown inside the attention kernels.  Runs
  * cp_attn_fwd (kernel = CP_K_FWD) or cp_attn_bwd (kernel = CP_K_BWD_DKDV or
- * CP_K_BWD_DQ) with the same arguments and checks as those calls (o and lse are
+ * CP_K_BWD_DQ: the two-pass backward; CP_K_BWD_FUSED: the one-pass backward,
+ * whatever problem->bwd_one_pass says) with the same arguments and checks as
+ * those calls (o and lse are
  * the forward's outputs or the backward's inputs; dout, dq, dk, dv are unused by
  * CP_K_FWD and may be NULL there), except that in the named kernel the producer
  * warp of CTA 0 skips its first K/V tile load.  The MMA warp of that CTA then
@@ -384,7 +394,9 @@ typedef enum {
     CP_K_BWD_DQ = 8,     /* backward: dQ                                    */
     CP_K_SELFTEST = 9,
     CP_K_SELFTEST_EXP2 = 10,
-    CP_K_CAST = 11       /* fp32 -> bf16 cast of summed dK / dV partials    */
+    CP_K_CAST = 11,      /* fp32 -> bf16 cast of summed dK / dV partials    */
+    CP_K_BWD_FUSED = 12, /* one-pass backward: dK, dV, dQ partials          */
+    CP_K_DQ_CONVERT = 13 /* one-pass backward: dQ accumulator -> bf16       */
 } cp_kernel_t;
 
 /* Number of kernels this library has launched in this process. */

@@ -42,11 +42,17 @@ def parity_stats(gpu: np.ndarray, ref: np.ndarray, max_abs: float = O_MAX) -> di
     err = np.abs(gpu - ref)
     bound = bf16_bound(ref, max_abs)
     worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    over = err > max_abs
+    # of the elements beyond the plain 2e-2, the one farthest from its reference in ulps
+    ulps_over = (err / bf16_ulp(ref))[over]
+    k = int(np.argmax(ulps_over)) if over.any() else -1
     return dict(n=int(err.size), max=float(err.max()), mean=float(err.mean()),
-                n_over_abs=int((err > max_abs).sum()), n_over_bound=int((err > bound).sum()),
+                n_over_abs=int(over.sum()), n_over_bound=int((err > bound).sum()),
                 worst_err=float(err[worst]), worst_ref=float(abs(ref[worst])),
                 worst_bound=float(bound[worst]),
-                worst_ulps=float(err[worst] / bf16_ulp(np.asarray(ref[worst]))))
+                worst_ulps=float(err[worst] / bf16_ulp(np.asarray(ref[worst]))),
+                over_abs_max_ulps=float(ulps_over[k]) if k >= 0 else 0.0,
+                over_abs_ref=float(np.abs(ref)[over][k]) if k >= 0 else 0.0)
 
 
 def assert_bf16_close(gpu: np.ndarray, ref: np.ndarray, what: str, max_abs=O_MAX, mean_abs=O_MEAN):

@@ -98,8 +98,10 @@ def test_workspace_query(lib):
     # cp partial O (fp32) + partial LSE (fp32), each rounded up to 256 B
     rows = 1 * 2 * 512
     assert st == 0 and n == 2 * rows * 64 * 4 + 2 * rows * 4
-    # backward: per-row dot(dO, O) and LSE*log2(e), fp32 each
+    # backward: per-row dot(dO, O) and LSE*log2(e), fp32 each; the one-pass form adds an
+    # fp32 dQ accumulator of head_dim values per row
     assert cz.bwd_workspace_bytes(prob()) == 2 * rows * 4
+    assert cz.bwd_workspace_bytes(prob(bwd_one_pass=True)) == 2 * rows * 4 + rows * 64 * 4
 
 
 def test_workspace_too_small_and_null_pointers(lib):

@@ -19,10 +19,11 @@ from helpers import (assert_bf16_close, bf16_operand_attention, f64, make_case, 
 pytestmark = pytest.mark.gpu
 
 
-def run_bwd(case, cp, rotate="allgather", merge="fused", scale=0.0, with_o=False):
+def run_bwd(case, cp, rotate="allgather", merge="fused", scale=0.0, with_o=False,
+            one_pass=False):
     prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, cp, rotate, merge, scale)
     (dos,) = plan.shard([case["do"].cuda()])
-    dq, dk, dv = cz.attn_bwd(prob, plan, qs, ks, vs, o, lse, dos)
+    dq, dk, dv = cz.attn_bwd(prob.with_one_pass(one_pass), plan, qs, ks, vs, o, lse, dos)
     torch.cuda.synchronize()
     assert cz.get_device_status() == 0
     if with_o:
@@ -32,12 +33,12 @@ def run_bwd(case, cp, rotate="allgather", merge="fused", scale=0.0, with_o=False
     return prob, plan, dq, dk, dv
 
 
-def check_full(case, cp, rotate, scale=0.0, emulate=False):
-    _, _, dq, dk, dv = run_bwd(case, cp, rotate, scale=scale)
+def check_full(case, cp, rotate, scale=0.0, emulate=False, one_pass=False):
+    _, _, dq, dk, dv = run_bwd(case, cp, rotate, scale=scale, one_pass=one_pass)
     q, k, v, do = (f64(case[n]) for n in ("q", "k", "v", "do"))
     o, lse = oracle.fwd(q, k, v, case["ds"], scale or None)
     rq, rk, rv = oracle.bwd(q, k, v, o, lse, do, case["ds"], scale or None)
-    tag = f"S={q.shape[2]} cp={cp} {rotate}"
+    tag = f"S={q.shape[2]} cp={cp} {rotate}" + (" one-pass" if one_pass else "")
     assert_bf16_close(f64(dq), rq, "dQ " + tag)
     assert_bf16_close(f64(dk), rk, "dK " + tag)
     assert_bf16_close(f64(dv), rv, "dV " + tag)
@@ -52,22 +53,38 @@ def check_full(case, cp, rotate, scale=0.0, emulate=False):
             assert d_emu.mean() < 0.5 * d_ref.mean(), (name, d_emu.mean(), d_ref.mean())
 
 
-def test_small_d64():
+# one_pass: the one-pass backward (dQ partials reduced into an fp32 accumulator);
+# otherwise the default two-pass backward (a dK/dV pass and a dQ pass)
+@pytest.mark.parametrize("one_pass", [False, True])
+def test_small_d64(one_pass):
     case = make_case(1, 2, 2, 512, 64, 2, 0, with_dout=True)
-    check_full(case, 2, "allgather")
+    check_full(case, 2, "allgather", one_pass=one_pass)
 
 
-def test_fb8k():
+@pytest.mark.parametrize("one_pass", [False, True])
+def test_fb8k(one_pass):
     """S 8192, cp 4, 8 heads MHA, head_dim 128, all-gather order."""
     case = make_case(1, 8, 8, 8192, 128, 4, 1, with_dout=True)
-    check_full(case, 4, "allgather")
+    check_full(case, 4, "allgather", one_pass=one_pass)
 
 
-@pytest.mark.parametrize("D", [64, 128])
-def test_gqa_docs_small(D):
+@pytest.mark.parametrize("D,one_pass", [(64, False), (128, False), (64, True), (128, True)])
+def test_gqa_docs_small(D, one_pass):
     cu = random_docs(4096, 21, 150.0)
     case = make_case(1, 8, 2, 4096, D, 2, 22, cu=cu, with_dout=True)
-    check_full(case, 2, "ring", emulate=(D == 128))
+    check_full(case, 2, "ring", emulate=(D == 128), one_pass=one_pass)
+
+
+def test_one_pass_matches_two_pass():
+    """The two backward forms compute the same sums in different orders: dK / dV
+    are bit-identical (same per-key accumulation order), dQ differs only by the
+    fp32 summation order of its partials."""
+    case = make_case(1, 8, 2, 4096, 128, 4, 24, with_dout=True)
+    _, _, dq1, dk1, dv1 = run_bwd(case, 4, "ring", one_pass=True)
+    _, _, dq2, dk2, dv2 = run_bwd(case, 4, "ring")
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    ulp = torch.exp2(torch.floor(torch.log2(dq2.double().abs().clamp_min(2.0 ** -126))) - 7)
+    assert ((dq1.double() - dq2.double()).abs() <= ulp + 1e-6).all()
 
 
 def test_batch2_cp3_scale():
@@ -139,14 +156,14 @@ def check_identities(name, S, g, Hkv, scale, cu, dq, dk, dv, q, o, do):
     return (ev / bv).max().item(), (ek / bk).max().item()
 
 
-def check_sampled(name, rotate, n_rows=96, n_keys=24, early=True):
+def check_sampled(name, rotate, n_rows=96, n_keys=24, early=True, one_pass=False):
     w = synth.WORKLOADS[name]
     t = synth.workload_inputs(w, with_dout=True)
     S, g = w.seq_len, w.num_heads // w.num_kv_heads
     cu = t["cu_seqlens"]
     ds = oracle.doc_start(S, cu)
     case = dict(q=t["q"], k=t["k"], v=t["v"], do=t["do"], cu_seqlens=cu, ds=ds)
-    _, _, dq, dk, dv, o_gpu = run_bwd(case, w.cp, rotate, with_o=True)
+    _, _, dq, dk, dv, o_gpu = run_bwd(case, w.cp, rotate, with_o=True, one_pass=one_pass)
     rng = np.random.default_rng(w.seed + 200)
     groups = [0, int(rng.integers(1, w.num_kv_heads))]
     qh = [gi * g + i for gi in groups for i in range(g)]
@@ -157,7 +174,8 @@ def check_sampled(name, rotate, n_rows=96, n_keys=24, early=True):
     flat = np.concatenate([hi * S + rows for hi in range(len(qh))])
     rq = oracle.bwd_dq_rows(q, k, v, do, flat, ds)
     gq = f64(dq[0, qh][:, rows]).reshape(-1, w.head_dim)
-    assert_bf16_close(gq, rq, f"dQ {name} {rotate} sampled rows")
+    tag = f"{name} {rotate}" + (" one-pass" if one_pass else "")
+    assert_bf16_close(gq, rq, f"dQ {tag} sampled rows")
     # dK / dV on keys whose attending rows are few: the last keys of the sequence
     # and of its documents
     ends = [S - 1 - i for i in range(n_keys // 2)]
@@ -168,9 +186,9 @@ def check_sampled(name, rotate, n_rows=96, n_keys=24, early=True):
     flatk = np.concatenate([gi * S + keys for gi in range(len(groups))])
     rk, rv = oracle.bwd_dkv_keys(q, k, v, do, flatk, ds)
     assert_bf16_close(f64(dk[0, groups][:, keys]).reshape(-1, w.head_dim), rk,
-                      f"dK {name} {rotate} late keys")
+                      f"dK {tag} late keys")
     assert_bf16_close(f64(dv[0, groups][:, keys]).reshape(-1, w.head_dim), rv,
-                      f"dV {name} {rotate} late keys")
+                      f"dV {tag} late keys")
     if early:
         # dK / dV on whole key tiles that collect over the most query rows (every
         # row after them), for one KV group: the oracle's forward of that group's
@@ -182,22 +200,23 @@ def check_sampled(name, rotate, n_rows=96, n_keys=24, early=True):
         o1, l1 = oracle.fwd(q1, k1, v1, ds)
         ek = key_tiles_early(S, cu, rng)
         fk, fv = oracle.bwd_dkv_keys_fwd(q1, k1, v1, o1, l1, do1, ek, ds)
-        assert_bf16_close(f64(dk[0, gi][ek]), fk, f"dK {name} {rotate} early key tiles")
-        assert_bf16_close(f64(dv[0, gi][ek]), fv, f"dV {name} {rotate} early key tiles")
+        assert_bf16_close(f64(dk[0, gi][ek]), fk, f"dK {tag} early key tiles")
+        assert_bf16_close(f64(dv[0, gi][ek]), fv, f"dV {tag} early key tiles")
     check_identities(name, S, g, w.num_kv_heads, 1.0 / np.sqrt(w.head_dim), cu, dq, dk, dv,
                      t["q"], o_gpu, t["do"])
 
 
-def test_gqa32k_ring_sampled():
-    check_sampled("gqa32k", "ring")
+@pytest.mark.parametrize("one_pass", [False, True])
+def test_gqa32k_ring_sampled(one_pass):
+    check_sampled("gqa32k", "ring", one_pass=one_pass)
 
 
 def test_docs64k_sampled():
     check_sampled("docs64k", "ring")
 
 
-@pytest.mark.parametrize("rotate", ["allgather", "ring"])
-def test_long128k_sampled(rotate):
+@pytest.mark.parametrize("rotate,one_pass", [("allgather", False), ("ring", True)])
+def test_long128k_sampled(rotate, one_pass):
     # the oracle forward of a whole KV group at 128k is too slow for a test: early
     # key tiles are covered at 32k and 64k
-    check_sampled("long128k", rotate, n_rows=48, n_keys=16, early=False)
+    check_sampled("long128k", rotate, n_rows=48, n_keys=16, early=False, one_pass=one_pass)

@@ -27,6 +27,7 @@ def test_ranks_reassemble_whole(Hq, Hkv, S, D, cp, docs, causal):
     case = make_case(1, Hq, Hkv, S, D, cp, 96 + S, cu=cu, with_dout=True, causal=causal)
     prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, cp, "ring", "fused")
     (dos,) = plan.shard([case["do"].cuda()])
+    # the per-rank backward is the two-pass form: compare with the whole two-pass one
     dq, dk, dv = cz.attn_bwd(prob, plan, qs, ks, vs, o, lse, dos)
     prob_sep = prob.with_merge("separate")
     o_sep, lse_sep = cz.attn_fwd(prob_sep, plan, qs, ks, vs)

@@ -1,6 +1,7 @@
 """The attention kernels' bounded waits, made to run out on the GPU.
 
-cp_selftest_stall runs a forward or backward in which CTA 0 of the named kernel
+cp_selftest_stall runs a forward or backward (the two-pass kernels or the
+one-pass kernel) in which CTA 0 of the named kernel
 never receives its first K/V tile: its MMA warp's wait must give up after the
 wait limit, record CP_ERR_TIMEOUT, and the CTA must drain and free its tensor
 memory.  The same process then runs a normal forward and backward and must
@@ -37,7 +38,7 @@ def _parity_after(case, cp, rotate):
     assert_bf16_close(f64(dv), rv, "dV after a timed-out kernel")
 
 
-@pytest.mark.parametrize("kernel", ["fwd", "bwd_dkdv", "bwd_dq"])
+@pytest.mark.parametrize("kernel", ["fwd", "bwd_dkdv", "bwd_dq", "bwd_fused"])
 def test_stalled_kernel_times_out_and_context_survives(kernel):
     case = make_case(1, 4, 2, 1024, 128, 2, 31, with_dout=True)
     prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, 2, "ring", "fused")
