@@ -208,10 +208,13 @@ KERNEL_FLOP_SHARE = {"fwd": 4.0, "bwd_fused": 8.0, "bwd_dkdv": 6.0, "bwd_dq": 2.
 # blank lines dropped, so comment edits keep it); after any code change it reads
 # as null.
 MEASURED_TRAFFIC = {
-    ("long128k", "allgather", "bwd_dkdv"): {"bytes": 42.76e9 + 0.551e9,
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum (1 pass) on the timed step's
+    # dK/dV pass of `bench.py --steps 1 --warmup 3 --no-cpu-baseline` (long128k)
+    ("long128k", "allgather", "bwd_dkdv"): {"bytes": 37.63e9 + 0.54344e9,
                                              "src": "context_zigzag_cp_b200/csrc/bwd.cuh",
-                                             "sha256_16": "01e6eae8f698ae33"},
+                                             "sha256_16": "d4f8f5285c5eba11"},
 }
+
 
 
 def measured_traffic(workload: str, rotate: str, kernel: str):
@@ -357,8 +360,10 @@ def run_native(args, w, rank, world, local_rank):
     hbm_bytes = {
         "gather": 2 * (2 * n_q + 2 * n_kv),                       # read + write Q, dO, K, V
         "merge": rows * w.cp * 4 + live * w.head_dim * 4 + rows * (row_bytes + 4),
-        # O, dO, LSE in; delta, -LSE*log2(e) out; the one-pass form's dQ accumulator zeroed
-        "bwd_prep": rows * (2 * row_bytes + 4) + rows * 8 + rows * w.head_dim * 4,
+        # O, dO, LSE in; delta, -LSE*log2(e) out (+ the dQ accumulator zeroed when the
+        # step runs the one-pass backward)
+        "bwd_prep": rows * (2 * row_bytes + 4) + rows * 8
+                    + (rows * w.head_dim * 4 if prob.bwd_one_pass else 0),
         "dq_convert": rows * w.head_dim * (4 + 2),                # fp32 accumulator in, bf16 dQ out
     }
     for n, b in hbm_bytes.items():
@@ -478,6 +483,10 @@ def run_native(args, w, rank, world, local_rank):
             "fwd_frac_of_peak": round(fwd_flops / 1e9 / fwd_ms / peaks["bf16"], 4),
             "fwd_fused_tflops": round(fwd_flops / 1e9 / fused_ms, 1),
             "fwd_fused_frac_of_peak": round(fwd_flops / 1e9 / fused_ms / peaks["bf16"], 4),
+            # the forward and its merge as they ran inside the traced step; the figures
+            # above time the forward alone, three calls back to back
+            "fwd_in_step_tflops": round(fwd_flops / 1e9 / (kernels["fwd"]["ms"] + kernels.get(
+                "merge", {"ms": 0.0})["ms"]), 1),
             "fwd_32k": fwd_32k,
             "bwd_tflops": round(2.0 * fwd_flops / 1e9 / bwd_ms, 1),
             "bwd_ms": round(bwd_ms, 3),

@@ -35,8 +35,9 @@ namespace cpattn {
 
 // ----------------------------------------------------------------------------
 // Preprocess: delta[row] = sum_d dO*O, nlse2[row] = -LSE * log2(e), and (for the
-// one-pass backward) the row of the fp32 dQ accumulator set to zero.  One warp
-// per row; lane l reads 4 consecutive elements (head_dim <= 128).
+// one-pass backward) the row of the fp32 dQ accumulator set to zero.  A row is
+// D/8 lanes of one warp, each reading 16 bytes (8 bf16) of O and of dO, so a
+// warp covers 32*8/D rows per step with full 16-byte accesses (D = 64 or 128).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
@@ -44,26 +45,34 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __rest
                 float* __restrict__ nlse2, int64_t rows, int D, float* __restrict__ dq_acc)
 {
     const int lane = threadIdx.x & 31;
+    const int lpr = D / 8;                      // lanes per row
+    const int rpw = 32 / lpr;                   // rows per warp step
+    const int sub = lane / lpr, e = lane - sub * lpr;
     const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t row = warp_g; row < rows; row += nwarps) {
+    for (int64_t base = warp_g * rpw; base < rows; base += nwarps * rpw) {
+        const int64_t row = base + sub;
         float acc = 0.f;
-        if (lane * 4 < D) {
-            const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + row * D) + lane);
-            const uint2 b = __ldg(reinterpret_cast<const uint2*>(dout + row * D) + lane);
+        if (row < rows) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + e);
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + e);
             const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
             const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const float2 x = __bfloat1622float2(a2[i]), y = __bfloat1622float2(b2[i]);
                 acc = fmaf(x.x, y.x, acc);
                 acc = fmaf(x.y, y.y, acc);
             }
+            if (dq_acc) {
+                float4* z = reinterpret_cast<float4*>(dq_acc + row * D) + 2 * e;
+                z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
-        if (dq_acc && lane * 4 < D)
-            reinterpret_cast<float4*>(dq_acc + row * D)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
+        // sum over the row's lpr lanes (a power of two, aligned inside the warp)
+        for (int off = lpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (e == 0 && row < rows) {
             delta[row] = acc;
             nlse2[row] = __ldg(lse + row) * -1.4426950408889634f;
         }
