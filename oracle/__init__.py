@@ -61,8 +61,8 @@ def _load():
         lib = ctypes.CDLL(build())
         I32, I64, F64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         lib.orc_doc_start.argtypes = [I32, I32, _i32p, _i32p]
-        lib.orc_plan.argtypes = [I32, I32, I32, I32, _i32p, I32, I32, _i32p, _i32p, _i32p, _i32p,
-                                 _i32p, _i32p, _i64p]
+        lib.orc_plan.argtypes = [I32, I32, I32, I32, _i32p, I32, I32, I32, _i32p, _i32p, _i32p,
+                                 _i32p, _i32p, _i32p, _i64p]
         lib.orc_fwd_rows.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _i32p,
                                      _i32p, I64, _i64p, _f64p, _f64p]
         lib.orc_fwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p, _i32p, _i32p,
@@ -116,11 +116,13 @@ def doc_start(seq_len: int, cu_seqlens=None) -> np.ndarray:
 
 
 def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None, window: int = 0,
-         causal: bool = True) -> dict:
+         causal: bool = True, shard: str = "sequence") -> dict:
     """The zigzag plan: perm, inv_perm, src, doc_start (shard order), rank_cu_off,
     rank_cu and pairs (int64), exactly as the library's planner must produce them.
     ``window`` > 0 counts pairs under a sliding window (keys q-W < k <= q);
-    ``causal`` False counts every key of the query's document."""
+    ``causal`` False counts every key of the query's document.  ``shard`` "doc"
+    cuts every document (not the sequence) into 2cp chunks, rank r taking chunks r
+    and 2cp-1-r of each document in turn (document lengths multiples of 2cp)."""
     lib = _load()
     cu = (np.zeros(1, dtype=np.int32) if cu_seqlens is None
           else np.ascontiguousarray(cu_seqlens, dtype=np.int32))
@@ -129,9 +131,9 @@ def plan(seq_len: int, cp: int, rotate: str = "allgather", cu_seqlens=None, wind
     out = dict(perm=np.zeros(S, np.int32), inv_perm=np.zeros(S, np.int32),
                src=np.zeros(cp * cp, np.int32), doc_start=np.zeros(S, np.int32),
                rank_cu_off=np.zeros(cp + 1, np.int32),
-               rank_cu=np.zeros(3 * cp + max(nd, 1), np.int32), pairs=np.zeros(cp, np.int64))
+               rank_cu=np.zeros(cp * (2 * max(nd, 1) + 3), np.int32), pairs=np.zeros(cp, np.int64))
     _check(lib.orc_plan(S, cp, ROTATE[rotate], nd, cu, int(window), int(bool(causal)),
-                        out["perm"], out["inv_perm"],
+                        {"sequence": 0, "doc": 1}[shard], out["perm"], out["inv_perm"],
                         out["src"], out["doc_start"], out["rank_cu_off"], out["rank_cu"],
                         out["pairs"]), "plan")
     out["rank_cu"] = out["rank_cu"][: out["rank_cu_off"][cp]].copy()
@@ -227,13 +229,13 @@ def lse_merge(o_parts, lse_parts):
 
 
 def cp_fwd(q, k, v, cp, rotate="allgather", cu_seqlens=None, scale=None, steps=None, window=0,
-           causal=True):
+           causal=True, shard="sequence"):
     """The sharded computation: for every rank r, the partials against K/V shard
     src[r][s] for each step s (all steps unless ``steps`` limits them), merged in
     visit order.  Returns O [B,Hq,S,D] and LSE [B,Hq,S] in SHARD order."""
     q = _f64(q)
     B, Hq, S, D = q.shape
-    pl = plan(S, cp, rotate, cu_seqlens, window, causal)
+    pl = plan(S, cp, rotate, cu_seqlens, window, causal, shard)
     ds = first_key(S, cu_seqlens, window)
     lk = last_key(S, cu_seqlens, causal)
     n2c = S // cp

@@ -66,7 +66,13 @@ int orc_doc_start(int32_t S, int32_t num_docs, const int32_t *cu, int32_t *ds_or
 
 /*
  * The zigzag shard plan.
- *   perm[r*2C + t]  = original index of local token t of rank r
+ *   perm[r*2C + t]  = original index of local token t of rank r.  Sequence-level
+ *                     sharding (per_doc = 0): rank r holds chunk r, then chunk
+ *                     2cp-1-r of the whole sequence.  Per-document sharding
+ *                     (per_doc = 1): every document is cut into 2cp equal
+ *                     chunks and rank r holds, document after document, its
+ *                     chunk r followed by its chunk 2cp-1-r (each document's
+ *                     length must be a multiple of 2cp).
  *   inv_perm[o]     = shard position of original index o
  *   src[r*cp + s]   = K/V shard visited by rank r at step s:
  *                     s (all-gather, rank order) or (r - s) mod cp (ring,
@@ -75,8 +81,10 @@ int orc_doc_start(int32_t S, int32_t num_docs, const int32_t *cu, int32_t *ds_or
  *   doc_start[p]    = doc start (original coordinates) of token perm[p]
  *   rank_cu_off[r]  = offset of rank r's list in rank_cu; rank_cu_off[cp] =
  *                     total entries.  rank r's list holds the local offsets
- *                     where a segment starts (local 0, the chunk boundary C,
- *                     and every document start inside its chunks), then 2C.
+ *                     where a segment starts, then 2C: sequence-level, local 0,
+ *                     the chunk boundary C and every document start inside its
+ *                     chunks; per-document, the start of each of its chunks
+ *                     (two per document).
  *   pairs[r]        = number of unmasked (q, k) pairs whose query is on rank r;
  *                     causal: the query at o sees keys ds(o) .. o, raised to
  *                     max(ds(o), o - W + 1) under a sliding window W > 0
@@ -86,36 +94,64 @@ int orc_doc_start(int32_t S, int32_t num_docs, const int32_t *cu, int32_t *ds_or
  * Returns ORC_EINVAL on a bad configuration.
  */
 int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int32_t *cu,
-             int32_t window, int32_t causal, int32_t *perm, int32_t *inv_perm, int32_t *src, int32_t *doc_start,
-             int32_t *rank_cu_off, int32_t *rank_cu, int64_t *pairs)
+             int32_t window, int32_t causal, int32_t per_doc, int32_t *perm, int32_t *inv_perm,
+             int32_t *src, int32_t *doc_start, int32_t *rank_cu_off, int32_t *rank_cu,
+             int64_t *pairs)
 {
     if (cp < 1 || S <= 0 || S % (2 * cp) != 0 || window < 0) return ORC_EINVAL;
     if (!causal && window != 0) return ORC_EINVAL;
     if (rotate != 0 && rotate != 1) return ORC_EINVAL;
+    if (per_doc && num_docs < 1) return ORC_EINVAL;
     int64_t C = S / (2 * cp);
     int32_t *ds_orig = (int32_t *)malloc(sizeof(int32_t) * (size_t)S);
     if (!ds_orig) return ORC_EINVAL;
     if (orc_doc_start(S, num_docs, cu, ds_orig) != ORC_OK) { free(ds_orig); return ORC_EINVAL; }
+    if (per_doc)
+        for (int64_t d = 0; d < num_docs; ++d)
+            if ((cu[d + 1] - cu[d]) % (2 * cp) != 0) { free(ds_orig); return ORC_EINVAL; }
 
-    for (int64_t r = 0; r < cp; ++r)
-        for (int64_t t = 0; t < 2 * C; ++t) {
-            int64_t o = orc_orig_of_local(C, cp, r, t);
-            perm[r * 2 * C + t] = (int32_t)o;
-            inv_perm[o] = (int32_t)(r * 2 * C + t);
+    int32_t n = 0;   /* entries written to rank_cu */
+    if (!per_doc) {
+        for (int64_t r = 0; r < cp; ++r)
+            for (int64_t t = 0; t < 2 * C; ++t) {
+                int64_t o = orc_orig_of_local(C, cp, r, t);
+                perm[r * 2 * C + t] = (int32_t)o;
+                inv_perm[o] = (int32_t)(r * 2 * C + t);
+            }
+    } else {
+        /* rank r's local tokens, appended document by document: its chunk r, then
+         * its chunk 2cp-1-r; each appended chunk starts a segment */
+        for (int64_t r = 0; r < cp; ++r) {
+            rank_cu_off[r] = n;
+            int64_t t = 0;
+            for (int64_t d = 0; d < num_docs; ++d) {
+                int64_t len = (cu[d + 1] - cu[d]) / (2 * cp);
+                int64_t chunks[2] = {r, 2 * cp - 1 - r};
+                for (int h = 0; h < 2; ++h) {
+                    rank_cu[n++] = (int32_t)t;
+                    for (int64_t w = 0; w < len; ++w, ++t) {
+                        int64_t o = cu[d] + chunks[h] * len + w;
+                        perm[r * 2 * C + t] = (int32_t)o;
+                        inv_perm[o] = (int32_t)(r * 2 * C + t);
+                    }
+                }
+            }
+            rank_cu[n++] = (int32_t)(2 * C);
         }
+        rank_cu_off[cp] = n;
+    }
     for (int64_t r = 0; r < cp; ++r)
         for (int64_t s = 0; s < cp; ++s)
             src[r * cp + s] = (int32_t)(rotate == 0 ? s : ((r - s) % cp + cp) % cp);
     for (int64_t p = 0; p < S; ++p) doc_start[p] = ds_orig[perm[p]];
 
-    int32_t n = 0;
     for (int64_t r = 0; r < cp; ++r) {
-        rank_cu_off[r] = n;
+        if (!per_doc) rank_cu_off[r] = n;
         int64_t cnt = 0;
         for (int64_t t = 0; t < 2 * C; ++t) {
-            int64_t o = orc_orig_of_local(C, cp, r, t);
+            int64_t o = perm[r * 2 * C + t];
             int is_start = (t == 0) || (t == C) || (ds_orig[o] == o);
-            if (is_start) rank_cu[n++] = (int32_t)t;
+            if (!per_doc && is_start) rank_cu[n++] = (int32_t)t;
             int64_t first = ds_orig[o];
             if (window > 0 && o - window + 1 > first) first = o - window + 1;
             int64_t last = o;
@@ -126,10 +162,10 @@ int orc_plan(int32_t S, int32_t cp, int32_t rotate, int32_t num_docs, const int3
             }
             cnt += last - first + 1; /* keys first..last are unmasked */
         }
-        rank_cu[n++] = (int32_t)(2 * C);
+        if (!per_doc) rank_cu[n++] = (int32_t)(2 * C);
         pairs[r] = cnt;
     }
-    rank_cu_off[cp] = n;
+    if (!per_doc) rank_cu_off[cp] = n;
     free(ds_orig);
     return ORC_OK;
 }

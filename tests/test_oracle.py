@@ -614,3 +614,64 @@ def test_noncausal_sampled_equals_full():
         sk, sv = fn()
         np.testing.assert_allclose(sk, dk.reshape(-1, D)[keys], atol=1e-13)
         np.testing.assert_allclose(sv, dv.reshape(-1, D)[keys], atol=1e-13)
+
+
+# ------------------------------------------------------- per-document zigzag sharding
+# (FlashCP abstract, "Per-Doc" sharding: every document, not only the sequence, is
+# split so each rank gets an equal share of its causal work)
+
+def test_per_doc_plan_golden():
+    """S 16, cp 2, two documents of 8: each cut into 4 chunks of 2 tokens; rank 0
+    holds chunks 0 and 3 of each document, rank 1 chunks 1 and 2 (worked by hand)."""
+    pl = oracle.plan(16, 2, "allgather", [0, 8, 16], shard="doc")
+    assert list(pl["perm"]) == [0, 1, 6, 7, 8, 9, 14, 15, 2, 3, 4, 5, 10, 11, 12, 13]
+    assert list(pl["inv_perm"][pl["perm"]]) == list(range(16))
+    assert list(pl["doc_start"]) == [0, 0, 0, 0, 8, 8, 8, 8, 0, 0, 0, 0, 8, 8, 8, 8]
+    assert list(pl["rank_cu_off"]) == [0, 5, 10]
+    assert list(pl["rank_cu"]) == [0, 2, 4, 6, 8, 0, 2, 4, 6, 8]
+    # causal pairs: rank 0 rows 0,1,6,7 | 8,9,14,15 -> (1+2+7+8) * 2; rank 1 -> (3+4+5+6) * 2
+    assert list(pl["pairs"]) == [36, 36]
+
+
+def test_per_doc_single_document_is_the_sequence_plan():
+    for S, cp in ((512, 2), (4096, 4), (2304, 3)):
+        a = oracle.plan(S, cp, "ring", [0, S], shard="doc")
+        b = oracle.plan(S, cp, "ring", [0, S])
+        for key in ("perm", "inv_perm", "src", "doc_start", "rank_cu_off", "rank_cu", "pairs"):
+            assert np.array_equal(a[key], b[key]), key
+
+
+def test_per_doc_balances_causal_work():
+    """Per document of length L = 2cp*c, rank r's two chunks carry c^2 (2cp-1) + c(c+1)
+    causal pairs whatever r is, so every rank gets the same work; the sequence-level
+    zigzag over the same documents does not."""
+    cp = 8
+    lens = synth.doc_lengths(65536, 3, 2048.0, 1.0, (128, 32768))
+    lens = [max(2 * cp, (n // (2 * cp)) * 2 * cp) for n in lens]
+    lens[-1] += 65536 - sum(lens)
+    assert lens[-1] > 0 and lens[-1] % (2 * cp) == 0
+    cu = synth.cu_seqlens(lens)
+    pd = oracle.plan(65536, cp, "ring", cu, shard="doc")
+    sq = oracle.plan(65536, cp, "ring", cu)
+    c = np.asarray(lens, dtype=np.int64) // (2 * cp)
+    assert (pd["pairs"] == (c * c * (2 * cp - 1) + c * (c + 1)).sum()).all()
+    assert pd["pairs"].sum() == sq["pairs"].sum() == oracle.causal_pairs(65536, cu)
+    assert sq["pairs"].max() / sq["pairs"].mean() > 1.5
+    assert np.array_equal(np.sort(pd["perm"]), np.arange(65536))
+
+
+def test_per_doc_sharded_merged_equals_unsharded():
+    S, cp, cu = 96, 2, [0, 24, 32, 96]
+    q, k, v = rnd((1, 2, S, 8), 81), rnd((1, 2, S, 8), 82), rnd((1, 2, S, 8), 83)
+    so, sl = oracle.cp_fwd(q, k, v, cp, "ring", cu, shard="doc")
+    o, lse = oracle.fwd(q, k, v, oracle.doc_start(S, cu))
+    perm = oracle.plan(S, cp, "ring", cu, shard="doc")["perm"]
+    np.testing.assert_allclose(so, o[:, :, perm], atol=1e-12)
+    np.testing.assert_allclose(sl, lse[:, :, perm], atol=1e-12)
+
+
+def test_per_doc_rejects_uneven_documents():
+    with pytest.raises(ValueError):
+        oracle.plan(16, 2, "allgather", [0, 6, 16], shard="doc")   # 6 is not a multiple of 4
+    with pytest.raises(ValueError):
+        oracle.plan(16, 2, "allgather", None, shard="doc")         # needs documents
