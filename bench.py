@@ -250,7 +250,7 @@ def forward_at(args, name, device, dist, peaks, reps=5):
     cu = None if t["cu_seqlens"] is None else torch.from_numpy(t["cu_seqlens"]).to(device)
     out = {"workload": name, "rotate": w.rotate}
     prob = cz.Problem(w.batch, w.seq_len, w.cp, w.num_heads, w.num_kv_heads, w.head_dim,
-                      w.rotate, cu, merge="separate")
+                      w.rotate, cu, merge="separate", shard=w.shard)
     plan = cz.Plan(prob)
     qs, ks, vs = plan.shard([t["q"], t["k"], t["v"]])
     o = torch.empty_like(qs)
@@ -289,7 +289,7 @@ def run_native(args, w, rank, world, local_rank):
     t = synth.workload_inputs(w, device=device, with_dout=True)
     cu = None if t["cu_seqlens"] is None else torch.from_numpy(t["cu_seqlens"]).to(device)
     prob = cz.Problem(w.batch, w.seq_len, w.cp, w.num_heads, w.num_kv_heads, w.head_dim, rotate,
-                      cu, merge="separate")
+                      cu, merge="separate", shard=w.shard)
     prob_fused = prob.with_merge("fused")
     plan = cz.Plan(prob)
     q, k, v, do = t["q"], t["k"], t["v"], t["do"]

@@ -88,6 +88,10 @@ def _check_plan(prob: "Problem", plan: "Plan", dev) -> None:
                          f"problem has seq_len {prob.seq_len}, cp {prob.cp}, {prob.rotate}")
     if getattr(pp, "causal", True) != getattr(prob, "causal", True):
         raise ValueError("plan: built for the other mask (causal / no causal mask)")
+    if getattr(pp, "shard", "sequence") != getattr(prob, "shard", "sequence"):
+        raise ValueError(f"plan: built for {pp.shard!r} sharding; the problem has {prob.shard!r}")
+    if getattr(pp, "window", 0) != getattr(prob, "window", 0):
+        raise ValueError(f"plan: built for window {pp.window}; the problem has {prob.window}")
     if pp.cu_seqlens is not prob.cu_seqlens:
         same = (pp.cu_seqlens is not None and prob.cu_seqlens is not None
                 and pp.cu_seqlens.shape == prob.cu_seqlens.shape
@@ -122,14 +126,20 @@ class Problem:
     sees keys q - window < k <= q); ``causal=False`` drops the causal mask (every
     query sees every key; no documents or window then); ``bwd_one_pass=True``
     selects the one-pass backward (dQ by fp32 atomic reductions; the default is the
-    two deterministic passes)."""
+    two deterministic passes); ``shard="doc"`` cuts every document, not the whole
+    sequence, into 2*cp zigzag chunks (needs ``cu_seqlens``, and every document's
+    length a multiple of 256*cp)."""
 
     def __init__(self, batch: int, seq_len: int, cp: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, rotate: str = "allgather", cu_seqlens: torch.Tensor | None = None,
                  merge: str = "fused", softmax_scale: float = 0.0, window: int = 0,
-                 causal: bool = True, bwd_one_pass: bool = False):
+                 causal: bool = True, bwd_one_pass: bool = False, shard: str = "sequence"):
         if not causal and (cu_seqlens is not None or window):
             raise ValueError("causal=False takes no cu_seqlens and no window")
+        if shard not in _lib.SHARD:
+            raise ValueError(f"shard: expected one of {sorted(_lib.SHARD)}, got {shard!r}")
+        if shard == "doc" and cu_seqlens is None:
+            raise ValueError("shard='doc' needs cu_seqlens")
         if cu_seqlens is not None:
             if not isinstance(cu_seqlens, torch.Tensor):
                 raise TypeError("cu_seqlens: expected a torch.Tensor")
@@ -145,23 +155,36 @@ class Problem:
         self.num_heads, self.num_kv_heads, self.head_dim = num_heads, num_kv_heads, head_dim
         self.rotate, self.merge, self.causal = rotate, merge, causal
         self.bwd_one_pass = bwd_one_pass
+        self.shard = shard
+        self.softmax_scale = float(softmax_scale)
         self.num_docs = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
         mask = "full" if not causal else ("causal" if cu_seqlens is None else "doc")
         self.c = CpProblem(batch, seq_len, cp, num_heads, num_kv_heads, head_dim,
                            _lib.ROTATE[rotate], _lib.MASK[mask],
-                           _lib.MERGE[merge], float(softmax_scale), self.num_docs, int(window),
-                           int(bool(bwd_one_pass)),
+                           _lib.MERGE[merge], self.softmax_scale, self.num_docs, int(window),
+                           int(bool(bwd_one_pass)), _lib.SHARD[shard],
                            None if cu_seqlens is None else cu_seqlens.data_ptr())
 
+    def _replace(self, **kw) -> "Problem":
+        args = dict(batch=self.batch, seq_len=self.seq_len, cp=self.cp, num_heads=self.num_heads,
+                    num_kv_heads=self.num_kv_heads, head_dim=self.head_dim, rotate=self.rotate,
+                    cu_seqlens=self.cu_seqlens, merge=self.merge,
+                    softmax_scale=self.softmax_scale, window=self.window, causal=self.causal,
+                    bwd_one_pass=self.bwd_one_pass, shard=self.shard)
+        args.update(kw)
+        return Problem(**args)
+
     def with_merge(self, merge: str) -> "Problem":
-        return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
-                       self.head_dim, self.rotate, self.cu_seqlens, merge,
-                       self.c.softmax_scale, self.window, self.causal, self.bwd_one_pass)
+        return self._replace(merge=merge)
 
     def with_one_pass(self, bwd_one_pass: bool) -> "Problem":
-        return Problem(self.batch, self.seq_len, self.cp, self.num_heads, self.num_kv_heads,
-                       self.head_dim, self.rotate, self.cu_seqlens, self.merge,
-                       self.c.softmax_scale, self.window, self.causal, bwd_one_pass)
+        return self._replace(bwd_one_pass=bwd_one_pass)
+
+    def rank_cu_len(self) -> int:
+        """Entries of the plan's per-rank segment list (cp_plan_t.rank_cu)."""
+        if self.shard == "doc":
+            return self.cp * (2 * self.num_docs + 1)
+        return 3 * self.cp + max(self.num_docs, 1)
 
     @property
     def ref(self):
@@ -181,11 +204,14 @@ class Plan:
         self.src = torch.empty(cp * cp, **i32)
         self.doc_start = torch.empty(S, **i32)
         self.rank_cu_off = torch.empty(cp + 1, **i32)
-        self.rank_cu = torch.empty(3 * cp + max(prob.num_docs, 1), **i32)
+        self.rank_cu = torch.empty(prob.rank_cu_len(), **i32)
         self.pairs = torch.empty(cp, dtype=torch.int64, device=dev)
+        self.tile_orig = torch.empty((S + 127) // 128, **i32)
+        self.tile_shard = torch.empty((S + 127) // 128, **i32)
         self.c = CpPlan(*(t.data_ptr() for t in (self.perm, self.inv_perm, self.src,
                                                   self.doc_start, self.rank_cu_off,
-                                                  self.rank_cu, self.pairs)))
+                                                  self.rank_cu, self.pairs, self.tile_orig,
+                                                  self.tile_shard)))
         self.build(stream=stream)
 
     @property
@@ -235,7 +261,7 @@ class Plan:
 def fwd_workspace_bytes(prob: Problem) -> int:
     n = ctypes.c_size_t(0)
     dummy = ctypes.c_void_p(256)
-    plan = CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     _check(lib().cp_attn_fwd(prob.ref, ctypes.byref(plan), dummy, dummy, dummy, dummy, dummy,
                              None, ctypes.byref(n), None), "cp_attn_fwd(workspace query)")
     return n.value
@@ -244,7 +270,7 @@ def fwd_workspace_bytes(prob: Problem) -> int:
 def bwd_workspace_bytes(prob: Problem) -> int:
     n = ctypes.c_size_t(0)
     d = ctypes.c_void_p(256)
-    plan = CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     _check(lib().cp_attn_bwd(prob.ref, ctypes.byref(plan), d, d, d, d, d, d, d, d, d, None,
                              ctypes.byref(n), None), "cp_attn_bwd(workspace query)")
     return n.value

@@ -29,6 +29,8 @@ EXPORTED = ("cp_plan_shards", "cp_unshard", "cp_attn_fwd", "cp_attn_bwd", "cp_ls
 
 NOALLOC_MAX_ROWS = 4194304
 
+SHARD = {"sequence": 0, "doc": 1}
+
 KERNEL_NAMES = {1: "plan_meta", 2: "plan_index", 3: "gather", 4: "fwd", 5: "merge",
                 6: "bwd_prep", 7: "bwd_dkdv", 8: "bwd_dq", 9: "selftest", 10: "selftest_exp2",
                 11: "cast", 12: "bwd_fused", 13: "dq_convert"}
@@ -42,14 +44,15 @@ class CpProblem(ctypes.Structure):
                 ("rotate", ctypes.c_int32), ("mask", ctypes.c_int32), ("merge", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("num_docs", ctypes.c_int32),
                 ("window", ctypes.c_int32), ("bwd_one_pass", ctypes.c_int32),
-                ("cu_seqlens", ctypes.c_void_p)]
+                ("shard", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p)]
 
 
 class CpPlan(ctypes.Structure):
     _fields_ = [("perm", ctypes.c_void_p), ("inv_perm", ctypes.c_void_p),
                 ("src", ctypes.c_void_p), ("doc_start", ctypes.c_void_p),
                 ("rank_cu_off", ctypes.c_void_p), ("rank_cu", ctypes.c_void_p),
-                ("pairs", ctypes.c_void_p)]
+                ("pairs", ctypes.c_void_p), ("tile_orig", ctypes.c_void_p),
+                ("tile_shard", ctypes.c_void_p)]
 
 
 _lib = None

@@ -96,6 +96,8 @@ struct BwdParams {
     float* dk32;             // non-null: dK / dV written as fp32 partials here instead of bf16
     float* dv32;
     float* dq_acc;           // one-pass backward: fp32 dQ accumulator [B*Hq][q_rows][D] (unscaled)
+    const int32_t* tile_orig;   // per-document plans (as in FwdParams); null otherwise
+    const int32_t* tile_shard;
     const int32_t* src;      // [cp*cp]
     const int32_t* doc_start;  // [S] shard order
     const int32_t* cu;       // [num_docs+1] document offsets, original order (documents only)
@@ -240,13 +242,11 @@ __device__ __forceinline__ int dkdv_last_tile(const BwdParams& P, int ko, int nt
     }
     return t_end;
 }
-// True when the query tile starting at original qo belongs to the rank the pass
+// True when the query tile at shard position qpos belongs to the rank the pass
 // runs for (always, for a whole-sequence pass).
-__device__ __forceinline__ bool q_tile_on_rank(const BwdParams& P, int qo)
+__device__ __forceinline__ bool q_tile_on_rank(const BwdParams& P, int qpos)
 {
-    if (P.rank < 0) return true;
-    const int c = qo / P.C;
-    return (c < P.cp ? c : 2 * P.cp - 1 - c) == P.rank;
+    return P.rank < 0 || qpos / (2 * P.C) == P.rank;
 }
 
 constexpr int BWD_NWG = 4;                       // elementwise warpgroups
@@ -287,6 +287,7 @@ struct DkdvItem {
 // wave then read query tiles that lie within a window of about gridDim.x tiles
 // (first halves) or are the same tile (second halves), so each query tile comes
 // from DRAM about once per wave instead of once per CTA.
+template <bool PD>
 __device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int unit, int half)
 {
     DkdvItem it;
@@ -298,11 +299,11 @@ __device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int unit, in
     it.b = it.bkv / P.Hkv;
     it.hk = it.bkv - it.b * P.Hkv;
     it.ko = t * 128;
-    it.kpos = shard_of_orig(it.ko, P.C, P.cp);
+    it.kpos = shard_of_tile<PD>(P, it.ko);
     return it;
 }
 
-template <int D>
+template <int D, bool PD>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -374,7 +375,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             uint32_t nst = 0, iter = 0;
             bool ok = true, kv_issued = false;
             for (int w = blockIdx.x; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
-                const DkdvItem it = decode_dkdv(P, w, iter & 1);
+                const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
                 ok = mbar_wait(bar_kv_empty, (iter & 1) ^ 1, abort_flag);
                 if (!ok) break;
                 kv_issued = true;
@@ -389,10 +390,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
                 for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
-                    const int qpos = shard_of_orig(qo, P.C, P.cp);
+                    const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qo))
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qpos))
                         continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const int bh = it.b * P.Hq + it.hk * g + hq;
@@ -478,7 +479,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 return true;
             };
             for (int w = blockIdx.x; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
-                const DkdvItem it = decode_dkdv(P, w, iter & 1);
+                const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
                 ok = mbar_wait_warp(bar_kv_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -486,10 +487,10 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 uint32_t prev_qs = 0, prev_ds = 0;
                 for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
-                    const int qpos = shard_of_orig(qo, P.C, P.cp);
+                    const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qo))
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qpos))
                         continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
@@ -564,16 +565,16 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint32_t nst = 0, st_phase = 0, dp_phase = 0, a_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x, iter = 0; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
-            const DkdvItem it = decode_dkdv(P, w, iter & 1);
+            const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
             for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                 const int qo = t * 128;
-                const int qpos = shard_of_orig(qo, P.C, P.cp);
+                const int qpos = shard_of_tile<PD>(P, qo);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
                 const int cls = classify_tile(qo, dsf, dsl, it.ko, P.nc);
-                if (cls == TILE_SKIP || !q_tile_on_rank(P, qo)) continue;
+                if (cls == TILE_SKIP || !q_tile_on_rank(P, qpos)) continue;
                 for (int hq = 0; hq < g && ok; ++hq) {
                     const uint32_t qs = nst % Cfg::NQ, ds = nst % Cfg::NDO;
                     ++nst;
@@ -726,6 +727,7 @@ struct DqItem {
 // Items run GQA group by group; inside a group, query tiles by descending
 // original position (the longest first) with the group's query heads fastest,
 // so the CTAs in flight stream the same K/V tiles of one KV head.
+template <bool PD>
 __device__ __forceinline__ DqItem decode_dq(const BwdParams& P, int w)
 {
     DqItem it;
@@ -739,17 +741,21 @@ __device__ __forceinline__ DqItem decode_dq(const BwdParams& P, int w)
     it.bh = b * P.Hq + hk * g + hq;
     if (P.rank < 0) {
         it.qo = (ntiles - 1 - t) * 128;      // descending original position
+        it.qpos = shard_of_tile<PD>(P, it.qo);
+    } else if (PD) {                         // rank r, per-document plan: its tiles, last first
+        it.qpos = P.rank * 2 * P.C + (ntiles - 1 - t) * 128;
+        it.qo = orig_of_tile<PD>(P, it.qpos);
     } else {                                 // rank r: its tail chunk, then its head chunk
         const int half = P.C / 128;
         it.qo = t < half ? (2 * P.cp - 1 - P.rank) * P.C + (half - 1 - t) * 128
                          : P.rank * P.C + (2 * half - 1 - t) * 128;
+        it.qpos = shard_of_orig(it.qo, P.C, P.cp);
     }
-    it.qpos = shard_of_orig(it.qo, P.C, P.cp);
     it.r = it.qpos / (2 * P.C);
     return it;
 }
 
-template <int D>
+template <int D, bool PD>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -811,15 +817,15 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             uint32_t nload = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
-                const DqItem it = decode_dq(P, w);
+                const DqItem it = decode_dq<PD>(P, w);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, dsf, it.qo + 127 + P.nc, half, P.C, P.cp);
+                    const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int kpos = j * n2c + kt * 128;
-                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                        const int ko = tile_orig_of<PD>(P, j, kt, half);
                         if (classify_tile(it.qo, dsf, dsl, ko, P.nc) == TILE_SKIP) continue;
                         for (int kv = 0; kv < 2 && ok; ++kv, ++nload) {
                             const uint32_t slot = nload % Cfg::NSLOT, par = (nload / Cfg::NSLOT) & 1;
@@ -885,7 +891,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 return true;
             };
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
-                const DqItem it = decode_dq(P, w);
+                const DqItem it = decode_dq<PD>(P, w);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
                 ok = mbar_wait_warp(bar_qt_full, iter & 1, abort_flag);   // Q, dO rows in tensor memory
@@ -895,9 +901,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 uint32_t prev_kslot = 0;
                 for (int s = 0; s < P.cp && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, dsf, it.qo + 127 + P.nc, half, P.C, P.cp);
+                    const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
-                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                        const int ko = tile_orig_of<PD>(P, j, kt, half);
                         if (classify_tile(it.qo, dsf, dsl, ko, P.nc) == TILE_SKIP) continue;
                         const uint32_t kslot = nload % Cfg::NSLOT, kpar = (nload / Cfg::NSLOT) & 1;
                         const uint32_t vslot = (nload + 1) % Cfg::NSLOT, vpar = ((nload + 1) / Cfg::NSLOT) & 1;
@@ -972,7 +978,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         uint32_t st_phase = 0, dp_phase = 0, a_phase = 0, iter = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
-            const DqItem it = decode_dq(P, w);
+            const DqItem it = decode_dq<PD>(P, w);
             const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
             const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
             const size_t rowi = static_cast<size_t>(it.bh) * P.q_rows + (it.qpos - P.q_base) + row;
@@ -1005,9 +1011,9 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             bool had = false;
             for (int s = 0; s < P.cp && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
-                const KtSpan ks = kt_span(j, dsf, it.qo + 127 + P.nc, half, P.C, P.cp);
+                const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
-                    const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                    const int ko = tile_orig_of<PD>(P, j, kt, half);
                     const int cls = classify_tile(it.qo, dsf, dsl, ko, P.nc);
                     if (cls == TILE_SKIP) continue;
                     // ---- S: copy out, release, and form P while dP is still being computed

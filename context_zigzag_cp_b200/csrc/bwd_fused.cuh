@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
     }
 }
 
-template <int D>
+template <int D, bool PD>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -139,7 +139,7 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             uint32_t nst = 0, iter = 0;
             bool ok = true, kv_issued = false;
             for (int w = blockIdx.x; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
-                const DkdvItem it = decode_dkdv(P, w, iter & 1);
+                const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
                 ok = mbar_wait(bar_kv_empty, (iter & 1) ^ 1, abort_flag);
                 if (!ok) break;
                 kv_issued = true;
@@ -154,10 +154,10 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
-                    const int qpos = shard_of_orig(qo, P.C, P.cp);
+                    const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qo))
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qpos))
                         continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const int bh = it.b * P.Hq + it.hk * g + hq;
@@ -215,17 +215,17 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // partial sits in the dP^T columns and has not been read out yet
             bool ok = true, acc_busy = false, dq_pending = false;
             for (int w = blockIdx.x; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
-                const DkdvItem it = decode_dkdv(P, w, iter & 1);
+                const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
                 ok = mbar_wait_warp(bar_kv_full, iter & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 bool first = true;
                 for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                     const int qo = t * 128;
-                    const int qpos = shard_of_orig(qo, P.C, P.cp);
+                    const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
-                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qo))
+                    if (classify_tile(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qpos))
                         continue;
                     for (int hq = 0; hq < g && ok; ++hq) {
                         const uint32_t qs = nst % Cfg::NQ, qp = (nst / Cfg::NQ) & 1;
@@ -335,16 +335,16 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         uint32_t nst = 0, st_phase = 0, dp_phase = 0, dq_phase = 0, a_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x, iter = 0; w < P.n_items && ok; w = blockIdx.x + ((++iter) >> 1) * gridDim.x) {
-            const DkdvItem it = decode_dkdv(P, w, iter & 1);
+            const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
             for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
                 const int qo = t * 128;
-                const int qpos = shard_of_orig(qo, P.C, P.cp);
+                const int qpos = shard_of_tile<PD>(P, qo);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
                 const int cls = classify_tile(qo, dsf, dsl, it.ko, P.nc);
-                if (cls == TILE_SKIP || !q_tile_on_rank(P, qo)) continue;
+                if (cls == TILE_SKIP || !q_tile_on_rank(P, qpos)) continue;
                 for (int hq = 0; hq < g && ok; ++hq) {
                     const uint32_t qs = nst % Cfg::NQ, ds = nst % Cfg::NDO;
                     ++nst;

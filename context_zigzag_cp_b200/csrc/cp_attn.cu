@@ -92,6 +92,8 @@ cp_status_t check_problem(const cp_problem_t* p)
     // without the causal mask: no documents, and a window (one-sided) is not defined
     if (p->mask == CP_MASK_FULL && (p->cu_seqlens || p->num_docs != 0)) return CP_ERR_INVALID_ARG;
     if (p->mask == CP_MASK_FULL && p->window != 0) return CP_ERR_UNSUPPORTED;
+    if (p->shard != CP_SHARD_SEQUENCE && p->shard != CP_SHARD_PER_DOC) return CP_ERR_INVALID_ARG;
+    if (p->shard == CP_SHARD_PER_DOC && p->mask != CP_MASK_DOC_CAUSAL) return CP_ERR_INVALID_ARG;
     if (p->mask == CP_MASK_DOC_CAUSAL) {
         if (!p->cu_seqlens || p->num_docs < 1 || p->num_docs > p->seq_len) return CP_ERR_INVALID_ARG;
     }
@@ -114,13 +116,26 @@ cp_status_t check_attention(const cp_problem_t* p)
     return CP_OK;
 }
 
-cp_status_t check_plan(const cp_plan_t* pl, bool need_all)
+cp_status_t check_plan(const cp_plan_t* pl, bool need_all, const cp_problem_t* p = nullptr)
 {
     if (!pl) return CP_ERR_INVALID_ARG;
     if (!pl->src || !pl->doc_start) return CP_ERR_INVALID_ARG;
-    if (need_all && (!pl->perm || !pl->inv_perm || !pl->rank_cu_off || !pl->rank_cu || !pl->pairs))
+    if (need_all && (!pl->perm || !pl->inv_perm || !pl->rank_cu_off || !pl->rank_cu || !pl->pairs ||
+                     !pl->tile_orig || !pl->tile_shard))
         return CP_ERR_INVALID_ARG;
+    // per-document plans: the attention kernels read the tile tables
+    if (p && p->shard == CP_SHARD_PER_DOC && (!pl->tile_orig || !pl->tile_shard)) return CP_ERR_INVALID_ARG;
     return CP_OK;
+}
+
+// The tile tables for the attention kernels: only per-document plans need them.
+inline const int32_t* tables_orig(const cp_problem_t* p, const cp_plan_t* pl)
+{
+    return p->shard == CP_SHARD_PER_DOC ? pl->tile_orig : nullptr;
+}
+inline const int32_t* tables_shard(const cp_problem_t* p, const cp_plan_t* pl)
+{
+    return p->shard == CP_SHARD_PER_DOC ? pl->tile_shard : nullptr;
 }
 
 // Keys visible to the query at original position q start at q - wm1 (window W:
@@ -190,9 +205,10 @@ struct LaunchScope {
     }
 };
 
-cp_status_t launch_gather(const cp_problem_t* p, int32_t n_bufs, const void* const* bufs_in,
-                          void* const* bufs_out, const int64_t* buf_outer,
-                          const int64_t* buf_row_bytes, int to_shard, cudaStream_t stream)
+cp_status_t launch_gather(const cp_problem_t* p, const cp_plan_t* pl, int32_t n_bufs,
+                          const void* const* bufs_in, void* const* bufs_out,
+                          const int64_t* buf_outer, const int64_t* buf_row_bytes, int to_shard,
+                          cudaStream_t stream)
 {
     const int C = p->seq_len / (2 * p->cp_size);
     for (int i = 0; i < n_bufs; ++i) {
@@ -207,10 +223,16 @@ cp_status_t launch_gather(const cp_problem_t* p, int32_t n_bufs, const void* con
         G.C = C;
         G.cp = p->cp_size;
         G.to_shard = to_shard;
+        // per-document shards have no closed form: the plan's permutation tables
+        G.map = p->shard == CP_SHARD_PER_DOC ? (to_shard ? pl->perm : pl->inv_perm) : nullptr;
         const int64_t warps_needed = (G.rows + G.rpw * 4 - 1) / (G.rpw * 4);
         const int64_t blocks = std::min<int64_t>((warps_needed + 7) / 8, int64_t(num_sms()) * 8);
         LaunchScope ls(CP_K_GATHER, stream);
-        gather_rows_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0, stream>>>(G);
+        const unsigned grid = static_cast<unsigned>(std::max<int64_t>(blocks, 1));
+        if (G.map)
+            gather_rows_kernel<true><<<grid, 256, 0, stream>>>(G);
+        else
+            gather_rows_kernel<false><<<grid, 256, 0, stream>>>(G);
         if (launch_status() != CP_OK) return CP_ERR_CUDA;
     }
     return CP_OK;
@@ -284,7 +306,12 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.fused = fused;
     P.scale_log2 = softmax_scale(p) * 1.4426950408889634f;
     P.ppc = (P.C + 255) / 256;
-    P.n_items = P.BH * (L.rank < 0 ? 2 * P.cp : 2) * P.ppc;
+    // per-document shards: work units of 256 shard rows (two 128-row query
+    // tiles, not necessarily adjacent in the original order)
+    P.n_items = p->shard == CP_SHARD_PER_DOC ? P.BH * (L.q_rows / 256)
+                                              : P.BH * (L.rank < 0 ? 2 * P.cp : 2) * P.ppc;
+    P.tile_orig = tables_orig(p, pl);
+    P.tile_shard = tables_shard(p, pl);
     P.stall = stall;
     P.q_rows = L.q_rows;
     P.q_base = L.q_base;
@@ -300,13 +327,19 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.o_parts = o_parts;
     P.lse_parts = lse_parts;
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_FWD128 : ATTR_FWD64, [] {
-        return cudaFuncSetAttribute(cp_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    Cfg::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(cp_fwd_kernel<D, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(cp_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM_BYTES);
+        return e;
     });
     if (ast != CP_OK) return ast;
     const int grid = std::min(P.n_items, num_sms());
     LaunchScope ls(CP_K_FWD, stream);
-    cp_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, P);
+    // per-document plans take the instantiation that reads the tile tables
+    auto* kern = p->shard == CP_SHARD_PER_DOC ? cp_fwd_kernel<D, true> : cp_fwd_kernel<D, false>;
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, P);
     return launch_status();
 }
 
@@ -422,6 +455,9 @@ cp_status_t cp_plan_shards(const cp_problem_t* problem, const cp_plan_t* plan, i
     P.rank_cu_off = plan->rank_cu_off;
     P.rank_cu = plan->rank_cu;
     P.pairs = plan->pairs;
+    P.per_doc = problem->shard == CP_SHARD_PER_DOC;
+    P.tile_orig = plan->tile_orig;
+    P.tile_shard = plan->tile_shard;
     {
         LaunchScope ls(CP_K_PLAN_META, s);
         plan_meta_kernel<<<1, 256, 0, s>>>(P);
@@ -433,7 +469,7 @@ cp_status_t cp_plan_shards(const cp_problem_t* problem, const cp_plan_t* plan, i
         plan_index_kernel<<<blocks, 256, 0, s>>>(P);
     }
     if (launch_status() != CP_OK) return CP_ERR_CUDA;
-    return launch_gather(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes, 1, s);
+    return launch_gather(problem, plan, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes, 1, s);
 }
 
 cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan, int32_t n_bufs,
@@ -443,9 +479,10 @@ cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan, int32
     cp_status_t st = check_problem(problem);
     if (st != CP_OK) return st;
     if (!plan) return CP_ERR_INVALID_ARG;
+    if (problem->shard == CP_SHARD_PER_DOC && !plan->inv_perm) return CP_ERR_INVALID_ARG;
     if ((st = check_bufs(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes)) != CP_OK)
         return st;
-    return launch_gather(problem, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes, 0,
+    return launch_gather(problem, plan, n_bufs, bufs_in, bufs_out, buf_outer, buf_row_bytes, 0,
                          as_stream(stream));
 }
 
@@ -459,7 +496,7 @@ cp_status_t attn_fwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
 {
     cp_status_t st = check_attention(problem);
     if (st != CP_OK) return st;
-    if ((st = check_plan(plan, false)) != CP_OK) return st;
+    if ((st = check_plan(plan, false, problem)) != CP_OK) return st;
     if (!q || !k || !v || !o || !lse) return CP_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return CP_ERR_INVALID_ARG;
@@ -596,27 +633,37 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.dk32 = dk32;
     P.dv32 = dv32;
     P.dq_acc = dq_acc;
+    P.tile_orig = tables_orig(p, pl);
+    P.tile_shard = tables_shard(p, pl);
+    const bool pd = p->shard == CP_SHARD_PER_DOC;
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_BWD128 : ATTR_BWD64, [] {
-        cudaError_t e = cudaFuncSetAttribute(cp_bwd_dkdv_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             DkdvCfg<D>::SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(cp_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     DqCfg<D>::SMEM_BYTES);
+        cudaError_t e = cudaSuccess;
+        for (auto* kd : {cp_bwd_dkdv_kernel<D, false>, cp_bwd_dkdv_kernel<D, true>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvCfg<D>::SMEM_BYTES);
+        for (auto* kq : {cp_bwd_dq_kernel<D, false>, cp_bwd_dq_kernel<D, true>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::SMEM_BYTES);
         return e;
     });
     if (ast != CP_OK) return ast;
     P.n_items = B * Hkv * (S / 256);   // pairs of key tiles (S / 128 is even)
     if (dq_acc) {
         const cp_status_t fst = ensure_attr(D == 128 ? ATTR_FUSED128 : ATTR_FUSED64, [] {
-            return cudaFuncSetAttribute(cp_bwd_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        FusedCfg<D>::SMEM_BYTES);
+            cudaError_t e = cudaFuncSetAttribute(cp_bwd_fused_kernel<D, false>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 FusedCfg<D>::SMEM_BYTES);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(cp_bwd_fused_kernel<D, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<D>::SMEM_BYTES);
+            return e;
         });
         if (fst != CP_OK) return fst;
         {
             LaunchScope ls(CP_K_BWD_FUSED, stream);
-            cp_bwd_fused_kernel<D><<<std::min(P.n_items, num_sms()), FusedCfg<D>::THREADS,
-                                     FusedCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, P);
+            auto* kern = pd ? cp_bwd_fused_kernel<D, true> : cp_bwd_fused_kernel<D, false>;
+            kern<<<std::min(P.n_items, num_sms()), FusedCfg<D>::THREADS, FusedCfg<D>::SMEM_BYTES, stream>>>(
+                tq, tk, tv, tdo, P);
         }
         if (launch_status() != CP_OK) return CP_ERR_CUDA;
         const int64_t n8 = rows * D / 8;
@@ -628,14 +675,15 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     }
     {
     LaunchScope ls(CP_K_BWD_DKDV, stream);
-    cp_bwd_dkdv_kernel<D><<<std::min(P.n_items, num_sms()), DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES,
-                            stream>>>(tq, tk, tv, tdo, P);
+    auto* kdkdv = pd ? cp_bwd_dkdv_kernel<D, true> : cp_bwd_dkdv_kernel<D, false>;
+    kdkdv<<<std::min(P.n_items, num_sms()), DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, P);
     }
     if (launch_status() != CP_OK) return CP_ERR_CUDA;
     P.n_items = B * Hq * (L.q_rows / 128);
     LaunchScope ls(CP_K_BWD_DQ, stream);
-    cp_bwd_dq_kernel<D><<<std::min(P.n_items, num_sms()), DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, P);
+    auto* kdq = pd ? cp_bwd_dq_kernel<D, true> : cp_bwd_dq_kernel<D, false>;
+    kdq<<<std::min(P.n_items, num_sms()), DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, P);
     return launch_status();
 }
 
@@ -650,7 +698,7 @@ cp_status_t attn_bwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
 {
     cp_status_t st = check_attention(problem);
     if (st != CP_OK) return st;
-    if ((st = check_plan(plan, false)) != CP_OK) return st;
+    if ((st = check_plan(plan, false, problem)) != CP_OK) return st;
     const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
     for (const void* x : ptrs)
         if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
@@ -740,7 +788,7 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
 {
     cp_status_t st = check_attention(problem);
     if (st != CP_OK) return st;
-    if ((st = check_plan(plan, false)) != CP_OK) return st;
+    if ((st = check_plan(plan, false, problem)) != CP_OK) return st;
     const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
     for (const void* x : ptrs)
         if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;

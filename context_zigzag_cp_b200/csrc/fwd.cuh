@@ -57,6 +57,10 @@ struct FwdParams {
     int32_t q_rows, q_base, kv_rows, kv_base;
     int32_t rank;                   // -1: the items of every rank; r: rank r's only
     int32_t s0, s1;                 // visit steps s0 .. s1-1 (partials indexed s - s0)
+    // per-document plans: original start of each 128-row shard tile and its inverse
+    // ([S/128] each); null for the sequence-level zigzag (closed forms instead)
+    const int32_t* tile_orig;
+    const int32_t* tile_shard;
     const int32_t* src;             // [cp*cp]
     const int32_t* doc_start;       // [S] shard order
     __nv_bfloat16* o;               // [BH][S][D]  (fused)
@@ -80,7 +84,8 @@ __device__ __forceinline__ int classify_tile(int qo, int dsf, int dsl, int ko, i
 }
 
 struct FwdItem {
-    int bh, bkv, r, p0, qo0, ntq;
+    int bh, bkv, r, p0, ntq;
+    int qo[2];   // original start of the item's query tiles
 };
 
 // Original start of key tile kt (0 <= kt < 2C/128) of shard j: the first C/128
@@ -121,13 +126,87 @@ __device__ __forceinline__ KtSpan kt_span(int j, int lo, int hi, int half, int C
 __device__ __forceinline__ int kt_first(const KtSpan& r) { return r.a0 < r.b0 ? r.a0 : r.a1; }
 __device__ __forceinline__ int kt_next(const KtSpan& r, int kt) { return kt + 1 == r.b0 ? r.a1 : kt + 1; }
 
+// The zigzag maps, from the plan's tile tables for per-document plans (PD: tiles
+// of a shard are then pieces of many documents) and in closed form otherwise.
+// The kernels are compiled once for each, so the sequence path carries no table
+// code.  PP is FwdParams or BwdParams.
+// Original start of key tile kt (0 <= kt < 2C/128) of shard j.
+template <bool PD, class PP>
+__device__ __forceinline__ int tile_orig_of(const PP& P, int j, int kt, int half)
+{
+    if (PD) return __ldg(P.tile_orig + j * 2 * half + kt);
+    return key_tile_orig(j, kt, half, P.C, P.cp);
+}
+// The key tiles of shard j that can hold a key in [lo, hi].  Under a
+// per-document plan a shard holds its two chunks of every document in document
+// order (chunk j before chunk 2cp-1-j), so the original starts of its tiles
+// increase along the shard and the tiles that can hold such a key are one run,
+// found by two binary searches of the tile table (both stay inside the shard's
+// 2C/128 entries whatever the table holds).
+template <bool PD, class PP>
+__device__ __forceinline__ KtSpan kv_span(const PP& P, int j, int lo, int hi, int half)
+{
+    if (PD) {
+        const int32_t* t = P.tile_orig + j * 2 * half;
+        int a = 0, b = 2 * half;
+        while (a < b) {                        // first tile whose last key is >= lo
+            const int m = (a + b) >> 1;
+            if (__ldg(t + m) + 127 < lo) a = m + 1; else b = m;
+        }
+        const int first = a;
+        b = 2 * half;
+        while (a < b) {                        // first tile starting after hi
+            const int m = (a + b) >> 1;
+            if (__ldg(t + m) <= hi) a = m + 1; else b = m;
+        }
+        KtSpan r;
+        r.a0 = first;
+        r.b0 = r.a1 = r.b1 = a;
+        return r;
+    }
+    return kt_span(j, lo, hi, half, P.C, P.cp);
+}
+// Shard position of the 128-row tile that starts at original position qo.
+template <bool PD, class PP>
+__device__ __forceinline__ int shard_of_tile(const PP& P, int qo)
+{
+    if (PD) return __ldg(P.tile_shard + (qo >> 7)) * 128;
+    return shard_of_orig(qo, P.C, P.cp);
+}
+// Original start of the 128-row tile at shard position qpos.
+template <bool PD, class PP>
+__device__ __forceinline__ int orig_of_tile(const PP& P, int qpos)
+{
+    if (PD) return __ldg(P.tile_orig + (qpos >> 7));
+    return orig_of_shard(qpos, P.C, P.cp);
+}
+
 // Chunks an item list covers: all 2cp, or rank r's two (its tail chunk first).
 __device__ __forceinline__ int fwd_nchunks(const FwdParams& P) { return P.rank < 0 ? 2 * P.cp : 2; }
 
+template <bool PD>
 __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
 {
     FwdItem it;
     const int g = P.Hq / P.Hkv;
+    if (PD) {
+        // per-document plans: 256-row units of shard positions (the rank's, or all),
+        // by descending shard position; each unit holds two whole tiles (2C is a
+        // multiple of 256) whose original starts come from the plan
+        const int nunits = (P.rank < 0 ? P.S : 2 * P.C) / 256;
+        const int per_group_d = g * nunits;
+        it.bkv = w / per_group_d;
+        const int rem = w - it.bkv * per_group_d;
+        const int t = rem / g, hq = rem - t * g;
+        const int b = it.bkv / P.Hkv, hk = it.bkv - b * P.Hkv;
+        it.bh = b * P.Hq + hk * g + hq;
+        it.p0 = (P.rank < 0 ? 0 : P.rank * 2 * P.C) + (nunits - 1 - t) * 256;
+        it.r = it.p0 / (2 * P.C);
+        it.qo[0] = __ldg(P.tile_orig + (it.p0 >> 7));
+        it.qo[1] = __ldg(P.tile_orig + (it.p0 >> 7) + 1);
+        it.ntq = 2;
+        return it;
+    }
     const int per_group = g * fwd_nchunks(P) * P.ppc;
     it.bkv = w / per_group;
     const int rem = w - it.bkv * per_group;
@@ -140,7 +219,8 @@ __device__ __forceinline__ FwdItem decode_item(const FwdParams& P, int w)
     int half;
     if (c < P.cp) { it.r = c; half = 0; } else { it.r = 2 * P.cp - 1 - c; half = 1; }
     it.p0 = it.r * 2 * P.C + half * P.C + u * 256;
-    it.qo0 = c * P.C + u * 256;
+    it.qo[0] = c * P.C + u * 256;
+    it.qo[1] = it.qo[0] + 128;
     it.ntq = (u * 256 + 256 <= P.C) ? 2 : 1;
     return it;
 }
@@ -177,7 +257,7 @@ __device__ __forceinline__ TileIter load_tile_iter(const FwdParams& P, const Fwd
 {
     TileIter ti;
     for (int x = 0; x < 2; ++x) {
-        ti.qo[x] = it.qo0 + 128 * x;
+        ti.qo[x] = it.qo[x];
         ti.dsf[x] = 0;
         ti.dsl[x] = 0;
         if (P.docs && x < it.ntq) {
@@ -238,7 +318,7 @@ __device__ __forceinline__ float exp_pack_store(const float* sf, float scale_log
     return a + b;
 }
 
-template <int D>
+template <int D, bool PD>
 __global__ void __launch_bounds__(384, 1)
 cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const FwdParams P)
@@ -293,7 +373,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             uint32_t nload = 0, iter = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
-                const FwdItem it = decode_item(P, w);
+                const FwdItem it = decode_item<PD>(P, w);
                 const TileIter ti = load_tile_iter(P, it);
                 ok = mbar_wait(bar_q_empty, (iter & 1) ^ 1, abort_flag);
                 if (!ok) break;
@@ -304,10 +384,10 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                     it.bh * P.q_rows + (it.p0 - P.q_base) + 128 * x, bar_q_full);
                 for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
+                    const KtSpan ks = kv_span<PD>(P, j, ti.dsf[0], (it.ntq == 2 ? ti.qo[1] : ti.qo[0]) + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
                         const int kpos = j * n2c + kt * 128;
-                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                        const int ko = tile_orig_of<PD>(P, j, kt, half);
                         const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko, P.nc) != TILE_SKIP;
                         const bool v1 = it.ntq == 2 &&
                                         classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko, P.nc) != TILE_SKIP;
@@ -353,16 +433,16 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             uint32_t p_phase0 = 0, p_phase1 = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x, ++iter) {
-                const FwdItem it = decode_item(P, w);
+                const FwdItem it = decode_item<PD>(P, w);
                 const TileIter ti = load_tile_iter(P, it);
                 // number of loaded tiles of this item: Q is released to the producer
                 // right after the last S = Q K^T, before the item's final PVs
                 int n_tiles = 0;
                 for (int s = P.s0; s < P.s1; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
+                    const KtSpan ks = kv_span<PD>(P, j, ti.dsf[0], (it.ntq == 2 ? ti.qo[1] : ti.qo[0]) + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1; kt = kt_next(ks, kt)) {
-                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                        const int ko = tile_orig_of<PD>(P, j, kt, half);
                         if (classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko, P.nc) != TILE_SKIP ||
                             (it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko, P.nc) != TILE_SKIP))
                             ++n_tiles;
@@ -410,9 +490,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
                 for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
-                    const KtSpan ks = kt_span(j, ti.dsf[0], ti.qo[0] + 128 * it.ntq - 1 + P.nc, half, P.C, P.cp);
+                    const KtSpan ks = kv_span<PD>(P, j, ti.dsf[0], (it.ntq == 2 ? ti.qo[1] : ti.qo[0]) + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
-                        const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                        const int ko = tile_orig_of<PD>(P, j, kt, half);
                         const bool v0 = classify_tile(ti.qo[0], ti.dsf[0], ti.dsl[0], ko, P.nc) != TILE_SKIP;
                         const bool v1 = it.ntq == 2 && classify_tile(ti.qo[1], ti.dsf[1], ti.dsl[1], ko, P.nc) != TILE_SKIP;
                         if (!v0 && !v1) continue;
@@ -477,7 +557,7 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < P.n_items && ok; w += gridDim.x) {
-            const FwdItem it = decode_item(P, w);
+            const FwdItem it = decode_item<PD>(P, w);
             if (X >= it.ntq) continue;
             const TileIter ti = load_tile_iter(P, it);
             const int prow = it.p0 + 128 * X + row;      // shard position of my row
@@ -487,9 +567,9 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool first = true, had = false;
             for (int s = P.s0; s < P.s1 && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
-                const KtSpan ks = kt_span(j, ti.dsf[X], ti.qo[X] + 127 + P.nc, half, P.C, P.cp);
+                const KtSpan ks = kv_span<PD>(P, j, ti.dsf[X], ti.qo[X] + 127 + P.nc, half);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
-                    const int ko = key_tile_orig(j, kt, half, P.C, P.cp);
+                    const int ko = tile_orig_of<PD>(P, j, kt, half);
                     const int cls = classify_tile(ti.qo[X], ti.dsf[X], ti.dsl[X], ko, P.nc);
                     if (cls == TILE_SKIP) continue;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * X, s_phase, abort_flag));

@@ -71,6 +71,17 @@ typedef enum { CP_ROTATE_ALLGATHER = 0, CP_ROTATE_RING = 1 } cp_rotate_t;
  * it takes no documents (cu_seqlens NULL, num_docs 0) and no window. */
 typedef enum { CP_MASK_CAUSAL = 0, CP_MASK_DOC_CAUSAL = 1, CP_MASK_FULL = 2 } cp_mask_t;
 
+/* How the sequence is cut into shards.
+ *   CP_SHARD_SEQUENCE: the sequence in 2*cp chunks, rank r holding chunks r and
+ *     2cp-1-r (the zigzag of the pages).
+ *   CP_SHARD_PER_DOC: every packed document in 2*cp chunks, rank r holding,
+ *     document after document, its chunk r then its chunk 2cp-1-r, so every rank
+ *     gets an equal share of every document's causal work (FlashCP abstract:
+ *     "Per-Doc" sharding).  Needs CP_MASK_DOC_CAUSAL; every document's length a
+ *     multiple of 256*cp_size (chunks of whole 128-row tiles), else
+ *     cp_plan_shards records CP_ERR_UNSUPPORTED in the device status word. */
+typedef enum { CP_SHARD_SEQUENCE = 0, CP_SHARD_PER_DOC = 1 } cp_shard_t;
+
 /* How cp_attn_fwd combines the per-step partial attentions.
  *   CP_MERGE_SEPARATE: each (rank, step) unit writes its partial (O, LSE) in
  *     fp32 to the workspace, then the cp_lse_merge kernel folds the cp
@@ -98,6 +109,7 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *                 q - W < k <= q (and, with documents, k in q's document).
  *                 Negative values are CP_ERR_INVALID_ARG; W > 0 with
  *                 CP_MASK_FULL is CP_ERR_UNSUPPORTED.
+ *   shard         cp_shard_t (CP_SHARD_PER_DOC needs the document mask)
  *   bwd_one_pass  backward only.  0 (default): two passes, a dK/dV pass and a
  *                 dQ pass that recomputes S and dP; bit-for-bit reproducible,
  *                 and the faster form on B200 (128k: 438 vs 475 ms).
@@ -129,6 +141,7 @@ typedef struct {
     int32_t num_docs;
     int32_t window;
     int32_t bwd_one_pass;
+    int32_t shard;
     const int32_t* cu_seqlens;
 } cp_problem_t;
 
@@ -140,10 +153,21 @@ typedef struct {
  *   doc_start   int32 [S]          original start of the document of token
  *                                  perm[p] (0 everywhere for CP_MASK_CAUSAL)
  *   rank_cu_off int32 [cp+1]       rank r's entries are rank_cu[off[r]..off[r+1])
- *   rank_cu     int32 [3*cp + num_docs]  per rank, local offsets where a
- *                                  segment starts (0, the chunk boundary C,
- *                                  every document start inside the rank's
- *                                  chunks), then 2C
+ *   rank_cu     int32 [3*cp + num_docs] (CP_SHARD_SEQUENCE) or
+ *               int32 [cp*(2*num_docs + 1)] (CP_SHARD_PER_DOC)
+ *                                  per rank, local offsets where a segment
+ *                                  starts, then 2C: sequence sharding, 0, the
+ *                                  chunk boundary C and every document start
+ *                                  inside the rank's chunks; per-document
+ *                                  sharding, the start of each of the rank's
+ *                                  two chunks of every document
+ *   tile_orig   int32 [ceil(S/128)] original start of the 128-row tile at shard
+ *                                  position 128*i
+ *   tile_shard  int32 [ceil(S/128)] shard tile index of the tile starting at
+ *                                  original position 128*i (inverse of tile_orig);
+ *                                  both defined when the chunks are whole tiles
+ *                                  (what the attention calls need) and read by
+ *                                  them for per-document plans only
  *   pairs       int64 [cp]         unmasked (q, k) pairs whose query lives on
  *                                  rank r (equal across ranks for the plain
  *                                  causal mask without a window; 2C * S each
@@ -156,6 +180,8 @@ typedef struct {
     int32_t* rank_cu_off;
     int32_t* rank_cu;
     int64_t* pairs;
+    int32_t* tile_orig;
+    int32_t* tile_shard;
 } cp_plan_t;
 
 /*

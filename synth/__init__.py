@@ -13,8 +13,10 @@ Draw recipe (one torch CPU generator per call, seeded):
   [B, H, S, D] in ORIGINAL token order, multiplied by ``amp`` and rounded to
   bf16 (round-to-nearest-even by ``Tensor.to``).
 Document lengths: numpy ``default_rng(seed).lognormal(ln(median), sigma)``,
-rounded with ``rint``, clipped to [lo, hi], drawn one at a time until their sum
-reaches S; the last document is cut so the lengths sum to exactly S.
+rounded with ``rint``, clipped to [lo, hi], then (for per-document sharding,
+whose chunks must be whole 128-row tiles) rounded to the nearest multiple of
+``quantum`` (at least one quantum), drawn one at a time until their sum reaches
+S; the last document is cut so the lengths sum to exactly S.
 """
 from __future__ import annotations
 
@@ -42,6 +44,8 @@ class Workload:
     doc_median: float = 2048.0
     doc_sigma: float = 1.0
     doc_clip: tuple = (128, 32768)
+    shard: str = "sequence"          # "sequence" | "doc" (per-document zigzag)
+    doc_quantum: int = 1             # document lengths a multiple of this
     extra: dict = field(default_factory=dict)
 
 
@@ -51,18 +55,26 @@ WORKLOADS = {
     "gqa32k": Workload("gqa32k", 1, 32768, 8, 32, 8, 128, "ring", amp=0.5, seed=2),
     "docs64k": Workload("docs64k", 1, 65536, 8, 32, 8, 128, "ring", docs=True, seed=3),
     "long128k": Workload("long128k", 1, 131072, 8, 32, 8, 128, "allgather", seed=4),
+    # the docs64k mix with every document cut into 2cp chunks of whole 128-row tiles
+    "docs64k_perdoc": Workload("docs64k_perdoc", 1, 65536, 8, 32, 8, 128, "ring", docs=True,
+                               seed=3, shard="doc", doc_quantum=2048),
 }
 
 
 def doc_lengths(seq_len: int, seed: int, median: float = 2048.0, sigma: float = 1.0,
-                clip: tuple = (128, 32768)) -> list[int]:
-    """Seeded lognormal document lengths summing to exactly ``seq_len``."""
+                clip: tuple = (128, 32768), quantum: int = 1) -> list[int]:
+    """Seeded lognormal document lengths summing to exactly ``seq_len``, each a
+    multiple of ``quantum`` (``seq_len`` must then be one too)."""
+    if quantum < 1 or seq_len % quantum:
+        raise ValueError(f"seq_len {seq_len} is not a multiple of quantum {quantum}")
     rng = np.random.default_rng(seed)
     lens: list[int] = []
     total = 0
     while total < seq_len:
         x = float(rng.lognormal(mean=math.log(median), sigma=sigma))
         n = int(np.clip(np.rint(x), clip[0], clip[1]))
+        if quantum > 1:
+            n = max(quantum, int(np.rint(n / quantum)) * quantum)
         lens.append(n)
         total += n
     lens[-1] -= total - seq_len
@@ -108,5 +120,5 @@ def workload_inputs(w: Workload, device="cpu", with_dout=None) -> dict:
     t = attn_inputs(w.batch, w.num_heads, w.num_kv_heads, w.seq_len, w.head_dim, w.seed,
                     amp=w.amp, with_dout=wd, device=device)
     t["cu_seqlens"] = (cu_seqlens(doc_lengths(w.seq_len, w.seed, w.doc_median, w.doc_sigma,
-                                              w.doc_clip)) if w.docs else None)
+                                              w.doc_clip, w.doc_quantum)) if w.docs else None)
     return t

@@ -78,13 +78,14 @@ def assert_lse_close(gpu: np.ndarray, ref: np.ndarray, what: str, tol=LSE_MAX):
     return err
 
 
-def random_docs(seq_len: int, seed: int, median: float, lo: int = 1, hi: int | None = None):
+def random_docs(seq_len: int, seed: int, median: float, lo: int = 1, hi: int | None = None,
+                quantum: int = 1):
     return synth.cu_seqlens(synth.doc_lengths(seq_len, seed, median, 1.0,
-                                              (lo, hi or seq_len)))
+                                              (lo, hi or seq_len), quantum))
 
 
 def make_case(B, Hq, Hkv, S, D, cp, seed, amp=1.0, cu=None, with_dout=False, window=0,
-              causal=True):
+              causal=True, shard="sequence"):
     """Seeded inputs on the CPU (original order) plus, per original position, the
     first key it attends to (document start, raised by a sliding window) and the
     last (itself under the causal mask, else the end of its document)."""
@@ -92,6 +93,7 @@ def make_case(B, Hq, Hkv, S, D, cp, seed, amp=1.0, cu=None, with_dout=False, win
     t["cu_seqlens"] = cu
     t["window"] = window
     t["causal"] = causal
+    t["shard"] = shard
     t["ds"] = oracle.first_key(S, cu, window)
     t["lk"] = oracle.last_key(S, cu, causal)
     return t
@@ -104,7 +106,7 @@ def run_fwd(cz, case, cp, rotate="allgather", merge="fused", scale=0.0, dev="cud
     B, Hq, S, D = q.shape
     cu = None if case["cu_seqlens"] is None else torch.from_numpy(case["cu_seqlens"]).to(dev)
     prob = cz.Problem(B, S, cp, Hq, k.shape[1], D, rotate, cu, merge, scale, case.get("window", 0),
-                      case.get("causal", True))
+                      case.get("causal", True), shard=case.get("shard", "sequence"))
     plan = cz.Plan(prob)
     qs, ks, vs = plan.shard([q, k, v])
     o, lse = cz.attn_fwd(prob, plan, qs, ks, vs)

@@ -48,7 +48,7 @@ def prob(**kw):
 def fwd_query(p):
     n = ctypes.c_size_t(0)
     d = ctypes.c_void_p(256)
-    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     st = cz.lib().cp_attn_fwd(p.ref, ctypes.byref(plan), d, d, d, d, d, None, ctypes.byref(n),
                               None)
     return st, n.value
@@ -107,7 +107,7 @@ def test_workspace_query(lib):
 def test_workspace_too_small_and_null_pointers(lib):
     p = prob(merge="separate")
     d = ctypes.c_void_p(256)
-    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     n = ctypes.c_size_t(16)
     assert cz.lib().cp_attn_fwd(p.ref, ctypes.byref(plan), d, d, d, d, d, d, ctypes.byref(n),
                                 None) == _lib.CP_ERR_WORKSPACE
@@ -115,14 +115,14 @@ def test_workspace_too_small_and_null_pointers(lib):
                                 ctypes.byref(n), None) == _lib.CP_ERR_INVALID_ARG
     assert cz.lib().cp_attn_fwd(None, ctypes.byref(plan), d, d, d, d, d, None, ctypes.byref(n),
                                 None) == _lib.CP_ERR_INVALID_ARG
-    bad_plan = _lib.CpPlan(256, 256, None, 256, 256, 256, 256)
+    bad_plan = _lib.CpPlan(256, 256, None, 256, 256, 256, 256, 256, 256)
     assert cz.lib().cp_attn_fwd(p.ref, ctypes.byref(bad_plan), d, d, d, d, d, None,
                                 ctypes.byref(n), None) == _lib.CP_ERR_INVALID_ARG
 
 
 def test_plan_host_checks(lib):
     p = prob(seq_len=102)       # 102 % 4 != 0
-    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     assert cz.lib().cp_plan_shards(p.ref, ctypes.byref(plan), 0, None, None, None, None, None,
                                    None, None) == _lib.CP_ERR_INVALID_ARG
     p = prob()
@@ -176,7 +176,7 @@ def test_noalloc_limit_checked_on_host(lib):
     p = prob(seq_len=4096, cp=2, num_heads=_lib.NOALLOC_MAX_ROWS // 4096 + 1, num_kv_heads=1,
              head_dim=128)
     d = ctypes.c_void_p(256)
-    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     assert cz.lib().cp_attn_bwd_noalloc(p.ref, ctypes.byref(plan), d, d, d, d, d, d, d, d, d,
                                         None) == _lib.CP_ERR_WORKSPACE
     assert cz.lib().cp_attn_bwd_noalloc(p.ref, ctypes.byref(plan), None, d, d, d, d, d, d, d, d,
@@ -200,3 +200,34 @@ def test_full_mask_host_checks(lib):
     assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
     with pytest.raises(ValueError, match="causal=False"):
         prob(causal=False, window=4)
+
+
+def test_shard_host_checks(lib):
+    """cp_problem_t.shard: CP_SHARD_SEQUENCE or CP_SHARD_PER_DOC, the latter only with
+    the document mask; a per-document plan must carry its tile tables."""
+    p = prob()
+    p.c.shard = 2                    # no such sharding
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob()
+    p.c.shard = 1                    # per-document sharding without documents
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob(causal=False)
+    p.c.shard = 1
+    assert fwd_query(p)[0] == _lib.CP_ERR_INVALID_ARG
+    p = prob()
+    p.c.mask, p.c.num_docs, p.c.cu_seqlens, p.c.shard = 1, 2, 256, 1
+    assert fwd_query(p)[0] == _lib.CP_OK
+    d = ctypes.c_void_p(256)
+    n = ctypes.c_size_t(0)
+    no_tables = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, None, None)
+    assert cz.lib().cp_attn_fwd(p.ref, ctypes.byref(no_tables), d, d, d, d, d, None,
+                                ctypes.byref(n), None) == _lib.CP_ERR_INVALID_ARG
+    assert cz.lib().cp_plan_shards(p.ref, ctypes.byref(no_tables), 0, None, None, None, None,
+                                   None, None, None) == _lib.CP_ERR_INVALID_ARG
+    no_inv = _lib.CpPlan(256, None, 256, 256, 256, 256, 256, 256, 256)
+    ptrs = (ctypes.c_void_p * 1)(256)
+    outs = (ctypes.c_void_p * 1)(1 << 20)
+    outer = (ctypes.c_int64 * 1)(1)
+    row = (ctypes.c_int64 * 1)(128)
+    assert cz.lib().cp_unshard(p.ref, ctypes.byref(no_inv), 1, ptrs, outs, outer, row,
+                               None) == _lib.CP_ERR_INVALID_ARG

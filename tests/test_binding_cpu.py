@@ -139,7 +139,7 @@ def _cpu_plan(p):
     plan = object.__new__(cz.Plan)
     plan.prob = p
     plan.perm = torch.zeros(p.seq_len, dtype=torch.int32)
-    plan.c = cz.CpPlan(0, 0, 0, 0, 0, 0, 0)
+    plan.c = cz.CpPlan(0, 0, 0, 0, 0, 0, 0, 0, 0)
     return plan
 
 
@@ -243,3 +243,26 @@ def test_plan_must_fit_problem(cpu_binding):
     plan.perm = torch.zeros(S, dtype=torch.int32, device="meta")
     with pytest.raises(ValueError, match="plan: on"):
         cz.attn_fwd(p, plan, *args)
+
+
+def test_problem_shard_option(cpu_binding):
+    """shard: "sequence" (default) or "doc"; per-document sharding needs documents, and
+    a plan made for one sharding does not serve the other."""
+    with pytest.raises(ValueError, match="shard"):
+        cz.Problem(B, S, CP, Hq, Hkv, D, shard="tile")
+    with pytest.raises(ValueError, match="needs cu_seqlens"):
+        cz.Problem(B, S, CP, Hq, Hkv, D, shard="doc")
+    p = cz.Problem(B, S, CP, Hq, Hkv, D)
+    assert p.c.shard == 0 and p.rank_cu_len() == 3 * CP + 1
+    assert p.with_merge("separate").shard == "sequence"
+    doc = object.__new__(cz.Problem)
+    doc.__dict__.update(p.__dict__)
+    doc.shard, doc.num_docs = "doc", 5
+    assert doc.rank_cu_len() == CP * 11
+    t = tensors()
+    args = (t["q"], t["k"], t["v"], t["o"], t["lse"])
+    with pytest.raises(ValueError, match="'sequence' sharding"):
+        cz.attn_fwd(doc, _cpu_plan(p), *args)
+    windowed = cz.Problem(B, S, CP, Hq, Hkv, D, window=64)
+    with pytest.raises(ValueError, match="window"):
+        cz.attn_fwd(windowed, _cpu_plan(p), *args)

@@ -162,7 +162,7 @@ def check_sampled(name, rotate, n_rows=96, n_keys=24, early=True, one_pass=False
     S, g = w.seq_len, w.num_heads // w.num_kv_heads
     cu = t["cu_seqlens"]
     ds = oracle.doc_start(S, cu)
-    case = dict(q=t["q"], k=t["k"], v=t["v"], do=t["do"], cu_seqlens=cu, ds=ds)
+    case = dict(q=t["q"], k=t["k"], v=t["v"], do=t["do"], cu_seqlens=cu, ds=ds, shard=w.shard)
     _, _, dq, dk, dv, o_gpu = run_bwd(case, w.cp, rotate, with_o=True, one_pass=one_pass)
     rng = np.random.default_rng(w.seed + 200)
     groups = [0, int(rng.integers(1, w.num_kv_heads))]
@@ -213,6 +213,11 @@ def test_gqa32k_ring_sampled(one_pass):
 
 def test_docs64k_sampled():
     check_sampled("docs64k", "ring")
+
+
+@pytest.mark.parametrize("one_pass", [False, True])
+def test_docs64k_perdoc_sampled(one_pass):
+    check_sampled("docs64k_perdoc", "ring", one_pass=one_pass)
 
 
 @pytest.mark.parametrize("rotate,one_pass", [("allgather", False), ("ring", True)])

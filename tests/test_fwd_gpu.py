@@ -77,9 +77,17 @@ def test_local_only_differs():
 
 # ----------------------------------------------------------------- full sizes, sampled
 
-def sampled_rows(S, cp, rng, per_head):
-    C = S // (2 * cp)
-    edges = np.concatenate([np.arange(2 * cp) * C, np.arange(1, 2 * cp + 1) * C - 1])
+def sampled_rows(S, cp, rng, per_head, cu=None, per_doc=False):
+    """Random rows plus the first and last row of every chunk (of the sequence, or
+    with per-document sharding, of every document)."""
+    if per_doc:
+        cu = np.asarray(cu, dtype=np.int64)
+        c = np.diff(cu) // (2 * cp)
+        starts = (cu[:-1, None] + np.arange(2 * cp)[None, :] * c[:, None]).ravel()
+        edges = np.concatenate([starts, starts + np.repeat(c, 2 * cp) - 1])
+    else:
+        C = S // (2 * cp)
+        edges = np.concatenate([np.arange(2 * cp) * C, np.arange(1, 2 * cp + 1) * C - 1])
     return np.unique(np.concatenate([edges, rng.integers(0, S, per_head)]))
 
 
@@ -87,7 +95,7 @@ def check_sampled(name, rotate, merge="fused", per_head=192):
     w = synth.WORKLOADS[name]
     t = synth.workload_inputs(w, with_dout=False)
     case = dict(q=t["q"], k=t["k"], v=t["v"], cu_seqlens=t["cu_seqlens"],
-                ds=oracle.doc_start(w.seq_len, t["cu_seqlens"]))
+                ds=oracle.doc_start(w.seq_len, t["cu_seqlens"]), shard=w.shard)
     prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, w.cp, rotate, merge)
     g = w.num_heads // w.num_kv_heads
     rng = np.random.default_rng(w.seed + 100)
@@ -96,7 +104,7 @@ def check_sampled(name, rotate, merge="fused", per_head=192):
     q = f64(t["q"][:, qh])
     k = f64(t["k"][:, groups])
     v = f64(t["v"][:, groups])
-    rows_orig = sampled_rows(w.seq_len, w.cp, rng, per_head)
+    rows_orig = sampled_rows(w.seq_len, w.cp, rng, per_head, t["cu_seqlens"], w.shard == "doc")
     S = w.seq_len
     flat = np.concatenate([hi * S + rows_orig for hi in range(len(qh))])
     ro, rl = oracle.fwd_rows(q, k, v, flat, case["ds"])
@@ -116,6 +124,12 @@ def test_gqa32k_ring_sampled():
 def test_docs64k_sampled():
     check_sampled("docs64k", "ring", "separate")
     check_sampled("docs64k", "allgather", "fused")
+
+
+def test_docs64k_perdoc_sampled():
+    """The docs64k length mix in whole-tile multiples, every document cut into 2cp chunks."""
+    check_sampled("docs64k_perdoc", "ring", "fused")
+    check_sampled("docs64k_perdoc", "allgather", "separate")
 
 
 @pytest.mark.parametrize("rotate", ["allgather", "ring"])

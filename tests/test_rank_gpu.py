@@ -19,12 +19,18 @@ def _local(x, r, n2c):
     return x[:, :, r * n2c:(r + 1) * n2c].contiguous()
 
 
+# docs: False (no documents), True (packed documents, sequence zigzag) or "per_doc"
+# (whole-tile documents, every one cut into 2cp chunks)
 @pytest.mark.parametrize("Hq,Hkv,S,D,cp,docs,causal", [
     (8, 2, 4096, 128, 4, False, True), (4, 2, 2304, 128, 3, True, True),
-    (4, 4, 2048, 64, 2, False, True), (4, 2, 2048, 128, 4, False, False)])
+    (4, 4, 2048, 64, 2, False, True), (4, 2, 2048, 128, 4, False, False),
+    (8, 2, 6144, 128, 2, "per_doc", True), (4, 2, 6144, 64, 3, "per_doc", True)])
 def test_ranks_reassemble_whole(Hq, Hkv, S, D, cp, docs, causal):
-    cu = random_docs(S, 95, 300.0) if docs else None
-    case = make_case(1, Hq, Hkv, S, D, cp, 96 + S, cu=cu, with_dout=True, causal=causal)
+    per_doc = docs == "per_doc"
+    cu = (random_docs(S, 95, 1500.0, quantum=256 * cp) if per_doc else
+          random_docs(S, 95, 300.0) if docs else None)
+    case = make_case(1, Hq, Hkv, S, D, cp, 96 + S, cu=cu, with_dout=True, causal=causal,
+                     shard="doc" if per_doc else "sequence")
     prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, cp, "ring", "fused")
     (dos,) = plan.shard([case["do"].cuda()])
     # the per-rank backward is the two-pass form: compare with the whole two-pass one

@@ -50,7 +50,7 @@ def test_noalloc_rejects_problems_beyond_the_array():
     rows_over = _lib.NOALLOC_MAX_ROWS // 4096 + 1      # heads so that rows exceed the limit
     prob = cz.Problem(1, 4096, 2, rows_over, 1, 128)
     d = ctypes.c_void_p(256)
-    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
     st = cz.lib().cp_attn_bwd_noalloc(prob.ref, ctypes.byref(plan), d, d, d, d, d, d, d, d, d,
                                       None)
     assert st == _lib.CP_ERR_WORKSPACE
