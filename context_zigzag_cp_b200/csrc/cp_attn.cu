@@ -16,6 +16,7 @@
 #include "fwd.cuh"
 #include "bwd.cuh"
 #include "bwd_fused.cuh"
+#include "fwd256.cuh"
 
 using namespace cpattn;
 
@@ -36,7 +37,8 @@ int g_num_sms[kMaxDevices] = {};
 uint32_t g_attr_done[kMaxDevices] = {};   // bit per kernel family (AttrSet)
 
 enum AttrSet : uint32_t {
-    ATTR_FWD64 = 1, ATTR_FWD128 = 2, ATTR_BWD64 = 4, ATTR_BWD128 = 8, ATTR_FUSED64 = 16, ATTR_FUSED128 = 32
+    ATTR_FWD64 = 1, ATTR_FWD128 = 2, ATTR_BWD64 = 4, ATTR_BWD128 = 8, ATTR_FUSED64 = 16, ATTR_FUSED128 = 32,
+    ATTR_FWD256 = 64, ATTR_BWD256 = 128
 };
 
 inline int current_device()
@@ -108,7 +110,7 @@ cp_status_t check_attention(const cp_problem_t* p)
 {
     cp_status_t st = check_problem(p);
     if (st != CP_OK) return st;
-    if (p->head_dim != 64 && p->head_dim != 128) return CP_ERR_UNSUPPORTED;
+    if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) return CP_ERR_UNSUPPORTED;
     // the kernels' tile bounds (key tile end + window or sequence length) stay in int32
     if (p->seq_len > (1 << 29)) return CP_ERR_UNSUPPORTED;
     const int C = p->seq_len / (2 * p->cp_size);
@@ -286,12 +288,13 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
                        const void* v, void* o, float* lse, float* o_parts, float* lse_parts,
                        cudaStream_t stream, int stall, const Layout& L, bool fused)
 {
-    using Cfg = FwdCfg<D>;
     const int B = p->batch, Hq = p->num_heads, Hkv = p->num_kv_heads, S = p->seq_len;
+    // head_dim 256: 64-row K/V boxes, Q read by the kernel itself (into tensor memory)
+    constexpr int KV_BOX_ROWS = D == 256 ? Fwd256Cfg::KT : 128;
     CUtensorMap tq, tk, tv;
-    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128))
+    if ((D != 256 && !make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128)) ||
+        !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, KV_BOX_ROWS) ||
+        !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, KV_BOX_ROWS))
         return CP_ERR_CUDA;
     FwdParams P;
     P.BH = B * Hq;
@@ -322,10 +325,31 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.s1 = L.s1;
     P.src = pl->src;
     P.doc_start = pl->doc_start;
+    P.q = static_cast<const __nv_bfloat16*>(q);
     P.o = static_cast<__nv_bfloat16*>(o);
     P.lse = lse;
     P.o_parts = o_parts;
     P.lse_parts = lse_parts;
+    if constexpr (D == 256) {
+        // one 128-row query tile per work item
+        P.n_items = P.BH * (L.q_rows / 128);
+        const cp_status_t ast = ensure_attr(ATTR_FWD256, [] {
+            cudaError_t e = cudaFuncSetAttribute(cp_fwd256_kernel<false>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 Fwd256Cfg::SMEM_BYTES);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(cp_fwd256_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Fwd256Cfg::SMEM_BYTES);
+            return e;
+        });
+        if (ast != CP_OK) return ast;
+        const int grid = std::min(P.n_items, num_sms());
+        LaunchScope ls(CP_K_FWD, stream);
+        auto* kern = p->shard == CP_SHARD_PER_DOC ? cp_fwd256_kernel<true> : cp_fwd256_kernel<false>;
+        kern<<<grid, Fwd256Cfg::THREADS, Fwd256Cfg::SMEM_BYTES, stream>>>(tk, tv, P);
+        return launch_status();
+    } else {
+    using Cfg = FwdCfg<D>;
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_FWD128 : ATTR_FWD64, [] {
         cudaError_t e = cudaFuncSetAttribute(cp_fwd_kernel<D, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
@@ -341,6 +365,19 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     auto* kern = p->shard == CP_SHARD_PER_DOC ? cp_fwd_kernel<D, true> : cp_fwd_kernel<D, false>;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, P);
     return launch_status();
+    }
+}
+
+// The forward for the problem's head_dim.
+cp_status_t launch_fwd_any(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
+                           const void* v, void* o, float* lse, float* o_parts, float* lse_parts,
+                           cudaStream_t stream, int stall, const Layout& L, bool fused)
+{
+    switch (p->head_dim) {
+    case 256: return launch_fwd<256>(p, pl, q, k, v, o, lse, o_parts, lse_parts, stream, stall, L, fused);
+    case 128: return launch_fwd<128>(p, pl, q, k, v, o, lse, o_parts, lse_parts, stream, stall, L, fused);
+    default: return launch_fwd<64>(p, pl, q, k, v, o, lse, o_parts, lse_parts, stream, stall, L, fused);
+    }
 }
 
 cp_status_t launch_merge(int64_t rows, int32_t D, int32_t n_parts, const float* o_parts,
@@ -510,9 +547,7 @@ cp_status_t attn_fwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
     cudaStream_t s = as_stream(stream);
     const Layout L = whole_layout(problem);
     const bool fused = problem->merge == CP_MERGE_FUSED;
-    st = problem->head_dim == 128
-             ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall, L, fused)
-             : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall, L, fused);
+    st = launch_fwd_any(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall, L, fused);
     if (st != CP_OK || !separate) return st;
     return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
 }
@@ -713,6 +748,7 @@ cp_status_t attn_bwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     float* dq_acc = one_pass ? reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * row_bytes) : nullptr;
     cudaStream_t s = as_stream(stream);
+    if (problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // backward at head_dim 256: not yet
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
                                  whole_layout(problem), nullptr, nullptr, dq_acc)
@@ -799,6 +835,7 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
     if ((st = noalloc_scratch(s, &scratch)) != CP_OK) return st;
     float* delta = static_cast<float*>(scratch);
     float* nlse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
+    if (problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // backward at head_dim 256: not yet
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
                                  whole_layout(problem), nullptr, nullptr, nullptr)
@@ -857,9 +894,7 @@ extern "C" cp_status_t cp_attn_fwd_rank(const cp_problem_t* problem, const cp_pl
     float* lse_parts = separate ? reinterpret_cast<float*>(static_cast<char*>(ws) + o_parts_bytes) : nullptr;
     cudaStream_t s = as_stream(stream);
     const Layout L = rank_layout(problem, rank, -1);
-    st = problem->head_dim == 128
-             ? launch_fwd<128>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, 0, L, !separate)
-             : launch_fwd<64>(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, 0, L, !separate);
+    st = launch_fwd_any(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, 0, L, !separate);
     if (st != CP_OK || !separate) return st;
     return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
 }
@@ -875,9 +910,7 @@ extern "C" cp_status_t cp_attn_fwd_step(const cp_problem_t* problem, const cp_pl
         if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
     const Layout L = rank_layout(problem, rank, step);
-    return problem->head_dim == 128
-               ? launch_fwd<128>(problem, plan, q, k, v, nullptr, nullptr, o_part, lse_part, s, 0, L, false)
-               : launch_fwd<64>(problem, plan, q, k, v, nullptr, nullptr, o_part, lse_part, s, 0, L, false);
+    return launch_fwd_any(problem, plan, q, k, v, nullptr, nullptr, o_part, lse_part, s, 0, L, false);
 }
 
 extern "C" cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_plan_t* plan,
@@ -899,6 +932,7 @@ extern "C" cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_pl
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     cudaStream_t s = as_stream(stream);
     const Layout L = rank_layout(problem, rank, -1);
+    if (problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // backward at head_dim 256: not yet
     return problem->head_dim == 128
                ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
                                  s, 0, L, dk_part, dv_part, nullptr)

@@ -63,6 +63,7 @@ struct FwdParams {
     const int32_t* tile_shard;
     const int32_t* src;             // [cp*cp]
     const int32_t* doc_start;       // [S] shard order
+    const __nv_bfloat16* q;         // [BH][q_rows][D] (read directly by the head_dim-256 kernel)
     __nv_bfloat16* o;               // [BH][S][D]  (fused)
     float* lse;                     // [BH][S]     (fused)
     float* o_parts;                 // [cp][BH][S][D] (separate)
