@@ -17,6 +17,7 @@
 #include "bwd.cuh"
 #include "bwd_fused.cuh"
 #include "fwd256.cuh"
+#include "bwd256.cuh"
 
 using namespace cpattn;
 
@@ -630,11 +631,13 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
             nlse2, rows, D, dq_acc);
         if (launch_status() != CP_OK) return CP_ERR_CUDA;
     }
+    // head_dim 256: the dK / dV passes stream 64-row query units
+    constexpr int QBOX_ROWS = D == 256 ? Kv256Cfg<0>::QT : 128;
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128) ||
+    if (!make_tmap_bf16_2d(&tq, q, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, QBOX_ROWS) ||
         !make_tmap_bf16_2d(&tk, k, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128) ||
         !make_tmap_bf16_2d(&tv, v, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, 128) ||
-        !make_tmap_bf16_2d(&tdo, dout, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128))
+        !make_tmap_bf16_2d(&tdo, dout, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, QBOX_ROWS))
         return CP_ERR_CUDA;
     BwdParams P;
     P.B = B;
@@ -671,6 +674,49 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.tile_orig = tables_orig(p, pl);
     P.tile_shard = tables_shard(p, pl);
     const bool pd = p->shard == CP_SHARD_PER_DOC;
+    if constexpr (D == 256) {
+        // three passes: dV, dK (64-row query units against 128-key tiles), dQ (64-key
+        // tiles against 128-row query tiles); no one-pass form
+        if (dq_acc) return CP_ERR_UNSUPPORTED;
+        CUtensorMap tk64, tv64, tdo128;
+        if (!make_tmap_bf16_2d(&tk64, k, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, Dq256Cfg::KT) ||
+            !make_tmap_bf16_2d(&tv64, v, D, static_cast<uint64_t>(B) * Hkv * L.kv_rows, D * 2, 64, Dq256Cfg::KT) ||
+            !make_tmap_bf16_2d(&tdo128, dout, D, static_cast<uint64_t>(B) * Hq * L.q_rows, D * 2, 64, 128))
+            return CP_ERR_CUDA;
+        const cp_status_t ast = ensure_attr(ATTR_BWD256, [] {
+            cudaError_t e = cudaSuccess;
+            for (auto* kd : {cp_bwd256_kv_kernel<false, 0>, cp_bwd256_kv_kernel<true, 0>})
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, Kv256Cfg<0>::SMEM_BYTES);
+            for (auto* kd : {cp_bwd256_kv_kernel<false, 1>, cp_bwd256_kv_kernel<true, 1>})
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, Kv256Cfg<1>::SMEM_BYTES);
+            for (auto* kq : {cp_bwd256_dq_kernel<false>, cp_bwd256_dq_kernel<true>})
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, Dq256Cfg::SMEM_BYTES);
+            return e;
+        });
+        if (ast != CP_OK) return ast;
+        P.n_items = B * Hkv * (S / 256);   // pairs of key tiles
+        const int grid_kv = std::min(P.n_items, num_sms());
+        {
+            LaunchScope ls(CP_K_BWD_DKDV, stream);
+            auto* kv = pd ? cp_bwd256_kv_kernel<true, 0> : cp_bwd256_kv_kernel<false, 0>;
+            kv<<<grid_kv, BWD_THREADS, Kv256Cfg<0>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, P);
+        }
+        if (launch_status() != CP_OK) return CP_ERR_CUDA;
+        {
+            LaunchScope ls(CP_K_BWD_DKDV, stream);
+            auto* kk = pd ? cp_bwd256_kv_kernel<true, 1> : cp_bwd256_kv_kernel<false, 1>;
+            kk<<<grid_kv, BWD_THREADS, Kv256Cfg<1>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, P);
+        }
+        if (launch_status() != CP_OK) return CP_ERR_CUDA;
+        P.n_items = B * Hq * (L.q_rows / 128);
+        LaunchScope ls(CP_K_BWD_DQ, stream);
+        auto* kq = pd ? cp_bwd256_dq_kernel<true> : cp_bwd256_dq_kernel<false>;
+        kq<<<std::min(P.n_items, num_sms()), BWD_THREADS, Dq256Cfg::SMEM_BYTES, stream>>>(tk64, tv64, tdo128, P);
+        return launch_status();
+    } else {
     const cp_status_t ast = ensure_attr(D == 128 ? ATTR_BWD128 : ATTR_BWD64, [] {
         cudaError_t e = cudaSuccess;
         for (auto* kd : {cp_bwd_dkdv_kernel<D, false>, cp_bwd_dkdv_kernel<D, true>})
@@ -720,6 +766,26 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     auto* kdq = pd ? cp_bwd_dq_kernel<D, true> : cp_bwd_dq_kernel<D, false>;
     kdq<<<std::min(P.n_items, num_sms()), DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, P);
     return launch_status();
+    }
+}
+
+// The backward for the problem's head_dim.
+cp_status_t launch_bwd_any(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
+                           const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                           void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream,
+                           int stall, const Layout& L, float* dk32, float* dv32, float* dq_acc)
+{
+    switch (p->head_dim) {
+    case 256:
+        return launch_bwd<256>(p, pl, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, stream, stall, L,
+                               dk32, dv32, dq_acc);
+    case 128:
+        return launch_bwd<128>(p, pl, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, stream, stall, L,
+                               dk32, dv32, dq_acc);
+    default:
+        return launch_bwd<64>(p, pl, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, stream, stall, L,
+                              dk32, dv32, dq_acc);
+    }
 }
 
 }  // namespace
@@ -742,18 +808,14 @@ cp_status_t attn_bwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
     // the two deterministic passes unless the caller asks for the one-pass form (the
     // stall hook picks the form of the kernel it targets)
     const bool one_pass = stall == CP_K_BWD_FUSED || (problem->bwd_one_pass && stall == 0);
+    if (one_pass && problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // three passes only
     const size_t acc_bytes = one_pass ? round_up(size_t(rows) * problem->head_dim * 4, 256) : 0;
     if (workspace_gate(2 * row_bytes + acc_bytes, ws, ws_bytes, &st)) return st;
     float* delta = static_cast<float*>(ws);
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     float* dq_acc = one_pass ? reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * row_bytes) : nullptr;
     cudaStream_t s = as_stream(stream);
-    if (problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // backward at head_dim 256: not yet
-    return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
-                                 whole_layout(problem), nullptr, nullptr, dq_acc)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall,
-                                whole_layout(problem), nullptr, nullptr, dq_acc);
+    return launch_bwd_any(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, stall, whole_layout(problem), nullptr, nullptr, dq_acc);
 }
 
 }  // namespace
@@ -835,12 +897,7 @@ extern "C" cp_status_t cp_attn_bwd_noalloc(const cp_problem_t* problem, const cp
     if ((st = noalloc_scratch(s, &scratch)) != CP_OK) return st;
     float* delta = static_cast<float*>(scratch);
     float* nlse2 = delta + CP_NOALLOC_MAX_ROWS;   // 16 MiB further: 256-byte aligned
-    if (problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // backward at head_dim 256: not yet
-    return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
-                                 whole_layout(problem), nullptr, nullptr, nullptr)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0,
-                                whole_layout(problem), nullptr, nullptr, nullptr);
+    return launch_bwd_any(problem, plan, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, s, 0, whole_layout(problem), nullptr, nullptr, nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -932,12 +989,7 @@ extern "C" cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_pl
     float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
     cudaStream_t s = as_stream(stream);
     const Layout L = rank_layout(problem, rank, -1);
-    if (problem->head_dim == 256) return CP_ERR_UNSUPPORTED;   // backward at head_dim 256: not yet
-    return problem->head_dim == 128
-               ? launch_bwd<128>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
-                                 s, 0, L, dk_part, dv_part, nullptr)
-               : launch_bwd<64>(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2,
-                                s, 0, L, dk_part, dv_part, nullptr);
+    return launch_bwd_any(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2, s, 0, L, dk_part, dv_part, nullptr);
 }
 
 extern "C" cp_status_t cp_f32_to_bf16(const float* in, void* out, int64_t n, void* stream)

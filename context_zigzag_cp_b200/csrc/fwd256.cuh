@@ -37,6 +37,7 @@ struct Fwd256Cfg {
     static constexpr int NBAR = 8 + 2 * NSLOT;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;  // + alignment slack
     static constexpr int THREADS = 192;
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 // A 64-key tile [ko, ko+63] against the query tile [qo, qo+127] (as

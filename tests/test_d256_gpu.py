@@ -93,3 +93,85 @@ def test_rank_calls_reassemble_whole():
         assert torch.equal(lm.view_as(l_r), loc(lse_sep, r))
     torch.cuda.synchronize()
     assert cz.get_device_status() == 0
+
+
+# ------------------------------------------------------------------ backward
+# Three passes at head_dim 256 (dV, dK: 64-row query units against 128-key
+# tiles; dQ: 64-key tiles against 128-row query tiles), against the oracle's
+# explicit-P gradients in original order.
+
+def check_bwd(case, cp, rotate, tag):
+    prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, cp, rotate, "fused")
+    (dos,) = plan.shard([case["do"].cuda()])
+    dq, dk, dv = cz.attn_bwd(prob, plan, qs, ks, vs, o, lse, dos)
+    torch.cuda.synchronize()
+    assert cz.get_device_status() == 0
+    dq, dk, dv = plan.unshard([dq, dk, dv])
+    q, k, v, do = (f64(case[n]) for n in ("q", "k", "v", "do"))
+    ro, rl = oracle.fwd(q, k, v, case["ds"], None, case["lk"])
+    rq, rk, rv = oracle.bwd(q, k, v, ro, rl, do, case["ds"], None, case["lk"])
+    tag = f"D=256 {tag} S={q.shape[2]} cp={cp} {rotate}"
+    assert_bf16_close(f64(dq), rq, "dQ " + tag)
+    assert_bf16_close(f64(dk), rk, "dK " + tag)
+    assert_bf16_close(f64(dv), rv, "dV " + tag)
+
+
+@pytest.mark.parametrize("rotate", ["allgather", "ring"])
+def test_bwd_causal_gqa(rotate):
+    case = make_case(1, 8, 2, 2048, 256, 2, 221, with_dout=True)
+    check_bwd(case, 2, rotate, "causal GQA 8/2")
+
+
+def test_bwd_cp3_batch2():
+    case = make_case(2, 4, 4, 2304, 256, 3, 222, with_dout=True)
+    check_bwd(case, 3, "ring", "causal MHA batch 2")
+
+
+def test_bwd_documents_window():
+    cu = random_docs(4096, 223, 300.0)
+    case = make_case(1, 4, 2, 4096, 256, 2, 224, cu=cu, with_dout=True)
+    check_bwd(case, 2, "ring", "documents")
+    case = make_case(1, 4, 2, 4096, 256, 2, 225, cu=cu, with_dout=True, window=200)
+    check_bwd(case, 2, "allgather", "documents + window 200")
+
+
+def test_bwd_no_causal_mask_and_per_doc():
+    case = make_case(1, 4, 2, 2048, 256, 2, 226, with_dout=True, causal=False)
+    check_bwd(case, 2, "allgather", "no causal mask")
+    cu = random_docs(4096, 227, 900.0, 128, quantum=512)
+    case = make_case(1, 4, 2, 4096, 256, 2, 228, cu=cu, with_dout=True, shard="doc")
+    check_bwd(case, 2, "ring", "per-doc")
+
+
+def test_bwd_one_pass_unsupported():
+    case = make_case(1, 2, 2, 512, 256, 2, 229, with_dout=True)
+    prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, 2, "ring", "fused")
+    (dos,) = plan.shard([case["do"].cuda()])
+    with pytest.raises(cz.CPError, match="UNSUPPORTED"):
+        cz.attn_bwd(prob.with_one_pass(True), plan, qs, ks, vs, o, lse, dos)
+
+
+def test_bwd_rank_calls_sum_to_whole():
+    S, cp, D = 2048, 2, 256
+    case = make_case(1, 4, 2, S, D, cp, 230, with_dout=True)
+    prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, cp, "ring", "fused")
+    (dos,) = plan.shard([case["do"].cuda()])
+    dq, dk, dv = cz.attn_bwd(prob, plan, qs, ks, vs, o, lse, dos)
+    n2c = S // cp
+    loc = lambda x, r: x[:, :, r * n2c:(r + 1) * n2c].contiguous()
+    dk_sum = torch.zeros(ks.shape, dtype=torch.float32, device="cuda")
+    dv_sum = torch.zeros_like(dk_sum)
+    for r in range(cp):
+        dq_r, dkp, dvp = cz.attn_bwd_rank(prob, plan, r, loc(qs, r), ks, vs, loc(o, r), loc(lse, r),
+                                          loc(dos, r))
+        assert torch.equal(dq_r, loc(dq, r))
+        dk_sum += dkp
+        dv_sum += dvp
+    torch.cuda.synchronize()
+    assert cz.get_device_status() == 0
+    dk_u, dv_u = plan.unshard([cz.f32_to_bf16(dk_sum), cz.f32_to_bf16(dv_sum)])
+    q, k, v, do = (f64(case[n]) for n in ("q", "k", "v", "do"))
+    ro, rl = oracle.fwd(q, k, v, case["ds"])
+    _, rk, rv = oracle.bwd(q, k, v, ro, rl, do, case["ds"])
+    assert_bf16_close(f64(dk_u), rk, f"dK D=256 S={S} cp={cp} per-rank sum")
+    assert_bf16_close(f64(dv_u), rv, f"dV D=256 S={S} cp={cp} per-rank sum")
