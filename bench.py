@@ -345,10 +345,12 @@ def run_native(args, w, rank, world, local_rank):
         a[0] += 1
         a[1] += kms
     kernels = {n: {"launches": c, "ms": round(t_, 4)} for n, (c, t_) in per.items()}
+    # a share is the step's work of that kernel name over all its launches (at head_dim
+    # 256 the dK/dV work is two launches, the dV pass and the dK pass)
     for n, share in KERNEL_FLOP_SHARE.items():
         if n in kernels:
             kernels[n]["tflops"] = round(share * w.head_dim * w.num_heads * pairs /
-                                         (kernels[n]["ms"] / kernels[n]["launches"]) / 1e9, 1)
+                                         kernels[n]["ms"] / 1e9, 1)
     # HBM-bound kernels: achieved GB/s from their algorithmic bytes
     rows = w.batch * w.num_heads * w.seq_len
     row_bytes = w.head_dim * 2
@@ -372,8 +374,7 @@ def run_native(args, w, rank, world, local_rank):
             kernels[n]["frac_of_hbm_peak"] = round(kernels[n]["gbs"] / peaks["hbm"], 4)
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     dom_flops = KERNEL_FLOP_SHARE.get(dom, 0.0) * w.head_dim * w.num_heads * pairs
-    dom_ms = kernels[dom]["ms"] / kernels[dom]["launches"]
-    achieved = dom_flops / dom_ms / 1e9 if dom_flops else 0.0
+    achieved = dom_flops / kernels[dom]["ms"] / 1e9 if dom_flops else 0.0
     peak = peaks["bf16_sustained"]
 
     # ---- forward alone, both merge modes (device time of the cp_attn_fwd call)
@@ -406,7 +407,8 @@ def run_native(args, w, rank, world, local_rank):
         return e0.elapsed_time(e1) / n
 
     bwd_ms = dist_max(dist, time_bwd(prob), device)
-    bwd1_ms = dist_max(dist, time_bwd(prob.with_one_pass(True)), device)
+    # the one-pass option exists at head_dim 64 and 128 only
+    bwd1_ms = dist_max(dist, time_bwd(prob.with_one_pass(True)), device) if w.head_dim != 256 else None
     fwd_32k = forward_at(args, "gqa32k", device, dist, peaks) if w.name != "gqa32k" else None
 
     # ---- end to end through the public API with pinned host buffers
@@ -519,8 +521,8 @@ def run_native(args, w, rank, world, local_rank):
             "fwd_32k": fwd_32k,
             "bwd_tflops": round(2.0 * fwd_flops / 1e9 / bwd_ms, 1),
             "bwd_ms": round(bwd_ms, 3),
-            "bwd_one_pass_tflops": round(2.0 * fwd_flops / 1e9 / bwd1_ms, 1),
-            "bwd_one_pass_ms": round(bwd1_ms, 3),
+            "bwd_one_pass_tflops": round(2.0 * fwd_flops / 1e9 / bwd1_ms, 1) if bwd1_ms else None,
+            "bwd_one_pass_ms": round(bwd1_ms, 3) if bwd1_ms else None,
             "step_frac_of_peak": round(value / world / peaks["bf16_sustained"], 4),
             "peak_source": peaks["source"],
             "pairs": pairs,

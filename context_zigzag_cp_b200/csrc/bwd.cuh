@@ -37,7 +37,7 @@ namespace cpattn {
 // Preprocess: delta[row] = sum_d dO*O, nlse2[row] = -LSE * log2(e), and (for the
 // one-pass backward) the row of the fp32 dQ accumulator set to zero.  A row is
 // D/8 lanes of one warp, each reading 16 bytes (8 bf16) of O and of dO, so a
-// warp covers 32*8/D rows per step with full 16-byte accesses (D = 64 or 128).
+// warp covers 32*8/D rows per step with full 16-byte accesses (D = 64, 128 or 256).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,

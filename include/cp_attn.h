@@ -111,11 +111,13 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *                 CP_MASK_FULL is CP_ERR_UNSUPPORTED.
  *   shard         cp_shard_t (CP_SHARD_PER_DOC needs the document mask)
  *   bwd_one_pass  backward only.  0 (default): two passes, a dK/dV pass and a
- *                 dQ pass that recomputes S and dP; bit-for-bit reproducible,
- *                 and the faster form on B200 (128k: 438 vs 475 ms).
+ *                 dQ pass that recomputes S and dP (three at head_dim 256: dV,
+ *                 dK and dQ); bit-for-bit reproducible, and the faster form on
+ *                 B200 (128k: 438 vs 475 ms).
  *                 1: one pass, dK, dV and dQ from one recomputation of S and dP,
  *                 dQ summed in an fp32 accumulator by atomic reductions (its
  *                 last bits depend on their order); bound by those reductions.
+ *                 head_dim 64 and 128 only (256: CP_ERR_UNSUPPORTED).
  *   cu_seqlens    DEVICE int32 [num_docs+1], 0 = cu[0] < cu[1] < ... <
  *                 cu[num_docs] = S, original order; the same documents apply to
  *                 every batch entry.  NULL for the plain causal mask.
@@ -224,7 +226,8 @@ CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan
  *   k, v  bf16 [B][Hkv][S][D] shard order
  *   o     bf16 [B][Hq][S][D]  output, shard order
  *   lse   fp32 [B][Hq][S]     output, natural-log LSE of the scaled scores
- * Supported: head_dim 64 or 128; C = S/(2cp) a multiple of 128; S <= 2^29.
+ * Supported: head_dim 64, 128 or 256; C = S/(2cp) a multiple of 128;
+ * S <= 2^29.
  * Workspace: CP_MERGE_SEPARATE needs cp fp32 partial (O, LSE) sets (each
  * region rounded up to 256 bytes); CP_MERGE_FUSED needs none (0 bytes).
  * Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_WORKSPACE, CP_ERR_CUDA.

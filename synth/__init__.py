@@ -55,6 +55,8 @@ WORKLOADS = {
     "gqa32k": Workload("gqa32k", 1, 32768, 8, 32, 8, 128, "ring", amp=0.5, seed=2),
     "docs64k": Workload("docs64k", 1, 65536, 8, 32, 8, 128, "ring", docs=True, seed=3),
     "long128k": Workload("long128k", 1, 131072, 8, 32, 8, 128, "allgather", seed=4),
+    # gqa32k at head_dim 256
+    "gqa32k_d256": Workload("gqa32k_d256", 1, 32768, 8, 32, 8, 256, "ring", amp=0.5, seed=5),
     # the docs64k mix with every document cut into 2cp chunks of whole 128-row tiles
     "docs64k_perdoc": Workload("docs64k_perdoc", 1, 65536, 8, 32, 8, 128, "ring", docs=True,
                                seed=3, shard="doc", doc_quantum=2048),

@@ -231,3 +231,15 @@ def test_shard_host_checks(lib):
     row = (ctypes.c_int64 * 1)(128)
     assert cz.lib().cp_unshard(p.ref, ctypes.byref(no_inv), 1, ptrs, outs, outer, row,
                                None) == _lib.CP_ERR_INVALID_ARG
+
+
+def test_head_dim_256(lib):
+    """head_dim 256 has its own forward and three-pass backward; no one-pass form."""
+    st, n = fwd_query(prob(head_dim=256, merge="separate"))
+    rows = 1 * 2 * 512
+    assert st == _lib.CP_OK and n == 2 * rows * 256 * 4 + 2 * rows * 4
+    assert cz.bwd_workspace_bytes(prob(head_dim=256)) == 2 * rows * 4
+    with pytest.raises(cz.CPError, match="UNSUPPORTED"):
+        cz.bwd_workspace_bytes(prob(head_dim=256, bwd_one_pass=True))
+    assert fwd_query(prob(head_dim=192))[0] == _lib.CP_ERR_UNSUPPORTED
+

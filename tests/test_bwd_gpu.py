@@ -215,6 +215,11 @@ def test_docs64k_sampled():
     check_sampled("docs64k", "ring")
 
 
+def test_gqa32k_d256_sampled():
+    """gqa32k at head_dim 256: the three-pass backward."""
+    check_sampled("gqa32k_d256", "ring")
+
+
 @pytest.mark.parametrize("one_pass", [False, True])
 def test_docs64k_perdoc_sampled(one_pass):
     check_sampled("docs64k_perdoc", "ring", one_pass=one_pass)

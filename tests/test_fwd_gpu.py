@@ -126,6 +126,12 @@ def test_docs64k_sampled():
     check_sampled("docs64k", "allgather", "fused")
 
 
+def test_gqa32k_d256_sampled():
+    """gqa32k at head_dim 256 (its own forward kernel)."""
+    check_sampled("gqa32k_d256", "ring", "separate")
+    check_sampled("gqa32k_d256", "allgather", "fused", per_head=96)
+
+
 def test_docs64k_perdoc_sampled():
     """The docs64k length mix in whole-tile multiples, every document cut into 2cp chunks."""
     check_sampled("docs64k_perdoc", "ring", "fused")

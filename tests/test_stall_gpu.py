@@ -38,9 +38,11 @@ def _parity_after(case, cp, rotate):
     assert_bf16_close(f64(dv), rv, "dV after a timed-out kernel")
 
 
-@pytest.mark.parametrize("kernel", ["fwd", "bwd_dkdv", "bwd_dq", "bwd_fused"])
-def test_stalled_kernel_times_out_and_context_survives(kernel):
-    case = make_case(1, 4, 2, 1024, 128, 2, 31, with_dout=True)
+# head_dim 256 runs its own kernels (one forward; dV, dK and dQ passes; no one-pass form)
+@pytest.mark.parametrize("kernel,D", [("fwd", 128), ("bwd_dkdv", 128), ("bwd_dq", 128), ("bwd_fused", 128),
+                                      ("fwd", 256), ("bwd_dkdv", 256), ("bwd_dq", 256)])
+def test_stalled_kernel_times_out_and_context_survives(kernel, D):
+    case = make_case(1, 4, 2, 1024, D, 2, 31, with_dout=True)
     prob, plan, qs, ks, vs, o, lse = run_fwd(cz, case, 2, "ring", "fused")
     (dos,) = plan.shard([case["do"].cuda()])
     torch.cuda.synchronize()
