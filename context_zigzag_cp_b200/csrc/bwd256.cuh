@@ -64,8 +64,8 @@ struct Kv256Cfg {
     static constexpr int DO_OFF = Q_OFF + NQ * QTILE;
     static constexpr int BAR_OFF = DO_OFF + NDO * QTILE;
     // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NDO], do_empty[NDO], st_ready,
-    // dp_ready, s_free, p_full, acc_full, drain, acc_empty
-    static constexpr int NBAR = 9 + 2 * NQ + 2 * NDO;
+    // dp_ready, s_free, p_full[2], acc_full, drain, acc_empty
+    static constexpr int NBAR = 10 + 2 * NQ + 2 * NDO;
     static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 64 + 1024;   // + alignment slack
     static constexpr int THREADS = BWD_THREADS;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -90,8 +90,11 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t bar_q_full = bars + 16, bar_q_empty = bar_q_full + 8 * Cfg::NQ;
     const uint32_t bar_do_full = bar_q_empty + 8 * Cfg::NQ, bar_do_empty = bar_do_full + 8 * Cfg::NDO;
     const uint32_t bar_st_ready = bar_do_empty + 8 * Cfg::NDO, bar_dp_ready = bar_st_ready + 8;
-    const uint32_t bar_s_free = bar_dp_ready + 8, bar_p_full = bar_s_free + 8;
-    const uint32_t bar_acc_full = bar_p_full + 8, bar_drain = bar_acc_full + 8;
+    // p_full[u & 1] for unit u: in the dV pass nothing orders the elementwise step of
+    // unit u+1 after the MMA warp's wait for unit u (S^T(u+1) is issued first), so one
+    // barrier could complete twice before that wait and its parity would alias
+    const uint32_t bar_s_free = bar_dp_ready + 8, bar_p_full = bar_s_free + 8;   // [2]
+    const uint32_t bar_acc_full = bar_p_full + 16, bar_drain = bar_acc_full + 8;
     const uint32_t bar_acc_empty = bar_drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + Cfg::NBAR * 8 + 8);
@@ -117,6 +120,7 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(bar_dp_ready, 1);
         mbar_init(bar_s_free, 4 * BWD_NWG);
         mbar_init(bar_p_full, 4 * BWD_NWG);
+        mbar_init(bar_p_full + 8, 4 * BWD_NWG);
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_drain, 1);
         mbar_init(bar_acc_empty, 4 * BWD_NWG);
@@ -200,7 +204,8 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const uint64_t dKk = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
             const uint64_t dQk = sdesc_sw128(sQ, 16, 1024), dQmn = sdesc_sw128(sQ, Cfg::QBOX, 1024);
             const uint64_t dOk = sdesc_sw128(sdO, 16, 1024), dOmn = sdesc_sw128(sdO, Cfg::QBOX, 1024);
-            uint32_t nst = 0, iter = 0, sf_phase = 0, ae_phase = 0, p_phase = 0;
+            uint32_t nst = 0, iter = 0, sf_phase = 0, ae_phase = 0;
+            uint32_t p_phase = 0;             // bit b: parity of the next wait on p_full[b]
             bool ok = true, acc_busy = false, s_pending = false;
             // the products of one finished unit: MODE 0 dV += P^T dO (P^T at columns 64 + 32pb,
             // query rows 16w .. +15 at + 8w); MODE 1 dK += dS^T Q (dS^T over the dP^T columns,
@@ -211,8 +216,8 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     ae_phase ^= 1;
                     acc_busy = false;
                 }
-                if (!mbar_wait_warp(bar_p_full, p_phase, abort_flag)) return false;
-                p_phase ^= 1;
+                if (!mbar_wait_warp(bar_p_full + 8 * pb, (p_phase >> pb) & 1u, abort_flag)) return false;
+                p_phase ^= 1u << pb;
                 // MODE 0: the unit's dO (MODE 1 waited for it before its dP^T)
                 if (MODE == 0 && !mbar_wait_warp(bar_do_full + 8 * ds, dpar, abort_flag)) return false;
                 tc_fence_after();
@@ -401,7 +406,7 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bar_p_full);
+                        if (lane == 0) mbar_arrive(bar_p_full + 8 * pb);
                         had = true;
                     }
                 }
