@@ -39,7 +39,7 @@ uint32_t g_attr_done[kMaxDevices] = {};   // bit per kernel family (AttrSet)
 
 enum AttrSet : uint32_t {
     ATTR_FWD64 = 1, ATTR_FWD128 = 2, ATTR_BWD64 = 4, ATTR_BWD128 = 8, ATTR_FUSED64 = 16, ATTR_FUSED128 = 32,
-    ATTR_FWD256 = 64, ATTR_BWD256 = 128
+    ATTR_FWD256 = 64, ATTR_BWD256 = 128, ATTR_MERGE_TILED = 256
 };
 
 inline int current_device()
@@ -331,6 +331,9 @@ cp_status_t launch_fwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.lse = lse;
     P.o_parts = o_parts;
     P.lse_parts = lse_parts;
+    // partials into the caller's buffers (cp_attn_fwd_step: no o) stay row-major;
+    // the library's own workspace is tile-interleaved for lse_merge_tiled_kernel
+    P.parts_tiled = o != nullptr;
     if constexpr (D == 256) {
         // one 128-row query tile per work item
         P.n_items = P.BH * (L.q_rows / 128);
@@ -382,7 +385,8 @@ cp_status_t launch_fwd_any(const cp_problem_t* p, const cp_plan_t* pl, const voi
 }
 
 cp_status_t launch_merge(int64_t rows, int32_t D, int32_t n_parts, const float* o_parts,
-                         const float* lse_parts, void* o_out, float* lse_out, cudaStream_t stream)
+                         const float* lse_parts, void* o_out, float* lse_out, cudaStream_t stream,
+                         bool tiled = false)
 {
     if (rows == 0) return CP_OK;
     MergeParams M;
@@ -393,6 +397,19 @@ cp_status_t launch_merge(int64_t rows, int32_t D, int32_t n_parts, const float* 
     M.lse_parts = lse_parts;
     M.o_out = static_cast<__nv_bfloat16*>(o_out);
     M.lse_out = lse_out;
+    if (tiled) {
+        // the forward's own partials (rows a multiple of 128, tile-interleaved)
+        const cp_status_t ast = ensure_attr(ATTR_MERGE_TILED, [] {
+            return cudaFuncSetAttribute(lse_merge_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        232448);
+        });
+        if (ast != CP_OK) return ast;
+        const size_t smem = size_t(n_parts) * 128 * 4 + size_t(128) * (D / 4 + 1) * 8;
+        const int64_t blocks = std::min<int64_t>(rows / 128, int64_t(num_sms()) * 8);
+        LaunchScope ls(CP_K_MERGE, stream);
+        lse_merge_tiled_kernel<<<static_cast<unsigned>(blocks), 128, smem, stream>>>(M);
+        return launch_status();
+    }
     const int64_t blocks = std::min<int64_t>((rows + 7) / 8, int64_t(num_sms()) * 16);
     LaunchScope ls(CP_K_MERGE, stream);
     lse_merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(M);
@@ -550,7 +567,7 @@ cp_status_t attn_fwd_impl(const cp_problem_t* problem, const cp_plan_t* plan, co
     const bool fused = problem->merge == CP_MERGE_FUSED;
     st = launch_fwd_any(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, stall, L, fused);
     if (st != CP_OK || !separate) return st;
-    return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
+    return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s, true);
 }
 
 }  // namespace
@@ -953,7 +970,7 @@ extern "C" cp_status_t cp_attn_fwd_rank(const cp_problem_t* problem, const cp_pl
     const Layout L = rank_layout(problem, rank, -1);
     st = launch_fwd_any(problem, plan, q, k, v, o, lse, o_parts, lse_parts, s, 0, L, !separate);
     if (st != CP_OK || !separate) return st;
-    return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s);
+    return launch_merge(rows, problem->head_dim, problem->cp_size, o_parts, lse_parts, o, lse, s, true);
 }
 
 extern "C" cp_status_t cp_attn_fwd_step(const cp_problem_t* problem, const cp_plan_t* plan,

@@ -46,6 +46,8 @@ struct FwdParams {
     int32_t wm1;                    // sliding window - 1 (larger than S: no window)
     int32_t nc;                     // last visible key of query q is q + nc: 0 causal, S none
     int32_t fused;                  // 1 = CP_MERGE_FUSED
+    int32_t parts_tiled;            // separate merge: partials tile-interleaved (lse_merge_tiled_kernel)
+                                    // rather than row-major [parts][rows][D]
     float scale_log2;               // softmax scale * log2(e)
     int32_t n_items, ppc;           // items, query-tile pairs per chunk
     int32_t stall;                  // test hook: 1 = CTA 0 skips its first K/V load
@@ -669,14 +671,18 @@ cp_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                     dst[i] = u;
                                 }
                             } else {
-                                float4* dst = reinterpret_cast<float4*>(
-                                    P.o_parts + (static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi) * D + c0);
+                                const size_t prow_all = static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi;
+                                // tile-interleaved: the warp's 32 rows store 512 contiguous bytes
+                                float4* dst = P.parts_tiled
+                                    ? reinterpret_cast<float4*>(P.o_parts) + ((prow_all >> 7) * (D / 4) + c0 / 4) * 128 + (prow_all & 127)
+                                    : reinterpret_cast<float4*>(P.o_parts + prow_all * D + c0);
+                                const size_t step = P.parts_tiled ? 128 : 1;
 #pragma unroll
                                 for (int i = 0; i < 8; ++i)
-                                    dst[i] = make_float4(__uint_as_float(orr[4 * i + 0]) * inv_l,
-                                                         __uint_as_float(orr[4 * i + 1]) * inv_l,
-                                                         __uint_as_float(orr[4 * i + 2]) * inv_l,
-                                                         __uint_as_float(orr[4 * i + 3]) * inv_l);
+                                    dst[i * step] = make_float4(__uint_as_float(orr[4 * i + 0]) * inv_l,
+                                                                __uint_as_float(orr[4 * i + 1]) * inv_l,
+                                                                __uint_as_float(orr[4 * i + 2]) * inv_l,
+                                                                __uint_as_float(orr[4 * i + 3]) * inv_l);
                             }
                         }
                         if (P.fused) P.lse[rowi] = lse_v;

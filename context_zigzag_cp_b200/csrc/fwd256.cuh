@@ -449,12 +449,16 @@ cp_fwd256_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                                     dst[i] = u;
                                 }
                             } else {
-                                float4* dst = reinterpret_cast<float4*>(
-                                    P.o_parts + (static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi) * D + c0);
+                                const size_t prow_all = static_cast<size_t>(s - P.s0) * P.BH * P.q_rows + rowi;
+                                // tile-interleaved: the warp's 32 rows store 512 contiguous bytes
+                                float4* dst = P.parts_tiled
+                                    ? reinterpret_cast<float4*>(P.o_parts) + ((prow_all >> 7) * (D / 4) + c0 / 4) * 128 + (prow_all & 127)
+                                    : reinterpret_cast<float4*>(P.o_parts + prow_all * D + c0);
+                                const size_t step = P.parts_tiled ? 128 : 1;
 #pragma unroll
                                 for (int i = 0; i < 8; ++i)
-                                    dst[i] = make_float4(of[4 * i + 0] * inv_l, of[4 * i + 1] * inv_l,
-                                                         of[4 * i + 2] * inv_l, of[4 * i + 3] * inv_l);
+                                    dst[i * step] = make_float4(of[4 * i + 0] * inv_l, of[4 * i + 1] * inv_l,
+                                                                of[4 * i + 2] * inv_l, of[4 * i + 3] * inv_l);
                             }
                         }
                         if (P.fused) P.lse[rowi] = lse_v;

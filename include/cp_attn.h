@@ -229,7 +229,9 @@ CP_API cp_status_t cp_unshard(const cp_problem_t* problem, const cp_plan_t* plan
  * Supported: head_dim 64, 128 or 256; C = S/(2cp) a multiple of 128;
  * S <= 2^29.
  * Workspace: CP_MERGE_SEPARATE needs cp fp32 partial (O, LSE) sets (each
- * region rounded up to 256 bytes); CP_MERGE_FUSED needs none (0 bytes).
+ * region rounded up to 256 bytes; the O partials in an internal 128-row
+ * tile-interleaved layout, not the row layout cp_lse_merge takes);
+ * CP_MERGE_FUSED needs none (0 bytes).
  * Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_WORKSPACE, CP_ERR_CUDA.
  */
 CP_API cp_status_t cp_attn_fwd(const cp_problem_t* problem, const cp_plan_t* plan, const void* q,
