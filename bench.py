@@ -379,20 +379,25 @@ def run_native(args, w, rank, world, local_rank):
     achieved = dom_flops / kernels[dom]["ms"] / 1e9 if dom_flops else 0.0
     peak = peaks["bf16_sustained"]
 
-    # ---- forward alone, both merge modes (device time of the cp_attn_fwd call)
+    # ---- forward alone, both merge modes (device time of the cp_attn_fwd call), with
+    # the clocks of that stretch and the time of each call: the forward alone runs
+    # several calls back to back under the power cap, the in-step figure one call
     def time_fwd(pr, n=3):
         cz.attn_fwd(pr, plan, qs, ks, vs, o, lse, ws=ws_f)
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(n):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        ev[0].record()
+        for i in range(n):
             cz.attn_fwd(pr, plan, qs, ks, vs, o, lse, ws=ws_f)
-        e1.record()
+            ev[i + 1].record()
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / n
+        calls = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+        return sum(calls) / n, calls
 
-    fwd_ms = dist_max(dist, time_fwd(prob), device)
-    fused_ms = dist_max(dist, time_fwd(prob_fused), device)
+    with ClockSampler(local_rank) as fwd_clocks:
+        fwd_ms, fwd_calls = time_fwd(prob)
+    fwd_ms = dist_max(dist, fwd_ms, device)
+    fused_ms = dist_max(dist, time_fwd(prob_fused)[0], device)
 
     # ---- the backward alone, both forms (one pass with dQ reductions; two passes)
     def time_bwd(pr, n=3):
@@ -514,6 +519,8 @@ def run_native(args, w, rank, world, local_rank):
             "config": config_dict(w, rotate, world),
             "fwd_tflops": round(fwd_flops / 1e9 / fwd_ms, 1),
             "fwd_frac_of_peak": round(fwd_flops / 1e9 / fwd_ms / peaks["bf16"], 4),
+            "fwd_alone_calls_ms": [round(c, 3) for c in fwd_calls],
+            "fwd_alone_clocks": fwd_clocks.summary(),
             "fwd_fused_tflops": round(fwd_flops / 1e9 / fused_ms, 1),
             "fwd_fused_frac_of_peak": round(fwd_flops / 1e9 / fused_ms / peaks["bf16"], 4),
             # the forward and its merge as they ran inside the traced step; the figures

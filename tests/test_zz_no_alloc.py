@@ -25,11 +25,12 @@ def _call_noalloc(prob, plan, qs, ks, vs, o, lse, dos, dq, dk, dv):
                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-def test_noalloc_matches_workspace_backward_twice():
-    case = make_case(1, 8, 2, 4096, 128, 4, 31, with_dout=True)
+@pytest.mark.parametrize("D", [128, 256])
+def test_noalloc_matches_workspace_backward_twice(D):
+    case = make_case(1, 8, 2, 4096, D, 4, 31, with_dout=True)
     dev = "cuda"
     q, k, v, do = (case[n].to(dev) for n in ("q", "k", "v", "do"))
-    prob = cz.Problem(1, 4096, 4, 8, 2, 128, "ring")
+    prob = cz.Problem(1, 4096, 4, 8, 2, D, "ring")
     plan = cz.Plan(prob)
     qs, ks, vs, dos = plan.shard([q, k, v, do])
     o, lse = cz.attn_fwd(prob, plan, qs, ks, vs)
@@ -43,7 +44,7 @@ def test_noalloc_matches_workspace_backward_twice():
         torch.cuda.synchronize()
         assert cz.get_device_status() == 0
         for name, got, want in zip(("dQ", "dK", "dV"), outs, ref):
-            assert_bf16_close(f64(got), want, f"{name} no-alloc call {call}")
+            assert_bf16_close(f64(got), want, f"{name} no-alloc D={D} call {call}")
 
 
 def test_noalloc_rejects_problems_beyond_the_array():
