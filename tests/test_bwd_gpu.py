@@ -230,3 +230,10 @@ def test_long128k_sampled(rotate, one_pass):
     # the oracle forward of a whole KV group at 128k is too slow for a test: early
     # key tiles are covered at 32k and 64k
     check_sampled("long128k", rotate, n_rows=48, n_keys=16, early=False, one_pass=one_pass)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_one_kv_head_eight_query_heads(D):
+    """GQA group of 8 (one KV head): dK / dV sum over eight query heads."""
+    case = make_case(1, 8, 1, 2048, D, 2, 240 + D, with_dout=True)
+    check_full(case, 2, "ring")

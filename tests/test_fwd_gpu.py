@@ -141,3 +141,11 @@ def test_docs64k_perdoc_sampled():
 @pytest.mark.parametrize("rotate", ["allgather", "ring"])
 def test_long128k_sampled(rotate):
     check_sampled("long128k", rotate, per_head=96)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_one_kv_head_eight_query_heads(D):
+    """GQA group of 8 (one KV head), both merges."""
+    case = make_case(1, 8, 1, 2048, D, 2, 250 + D)
+    check_full(case, 2, "ring", "fused")
+    check_full(case, 2, "allgather", "separate")

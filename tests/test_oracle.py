@@ -675,3 +675,13 @@ def test_per_doc_rejects_uneven_documents():
         oracle.plan(16, 2, "allgather", [0, 6, 16], shard="doc")   # 6 is not a multiple of 4
     with pytest.raises(ValueError):
         oracle.plan(16, 2, "allgather", None, shard="doc")         # needs documents
+
+
+def test_per_doc_cp1_is_identity():
+    """cp 1: every document is cut into its two halves and rank 0 holds them in
+    order, so the per-document plan is the identity (as the sequence plan is)."""
+    cu = [0, 8, 24, 64]
+    pl = oracle.plan(64, 1, "allgather", cu, shard="doc")
+    assert list(pl["perm"]) == list(range(64))
+    assert list(pl["rank_cu"]) == [0, 4, 8, 16, 24, 44, 64]
+    assert int(pl["pairs"][0]) == oracle.causal_pairs(64, cu)
