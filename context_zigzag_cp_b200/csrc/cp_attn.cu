@@ -404,10 +404,10 @@ cp_status_t launch_merge(int64_t rows, int32_t D, int32_t n_parts, const float* 
                                         232448);
         });
         if (ast != CP_OK) return ast;
-        const size_t smem = size_t(n_parts) * 128 * 4 + size_t(128) * (D / 4 + 1) * 8;
+        const size_t smem = size_t(n_parts) * 128 * 4 + 128 * 4 + size_t(128) * (D / 4 + 1) * 8;
         const int64_t blocks = std::min<int64_t>(rows / 128, int64_t(num_sms()) * 8);
         LaunchScope ls(CP_K_MERGE, stream);
-        lse_merge_tiled_kernel<<<static_cast<unsigned>(blocks), 128, smem, stream>>>(M);
+        lse_merge_tiled_kernel<<<static_cast<unsigned>(blocks), 256, smem, stream>>>(M);
         return launch_status();
     }
     const int64_t blocks = std::min<int64_t>((rows + 7) / 8, int64_t(num_sms()) * 16);

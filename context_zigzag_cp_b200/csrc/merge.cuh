@@ -79,47 +79,55 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeParams M)
 // floats) and row r of the tile, the float4 at ((p * ntile + t) * D/4 + c4) * 128 + r.
 // The forward writes this layout for its own workspace because a warp's 32
 // rows then store 512 contiguous bytes per instruction (row-major partials
-// would put each lane of every store in a different line).  One CTA of 128
-// threads per tile, one thread per row: the weights go to shared memory, the
-// loads of each (part, column group) are 512 contiguous bytes per warp, and the
-// tile's bf16 output is staged in shared memory (rows padded by 8 bytes) and
-// written back as one contiguous block.
-__global__ void __launch_bounds__(128) lse_merge_tiled_kernel(MergeParams M)
+// would put each lane of every store in a different line).  One CTA of 256
+// threads per tile, two threads per row (each half of the column groups): the
+// weights go to shared memory, the loads of each (part, column group) are 512
+// contiguous bytes per warp, and the tile's bf16 output is staged in shared
+// memory (rows padded by 8 bytes) and written back as one contiguous block.
+__global__ void __launch_bounds__(256) lse_merge_tiled_kernel(MergeParams M)
 {
     extern __shared__ float msm[];
-    const int r = threadIdx.x;
+    const int r = threadIdx.x & 127, hh = threadIdx.x >> 7;
     const int nvec = M.D / 4;
     const int64_t ntile = M.rows / 128;
     float* w_s = msm;                                                  // [n_parts][128]
-    uint2* o_s = reinterpret_cast<uint2*>(msm + M.n_parts * 128);     // [128][nvec + 1]
+    float* inv_s = msm + M.n_parts * 128;                              // [128]
+    uint2* o_s = reinterpret_cast<uint2*>(msm + M.n_parts * 128 + 128);   // [128][nvec + 1]
     const float4* parts = reinterpret_cast<const float4*>(M.o_parts);
     for (int64_t t = blockIdx.x; t < ntile; t += gridDim.x) {
         const int64_t row = t * 128 + r;
-        float m = -INFINITY;
-        for (int p = 0; p < M.n_parts; ++p) {
-            const float l = __ldg(M.lse_parts + static_cast<int64_t>(p) * M.rows + row);
-            w_s[p * 128 + r] = l;
-            m = fmaxf(m, l);
+        if (hh == 0) {
+            float m = -INFINITY;
+            for (int p = 0; p < M.n_parts; ++p) {
+                const float l = __ldg(M.lse_parts + static_cast<int64_t>(p) * M.rows + row);
+                w_s[p * 128 + r] = l;
+                m = fmaxf(m, l);
+            }
+            for (int p = 0; p < M.n_parts; ++p) {
+                const float l = w_s[p * 128 + r];
+                w_s[p * 128 + r] = (m == -INFINITY || l == -INFINITY) ? 0.f : expf(l - m);
+            }
+            // sum of the weights in the order of lse_merge_kernel's warp reduction (part
+            // pairs p, p+32, then a butterfly over the 32 lanes), folded in place, so the
+            // two kernels give the same bits for the same partials
+            float v[32];
+#pragma unroll
+            for (int l = 0; l < 32; ++l)
+                v[l] = (l < M.n_parts ? w_s[l * 128 + r] : 0.f) +
+                       (l + 32 < M.n_parts ? w_s[(l + 32) * 128 + r] : 0.f);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                for (int l = 0; l < off; ++l) v[l] = v[l] + v[l + off];
+            const float wsum = m == -INFINITY ? 0.f : v[0];
+            inv_s[r] = wsum > 0.f ? 1.f / wsum : 0.f;
+            M.lse_out[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
         }
-        for (int p = 0; p < M.n_parts; ++p) {
-            const float l = w_s[p * 128 + r];
-            w_s[p * 128 + r] = (m == -INFINITY || l == -INFINITY) ? 0.f : expf(l - m);
-        }
-        // sum of the weights in the order of lse_merge_kernel's warp reduction (part
-        // pairs p, p+32, then a butterfly over the 32 lanes), folded in place, so the
-        // two kernels give the same bits for the same partials
-        float v[32];
-#pragma unroll
-        for (int l = 0; l < 32; ++l)
-            v[l] = (l < M.n_parts ? w_s[l * 128 + r] : 0.f) + (l + 32 < M.n_parts ? w_s[(l + 32) * 128 + r] : 0.f);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-            for (int l = 0; l < off; ++l) v[l] = v[l] + v[l + off];
-        const float wsum = m == -INFINITY ? 0.f : v[0];
-        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-        // four column groups at a time: four independent 16-byte loads per live part
-        for (int c0 = 0; c0 < nvec; c0 += 4) {
+        __syncthreads();
+        const float inv = inv_s[r];
+        // this thread's half of the column groups, four at a time: four independent
+        // 16-byte loads per live part
+        for (int c0 = hh * (nvec / 2); c0 < (hh + 1) * (nvec / 2); c0 += 4) {
             float4 acc[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -147,11 +155,10 @@ __global__ void __launch_bounds__(128) lse_merge_tiled_kernel(MergeParams M)
                 o_s[r * (nvec + 1) + c0 + j] = make_uint2(pack_bf16(acc[j].x * inv, acc[j].y * inv),
                                                           pack_bf16(acc[j].z * inv, acc[j].w * inv));
         }
-        M.lse_out[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
         __syncthreads();
         // the tile's 128 output rows are contiguous: 8-byte stores, 256 contiguous bytes per warp
         uint2* dst = reinterpret_cast<uint2*>(M.o_out + t * 128 * M.D);
-        for (int i = r; i < 128 * nvec; i += 128) {
+        for (int i = threadIdx.x; i < 128 * nvec; i += 256) {
             const int rr = i / nvec, cc = i - rr * nvec;
             dst[i] = o_s[rr * (nvec + 1) + cc];
         }
