@@ -87,7 +87,12 @@ class OracleKernels:
         return x.to(torch.bfloat16)
 
 
-def _worker(rank, world, port, rotate, q_out):
+# documents for the per-document runs: lengths multiples of 2cp = 4, so every
+# document is cut into four chunks of whole rows
+CU_DOC = [0, 20, 32, 84, 128]
+
+
+def _worker(rank, world, port, rotate, shard, q_out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -98,8 +103,9 @@ def _worker(rank, world, port, rotate, q_out):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     cp = world
-    pl = oracle.plan(S, cp, rotate)
-    ds = oracle.doc_start(S)
+    cu = CU_DOC if shard == "doc" else None
+    pl = oracle.plan(S, cp, rotate, cu, shard=shard)
+    ds = oracle.doc_start(S, cu)
     t = synth.attn_inputs(B, HQ, HKV, S, D, seed=91, with_dout=True)   # the same on every rank
     n2c = S // cp
     local = lambda x: x[:, :, pl["perm"][rank * n2c:(rank + 1) * n2c]].contiguous()
@@ -115,12 +121,16 @@ def _worker(rank, world, port, rotate, q_out):
     q_out.put((rank, outs if rank == 0 else None))
 
 
-@pytest.mark.parametrize("rotate", ["allgather", "ring"])
-def test_two_ranks_match_unsharded(rotate):
+# shard "doc": the driver with a per-document plan (the permutation and the
+# document mask change; the exchange, the merge order and the reduce-scatter
+# are the same)
+@pytest.mark.parametrize("rotate,shard", [("allgather", "sequence"), ("ring", "sequence"),
+                                          ("ring", "doc")])
+def test_two_ranks_match_unsharded(rotate, shard):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, rotate, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, rotate, shard, q)) for r in range(2)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=240) for _ in procs)
@@ -134,12 +144,14 @@ def test_two_ranks_match_unsharded(rotate):
     from helpers import assert_bf16_close, assert_lse_close
     t = synth.attn_inputs(B, HQ, HKV, S, D, seed=91, with_dout=True)
     f = lambda x: x.double().numpy()
-    ro, rl = oracle.fwd(f(t["q"]), f(t["k"]), f(t["v"]))
-    rq, rk, rv = oracle.bwd(f(t["q"]), f(t["k"]), f(t["v"]), ro, rl, f(t["do"]))
-    perm = oracle.plan(S, 2, rotate)["perm"]
+    cu = CU_DOC if shard == "doc" else None
+    ds = oracle.doc_start(S, cu)
+    ro, rl = oracle.fwd(f(t["q"]), f(t["k"]), f(t["v"]), ds)
+    rq, rk, rv = oracle.bwd(f(t["q"]), f(t["k"]), f(t["v"]), ro, rl, f(t["do"]), ds)
+    perm = oracle.plan(S, 2, rotate, cu, shard=shard)["perm"]
     cat = lambda n: np.concatenate([outs[r][n] for r in range(2)], axis=2).astype(np.float64)
-    assert_bf16_close(cat("o"), ro[:, :, perm], f"O two ranks {rotate}")
-    assert_lse_close(cat("lse"), rl[:, :, perm], f"LSE two ranks {rotate}")
-    assert_bf16_close(cat("dq"), rq[:, :, perm], f"dQ two ranks {rotate}")
-    assert_bf16_close(cat("dk"), rk[:, :, perm], f"dK two ranks {rotate}")
-    assert_bf16_close(cat("dv"), rv[:, :, perm], f"dV two ranks {rotate}")
+    assert_bf16_close(cat("o"), ro[:, :, perm], f"O two ranks {rotate} {shard}")
+    assert_lse_close(cat("lse"), rl[:, :, perm], f"LSE two ranks {rotate} {shard}")
+    assert_bf16_close(cat("dq"), rq[:, :, perm], f"dQ two ranks {rotate} {shard}")
+    assert_bf16_close(cat("dk"), rk[:, :, perm], f"dK two ranks {rotate} {shard}")
+    assert_bf16_close(cat("dv"), rv[:, :, perm], f"dV two ranks {rotate} {shard}")
