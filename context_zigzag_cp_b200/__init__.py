@@ -27,7 +27,7 @@ __all__ = ["CPError", "Problem", "Plan", "attn_fwd", "attn_bwd", "lse_merge",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "get_device_status",
            "set_wait_limit_ns", "selftest_wait_timeout", "version", "lib", "launch_count",
            "LaunchTrace", "attn_bwd_noalloc", "selftest_stall", "attn_fwd_rank", "attn_fwd_step",
-           "attn_bwd_rank", "f32_to_bf16"]
+           "attn_bwd_rank", "attn_bwd_step", "f32_to_bf16"]
 
 
 class CPError(RuntimeError):
@@ -429,6 +429,32 @@ def attn_bwd_rank(prob: Problem, plan: Plan, rank: int, q, k, v, o, lse, do, dq=
                                   _ptr(dv_part), _ptr(w), ctypes.byref(n) if w is not None else None,
                                   _stream(stream)), "cp_attn_bwd_rank")
     return dq, dk_part, dv_part
+
+
+def attn_bwd_step(prob: Problem, plan: Plan, rank: int, step: int, q, k, v, o, lse, do,
+                  dq_sum, dk_sum, dv_sum, ws=None, stream=None):
+    """cp_attn_bwd_step: one ring step of the backward.  Adds the step's share of the
+    rank's dQ into dq_sum [B,Hq,2C,D] and of shard src[rank][step]'s dK / dV into
+    dk_sum / dv_sum [B,Hkv,2C,D] (fp32, zeroed by the caller before the first step)."""
+    qs, _, kv1, ls = _rank_shapes(prob)
+    bf16, f32 = torch.bfloat16, torch.float32
+    for t, name in ((dq_sum, "dq_sum"), (dk_sum, "dk_sum"), (dv_sum, "dv_sum")):
+        if t is None:
+            raise ValueError(f"{name}: the fp32 sum to add into is required")
+    _validate((q, qs, bf16, "q"), (k, kv1, bf16, "k"), (v, kv1, bf16, "v"), (o, qs, bf16, "o"),
+              (lse, ls, f32, "lse"), (do, qs, bf16, "do"), (dq_sum, qs, f32, "dq_sum"),
+              (dk_sum, kv1, f32, "dk_sum"), (dv_sum, kv1, f32, "dv_sum"))
+    _check_plan(prob, plan, q.device)
+    d = ctypes.c_void_p(256)
+    nbytes = _ws_query(lib().cp_attn_bwd_step, prob.ref, plan.ref, int(rank), int(step), d, d, d, d, d,
+                       d, d, d, d)
+    w = _workspace(nbytes, q.device, ws)
+    n = ctypes.c_size_t(nbytes)
+    _check(lib().cp_attn_bwd_step(prob.ref, plan.ref, int(rank), int(step), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(o), _ptr(lse), _ptr(do), _ptr(dq_sum), _ptr(dk_sum),
+                                  _ptr(dv_sum), _ptr(w), ctypes.byref(n) if w is not None else None,
+                                  _stream(stream)), "cp_attn_bwd_step")
+    return dq_sum, dk_sum, dv_sum
 
 
 def f32_to_bf16(x, out=None, stream=None):

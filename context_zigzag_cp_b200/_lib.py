@@ -25,7 +25,7 @@ EXPORTED = ("cp_plan_shards", "cp_unshard", "cp_attn_fwd", "cp_attn_bwd", "cp_ls
             "cp_get_device_status", "cp_set_wait_limit_ns", "cp_selftest_wait_timeout",
             "cp_launch_count", "cp_trace_begin", "cp_trace_end", "cp_selftest_exp2",
             "cp_attn_bwd_noalloc", "cp_selftest_stall", "cp_attn_fwd_rank", "cp_attn_fwd_step",
-            "cp_attn_bwd_rank", "cp_f32_to_bf16", "cp_version")
+            "cp_attn_bwd_rank", "cp_attn_bwd_step", "cp_f32_to_bf16", "cp_version")
 
 NOALLOC_MAX_ROWS = 4194304
 
@@ -93,6 +93,7 @@ def load() -> ctypes.CDLL:
     lib.cp_attn_fwd_rank.argtypes = [P, PL, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cp_attn_fwd_step.argtypes = [P, PL, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.cp_attn_bwd_rank.argtypes = [P, PL, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.cp_attn_bwd_step.argtypes = [P, PL, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cp_f32_to_bf16.argtypes = [vp, vp, ctypes.c_int64, vp]
     for name in EXPORTED:
         getattr(lib, name).restype = ctypes.c_int32

@@ -90,9 +90,14 @@ struct BwdParams {
     int32_t stall;           // test hook: the cp_kernel_t whose CTA 0 skips its first K/V load
     // Row layouts (as in FwdParams): Q, dO, dQ and the per-row workspace hold q_rows
     // rows per batch*head starting at shard position q_base; K, V hold kv_rows rows
-    // per batch*KV head starting at kv_base.  dK / dV always cover all S keys.
+    // per batch*KV head starting at kv_base (-1: only the shard visited, 2C rows).
+    // dK / dV cover all S keys, or with step_shard the visited shard's 2C keys.
     int32_t q_rows, q_base, kv_rows, kv_base;
     int32_t rank;            // -1: every rank's query rows; r: only rank r's
+    int32_t s0, s1;          // dQ pass: visit steps s0 .. s1-1 (0 .. cp: the whole visit)
+    int32_t step_shard;      // 1: the dK/dV pass covers only the shard rank `rank` visits at step s0
+    int32_t accumulate;      // 1: dq32 / dk32 / dv32 are fp32 sums that the pass adds into
+    float* dq32;             // non-null: dQ (scaled) in fp32 here instead of bf16 in dq
     float* dk32;             // non-null: dK / dV written as fp32 partials here instead of bf16
     float* dv32;
     float* dq_acc;           // one-pass backward: fp32 dQ accumulator [B*Hq][q_rows][D] (unscaled)
@@ -276,6 +281,7 @@ struct DkdvCfg {
 
 struct DkdvItem {
     int bkv, b, hk, kpos, ko;
+    int krow;                // the key tile's first row in K / V (and, with step_shard, in dK / dV)
 };
 
 // A work unit is a pair of key tiles of one KV head, original tiles p and
@@ -291,15 +297,24 @@ template <bool PD>
 __device__ __forceinline__ DkdvItem decode_dkdv(const BwdParams& P, int unit, int half)
 {
     DkdvItem it;
-    const int nkt = P.S / 128;
+    // with step_shard, the tiles of the one shard visited (zigzag pairs inside it)
+    const int nkt = P.step_shard ? 2 * P.C / 128 : P.S / 128;
     const int npair = nkt / 2;
     it.bkv = unit / npair;
     const int pidx = unit - it.bkv * npair;
     const int t = half ? nkt - 1 - pidx : pidx;
     it.b = it.bkv / P.Hkv;
     it.hk = it.bkv - it.b * P.Hkv;
-    it.ko = t * 128;
-    it.kpos = shard_of_tile<PD>(P, it.ko);
+    if (P.step_shard) {
+        const int j = __ldg(P.src + P.rank * P.cp + P.s0);
+        it.ko = tile_orig_of<PD>(P, j, t, P.C / 128);
+        it.kpos = j * 2 * P.C + t * 128;
+        it.krow = t * 128;
+    } else {
+        it.ko = t * 128;
+        it.kpos = shard_of_tile<PD>(P, it.ko);
+        it.krow = it.kpos - P.kv_base;
+    }
     return it;
 }
 
@@ -383,7 +398,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (!(P.stall == 7 /* CP_K_BWD_DKDV */ && blockIdx.x == 0 && iter == 0)) {
                     mbar_arrive_expect_tx(bar_kv_full, 2 * Cfg::TILE);
                     for (int h = 0; h < D / 64; ++h) {
-                        const int kvrow = it.bkv * P.kv_rows + (it.kpos - P.kv_base);
+                        const int kvrow = it.bkv * P.kv_rows + it.krow;
                         tma_load_2d(sK + h * 16384, &tmK, h * 64, kvrow, bar_kv_full);
                         tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);
                     }
@@ -632,7 +647,8 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             }
             if (!ok) break;
             // ---- epilogue: this group's 32 columns of dK (scaled) and dV
-            const size_t orow = static_cast<size_t>(it.bkv) * P.S + it.kpos + row;
+            const size_t orow = P.step_shard ? static_cast<size_t>(it.bkv) * 2 * P.C + it.krow + row
+                                             : static_cast<size_t>(it.bkv) * P.S + it.kpos + row;
             if (had) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_acc_full, a_phase, abort_flag));
                 if (!ok) break;
@@ -650,9 +666,16 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         float4* dk = reinterpret_cast<float4*>(P.dk32 + orow * D + 32 * wg);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            dv[i] = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
-                            dk[i] = make_float4(b[4 * i] * P.scale, b[4 * i + 1] * P.scale,
-                                                b[4 * i + 2] * P.scale, b[4 * i + 3] * P.scale);
+                            float4 x = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+                            float4 y = make_float4(b[4 * i] * P.scale, b[4 * i + 1] * P.scale,
+                                                   b[4 * i + 2] * P.scale, b[4 * i + 3] * P.scale);
+                            if (P.accumulate) {   // this CTA owns the rows: a plain read-modify-write
+                                const float4 u = dv[i], w = dk[i];
+                                x.x += u.x; x.y += u.y; x.z += u.z; x.w += u.w;
+                                y.x += w.x; y.y += w.y; y.z += w.z; y.w += w.w;
+                            }
+                            dv[i] = x;
+                            dk[i] = y;
                         }
                     } else {
                     uint4* dv = reinterpret_cast<uint4*>(P.dv + orow * D + 32 * wg);
@@ -671,7 +694,7 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty);
-            } else if (32 * wg < D) {
+            } else if (32 * wg < D && !P.accumulate) {
                 if (P.dk32) {
                     float4* dv = reinterpret_cast<float4*>(P.dv32 + orow * D + 32 * wg);
                     float4* dk = reinterpret_cast<float4*>(P.dk32 + orow * D + 32 * wg);
@@ -820,7 +843,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const DqItem it = decode_dq<PD>(P, w);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + it.qpos) : 0, it.qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + it.qpos + 127) : 0, it.qo + 127 - P.wm1);
-                for (int s = 0; s < P.cp && ok; ++s) {
+                for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -899,7 +922,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_kslot = 0;
-                for (int s = 0; s < P.cp && ok; ++s) {
+                for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -1009,7 +1032,7 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const int q_orig = it.qo + row;
             const int ds_q = max(P.docs ? __ldg(P.doc_start + it.qpos + row) : 0, q_orig - P.wm1);
             bool had = false;
-            for (int s = 0; s < P.cp && ok; ++s) {
+            for (int s = P.s0; s < P.s1 && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
                 const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -1070,6 +1093,19 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     tmem_ld32f(tdQ, a);
                     tmem_wait_ld();
                     reg_fence32f(a);
+                    if (P.dq32) {   // fp32 dQ, added into the caller's sum (this CTA owns the row)
+                        float4* dq = reinterpret_cast<float4*>(P.dq32 + rowi * D + 32 * wg);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float4 x = make_float4(a[4 * i] * P.scale, a[4 * i + 1] * P.scale,
+                                                   a[4 * i + 2] * P.scale, a[4 * i + 3] * P.scale);
+                            if (P.accumulate) {
+                                const float4 u = dq[i];
+                                x.x += u.x; x.y += u.y; x.z += u.z; x.w += u.w;
+                            }
+                            dq[i] = x;
+                        }
+                    } else {
                     uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 32 * wg);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
@@ -1077,13 +1113,19 @@ cp_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                            pack_bf16(a[8 * i + 2] * P.scale, a[8 * i + 3] * P.scale),
                                            pack_bf16(a[8 * i + 4] * P.scale, a[8 * i + 5] * P.scale),
                                            pack_bf16(a[8 * i + 6] * P.scale, a[8 * i + 7] * P.scale));
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty);
-            } else if (32 * wg < D) {
-                uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 32 * wg);
-                for (int i = 0; i < 4; ++i) dq[i] = make_uint4(0, 0, 0, 0);
+            } else if (32 * wg < D && !P.accumulate) {
+                if (P.dq32) {
+                    float4* dq = reinterpret_cast<float4*>(P.dq32 + rowi * D + 32 * wg);
+                    for (int i = 0; i < 8; ++i) dq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 32 * wg);
+                    for (int i = 0; i < 4; ++i) dq[i] = make_uint4(0, 0, 0, 0);
+                }
             }
         }
     }

@@ -150,7 +150,7 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // test hook (cp_selftest_stall): the first K/V tile of CTA 0 is never loaded
                 if (!(P.stall == 7 /* CP_K_BWD_DKDV */ && blockIdx.x == 0 && iter == 0)) {
                     mbar_arrive_expect_tx(bar_kv_full, (MODE == 1 ? 2 : 1) * Cfg::KTILE);
-                    const int kvrow = it.bkv * P.kv_rows + (it.kpos - P.kv_base);
+                    const int kvrow = it.bkv * P.kv_rows + it.krow;
                     for (int h = 0; h < D / 64; ++h) {
                         tma_load_2d(sK + h * 16384, &tmK, h * 64, kvrow, bar_kv_full);
                         if (MODE == 1) tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);
@@ -413,7 +413,8 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             if (!ok) break;
             // ---- epilogue: this group's 64 columns of dV (MODE 0) or dK (MODE 1, scaled)
-            const size_t orow = static_cast<size_t>(it.bkv) * P.S + it.kpos + row;
+            const size_t orow = P.step_shard ? static_cast<size_t>(it.bkv) * 2 * P.C + it.krow + row
+                                             : static_cast<size_t>(it.bkv) * P.S + it.kpos + row;
             const float mul = MODE == 0 ? 1.f : P.scale;
             float* out32 = MODE == 0 ? P.dv32 : P.dk32;
             __nv_bfloat16* out16 = MODE == 0 ? P.dv : P.dk;
@@ -432,9 +433,15 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     if (out32) {   // fp32 partials (one rank's share, summed across ranks later)
                         float4* dst = reinterpret_cast<float4*>(out32 + orow * D + col);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(a[4 * i] * mul, a[4 * i + 1] * mul, a[4 * i + 2] * mul,
-                                                 a[4 * i + 3] * mul);
+                        for (int i = 0; i < 8; ++i) {
+                            float4 x = make_float4(a[4 * i] * mul, a[4 * i + 1] * mul, a[4 * i + 2] * mul,
+                                                   a[4 * i + 3] * mul);
+                            if (P.accumulate) {   // this CTA owns the rows: a plain read-modify-write
+                                const float4 u = dst[i];
+                                x.x += u.x; x.y += u.y; x.z += u.z; x.w += u.w;
+                            }
+                            dst[i] = x;
+                        }
                     } else {
                         uint4* dst = reinterpret_cast<uint4*>(out16 + orow * D + col);
 #pragma unroll
@@ -448,6 +455,8 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty);
+            } else if (P.accumulate) {
+                // nothing to add
             } else if (out32) {
                 float4* dst = reinterpret_cast<float4*>(out32 + orow * D + 64 * wg);
                 for (int i = 0; i < 16; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -564,7 +573,7 @@ cp_bwd256_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 const int drow = static_cast<int>(static_cast<size_t>(it.bh) * P.q_rows + (it.qpos - P.q_base));
                 for (int h = 0; h < D / 64; ++h)
                     tma_load_2d(sdO + h * 16384, &tmdO, h * 64, drow, bar_do_full);
-                for (int s = 0; s < P.cp && ok; ++s) {
+                for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -642,7 +651,7 @@ cp_bwd256_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_kslot = 0;
-                for (int s = 0; s < P.cp && ok; ++s) {
+                for (int s = P.s0; s < P.s1 && ok; ++s) {
                     const int j = __ldg(P.src + it.r * P.cp + s);
                     const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                     for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -749,7 +758,7 @@ cp_bwd256_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const int q_orig = it.qo + row;
             const int ds_q = max(P.docs ? __ldg(P.doc_start + it.qpos + row) : 0, q_orig - P.wm1);
             bool had = false;
-            for (int s = 0; s < P.cp && ok; ++s) {
+            for (int s = P.s0; s < P.s1 && ok; ++s) {
                 const int j = __ldg(P.src + it.r * P.cp + s);
                 const KtSpan ks = kv_span<PD>(P, j, dsf, it.qo + 127 + P.nc, half);
                 for (int kt = kt_first(ks); kt < ks.b1 && ok; kt = kt_next(ks, kt)) {
@@ -806,6 +815,20 @@ cp_bwd256_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     tmem_ld32f(tdQ + 32 * h, a);
                     tmem_wait_ld();
                     reg_fence32f(a);
+                    if (P.dq32) {   // fp32 dQ, added into the caller's sum (this CTA owns the row)
+                        float4* dq = reinterpret_cast<float4*>(P.dq32 + rowi * D + 64 * wg + 32 * h);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float4 x = make_float4(a[4 * i] * P.scale, a[4 * i + 1] * P.scale,
+                                                   a[4 * i + 2] * P.scale, a[4 * i + 3] * P.scale);
+                            if (P.accumulate) {
+                                const float4 u = dq[i];
+                                x.x += u.x; x.y += u.y; x.z += u.z; x.w += u.w;
+                            }
+                            dq[i] = x;
+                        }
+                        continue;
+                    }
                     uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 64 * wg + 32 * h);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
@@ -817,9 +840,14 @@ cp_bwd256_dq_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty);
-            } else {
-                uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 64 * wg);
-                for (int i = 0; i < 8; ++i) dq[i] = make_uint4(0, 0, 0, 0);
+            } else if (!P.accumulate) {
+                if (P.dq32) {
+                    float4* dq = reinterpret_cast<float4*>(P.dq32 + rowi * D + 64 * wg);
+                    for (int i = 0; i < 16; ++i) dq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    uint4* dq = reinterpret_cast<uint4*>(P.dq + rowi * D + 64 * wg);
+                    for (int i = 0; i < 8; ++i) dq[i] = make_uint4(0, 0, 0, 0);
+                }
             }
         }
     }

@@ -146,7 +146,7 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // test hook (cp_selftest_stall): the first K/V tile of CTA 0 is never loaded
                 if (!(P.stall == 12 /* CP_K_BWD_FUSED */ && blockIdx.x == 0 && iter == 0)) {
                     mbar_arrive_expect_tx(bar_kv_full, 2 * Cfg::TILE);
-                    const int kvrow = it.bkv * P.kv_rows + (it.kpos - P.kv_base);
+                    const int kvrow = it.bkv * P.kv_rows + it.krow;
                     for (int h = 0; h < D / 64; ++h) {
                         tma_load_2d(sK + h * 16384, &tmK, h * 64, kvrow, bar_kv_full);
                         tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);

@@ -634,7 +634,8 @@ template <int D>
 cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                        const void* v, const void* o, const float* lse, const void* dout, void* dq,
                        void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream,
-                       int stall, const Layout& L, float* dk32, float* dv32, float* dq_acc)
+                       int stall, const Layout& L, float* dk32, float* dv32, float* dq_acc,
+                       float* dq32 = nullptr, bool ring_step = false)
 {
     // dq_acc non-null: the one-pass backward (cp_bwd_fused_kernel + dq_convert_kernel);
     // null: the two deterministic passes (cp_bwd_dkdv_kernel, cp_bwd_dq_kernel)
@@ -688,6 +689,13 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
     P.dk32 = dk32;
     P.dv32 = dv32;
     P.dq_acc = dq_acc;
+    P.s0 = L.s0;
+    P.s1 = L.s1;
+    // one ring step: the dK/dV pass covers the shard visited at that step, and dQ, dK,
+    // dV are added into the caller's fp32 sums
+    P.step_shard = ring_step;
+    P.accumulate = ring_step;
+    P.dq32 = dq32;
     P.tile_orig = tables_orig(p, pl);
     P.tile_shard = tables_shard(p, pl);
     const bool pd = p->shard == CP_SHARD_PER_DOC;
@@ -714,7 +722,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
             return e;
         });
         if (ast != CP_OK) return ast;
-        P.n_items = B * Hkv * (S / 256);   // pairs of key tiles
+        P.n_items = B * Hkv * (ring_step ? P.C / 128 : S / 256);   // pairs of key tiles
         const int grid_kv = std::min(P.n_items, num_sms());
         {
             LaunchScope ls(CP_K_BWD_DKDV, stream);
@@ -745,7 +753,7 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
         return e;
     });
     if (ast != CP_OK) return ast;
-    P.n_items = B * Hkv * (S / 256);   // pairs of key tiles (S / 128 is even)
+    P.n_items = B * Hkv * (ring_step ? P.C / 128 : S / 256);   // pairs of key tiles (S / 128 is even)
     if (dq_acc) {
         const cp_status_t fst = ensure_attr(D == 128 ? ATTR_FUSED128 : ATTR_FUSED64, [] {
             cudaError_t e = cudaFuncSetAttribute(cp_bwd_fused_kernel<D, false>,
@@ -790,18 +798,19 @@ cp_status_t launch_bwd(const cp_problem_t* p, const cp_plan_t* pl, const void* q
 cp_status_t launch_bwd_any(const cp_problem_t* p, const cp_plan_t* pl, const void* q, const void* k,
                            const void* v, const void* o, const float* lse, const void* dout, void* dq,
                            void* dk, void* dv, float* delta, float* nlse2, cudaStream_t stream,
-                           int stall, const Layout& L, float* dk32, float* dv32, float* dq_acc)
+                           int stall, const Layout& L, float* dk32, float* dv32, float* dq_acc,
+                           float* dq32 = nullptr, bool ring_step = false)
 {
     switch (p->head_dim) {
     case 256:
         return launch_bwd<256>(p, pl, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, stream, stall, L,
-                               dk32, dv32, dq_acc);
+                               dk32, dv32, dq_acc, dq32, ring_step);
     case 128:
         return launch_bwd<128>(p, pl, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, stream, stall, L,
-                               dk32, dv32, dq_acc);
+                               dk32, dv32, dq_acc, dq32, ring_step);
     default:
         return launch_bwd<64>(p, pl, q, k, v, o, lse, dout, dq, dk, dv, delta, nlse2, stream, stall, L,
-                              dk32, dv32, dq_acc);
+                              dk32, dv32, dq_acc, dq32, ring_step);
     }
 }
 
@@ -1007,6 +1016,29 @@ extern "C" cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_pl
     cudaStream_t s = as_stream(stream);
     const Layout L = rank_layout(problem, rank, -1);
     return launch_bwd_any(problem, plan, q, k, v, o, lse, dout, dq, nullptr, nullptr, delta, nlse2, s, 0, L, dk_part, dv_part, nullptr);
+}
+
+extern "C" cp_status_t cp_attn_bwd_step(const cp_problem_t* problem, const cp_plan_t* plan,
+                                        int32_t rank, int32_t step, const void* q, const void* k,
+                                        const void* v, const void* o, const float* lse,
+                                        const void* dout, float* dq_sum, float* dk_sum, float* dv_sum,
+                                        void* ws, size_t* ws_bytes, void* stream)
+{
+    cp_status_t st = check_rank_call(problem, plan, rank, step, true);
+    if (st != CP_OK) return st;
+    const void* ptrs[] = {q, k, v, o, lse, dout, dq_sum, dk_sum, dv_sum};
+    for (const void* x : ptrs)
+        if (!x || !aligned16(x)) return CP_ERR_INVALID_ARG;
+    const int n2c = problem->seq_len / problem->cp_size;
+    const int64_t rows = static_cast<int64_t>(problem->batch) * problem->num_heads * n2c;
+    const size_t row_bytes = round_up(size_t(rows) * 4, 256);
+    if (workspace_gate(2 * row_bytes, ws, ws_bytes, &st)) return st;
+    float* delta = static_cast<float*>(ws);
+    float* nlse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + row_bytes);
+    cudaStream_t s = as_stream(stream);
+    const Layout L = rank_layout(problem, rank, step);   // rank r's rows, the one shard of the step
+    return launch_bwd_any(problem, plan, q, k, v, o, lse, dout, nullptr, nullptr, nullptr, delta, nlse2, s, 0,
+                          L, dk_sum, dv_sum, nullptr, dq_sum, true);
 }
 
 extern "C" cp_status_t cp_f32_to_bf16(const float* in, void* out, int64_t n, void* stream)

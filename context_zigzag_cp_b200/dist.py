@@ -14,10 +14,18 @@ its "all-to-all vs all-gather" section:
     and receives the next one from rank r-1, and the cp partials are combined
     by the LSE-merge kernel (cp_lse_merge).
 
-The backward gathers K/V (both orders; every rank's queries see every shard),
-computes dQ_r and rank r's fp32 share of dK/dV for every key
-(cp_attn_bwd_rank), and a reduce-scatter hands rank j the sum for its shard j,
-cast to bf16 by cp_f32_to_bf16.
+The backward takes the same two orders:
+
+  * all-gather: K/V gathered, dQ_r and rank r's fp32 share of dK/dV for every
+    key in one call (cp_attn_bwd_rank), and a reduce-scatter hands rank j the
+    sum for its shard j;
+  * ring: cp steps (cp_attn_bwd_step); the shard visited at step s comes with
+    its fp32 dK/dV sums, the step adds rank r's share into them and into its
+    own fp32 dQ, and the sums travel on with the shard (one hop per step; after
+    the last step one more hop hands every shard's sums back to its owner).
+    No rank ever holds more than one other shard.
+
+Both cast the fp32 sums to bf16 with cp_f32_to_bf16.
 
 The library moves no data between GPUs; this module runs the collectives with
 torch.distributed (NCCL on GPUs).  The kernel calls go through a `kernels`
@@ -29,8 +37,8 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (Plan, Problem, attn_bwd_rank, attn_fwd_rank, attn_fwd_step, f32_to_bf16,
-               lse_merge)
+from . import (Plan, Problem, attn_bwd_rank, attn_bwd_step, attn_fwd_rank, attn_fwd_step,
+               f32_to_bf16, lse_merge)
 
 
 class LibraryKernels:
@@ -47,6 +55,9 @@ class LibraryKernels:
 
     def bwd_rank(self, prob, plan, rank, q, k_all, v_all, o, lse, do):
         return attn_bwd_rank(prob, plan, rank, q, k_all, v_all, o, lse, do)
+
+    def bwd_step(self, prob, plan, rank, step, q, k, v, o, lse, do, dq_sum, dk_sum, dv_sum):
+        attn_bwd_step(prob, plan, rank, step, q, k, v, o, lse, do, dq_sum, dk_sum, dv_sum)
 
     def to_bf16(self, x):
         return f32_to_bf16(x)
@@ -99,19 +110,11 @@ class ContextParallel:
 
     def _ring_forward(self, q, k, v):
         r, cp = self.rank, self.cp
-        nxt, prv = (r + 1) % cp, (r - 1) % cp
         kv = torch.stack([k, v]).contiguous()
         parts_o, parts_l = [], []
         for s in range(cp):
-            pending = None
-            if s + 1 < cp:
-                # pass the held shard on while this step computes with it
-                recv = torch.empty_like(kv)
-                ops = [dist.P2POp(dist.isend, kv, dist.get_global_rank(self.group, nxt)
-                                  if self.group is not None else nxt, self.group),
-                       dist.P2POp(dist.irecv, recv, dist.get_global_rank(self.group, prv)
-                                  if self.group is not None else prv, self.group)]
-                pending = (dist.batch_isend_irecv(ops), recv)
+            # pass the held shard on while this step computes with it
+            pending = self._shift(kv) if s + 1 < cp else None
             o_s, l_s = self.kernels.fwd_step(self.prob, self.plan, r, s, q, kv[0], kv[1])
             parts_o.append(o_s)
             parts_l.append(l_s)
@@ -125,8 +128,20 @@ class ContextParallel:
         o, lse = self.kernels.merge(o_parts, l_parts)
         return o.view(B, H, n2c, D), lse.view(B, H, n2c)
 
+    def _peer(self, r):
+        return dist.get_global_rank(self.group, r) if self.group is not None else r
+
+    def _shift(self, x):
+        """Send x to rank r+1 and return what rank r-1 sent (the ring's one hop)."""
+        recv = torch.empty_like(x)
+        ops = [dist.P2POp(dist.isend, x, self._peer((self.rank + 1) % self.cp), self.group),
+               dist.P2POp(dist.irecv, recv, self._peer((self.rank - 1) % self.cp), self.group)]
+        return dist.batch_isend_irecv(ops), recv
+
     def backward(self, q, k, v, o, lse, do):
         """Rank r's (dQ_r, dK_r, dV_r) from its local shards and the upstream dO_r."""
+        if self.prob.rotate == "ring":
+            return self._ring_backward(q, k, v, o, lse, do)
         k_all = _gather_shards(k, self.cp, self.group)
         v_all = _gather_shards(v, self.cp, self.group)
         dq, dk_part, dv_part = self.kernels.bwd_rank(self.prob, self.plan, self.rank, q, k_all,
@@ -134,3 +149,26 @@ class ContextParallel:
         dk = self.kernels.to_bf16(_reduce_scatter_shards(dk_part, self.cp, self.group))
         dv = self.kernels.to_bf16(_reduce_scatter_shards(dv_part, self.cp, self.group))
         return dq, dk, dv
+
+    def _ring_backward(self, q, k, v, o, lse, do):
+        # step s: rank r holds shard (r - s) mod cp with that shard's dK/dV sums so far
+        r, cp = self.rank, self.cp
+        kv = torch.stack([k, v]).contiguous()
+        acc = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)   # dK, dV sums
+        dq = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
+        for s in range(cp):
+            pending = self._shift(kv) if s + 1 < cp else None   # overlaps the step
+            self.kernels.bwd_step(self.prob, self.plan, r, s, q, kv[0], kv[1], o, lse, do, dq,
+                                  acc[0], acc[1])
+            # the sums move on with their shard; after the last step this hop brings
+            # rank r its own shard's sums, completed by every rank
+            if cp > 1:
+                works, acc = self._shift(acc)
+                for w in works:
+                    w.wait()
+            if pending is not None:
+                for w in pending[0]:
+                    w.wait()
+                kv = pending[1]
+        return (self.kernels.to_bf16(dq), self.kernels.to_bf16(acc[0].contiguous()),
+                self.kernels.to_bf16(acc[1].contiguous()))

@@ -374,6 +374,29 @@ CP_API cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_plan_t
                                     float* dk_part, float* dv_part, void* ws, size_t* ws_bytes,
                                     void* stream);
 
+/*
+ * cp_attn_bwd_step -- one step of the ring form of the backward: rank r's
+ * queries against the single K/V shard j = src[r][step] it holds at that step,
+ * their gradients added into fp32 sums:
+ *   q, o, dout      bf16 [B][Hq][2C][D], lse fp32 [B][Hq][2C]   rank r's shard
+ *   k, v            bf16 [B][Hkv][2C][D]                         shard j
+ *   dq_sum          fp32 [B][Hq][2C][D]   rank r's dQ, this step's share added
+ *   dk_sum, dv_sum  fp32 [B][Hkv][2C][D]  shard j's dK / dV, rank r's share added
+ * The sums are read and written (the caller zeroes them first).  In a ring the
+ * dK / dV sums travel with the K/V shard: after the cp steps (and one more hop)
+ * every shard's sums have been added to by every rank and are back with their
+ * owner; cp_f32_to_bf16 casts them (and dq_sum).  Two passes (a dK/dV pass over
+ * shard j's keys, a dQ pass over that step) whatever problem->bwd_one_pass says.
+ * Workspace: two fp32 values per local query row (as cp_attn_bwd_rank).
+ * Errors: as cp_attn_bwd; CP_ERR_INVALID_ARG for rank or step outside
+ * [0, cp_size).
+ */
+CP_API cp_status_t cp_attn_bwd_step(const cp_problem_t* problem, const cp_plan_t* plan,
+                                    int32_t rank, int32_t step, const void* q, const void* k,
+                                    const void* v, const void* o, const float* lse,
+                                    const void* dout, float* dq_sum, float* dk_sum, float* dv_sum,
+                                    void* ws, size_t* ws_bytes, void* stream);
+
 /* out[i] = bf16(in[i]) (round to nearest even) for n floats; n a multiple of 4, in
  * 16-byte and out 8-byte aligned. */
 CP_API cp_status_t cp_f32_to_bf16(const float* in, void* out, int64_t n, void* stream);

@@ -1,6 +1,7 @@
 """Context parallelism across processes (context_zigzag_cp_b200.dist) with gloo on
-CPU, world size 2: the K/V exchange (all-gather, ring send/recv), the order of the
-steps and of the merge, and the reduce-scatter of dK/dV, end to end.  The
+CPU, world sizes 2 and 3: the K/V exchange (all-gather, ring send/recv), the order
+of the steps and of the merge, the reduce-scatter of dK/dV (all-gather order)
+and the dK/dV sums that travel with their shard (ring order), end to end.  The
 per-rank kernels are stood in by the oracle (the library's own per-rank calls
 are checked on a GPU by test_rank_gpu.py); each rank ends up with its shard of
 O, LSE, dQ, dK, dV, and rank 0 compares the reassembled result with the oracle's
@@ -17,7 +18,7 @@ import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-B, HQ, HKV, S, D = 1, 4, 2, 128, 8
+B, HQ, HKV, D = 1, 4, 2, 8
 
 
 def _free_port():
@@ -34,19 +35,19 @@ class OracleKernels:
     K/V rows handed to it; they are placed at their original positions (from the
     plan's perm) in otherwise-zero full-length arrays for the oracle."""
 
-    def __init__(self, pl, ds, cp):
+    def __init__(self, pl, ds, cp, S):
         import oracle
-        self.o, self.pl, self.ds, self.cp = oracle, pl, ds, cp
+        self.o, self.pl, self.ds, self.cp, self.S = oracle, pl, ds, cp, S
         self.n2c = S // cp
 
     def _place(self, x, shard, nheads):
-        full = np.zeros((B, nheads, S, D))
+        full = np.zeros((B, nheads, self.S, D))
         pos = self.pl["perm"][shard * self.n2c:(shard + 1) * self.n2c]
         full[:, :, pos] = x.double().numpy()
         return full
 
     def _all(self, x_all, nheads):
-        full = np.zeros((B, nheads, S, D))
+        full = np.zeros((B, nheads, self.S, D))
         full[:, :, self.pl["perm"]] = x_all.double().numpy()
         return full
 
@@ -74,8 +75,7 @@ class OracleKernels:
     def bwd_rank(self, prob, plan, rank, q, k_all, v_all, o, lse, do):
         # rows of other ranks carry dO = 0: they add nothing to dK / dV
         qf, of, dof = (self._place(x, rank, HQ) for x in (q, o, do))
-        lf = np.zeros((B, HQ, S))
-        lf[:, :, self.pl["perm"][rank * self.n2c:(rank + 1) * self.n2c]] = lse.double().numpy()
+        lf = self._place_lse(lse, rank)
         dq, dk, dv = self.o.bwd(qf, self._all(k_all, HKV), self._all(v_all, HKV), of, lf, dof,
                                 self.ds)
         pos = self.pl["perm"][rank * self.n2c:(rank + 1) * self.n2c]
@@ -83,13 +83,32 @@ class OracleKernels:
                 torch.from_numpy(dk[:, :, self.pl["perm"]]).float(),
                 torch.from_numpy(dv[:, :, self.pl["perm"]]).float())
 
+    def _place_lse(self, lse, rank):
+        lf = np.zeros((B, HQ, self.S))
+        lf[:, :, self.pl["perm"][rank * self.n2c:(rank + 1) * self.n2c]] = lse.double().numpy()
+        return lf
+
+    def bwd_step(self, prob, plan, rank, step, q, k, v, o, lse, do, dq_sum, dk_sum, dv_sum):
+        # keys outside shard j are zero rows of K and V: with P taken from the true LSE
+        # they add nothing to dQ, and only shard j's dK / dV rows are read back
+        j = int(self.pl["src"][rank * self.cp + step])
+        qf, of, dof = (self._place(x, rank, HQ) for x in (q, o, do))
+        dq, dk, dv = self.o.bwd(qf, self._place(k, j, HKV), self._place(v, j, HKV), of,
+                                self._place_lse(lse, rank), dof, self.ds)
+        pos_r = self.pl["perm"][rank * self.n2c:(rank + 1) * self.n2c]
+        pos_j = self.pl["perm"][j * self.n2c:(j + 1) * self.n2c]
+        dq_sum += torch.from_numpy(dq[:, :, pos_r]).float()
+        dk_sum += torch.from_numpy(dk[:, :, pos_j]).float()
+        dv_sum += torch.from_numpy(dv[:, :, pos_j]).float()
+
     def to_bf16(self, x):
         return x.to(torch.bfloat16)
 
 
-# documents for the per-document runs: lengths multiples of 2cp = 4, so every
-# document is cut into four chunks of whole rows
-CU_DOC = [0, 20, 32, 84, 128]
+# documents for the per-document runs: lengths multiples of 2cp, so every
+# document is cut into 2cp chunks of whole rows
+CU_DOC = {2: [0, 20, 32, 84, 128], 3: [0, 48, 66, 150, 192]}
+SEQ = {2: 128, 3: 192}     # S / 2cp whole rows per chunk
 
 
 def _worker(rank, world, port, rotate, shard, q_out):
@@ -103,14 +122,15 @@ def _worker(rank, world, port, rotate, shard, q_out):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     cp = world
-    cu = CU_DOC if shard == "doc" else None
+    S = SEQ[cp]
+    cu = CU_DOC[cp] if shard == "doc" else None
     pl = oracle.plan(S, cp, rotate, cu, shard=shard)
     ds = oracle.doc_start(S, cu)
     t = synth.attn_inputs(B, HQ, HKV, S, D, seed=91, with_dout=True)   # the same on every rank
     n2c = S // cp
     local = lambda x: x[:, :, pl["perm"][rank * n2c:(rank + 1) * n2c]].contiguous()
     prob = cz.Problem(B, S, cp, HQ, HKV, D, rotate)
-    ctx = ContextParallel(prob, kernels=OracleKernels(pl, ds, cp), plan=object())
+    ctx = ContextParallel(prob, kernels=OracleKernels(pl, ds, cp, S), plan=object())
     o, lse = ctx.forward(local(t["q"]), local(t["k"]), local(t["v"]))
     dq, dk, dv = ctx.backward(local(t["q"]), local(t["k"]), local(t["v"]), o, lse, local(t["do"]))
     outs = [None] * world
@@ -124,13 +144,16 @@ def _worker(rank, world, port, rotate, shard, q_out):
 # shard "doc": the driver with a per-document plan (the permutation and the
 # document mask change; the exchange, the merge order and the reduce-scatter
 # are the same)
-@pytest.mark.parametrize("rotate,shard", [("allgather", "sequence"), ("ring", "sequence"),
-                                          ("ring", "doc")])
-def test_two_ranks_match_unsharded(rotate, shard):
+# world 3: the ring's direction matters (rank r+1 and rank r-1 differ)
+@pytest.mark.parametrize("world,rotate,shard", [(2, "allgather", "sequence"), (2, "ring", "sequence"),
+                                                (2, "ring", "doc"), (3, "ring", "sequence"),
+                                                (3, "ring", "doc"), (3, "allgather", "doc")])
+def test_ranks_match_unsharded(world, rotate, shard):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, rotate, shard, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, rotate, shard, q))
+             for r in range(world)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=240) for _ in procs)
@@ -142,16 +165,17 @@ def test_two_ranks_match_unsharded(rotate, shard):
     import oracle
     import synth
     from helpers import assert_bf16_close, assert_lse_close
+    S = SEQ[world]
     t = synth.attn_inputs(B, HQ, HKV, S, D, seed=91, with_dout=True)
     f = lambda x: x.double().numpy()
-    cu = CU_DOC if shard == "doc" else None
+    cu = CU_DOC[world] if shard == "doc" else None
     ds = oracle.doc_start(S, cu)
     ro, rl = oracle.fwd(f(t["q"]), f(t["k"]), f(t["v"]), ds)
     rq, rk, rv = oracle.bwd(f(t["q"]), f(t["k"]), f(t["v"]), ro, rl, f(t["do"]), ds)
-    perm = oracle.plan(S, 2, rotate, cu, shard=shard)["perm"]
-    cat = lambda n: np.concatenate([outs[r][n] for r in range(2)], axis=2).astype(np.float64)
-    assert_bf16_close(cat("o"), ro[:, :, perm], f"O two ranks {rotate} {shard}")
-    assert_lse_close(cat("lse"), rl[:, :, perm], f"LSE two ranks {rotate} {shard}")
-    assert_bf16_close(cat("dq"), rq[:, :, perm], f"dQ two ranks {rotate} {shard}")
-    assert_bf16_close(cat("dk"), rk[:, :, perm], f"dK two ranks {rotate} {shard}")
-    assert_bf16_close(cat("dv"), rv[:, :, perm], f"dV two ranks {rotate} {shard}")
+    perm = oracle.plan(S, world, rotate, cu, shard=shard)["perm"]
+    cat = lambda n: np.concatenate([outs[r][n] for r in range(world)], axis=2).astype(np.float64)
+    assert_bf16_close(cat("o"), ro[:, :, perm], f"O {world} ranks {rotate} {shard}")
+    assert_lse_close(cat("lse"), rl[:, :, perm], f"LSE {world} ranks {rotate} {shard}")
+    assert_bf16_close(cat("dq"), rq[:, :, perm], f"dQ {world} ranks {rotate} {shard}")
+    assert_bf16_close(cat("dk"), rk[:, :, perm], f"dK {world} ranks {rotate} {shard}")
+    assert_bf16_close(cat("dv"), rv[:, :, perm], f"dV {world} ranks {rotate} {shard}")
