@@ -266,3 +266,40 @@ def test_problem_shard_option(cpu_binding):
     windowed = cz.Problem(B, S, CP, Hq, Hkv, D, window=64)
     with pytest.raises(ValueError, match="window"):
         cz.attn_fwd(windowed, _cpu_plan(p), *args)
+
+
+def _rank_tensors():
+    n2c = S // CP
+    q = torch.zeros(B, Hq, n2c, D, dtype=bf16)
+    k = torch.zeros(B, Hkv, n2c, D, dtype=bf16)
+    return dict(q=q, k=k, v=k.clone(), o=q.clone(), lse=torch.zeros(B, Hq, n2c, dtype=f32),
+                do=q.clone(), dq_sum=torch.zeros(q.shape, dtype=f32),
+                dk_sum=torch.zeros(k.shape, dtype=f32), dv_sum=torch.zeros(k.shape, dtype=f32))
+
+
+def _bwd_step(t):
+    return cz.attn_bwd_step(prob(), None, 0, 0, t["q"], t["k"], t["v"], t["o"], t["lse"], t["do"],
+                            t["dq_sum"], t["dk_sum"], t["dv_sum"])
+
+
+@pytest.mark.parametrize("name,bad,what", [
+    ("dq_sum", lambda t: t["dq_sum"].to(bf16), "dtype"),            # the sums are fp32
+    ("dk_sum", lambda t: torch.zeros(B, Hkv, S, D, dtype=f32), "shape"),   # one shard, not all S
+    ("k", lambda t: torch.zeros(B, Hkv, S, D, dtype=bf16), "shape"),       # the one shard held
+    ("lse", lambda t: t["lse"].to(bf16), "dtype"),
+    ("o", lambda t: torch.zeros(B, Hq, S, D, dtype=bf16), "shape")])
+def test_bwd_step_rejects(name, bad, what):
+    """cp_attn_bwd_step: rank-local q/o/do/lse, one K/V shard, fp32 sums of the same shapes."""
+    t = _rank_tensors()
+    t[name] = bad(t)
+    with pytest.raises(ValueError, match=what):
+        _bwd_step(t)
+
+
+def test_bwd_step_needs_every_sum():
+    t = _rank_tensors()
+    t["dv_sum"] = None
+    with pytest.raises(ValueError, match="dv_sum"):
+        _bwd_step(t)
+    with pytest.raises(ValueError, match="CUDA device"):   # right shapes: stops at the device check
+        _bwd_step(_rank_tensors())
