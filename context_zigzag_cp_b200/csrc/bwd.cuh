@@ -247,6 +247,21 @@ __device__ __forceinline__ int dkdv_last_tile(const BwdParams& P, int ko, int nt
     }
     return t_end;
 }
+// The order in which a work unit's half visits its key tile's query tiles
+// [t0, t1): u runs over [u0, u1) and the query tile is |u|.  The first half's key
+// tile (attended by the long run of query tiles from its own position to the end)
+// walks them from the end down (u from 1 - t1 to -t0), the second half's (the
+// short run at the end) upwards (u = t).  Every CTA of a wave starts its two halves
+// at the same times, so at any moment the first halves all read one query tile
+// and the second halves another, each from L2 after its first reader; walked
+// upwards, the first halves would read a window as wide as the wave.
+struct DkdvWalk {
+    int u0, u1;
+};
+__device__ __forceinline__ DkdvWalk dkdv_walk(int t0, int t1, int iter)
+{
+    return (iter & 1) ? DkdvWalk{t0, t1} : DkdvWalk{1 - t1, 1 - t0};
+}
 // True when the query tile at shard position qpos belongs to the rank the pass
 // runs for (always, for a whole-sequence pass).
 __device__ __forceinline__ bool q_tile_on_rank(const BwdParams& P, int qpos)
@@ -403,8 +418,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);
                     }
                 }
-                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                    const int qo = t * 128;
+                const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+                for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                    const int qo = abs(u) * 128;
                     const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
@@ -500,8 +516,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0;
-                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                    const int qo = t * 128;
+                const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+                for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                    const int qo = abs(u) * 128;
                     const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
@@ -583,8 +600,9 @@ cp_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                const int qo = t * 128;
+            const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+            for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                const int qo = abs(u) * 128;
                 const int qpos = shard_of_tile<PD>(P, qo);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);

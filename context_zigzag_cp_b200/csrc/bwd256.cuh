@@ -156,10 +156,12 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         if (MODE == 1) tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);
                     }
                 }
-                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                    const int qpos128 = shard_of_tile<PD>(P, t * 128);
+                const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+                for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                    const int tq = abs(u);
+                    const int qpos128 = shard_of_tile<PD>(P, tq * 128);
                     for (int qh = 0; qh < 2 && ok; ++qh) {
-                        const int qo = t * 128 + 64 * qh, qpos = qpos128 + 64 * qh;
+                        const int qo = tq * 128 + 64 * qh, qpos = qpos128 + 64 * qh;
                         const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                         const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 63) : 0, qo + 63 - P.wm1);
                         if (classify_q64(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qpos))
@@ -245,10 +247,12 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tc_fence_after();
                 bool first = true, prev_live = false;
                 uint32_t prev_qs = 0, prev_ds = 0, prev_dpar = 0, prev_pb = 0;
-                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                    const int qpos128 = shard_of_tile<PD>(P, t * 128);
+                const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+                for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                    const int tq = abs(u);
+                    const int qpos128 = shard_of_tile<PD>(P, tq * 128);
                     for (int qh = 0; qh < 2 && ok; ++qh) {
-                        const int qo = t * 128 + 64 * qh, qpos = qpos128 + 64 * qh;
+                        const int qo = tq * 128 + 64 * qh, qpos = qpos128 + 64 * qh;
                         const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                         const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 63) : 0, qo + 63 - P.wm1);
                         if (classify_q64(qo, dsf, dsl, it.ko, P.nc) == TILE_SKIP || !q_tile_on_rank(P, qpos))
@@ -338,10 +342,12 @@ cp_bwd256_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                const int qpos128 = shard_of_tile<PD>(P, t * 128);
+            const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+            for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                const int tq = abs(u);
+                const int qpos128 = shard_of_tile<PD>(P, tq * 128);
                 for (int qh = 0; qh < 2 && ok; ++qh) {
-                    const int qo = t * 128 + 64 * qh, qpos = qpos128 + 64 * qh;
+                    const int qo = tq * 128 + 64 * qh, qpos = qpos128 + 64 * qh;
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 63) : 0, qo + 63 - P.wm1);
                     const int cls = classify_q64(qo, dsf, dsl, it.ko, P.nc);

@@ -152,8 +152,9 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         tma_load_2d(sV + h * 16384, &tmV, h * 64, kvrow, bar_kv_full);
                     }
                 }
-                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                    const int qo = t * 128;
+                const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+                for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                    const int qo = abs(u) * 128;
                     const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
@@ -220,8 +221,9 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (!ok) break;
                 tc_fence_after();
                 bool first = true;
-                for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                    const int qo = t * 128;
+                const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+                for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                    const int qo = abs(u) * 128;
                     const int qpos = shard_of_tile<PD>(P, qo);
                     const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                     const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
@@ -338,8 +340,9 @@ cp_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const DkdvItem it = decode_dkdv<PD>(P, w, iter & 1);
             const int k_orig = it.ko + row;
             bool had = false;
-            for (int t = max(0, it.ko - P.nc) / 128, t_end = dkdv_last_tile(P, it.ko, ntq); t < t_end && ok; ++t) {
-                const int qo = t * 128;
+            const DkdvWalk wk = dkdv_walk(max(0, it.ko - P.nc) / 128, dkdv_last_tile(P, it.ko, ntq), iter);
+            for (int u = wk.u0; u < wk.u1 && ok; ++u) {
+                const int qo = abs(u) * 128;
                 const int qpos = shard_of_tile<PD>(P, qo);
                 const int dsf = max(P.docs ? __ldg(P.doc_start + qpos) : 0, qo - P.wm1);
                 const int dsl = max(P.docs ? __ldg(P.doc_start + qpos + 127) : 0, qo + 127 - P.wm1);
