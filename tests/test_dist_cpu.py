@@ -107,8 +107,8 @@ class OracleKernels:
 
 # documents for the per-document runs: lengths multiples of 2cp, so every
 # document is cut into 2cp chunks of whole rows
-CU_DOC = {2: [0, 20, 32, 84, 128], 3: [0, 48, 66, 150, 192]}
-SEQ = {2: 128, 3: 192}     # S / 2cp whole rows per chunk
+CU_DOC = {1: [0, 20, 32, 84, 128], 2: [0, 20, 32, 84, 128], 3: [0, 48, 66, 150, 192]}
+SEQ = {1: 128, 2: 128, 3: 192}     # S / 2cp whole rows per chunk
 
 
 def _worker(rank, world, port, rotate, shard, q_out):
@@ -144,8 +144,10 @@ def _worker(rank, world, port, rotate, shard, q_out):
 # shard "doc": the driver with a per-document plan (the permutation and the
 # document mask change; the exchange, the merge order and the reduce-scatter
 # are the same)
-# world 3: the ring's direction matters (rank r+1 and rank r-1 differ)
-@pytest.mark.parametrize("world,rotate,shard", [(2, "allgather", "sequence"), (2, "ring", "sequence"),
+# world 3: the ring's direction matters (rank r+1 and rank r-1 differ); world 1:
+# a ring of one rank has no hop
+@pytest.mark.parametrize("world,rotate,shard", [(1, "ring", "sequence"), (1, "allgather", "doc"),
+                                                (2, "allgather", "sequence"), (2, "ring", "sequence"),
                                                 (2, "ring", "doc"), (3, "ring", "sequence"),
                                                 (3, "ring", "doc"), (3, "allgather", "doc")])
 def test_ranks_match_unsharded(world, rotate, shard):
