@@ -219,6 +219,42 @@ def test_sharded_merged_equals_unsharded(cp, rotate, docs):
     np.testing.assert_allclose(sl, lse[:, :, perm], atol=1e-12)
 
 
+@pytest.mark.parametrize("cp,S,docs,shard", [(3, 72, None, "sequence"),
+                                             (2, 64, [0, 3, 40, 41, 64], "sequence"),
+                                             (2, 64, [0, 16, 24, 64], "doc")])
+def test_bwd_ring_steps_sum_to_whole(cp, S, docs, shard):
+    """The backward split by ring step: rank r's queries against the one shard j =
+    src[r][s] it holds at step s (every other key's K, V rows zero, P taken from the
+    final LSE) give pieces of the gradients; over the steps the pieces of dQ_r, and
+    over the ranks those of dK_j / dV_j, add up to the unsharded gradients, and
+    leaving out the last step's pieces does not."""
+    D = 8
+    q, k, v, do = rnd((1, 4, S, D), 24), rnd((1, 2, S, D), 25), rnd((1, 2, S, D), 26), rnd((1, 4, S, D), 27)
+    cu = None if docs is None else np.array(docs, np.int32)
+    ds = oracle.doc_start(S, cu)
+    o, lse = oracle.fwd(q, k, v, ds)
+    rq, rk, rv = oracle.bwd(q, k, v, o, lse, do, ds)
+    pl = oracle.plan(S, cp, "ring", cu, shard=shard)
+    perm, src, n2c = pl["perm"], pl["src"], S // cp
+    rows = lambda r: perm[r * n2c:(r + 1) * n2c]
+    keep = lambda x, p: np.where(np.isin(np.arange(S), p)[None, None, :, None], x, 0.0)
+    got = [np.zeros_like(rq), np.zeros_like(rk), np.zeros_like(rv)]
+    last = [np.zeros_like(rq), np.zeros_like(rk), np.zeros_like(rv)]
+    for s in range(cp):
+        for r in range(cp):
+            j = int(src[r * cp + s])
+            lr = np.where(np.isin(np.arange(S), rows(r))[None, None, :], lse, 0.0)
+            gq, gk, gv = oracle.bwd(keep(q, rows(r)), keep(k, rows(j)), keep(v, rows(j)),
+                                    keep(o, rows(r)), lr, keep(do, rows(r)), ds)
+            for acc in ([got] + ([last] if s == cp - 1 else [])):
+                acc[0][:, :, rows(r)] += gq[:, :, rows(r)]
+                acc[1][:, :, rows(j)] += gk[:, :, rows(j)]
+                acc[2][:, :, rows(j)] += gv[:, :, rows(j)]
+    for g, ref in zip(got, (rq, rk, rv)):
+        np.testing.assert_allclose(g, ref, atol=1e-12)
+    assert max(np.abs(g - l - ref).max() for g, l, ref in zip(got, last, (rq, rk, rv))) > 1e-2
+
+
 def test_local_only_attention_breaks_parity():
     """If only the local shard is attended (CP communication silently off), the result
     is wrong: dropping steps s > 0 must fail parity."""
