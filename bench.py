@@ -428,29 +428,33 @@ def run_native(args, w, rank, world, local_rank):
 
     # The same work as step(), step after step, with the copies pipelined the way a
     # training loop would run them: the device holds two sets of input and gradient
-    # buffers, step i+1's Q, K, V, dO go up on a side stream while step i computes,
-    # and step i's O, LSE (during its backward) and dQ, dK, dV (during step i+1) come
-    # down on another.  Every step's copies are inside the timed region: it starts
+    # buffers, step i+1's Q, K, V, dO go up on a side stream while step i computes
+    # (dO last: only the backward waits for it), and step i's O, LSE (during its
+    # backward) and dQ, dK, dV (during step i+1) come down on another.  Every step's copies are inside the timed region: it starts
     # before the first upload and ends after the last download has landed.
     main_s = torch.cuda.current_stream(device)
     up_s, down_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
     ins = [(q, k, v, do), tuple(torch.empty_like(x) for x in (q, k, v, do))]
     grads = [(dq, dk, dv), tuple(torch.empty_like(x) for x in (dq, dk, dv))]
-    in_ready, in_free, grads_out, o_out = [None, None], [None, None], [None, None], [None]
+    qkv_ready, do_ready = [None, None], [None, None]
+    in_free, grads_out, o_out = [None, None], [None, None], [None]
 
     def upload(i):
+        # Q, K, V first (the forward waits for them), then dO (only the backward does)
         b = i % 2
         with torch.cuda.stream(up_s):
             if in_free[b] is not None:            # step i-2 has gathered these buffers
                 up_s.wait_event(in_free[b])
-            for dst, src in zip(ins[b], (hq, hk, hv, hdo)):
+            for dst, src in zip(ins[b][:3], (hq, hk, hv)):
                 dst.copy_(src, non_blocking=True)
-            in_ready[b] = up_s.record_event()
+            qkv_ready[b] = up_s.record_event()
+            ins[b][3].copy_(hdo, non_blocking=True)
+            do_ready[b] = up_s.record_event()
 
     def compute(i):
         b = i % 2
         xq, xk, xv, xdo = ins[b]
-        main_s.wait_event(in_ready[b])
+        main_s.wait_event(qkv_ready[b])
         if o_out[0] is not None:                  # the previous O / LSE have come down
             main_s.wait_event(o_out[0])
         plan.build([xq, xk, xv], [qs, ks, vs])
@@ -461,6 +465,7 @@ def run_native(args, w, rank, world, local_rank):
             ho.copy_(o, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
             o_out[0] = down_s.record_event()
+        main_s.wait_event(do_ready[b])
         plan.build([xdo], [dos])
         in_free[b] = main_s.record_event()
         gq, gk, gv = grads[b]
@@ -545,8 +550,9 @@ def run_native(args, w, rank, world, local_rank):
                     "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
                     "overlap": "inputs of step i+1 up and gradients of step i down while "
-                               "step i / i+1 compute (two buffer sets); O/LSE down during "
-                               "the backward"},
+                               "step i / i+1 compute (two buffer sets); dO up after Q/K/V "
+                               "(the forward waits for Q/K/V only); O/LSE down during the "
+                               "backward"},
             "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": base,
