@@ -243,3 +243,53 @@ def test_head_dim_256(lib):
         cz.bwd_workspace_bytes(prob(head_dim=256, bwd_one_pass=True))
     assert fwd_query(prob(head_dim=192))[0] == _lib.CP_ERR_UNSUPPORTED
 
+
+
+def _rank_calls(p, rank, step, ws_bytes):
+    """The three per-rank entry points that take a workspace, with dummy aligned
+    device pointers and ws = NULL (a workspace query when the arguments pass, so
+    nothing launches): their statuses; the byte counts go to ws_bytes."""
+    d = ctypes.c_void_p(256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
+    pl = ctypes.byref(plan)
+    L = cz.lib()
+    n = [ctypes.c_size_t(0) for _ in range(3)]
+    st = [L.cp_attn_fwd_rank(p.ref, pl, rank, d, d, d, d, d, None, ctypes.byref(n[0]), None),
+          L.cp_attn_bwd_rank(p.ref, pl, rank, d, d, d, d, d, d, d, d, d, None, ctypes.byref(n[1]), None),
+          L.cp_attn_bwd_step(p.ref, pl, rank, step, d, d, d, d, d, d, d, d, d, None, ctypes.byref(n[2]),
+                             None)]
+    ws_bytes.extend(x.value for x in n)
+    return st
+
+
+def test_rank_calls_host_checks(lib):
+    """Rank and step must lie in [0, cp) (refused on the host, before any launch);
+    the workspace query of a good call reports the per-row scratch: the step
+    backward needs two fp32 values per local query row, like the per-rank one."""
+    p = prob()
+    sizes = []
+    assert _rank_calls(p, 0, 1, sizes) == [_lib.CP_OK] * 3
+    rows = 1 * 2 * (512 // 2)                           # batch x heads x 2C local rows
+    assert sizes[1] == sizes[2] and sizes[2] >= 2 * rows * 4
+    d = ctypes.c_void_p(256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
+    for rank, step in ((2, 0), (-1, 0), (0, 2), (0, -1)):
+        st = _rank_calls(p, rank, step, [])
+        assert st[2] == _lib.CP_ERR_INVALID_ARG, (rank, step, st)
+        assert cz.lib().cp_attn_fwd_step(p.ref, ctypes.byref(plan), rank, step, d, d, d, d, d,
+                                         None) == _lib.CP_ERR_INVALID_ARG, (rank, step)
+        if rank not in (0, 1):
+            assert st[0] == _lib.CP_ERR_INVALID_ARG and st[1] == _lib.CP_ERR_INVALID_ARG
+
+
+def test_bwd_step_null_pointers(lib):
+    p = prob()
+    d = ctypes.c_void_p(256)
+    plan = _lib.CpPlan(256, 256, 256, 256, 256, 256, 256, 256, 256)
+    n = ctypes.c_size_t(0)
+    for i in range(9):                                  # q k v o lse dout dq_sum dk_sum dv_sum
+        args = [d] * 9
+        args[i] = None
+        st = cz.lib().cp_attn_bwd_step(p.ref, ctypes.byref(plan), 0, 0, *args, None,
+                                       ctypes.byref(n), None)
+        assert st == _lib.CP_ERR_INVALID_ARG, i
