@@ -124,11 +124,12 @@ typedef enum { CP_MERGE_SEPARATE = 0, CP_MERGE_FUSED = 1 } cp_merge_t;
  *                 cp_plan_shards checks it on the device: a list that is not
  *                 strictly increasing from 0 to S records CP_ERR_INVALID_ARG in
  *                 the device status word (the host cannot see device memory
- *                 without synchronising).  cp_attn_bwd (and cp_attn_bwd_noalloc)
- *                 read it again on the device, for the document end of each key
+ *                 without synchronising).  The backward calls (cp_attn_bwd,
+ *                 cp_attn_bwd_noalloc, cp_attn_bwd_rank, cp_attn_bwd_step) read
+ *                 it again on the device, for the document end of each key
  *                 tile, without checking it: the list must stay allocated and
  *                 unchanged from cp_plan_shards until the backward has run.
- *                 cp_attn_fwd reads only the plan. */
+ *                 The forward calls read only the plan. */
 typedef struct {
     int32_t batch;
     int32_t seq_len;
