@@ -16,7 +16,9 @@ What it computes, and where each step is defined:
     (concept guide, "So how does it work?", pseudocode), read as the exact
     log-sum-exp merge;
   * unsharded attention and its explicit-P backward (the definition of scaled
-    dot-product attention with the causal / packed-document mask).
+    dot-product attention with the causal / packed-document mask), and that
+    backward unit by unit in the visit order: rank r's queries against shard j,
+    dQ_r summed over the steps and dK_j / dV_j over the ranks.
 
 Inputs are numpy float64 arrays [B, H, S, D] in original token order.
 """
@@ -80,10 +82,13 @@ def _load():
         lib.orc_bwd_dkv_keys_fwd.argtypes = [I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
                                              _f64p, _f64p, _f64p, _i32p, _i32p, I64, _i64p, _f64p,
                                              _f64p]
+        lib.orc_bwd_partial.argtypes = [I32, I32, I32, I32, I32, I32, F64, _f64p, _f64p, _f64p,
+                                        _f64p, _f64p, _f64p, _i32p, _i32p, _i32p, I32, I32,
+                                        _f64p, _f64p, _f64p]
         lib.orc_num_threads.argtypes = []
         for name in ("orc_doc_start", "orc_plan", "orc_fwd_rows", "orc_fwd", "orc_partial",
                      "orc_bwd", "orc_bwd_dq_rows", "orc_bwd_dkv_keys", "orc_bwd_dkv_keys_fwd",
-                     "orc_num_threads"):
+                     "orc_bwd_partial", "orc_num_threads"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -265,6 +270,48 @@ def bwd(q, k, v, o, lse, dout, ds_orig=None, scale=None, lk_orig=None):
     dv = np.zeros(k.shape, np.float64)
     _check(_load().orc_bwd(B, Hq, Hkv, S, D, _scale(D, scale), q, k, v, o, lse, dout, ds,
                            _lk(S, lk_orig), dq, dk, dv), "bwd")
+    return dq, dk, dv
+
+
+def bwd_partial(q, k, v, o, lse, dout, perm, cp, r, j, ds_orig=None, scale=None, lk_orig=None):
+    """The backward of unit (rank r, shard j) with the final o [B,Hq,S,D] / lse
+    [B,Hq,S] (original order): dQ [B,Hq,2C,D] of rank r's rows, dK / dV
+    [B,Hkv,2C,D] of shard j's rows (local shard order)."""
+    q, k, v, o, lse, dout = map(_f64, (q, k, v, o, lse, dout))
+    B, Hq, Hkv, S, D = _dims(q, k)
+    ds = np.zeros(S, np.int32) if ds_orig is None else np.ascontiguousarray(ds_orig, np.int32)
+    n2c = S // cp
+    dq = np.zeros((B, Hq, n2c, D), np.float64)
+    dk = np.zeros((B, Hkv, n2c, D), np.float64)
+    dv = np.zeros((B, Hkv, n2c, D), np.float64)
+    _check(_load().orc_bwd_partial(B, Hq, Hkv, S, D, cp, _scale(D, scale), q, k, v, o, lse, dout,
+                                   ds, _lk(S, lk_orig), np.ascontiguousarray(perm, np.int32), r, j,
+                                   dq, dk, dv), "bwd_partial")
+    return dq, dk, dv
+
+
+def cp_bwd(q, k, v, o, lse, dout, cp, rotate="allgather", cu_seqlens=None, scale=None,
+           steps=None, window=0, causal=True, shard="sequence"):
+    """The sharded backward, unit by unit in visit order: at step s rank r's
+    pieces against shard src[r][s] add into its dQ and into that shard's dK / dV
+    (all steps unless ``steps`` limits them).  o / lse: the final forward results
+    in original order.  Returns dQ [B,Hq,S,D], dK / dV [B,Hkv,S,D] in SHARD order."""
+    q, k = _f64(q), _f64(k)
+    B, Hq, Hkv, S, D = _dims(q, k)
+    pl = plan(S, cp, rotate, cu_seqlens, window, causal, shard)
+    ds = first_key(S, cu_seqlens, window)
+    lk = last_key(S, cu_seqlens, causal)
+    n2c = S // cp
+    dq = np.zeros((B, Hq, S, D), np.float64)
+    dk = np.zeros((B, Hkv, S, D), np.float64)
+    dv = np.zeros((B, Hkv, S, D), np.float64)
+    for s in range(cp if steps is None else steps):
+        for r in range(cp):
+            j = int(pl["src"][r * cp + s])
+            gq, gk, gv = bwd_partial(q, k, v, o, lse, dout, pl["perm"], cp, r, j, ds, scale, lk)
+            dq[:, :, r * n2c:(r + 1) * n2c] += gq
+            dk[:, :, j * n2c:(j + 1) * n2c] += gk
+            dv[:, :, j * n2c:(j + 1) * n2c] += gv
     return dq, dk, dv
 
 

@@ -306,6 +306,64 @@ int orc_partial(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, int32_
 }
 
 /*
+ * The backward of one (rank, step) unit: rank r's queries (its 2C rows) against
+ * shard j's keys (its 2C rows), by the explicit-P formula with P taken from the
+ * final LSE and D_q = sum_d dO*O from the final O (the row's own forward is not
+ * redone).  Inputs in ORIGINAL order, the rank's and the shard's tokens located
+ * through perm.  Outputs in local shard order: dq_part[B*Hq][2C][D] for rank
+ * r's rows, dk_part / dv_part[B*Hkv][2C][D] for shard j's rows.  Summed over
+ * the steps (dQ_r) and over the ranks (dK_j, dV_j) they are the gradients of
+ * the unsharded attention.
+ */
+int orc_bwd_partial(int32_t B, int32_t Hq, int32_t Hkv, int32_t S, int32_t D, int32_t cp,
+                    double scale, const double *q, const double *k, const double *v,
+                    const double *o, const double *lse, const double *dout,
+                    const int32_t *ds_orig, const int32_t *lk_orig, const int32_t *perm, int32_t r,
+                    int32_t j, double *dq_part, double *dk_part, double *dv_part)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0 || cp < 1 || S % (2 * cp) != 0 || r < 0 || r >= cp || j < 0 ||
+        j >= cp)
+        return ORC_EINVAL;
+    int64_t g = Hq / Hkv, n2c = S / cp, SD = (int64_t)S * D;
+    memset(dq_part, 0, sizeof(double) * (size_t)((int64_t)B * Hq * n2c * D));
+    memset(dk_part, 0, sizeof(double) * (size_t)((int64_t)B * Hkv * n2c * D));
+    memset(dv_part, 0, sizeof(double) * (size_t)((int64_t)B * Hkv * n2c * D));
+    /* one KV head per task: its dK/dV rows collect over the group's query heads */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bkv = 0; bkv < (int64_t)B * Hkv; ++bkv) {
+        int64_t b = bkv / Hkv, hk = bkv % Hkv;
+        const double *kh = k + bkv * SD, *vh = v + bkv * SD;
+        double *dkh = dk_part + bkv * n2c * D, *dvh = dv_part + bkv * n2c * D;
+        for (int64_t h = hk * g; h < (hk + 1) * g; ++h) {
+            int64_t bh = b * Hq + h;
+            for (int64_t t = 0; t < n2c; ++t) {
+                int64_t qi = perm[(int64_t)r * n2c + t];
+                const double *qv = q + (bh * S + qi) * D, *ov = o + (bh * S + qi) * D;
+                const double *dov = dout + (bh * S + qi) * D;
+                double *dqv = dq_part + (bh * n2c + t) * D;
+                double L = lse[bh * S + qi], Dq = 0.0;
+                for (int64_t d = 0; d < D; ++d) Dq += dov[d] * ov[d];
+                for (int64_t u = 0; u < n2c; ++u) {
+                    int64_t kk = perm[(int64_t)j * n2c + u];
+                    if (kk < ds_orig[qi] || kk > lk_orig[qi]) continue;
+                    const double *kv = kh + kk * D, *vv = vh + kk * D;
+                    double dot = 0.0, dP = 0.0;
+                    for (int64_t d = 0; d < D; ++d) { dot += qv[d] * kv[d]; dP += dov[d] * vv[d]; }
+                    double P = exp(scale * dot - L);
+                    double dS = P * (dP - Dq);
+                    for (int64_t d = 0; d < D; ++d) {
+                        dvh[u * D + d] += P * dov[d];
+                        dqv[d] += scale * dS * kv[d];
+                        dkh[u * D + d] += scale * dS * qv[d];
+                    }
+                }
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/*
  * combine(): fold n_parts partial (O, LSE) pairs, in the given order, into one.
  * For the running pair (O_a, L_a) and the next (O_b, L_b):
  *   m = max(L_a, L_b); if m = -inf the result stays (0, -inf); otherwise

@@ -89,17 +89,15 @@ class OracleKernels:
         return lf
 
     def bwd_step(self, prob, plan, rank, step, q, k, v, o, lse, do, dq_sum, dk_sum, dv_sum):
-        # keys outside shard j are zero rows of K and V: with P taken from the true LSE
-        # they add nothing to dQ, and only shard j's dK / dV rows are read back
+        # the oracle's unit backward: rank r's rows against shard j's keys
         j = int(self.pl["src"][rank * self.cp + step])
-        qf, of, dof = (self._place(x, rank, HQ) for x in (q, o, do))
-        dq, dk, dv = self.o.bwd(qf, self._place(k, j, HKV), self._place(v, j, HKV), of,
-                                self._place_lse(lse, rank), dof, self.ds)
-        pos_r = self.pl["perm"][rank * self.n2c:(rank + 1) * self.n2c]
-        pos_j = self.pl["perm"][j * self.n2c:(j + 1) * self.n2c]
-        dq_sum += torch.from_numpy(dq[:, :, pos_r]).float()
-        dk_sum += torch.from_numpy(dk[:, :, pos_j]).float()
-        dv_sum += torch.from_numpy(dv[:, :, pos_j]).float()
+        dq, dk, dv = self.o.bwd_partial(self._place(q, rank, HQ), self._place(k, j, HKV),
+                                        self._place(v, j, HKV), self._place(o, rank, HQ),
+                                        self._place_lse(lse, rank), self._place(do, rank, HQ),
+                                        self.pl["perm"], self.cp, rank, j, self.ds)
+        dq_sum += torch.from_numpy(dq).float()
+        dk_sum += torch.from_numpy(dk).float()
+        dv_sum += torch.from_numpy(dv).float()
 
     def to_bf16(self, x):
         return x.to(torch.bfloat16)

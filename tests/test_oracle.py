@@ -219,40 +219,50 @@ def test_sharded_merged_equals_unsharded(cp, rotate, docs):
     np.testing.assert_allclose(sl, lse[:, :, perm], atol=1e-12)
 
 
-@pytest.mark.parametrize("cp,S,docs,shard", [(3, 72, None, "sequence"),
-                                             (2, 64, [0, 3, 40, 41, 64], "sequence"),
-                                             (2, 64, [0, 16, 24, 64], "doc")])
-def test_bwd_ring_steps_sum_to_whole(cp, S, docs, shard):
-    """The backward split by ring step: rank r's queries against the one shard j =
-    src[r][s] it holds at step s (every other key's K, V rows zero, P taken from the
-    final LSE) give pieces of the gradients; over the steps the pieces of dQ_r, and
-    over the ranks those of dK_j / dV_j, add up to the unsharded gradients, and
-    leaving out the last step's pieces does not."""
+@pytest.mark.parametrize("cp,S,rotate,docs,shard,window,causal", [
+    (3, 72, "ring", None, "sequence", 0, True), (4, 64, "allgather", None, "sequence", 0, True),
+    (2, 64, "ring", [0, 3, 40, 41, 64], "sequence", 0, True),
+    (2, 64, "ring", [0, 16, 24, 64], "doc", 0, True), (2, 64, "allgather", None, "sequence", 9, True),
+    (2, 64, "ring", None, "sequence", 0, False)])
+def test_sharded_bwd_equals_unsharded(cp, S, rotate, docs, shard, window, causal):
+    """The backward unit by unit (rank r's queries against shard src[r][s], P from
+    the final LSE): dQ_r summed over the steps and dK_j / dV_j over the ranks give
+    the unsharded gradients, and stopping one step short does not."""
     D = 8
     q, k, v, do = rnd((1, 4, S, D), 24), rnd((1, 2, S, D), 25), rnd((1, 2, S, D), 26), rnd((1, 4, S, D), 27)
     cu = None if docs is None else np.array(docs, np.int32)
+    ds, lk = oracle.first_key(S, cu, window), oracle.last_key(S, cu, causal)
+    o, lse = oracle.fwd(q, k, v, ds, None, lk)
+    rq, rk, rv = oracle.bwd(q, k, v, o, lse, do, ds, None, lk)
+    perm = oracle.plan(S, cp, rotate, cu, window, causal, shard)["perm"]
+    kw = dict(window=window, causal=causal, shard=shard)
+    got = oracle.cp_bwd(q, k, v, o, lse, do, cp, rotate, cu, **kw)
+    for g, ref in zip(got, (rq, rk, rv)):
+        np.testing.assert_allclose(g, ref[:, :, perm], atol=1e-12)
+    short = oracle.cp_bwd(q, k, v, o, lse, do, cp, rotate, cu, steps=cp - 1, **kw)
+    assert max(np.abs(g - ref[:, :, perm]).max() for g, ref in zip(short, (rq, rk, rv))) > 1e-2
+
+
+def test_bwd_partial_is_the_masked_full_backward():
+    """One unit by another route: the full backward with every row outside rank r's
+    queries and every key outside shard j zeroed (P from the final LSE, so zero K, V
+    rows add nothing to dQ) read back at rank r's and shard j's rows."""
+    S, D, cp, r, j = 64, 8, 4, 1, 2
+    q, k, v, do = rnd((1, 4, S, D), 28), rnd((1, 2, S, D), 29), rnd((1, 2, S, D), 30), rnd((1, 4, S, D), 31)
+    cu = np.array([0, 5, 33, 64], np.int32)
     ds = oracle.doc_start(S, cu)
     o, lse = oracle.fwd(q, k, v, ds)
-    rq, rk, rv = oracle.bwd(q, k, v, o, lse, do, ds)
-    pl = oracle.plan(S, cp, "ring", cu, shard=shard)
-    perm, src, n2c = pl["perm"], pl["src"], S // cp
-    rows = lambda r: perm[r * n2c:(r + 1) * n2c]
-    keep = lambda x, p: np.where(np.isin(np.arange(S), p)[None, None, :, None], x, 0.0)
-    got = [np.zeros_like(rq), np.zeros_like(rk), np.zeros_like(rv)]
-    last = [np.zeros_like(rq), np.zeros_like(rk), np.zeros_like(rv)]
-    for s in range(cp):
-        for r in range(cp):
-            j = int(src[r * cp + s])
-            lr = np.where(np.isin(np.arange(S), rows(r))[None, None, :], lse, 0.0)
-            gq, gk, gv = oracle.bwd(keep(q, rows(r)), keep(k, rows(j)), keep(v, rows(j)),
-                                    keep(o, rows(r)), lr, keep(do, rows(r)), ds)
-            for acc in ([got] + ([last] if s == cp - 1 else [])):
-                acc[0][:, :, rows(r)] += gq[:, :, rows(r)]
-                acc[1][:, :, rows(j)] += gk[:, :, rows(j)]
-                acc[2][:, :, rows(j)] += gv[:, :, rows(j)]
-    for g, ref in zip(got, (rq, rk, rv)):
-        np.testing.assert_allclose(g, ref, atol=1e-12)
-    assert max(np.abs(g - l - ref).max() for g, l, ref in zip(got, last, (rq, rk, rv))) > 1e-2
+    perm = oracle.plan(S, cp, "ring", cu)["perm"]
+    rows = lambda x: perm[x * (S // cp):(x + 1) * (S // cp)]
+    on = lambda p: np.isin(np.arange(S), p)
+    keep = lambda x, p: np.where(on(p)[None, None, :, None], x, 0.0)
+    fq, fk, fv = oracle.bwd(keep(q, rows(r)), keep(k, rows(j)), keep(v, rows(j)), keep(o, rows(r)),
+                            np.where(on(rows(r))[None, None, :], lse, 0.0), keep(do, rows(r)), ds)
+    pq, pk, pv = oracle.bwd_partial(q, k, v, o, lse, do, perm, cp, r, j, ds)
+    np.testing.assert_allclose(pq, fq[:, :, rows(r)], atol=1e-13)
+    np.testing.assert_allclose(pk, fk[:, :, rows(j)], atol=1e-13)
+    np.testing.assert_allclose(pv, fv[:, :, rows(j)], atol=1e-13)
+    assert np.abs(pk).max() > 1e-3
 
 
 def test_local_only_attention_breaks_parity():
