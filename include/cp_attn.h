@@ -377,13 +377,17 @@ CP_API cp_status_t cp_attn_bwd_rank(const cp_problem_t* problem, const cp_plan_t
 
 /*
  * cp_attn_bwd_step -- one step of the ring form of the backward: rank r's
- * queries against the single K/V shard j = src[r][step] it holds at that step,
- * their gradients added into fp32 sums:
+ * queries against the single K/V shard j = src[r][step] it holds at that step
+ * (the ring rotation of the concept guide's "all-to-all vs all-gather", run
+ * for the gradients of the attention it computes), their gradients added into
+ * fp32 sums:
  *   q, o, dout      bf16 [B][Hq][2C][D], lse fp32 [B][Hq][2C]   rank r's shard
  *   k, v            bf16 [B][Hkv][2C][D]                         shard j
  *   dq_sum          fp32 [B][Hq][2C][D]   rank r's dQ, this step's share added
  *   dk_sum, dv_sum  fp32 [B][Hkv][2C][D]  shard j's dK / dV, rank r's share added
- * The sums are read and written (the caller zeroes them first).  In a ring the
+ * The sums are read and written (the caller zeroes them first), without
+ * atomics: two calls that add into the same sums must not run concurrently
+ * (issue them on one stream, or order them with events).  In a ring the
  * dK / dV sums travel with the K/V shard: after the cp steps (and one more hop)
  * every shard's sums have been added to by every rank and are back with their
  * owner; cp_f32_to_bf16 casts them (and dq_sum).  Two passes (a dK/dV pass over
